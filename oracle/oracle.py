@@ -1,0 +1,312 @@
+"""Python side of the CPU oracle for the SVDQuant W4A4 + low-rank linear layer.
+
+TEST INFRASTRUCTURE: only the tests, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
+module.  It never imports the CUDA package and the CUDA package never imports
+it.
+
+The arithmetic lives in two places, both written from the SVDQuant paper
+("SVDQuant: Absorbing Outliers by Low-Rank Components for 4-Bit Diffusion
+Models", arXiv 2411.05007):
+  * ``svdq_oracle.c`` (plain C, fp32 where the decision is fp32): number
+    formats, the per-group quantizer (Sec. 3), the activation path and the
+    fp32-accumulated GEMM;
+  * this file (numpy fp64): the smoothing factor (Sec. 4.2, "migrate outliers
+    from activations to weights"), the truncated SVD of the smoothed weight
+    (Sec. 4.2, Eckart-Young-Mirsky), the residual and the LoRA fold
+    (Sec. 5.2, "Integrate LoRA into Nunchaku").
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional
+
+import numpy as np
+
+NVFP4, INT4 = 0, 1
+_FMT = {"nvfp4": NVFP4, "int4": INT4, NVFP4: NVFP4, INT4: INT4}
+GROUP = {NVFP4: 16, INT4: 64}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "svdq_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "_build", "libsvdq_oracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle with gcc (IEEE fp32, no contraction, no fast-math)."""
+    os.makedirs(os.path.dirname(_LIB_PATH), exist_ok=True)
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math", "-std=gnu11",
+           "-shared", "-fPIC", "-o", tmp, _SRC, "-lm"]
+    subprocess.check_call(cmd)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        _lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        I = ctypes.c_int
+        L = ctypes.c_long
+        _lib.oracle_bf16_decode.restype = ctypes.c_float
+        _lib.oracle_bf16_decode.argtypes = [ctypes.c_uint16]
+        _lib.oracle_bf16_round.restype = ctypes.c_uint16
+        _lib.oracle_bf16_round.argtypes = [ctypes.c_double]
+        _lib.oracle_e2m1_decode.restype = ctypes.c_float
+        _lib.oracle_e2m1_decode.argtypes = [ctypes.c_uint8]
+        _lib.oracle_e2m1_round.restype = ctypes.c_uint8
+        _lib.oracle_e2m1_round.argtypes = [ctypes.c_float]
+        _lib.oracle_e4m3_decode.restype = ctypes.c_float
+        _lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+        _lib.oracle_e4m3_round_sat.restype = ctypes.c_uint8
+        _lib.oracle_e4m3_round_sat.argtypes = [ctypes.c_float]
+        _lib.oracle_fp16_decode.restype = ctypes.c_float
+        _lib.oracle_fp16_decode.argtypes = [ctypes.c_uint16]
+        _lib.oracle_fp16_round_sat.restype = ctypes.c_uint16
+        _lib.oracle_fp16_round_sat.argtypes = [ctypes.c_float]
+        _lib.oracle_quant_group_nvfp4.argtypes = [P, P, P]
+        _lib.oracle_quant_group_int4.argtypes = [P, P, P]
+        for name in ("oracle_bf16_round_array", "oracle_e4m3_round_array",
+                     "oracle_e2m1_round_array", "oracle_fp16_round_array"):
+            getattr(_lib, name).argtypes = [P, L, P]
+            getattr(_lib, name).restype = None
+        _lib.oracle_act_quant.argtypes = [I, I, I, I, P, P, P, P, P, P]
+        _lib.oracle_weight_quant.argtypes = [I, I, I, P, P, P]
+        _lib.oracle_linear_rows.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, P, I, P]
+        _lib.oracle_dequant.argtypes = [I, I, I, P, P, P]
+    return _lib
+
+
+def _ptr(a: Optional[np.ndarray]):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"], "oracle arrays must be C-contiguous"
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+# --------------------------------------------------------------------------
+# number formats
+# --------------------------------------------------------------------------
+
+def bf16_round(x) -> np.ndarray:
+    """Nearest bf16 (ties to even) of each element, as uint16 bit patterns."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    out = np.empty(x.shape, dtype=np.uint16)
+    lib().oracle_bf16_round_array(_ptr(x), x.size, _ptr(out))
+    return out
+
+
+def bf16_decode(bits) -> np.ndarray:
+    bits = np.ascontiguousarray(bits, dtype=np.uint16)
+    return (bits.astype(np.uint32) << 16).view(np.float32)
+
+
+def e4m3_round(x) -> np.ndarray:
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty(x.shape, dtype=np.uint8)
+    lib().oracle_e4m3_round_array(_ptr(x), x.size, _ptr(out))
+    return out
+
+
+def e2m1_round(x) -> np.ndarray:
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty(x.shape, dtype=np.uint8)
+    lib().oracle_e2m1_round_array(_ptr(x), x.size, _ptr(out))
+    return out
+
+
+def fp16_round(x) -> np.ndarray:
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty(x.shape, dtype=np.uint16)
+    lib().oracle_fp16_round_array(_ptr(x), x.size, _ptr(out))
+    return out
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    L = lib()
+    return np.array([L.oracle_e4m3_decode(int(c)) for c in np.ravel(codes)],
+                    dtype=np.float32).reshape(np.shape(codes))
+
+
+def e2m1_decode(codes) -> np.ndarray:
+    L = lib()
+    return np.array([L.oracle_e2m1_decode(int(c)) for c in np.ravel(codes)],
+                    dtype=np.float32).reshape(np.shape(codes))
+
+
+def fp16_decode(codes) -> np.ndarray:
+    L = lib()
+    return np.array([L.oracle_fp16_decode(int(c)) for c in np.ravel(codes)],
+                    dtype=np.float32).reshape(np.shape(codes))
+
+
+def quant_group(fmt, v) -> tuple:
+    """One group (16 values NVFP4 / 64 values INT4) -> (codes one per byte, scale code)."""
+    fmt = _FMT[fmt]
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    assert v.size == GROUP[fmt]
+    codes = np.zeros(v.size, dtype=np.uint8)
+    if fmt == NVFP4:
+        sc = np.zeros(1, dtype=np.uint8)
+        lib().oracle_quant_group_nvfp4(_ptr(v), _ptr(codes), _ptr(sc))
+    else:
+        sc = np.zeros(1, dtype=np.uint16)
+        lib().oracle_quant_group_int4(_ptr(v), _ptr(codes), _ptr(sc))
+    return codes, int(sc[0])
+
+
+# --------------------------------------------------------------------------
+# preparation (offline, Sec. 4.2 and Sec. 5.2)
+# --------------------------------------------------------------------------
+
+def smoothing(x_absmax: Optional[np.ndarray], W_bits: np.ndarray):
+    """Per-input-channel smoothing factor lambda and its fp32 reciprocal.
+
+    lambda_j = sqrt(max|X_j| / max|W_j|) in fp64, rounded to fp32 (the
+    square-root balance of SmoothQuant, which SVDQuant Sec. 4.2 cites for
+    migrating outliers); lambda_j = 1 where either maximum is 0 or no
+    calibration maximum is given.  inv_lambda = fp32(1) / lambda (fp32 IEEE).
+    """
+    W = bf16_decode(W_bits).astype(np.float64)
+    K = W.shape[0]
+    if x_absmax is None:
+        lam = np.ones(K, dtype=np.float32)
+    else:
+        xm = np.asarray(x_absmax, dtype=np.float32).astype(np.float64)
+        wm = np.max(np.abs(W), axis=1)
+        ok = (xm > 0) & (wm > 0)
+        lam64 = np.ones(K, dtype=np.float64)
+        lam64[ok] = np.sqrt(xm[ok] / wm[ok])
+        lam = lam64.astype(np.float32)
+    inv = (np.float32(1.0) / lam).astype(np.float32)
+    return lam, inv
+
+
+def calib_absmax(X_bits: np.ndarray) -> np.ndarray:
+    """max_m |X[m, j]| per input channel (exact; the calibration statistic)."""
+    return np.max(np.abs(bf16_decode(X_bits)), axis=0).astype(np.float32)
+
+
+def prepare(W_bits: np.ndarray, x_absmax: Optional[np.ndarray], rank: int,
+            lora_A_bits: Optional[np.ndarray] = None,
+            lora_B_bits: Optional[np.ndarray] = None) -> dict:
+    """Smoothing, truncated SVD, residual and optional LoRA fold, in fp64.
+
+    W_hat = diag(lambda) W; W_hat = U S V^T (numpy/LAPACK fp64);
+    L1 = U[:, :r] S[:r] and L2 = V^T[:r, :] (the optimal rank-r factors),
+    rounded to bf16; R = fp32(W_hat - L1_bf16 L2_bf16), so the residual is
+    taken against the factors the layer actually uses.  A LoRA (A: K x rl,
+    B: rl x N) joins the branch as L1' = [L1 | bf16(diag(lambda) A)],
+    L2' = [L2 ; B] without touching R (no requantization).
+    """
+    W = bf16_decode(W_bits).astype(np.float64)
+    K, N = W.shape
+    lam, inv = smoothing(x_absmax, W_bits)
+    W_hat = lam.astype(np.float64)[:, None] * W
+    U, S, Vt = np.linalg.svd(W_hat, full_matrices=False)
+    r = int(rank)
+    L1_exact = U[:, :r] * S[:r]
+    L2_exact = Vt[:r, :]
+    L1 = bf16_round(L1_exact)
+    L2 = bf16_round(L2_exact)
+    R64 = W_hat - bf16_decode(L1).astype(np.float64) @ bf16_decode(L2).astype(np.float64)
+    R = R64.astype(np.float32)
+    out = {"lam": lam, "inv_lambda": inv, "W_hat": W_hat, "sigma": S,
+           "L1_exact": L1_exact, "L2_exact": L2_exact, "L1": L1, "L2": L2, "R": R,
+           "rank": r}
+    if lora_A_bits is not None:
+        A = bf16_decode(lora_A_bits).astype(np.float64)
+        L1_lora = bf16_round(lam.astype(np.float64)[:, None] * A)
+        out["L1"] = np.ascontiguousarray(np.concatenate([L1, L1_lora], axis=1))
+        out["L2"] = np.ascontiguousarray(np.concatenate([L2, lora_B_bits], axis=0))
+        out["rank"] = r + A.shape[1]
+    return out
+
+
+# --------------------------------------------------------------------------
+# quantization and the layer (C oracle)
+# --------------------------------------------------------------------------
+
+def weight_quant(fmt, R: np.ndarray):
+    """Quantize R (K x N fp32) along K per output column -> codes (N x K/2), scales (N x K/g)."""
+    fmt = _FMT[fmt]
+    R = np.ascontiguousarray(R, dtype=np.float32)
+    K, N = R.shape
+    g = GROUP[fmt]
+    codes = np.zeros((N, K // 2), dtype=np.uint8)
+    scales = np.zeros((N, K // g), dtype=np.uint8 if fmt == NVFP4 else np.uint16)
+    rc = lib().oracle_weight_quant(fmt, K, N, _ptr(R), _ptr(codes), _ptr(scales))
+    assert rc == 0
+    return codes, scales
+
+
+def act_quant(fmt, X_bits: np.ndarray, inv_lambda: Optional[np.ndarray], L1_bits: Optional[np.ndarray]):
+    """Smooth, quantize and down-project X (M x K bf16) -> codes, scales, XL1 (M x r bf16)."""
+    fmt = _FMT[fmt]
+    X_bits = np.ascontiguousarray(X_bits, dtype=np.uint16)
+    M, K = X_bits.shape
+    g = GROUP[fmt]
+    r = 0 if L1_bits is None else L1_bits.shape[1]
+    codes = np.zeros((M, K // 2), dtype=np.uint8)
+    scales = np.zeros((M, K // g), dtype=np.uint8 if fmt == NVFP4 else np.uint16)
+    XL1 = np.zeros((M, r), dtype=np.uint16)
+    inv = None if inv_lambda is None else np.ascontiguousarray(inv_lambda, dtype=np.float32)
+    L1 = None if L1_bits is None else np.ascontiguousarray(L1_bits, dtype=np.uint16)
+    rc = lib().oracle_act_quant(fmt, M, K, r, _ptr(X_bits), _ptr(inv), _ptr(L1),
+                                _ptr(codes), _ptr(scales), _ptr(XL1))
+    assert rc == 0
+    return codes, scales, XL1
+
+
+def linear(fmt, act, wq, L2_bits: Optional[np.ndarray], bias_bits: Optional[np.ndarray],
+           N: int, rows: Optional[np.ndarray] = None) -> np.ndarray:
+    """Y rows (bf16 bits): 4-bit GEMM over groups + XL1 L2 + bias, fp32 accumulation."""
+    fmt = _FMT[fmt]
+    cx, sx, XL1 = act
+    cw, sw = wq
+    M = cx.shape[0]
+    K = cx.shape[1] * 2
+    r = XL1.shape[1]
+    if r:
+        assert L2_bits is not None and L2_bits.shape == (r, N)
+    rows_arr = None if rows is None else np.ascontiguousarray(rows, dtype=np.int32)
+    n_rows = M if rows is None else len(rows_arr)
+    Y = np.zeros((n_rows, N), dtype=np.uint16)
+    L2 = None if not r else np.ascontiguousarray(L2_bits, dtype=np.uint16)
+    bias = None if bias_bits is None else np.ascontiguousarray(bias_bits, dtype=np.uint16)
+    rc = lib().oracle_linear_rows(fmt, M, N, K, r, _ptr(cx), _ptr(sx), _ptr(XL1), _ptr(cw),
+                                  _ptr(sw), _ptr(L2), _ptr(bias), _ptr(rows_arr), n_rows, _ptr(Y))
+    assert rc == 0
+    return Y
+
+
+def dequant(fmt, codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """s * deq(q) for packed codes (rows x K/2) -> fp32 rows x K."""
+    fmt = _FMT[fmt]
+    rows, K = codes.shape[0], codes.shape[1] * 2
+    out = np.zeros((rows, K), dtype=np.float32)
+    rc = lib().oracle_dequant(fmt, rows, K, _ptr(np.ascontiguousarray(codes)),
+                              _ptr(np.ascontiguousarray(scales)), _ptr(out))
+    assert rc == 0
+    return out
+
+
+def layer(fmt, X_bits, W_bits, rank: int, bias_bits=None, lora_A_bits=None, lora_B_bits=None,
+          x_absmax=None, smooth: bool = True, rows=None) -> dict:
+    """The whole layer: prepare (fp64), quantize W and X, GEMM; returns every intermediate."""
+    if smooth and x_absmax is None:
+        x_absmax = calib_absmax(X_bits)
+    prep = prepare(W_bits, x_absmax if smooth else None, rank, lora_A_bits, lora_B_bits)
+    wq = weight_quant(fmt, prep["R"])
+    r = prep["rank"]
+    act = act_quant(fmt, X_bits, prep["inv_lambda"], prep["L1"] if r else None)
+    Y = linear(fmt, act, wq, prep["L2"] if r else None, bias_bits, W_bits.shape[1], rows)
+    return {"prep": prep, "wq": wq, "act": act, "Y": Y}
