@@ -1,0 +1,350 @@
+#!/usr/bin/env python
+"""Benchmark of the SVDQuant W4A4 + low-rank linear layer on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+the fused activation kernel (smoothing + quantize + down-projection) and the
+fused 4-bit GEMM (+ up-projection + bias), both through the C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--config c2_qkv] [--layer qkv] [--M 4608]
+
+Default workload: the FLUX attention QKV projection, M = 4608 tokens
+(4096 image + 512 text), K = 3072 -> N = 9216, rank 32, NVFP4.  The metric is
+the effective throughput 2*M*K*N / (layer time), in TFLOP/s; the line also
+carries us/layer, the per-kernel times, the GEMM's roofline fraction against
+the FP4 tensor peak and the activation kernel's against HBM bandwidth.
+
+Between timed steps a 512 MiB buffer is rewritten to flush the 126 MB L2.
+Under torchrun every rank runs its own batch of the same layer (token-parallel
+weak scaling, no data-path collective); the time is the max over ranks.
+
+`--impl reference` times the CPU oracle (test infrastructure: a plain C /
+numpy restatement of the method) on a bounded sample of rows of the same
+workload and prints the same JSON line with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads as WL  # noqa: E402
+
+METRIC = "SVDQuant W4A4+low-rank linear: µs/layer, effective TFLOPS, % of FP4 peak"
+UNIT = "TFLOP/s"
+FLUSH_BYTES = 512 << 20
+
+
+def peaks():
+    """Roofline denominators: the machine's measured copy bandwidth and bf16 GEMM
+    throughput; dense FP4 / INT8 = measured bf16 x the nominal ratio (4x / 2x)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            m = json.load(f)
+        return {"hbm_gbs": float(m["hbm_gbs"]), "bf16": float(m["bf16_tflops"]),
+                "bf16_sustained": float(m["bf16_tflops_sustained"]), "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        try:
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = max(mx, float(parts[2]))
+                except ValueError:
+                    continue
+                for nm, val in zip(names, parts[5:9]):
+                    if val.lower() == "active":
+                        reasons.add(nm)
+        finally:
+            os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def layer_inputs(args):
+    spec = WL.layer_spec(args.config, args.layer)
+    M = args.M or WL.CONFIGS[args.config].Ms[-1 if args.config == "c5_block" else 0]
+    return spec, M
+
+
+# ----------------------------------------------------------------------------- ours
+def run_ours(args):
+    import w4a4_gemm_b200 as S
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    S.lib()
+    spec, M = layer_inputs(args)
+    K, N = spec.K, spec.N
+    W, bias, A, B = WL.make_weights(spec)
+    X = WL.make_activations(spec, M).to(dev)
+    W = W.to(dev)
+    xabs = S.svdq_calib_absmax(X)
+    w = S.svdq_prepare_weights(W, spec.rank, spec.fmt, x_absmax=xabs,
+                               bias=bias.to(dev) if bias is not None else None,
+                               lora_A=A.to(dev) if A is not None else None,
+                               lora_B=B.to(dev) if B is not None else None)
+    del W
+    ws = S.alloc_workspace(w, M, dev)
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    launches_per_step = 2 + (1 if (spec.fmt == "nvfp4" and K % 256) else 0)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        S.svdq_quantize_act(w, X, ws)
+        if ev:
+            ev[1].record(stream)
+        S.svdq_linear(w, ws, M, Y)
+        if ev:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if S.svdq_get_error():
+        raise RuntimeError("device wait timed out during warm-up")
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    for i in range(args.steps):
+        flush.zero_()          # L2 flush between steps, outside the timed events
+        step(events[i])
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if world > 1:
+        torch.distributed.barrier()
+    t_q = np.array([e[0].elapsed_time(e[1]) for e in events]) * 1e-3   # s
+    t_g = np.array([e[1].elapsed_time(e[2]) for e in events]) * 1e-3
+    t_layer = t_q + t_g
+    total = float(t_layer.sum())
+    if world > 1:
+        t = torch.tensor([total, float(t_q.mean()), float(t_g.mean())], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total, tq_mean, tg_mean = (float(v) for v in t.tolist())
+    else:
+        tq_mean, tg_mean = float(t_q.mean()), float(t_g.mean())
+
+    # end to end through the public API: pinned host X in, host Y out, every step
+    X_host = X.cpu().pin_memory()
+    Y_host = torch.empty(M, N, dtype=torch.bfloat16).pin_memory()
+    X_dev = torch.empty_like(X)
+    e2e_steps = max(3, min(args.steps, 10))
+    for _ in range(2):
+        X_dev.copy_(X_host, non_blocking=True)
+        S.svdq_forward(w, X_dev, Y, ws)
+        Y_host.copy_(Y, non_blocking=True)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        X_dev.copy_(X_host, non_blocking=True)
+        S.svdq_forward(w, X_dev, Y, ws)
+        Y_host.copy_(Y, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t_e2e = e0.elapsed_time(e1) * 1e-3 / e2e_steps
+    if S.svdq_get_error():
+        raise RuntimeError("device wait timed out during timing")
+
+    flops = 2.0 * M * K * N
+    r = w.rank
+    pk = peaks()
+    fp_peak = pk["bf16"] * (4.0 if spec.fmt == "nvfp4" else 2.0)
+    gemm_flops = flops + 2.0 * M * r * N
+    achieved = gemm_flops / tg_mean / 1e12
+    # activation kernel: algorithmic bytes (X read, codes + scales + XL1 written)
+    code_bytes = M * K / 2 if spec.fmt == "nvfp4" else M * K
+    scale_bytes = M * K / 16 if spec.fmt == "nvfp4" else M * K / 64 * 2
+    q_bytes = 2.0 * M * K + code_bytes + scale_bytes + 2.0 * M * w.rank_padded
+    q_gbs = q_bytes / tq_mean / 1e9
+    value = world * flops * args.steps / total / 1e12
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(total / args.steps * 1e3, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e2m1xe2m1+bf16 (fp32 acc)" if spec.fmt == "nvfp4" else "s8xs8+bf16 (fp32 acc)",
+        "data": "synthetic (seeded FLUX-shaped activations and weights; no checkpoints)",
+        "config": {"workload": f"{args.config}/{spec.name}: M={M} K={K} N={N} rank={r} {spec.fmt}",
+                   "M": M, "K": K, "N": N, "rank": r, "format": spec.fmt,
+                   "l2": "flushed between steps (512 MiB write)", "parallelism": f"dp{world} (token batches)"},
+        "us_per_layer": round(total / args.steps * 1e6, 2),
+        "us_quant": round(tq_mean * 1e6, 2), "us_gemm": round(tg_mean * 1e6, 2),
+        "pct_fp4_peak_layer": round(100.0 * flops / (total / args.steps) / 1e12 / fp_peak, 2),
+        "roofline": {"bound": "tensor", "kernel": "gemm_nvfp4_kernel" if spec.fmt == "nvfp4" else "gemm_int4_kernel",
+                     "achieved": round(achieved, 1), "peak": round(fp_peak, 1), "unit": "TFLOP/s",
+                     "frac": round(achieved / fp_peak, 4), "traffic": None,
+                     "peak_note": f"{pk['source']}: bf16 {pk['bf16']} TF/s x {'4 (FP4)' if spec.fmt == 'nvfp4' else '2 (INT8)'}"},
+        "roofline_quant": {"bound": "hbm", "kernel": "quant_act_kernel", "achieved": round(q_gbs, 1),
+                           "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": round(q_gbs / pk["hbm_gbs"], 4),
+                           "algorithmic_bytes": int(q_bytes)},
+        "e2e": {"value": round(flops / t_e2e / 1e12, 3), "unit": UNIT,
+                "h2d_bytes_per_step": int(X.numel() * 2), "d2h_bytes_per_step": int(Y.numel() * 2)},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(spec, M, args.cpu_rows)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    w.close()
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------- oracle
+def _oracle_setup(spec, M, rows):
+    import oracle as O
+    W, bias, A, B = WL.make_weights(spec)
+    X = WL.make_activations(spec, M)
+    Xb = WL.bf16_bits(X)
+    xm = O.calib_absmax(Xb)
+    prep = O.prepare(WL.bf16_bits(W), xm, spec.rank,
+                     WL.bf16_bits(A) if A is not None else None,
+                     WL.bf16_bits(B) if B is not None else None)
+    wq = O.weight_quant(spec.fmt, prep["R"])
+    sample = np.ascontiguousarray(Xb[:rows])
+    return O, prep, wq, sample, (WL.bf16_bits(bias) if bias is not None else None)
+
+
+def _oracle_step(O, spec, prep, wq, sample, bias):
+    act = O.act_quant(spec.fmt, sample, prep["inv_lambda"], prep["L1"] if prep["rank"] else None)
+    O.linear(spec.fmt, act, wq, prep["L2"] if prep["rank"] else None, bias, spec.N)
+
+
+def cpu_baseline(spec, M, rows):
+    O, prep, wq, sample, bias = _oracle_setup(spec, M, rows)
+    t0 = time.perf_counter()
+    _oracle_step(O, spec, prep, wq, sample, bias)
+    dt = time.perf_counter() - t0
+    cores = len(os.sched_getaffinity(0))
+    return {"value": round(2.0 * rows * spec.K * spec.N / dt / 1e12, 6), "unit": UNIT, "cores": cores,
+            "kind": "oracle",
+            "sample": f"first {rows} of {M} token rows (quantize + GEMM + low-rank + bias, all N); "
+                      f"OpenMP over rows; weight preparation untimed"}
+
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    spec, M = layer_inputs(args)
+    rows = args.cpu_rows
+    O, prep, wq, sample, bias = _oracle_setup(spec, M, rows)
+    for _ in range(args.warmup):
+        _oracle_step(O, spec, prep, wq, sample, bias)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        _oracle_step(O, spec, prep, wq, sample, bias)
+    dt = (time.perf_counter() - t0) / args.steps
+    value = 2.0 * rows * spec.K * spec.N / dt / 1e12
+    cores = len(os.sched_getaffinity(0))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp32 (CPU oracle)",
+        "data": "synthetic (seeded FLUX-shaped activations and weights; no checkpoints)",
+        "config": {"workload": f"{args.config}/{spec.name}: M={M} K={spec.K} N={spec.N} rank={spec.rank} {spec.fmt}",
+                   "sample_rows": rows},
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"first {rows} of {M} token rows per step"},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="c2_qkv", choices=sorted(WL.CONFIGS))
+    ap.add_argument("--layer", default=None)
+    ap.add_argument("--M", type=int, default=None)
+    ap.add_argument("--cpu-rows", type=int, default=64)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

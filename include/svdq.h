@@ -1,0 +1,172 @@
+/*
+ * svdq.h -- C ABI of the B200 (sm_100a) SVDQuant W4A4 + low-rank linear layer.
+ *
+ * The layer is the one of "SVDQuant: Absorbing Outliers by Low-Rank
+ * Components for 4-Bit Diffusion Models" (arXiv 2411.05007), Sec. 4.2, Eq. 5:
+ *
+ *     Y = X_hat L1 L2 + Q(X_hat) Q(R) + bias,     X_hat = X diag(lambda)^-1,
+ *
+ * where lambda smooths each input channel, L1 (K x r) and L2 (r x N) are the
+ * 16-bit rank-r factors of the smoothed weight W_hat = diag(lambda) W from its
+ * truncated SVD, R = W_hat - L1 L2 is the residual, and Q is the symmetric
+ * per-group 4-bit quantizer of Sec. 3.  Two 4-bit formats are supported:
+ *   SVDQ_NVFP4: E2M1 codes with one E4M3 scale per 16 values along K;
+ *   SVDQ_INT4 : signed 4-bit integers in [-7, 7] with one fp16 scale per 64
+ *               values along K (Sec. 5.1).
+ *
+ * Conventions for every call:
+ *   - "device" pointers are CUDA global-memory pointers on the current device;
+ *     "host" pointers are ordinary CPU memory.  The caller owns every pointer
+ *     it passes; the library owns the memory behind an svdq_weights handle.
+ *   - bf16 tensors are raw IEEE bfloat16 (2 bytes), row-major and contiguous.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  The hot
+ *     calls (svdq_quantize_act, svdq_linear, svdq_forward) are asynchronous on
+ *     it, never allocate and never synchronize.  Preparation, LoRA appending
+ *     and the export calls may allocate and synchronize.
+ *   - Every call returns an svdq_status; on failure nothing has been launched
+ *     unless the status is SVDQ_ERR_CUDA.
+ *
+ * Shape rules: K % 64 == 0, N % 16 == 0, M >= 0 (M == 0 is a no-op),
+ * 0 <= rank (+ LoRA rank) <= 256 and rank <= min(K, N).  Device pointers to
+ * X, Y and the workspace must be 16-byte aligned (cudaMalloc gives 256).
+ */
+#ifndef SVDQ_H_
+#define SVDQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define SVDQ_API __attribute__((visibility("default")))
+#else
+#define SVDQ_API
+#endif
+
+typedef enum {
+  SVDQ_OK = 0,
+  SVDQ_ERR_INVALID_ARG = 1,       /* null pointer, bad enum, misaligned pointer */
+  SVDQ_ERR_UNSUPPORTED_SHAPE = 2, /* violates the shape rules above */
+  SVDQ_ERR_ALLOC = 3,             /* a preparation-time cudaMalloc failed */
+  SVDQ_ERR_CUDA = 4,              /* a CUDA runtime / driver call failed */
+  SVDQ_ERR_TIMEOUT = 5,           /* a bounded device wait ran out (svdq_get_error) */
+  SVDQ_ERR_LIBRARY = 6            /* cuSOLVER / cuBLAS failed during preparation */
+} svdq_status;
+
+typedef enum { SVDQ_NVFP4 = 0, SVDQ_INT4 = 1 } svdq_format;
+
+/* Opaque prepared layer: 4-bit residual codes and scales, the bf16 low-rank
+ * factors, 1/lambda and the bias, all in device memory owned by the handle. */
+typedef struct svdq_weights svdq_weights;
+
+/* Inputs of svdq_prepare_weights (all device pointers). */
+typedef struct {
+  int fmt;                 /* svdq_format */
+  int K, N;                /* W is K x N: input channels x output channels */
+  int rank;                /* r of the SVD branch, 0 = plain W4A4 */
+  const void* W;           /* bf16 K x N */
+  const float* x_absmax;   /* K calibration maxima max|X_j|, or NULL (lambda = 1) */
+  const void* bias;        /* bf16 N, or NULL */
+  const void* lora_A;      /* bf16 K x lora_rank, or NULL */
+  const void* lora_B;      /* bf16 lora_rank x N, or NULL */
+  int lora_rank;           /* 0 = no LoRA */
+} svdq_prepare_desc;
+
+/* Inputs of svdq_load_weights: an already decomposed layer (device pointers). */
+typedef struct {
+  int fmt, K, N, rank;
+  const float* inv_lambda; /* K values of 1/lambda, or NULL (all ones) */
+  const float* lambda;     /* K values of lambda (used by svdq_append_lora), or NULL = 1/inv_lambda */
+  const void* L1;          /* bf16 K x rank (ignored if rank == 0) */
+  const void* L2;          /* bf16 rank x N (ignored if rank == 0) */
+  const float* R;          /* fp32 K x N residual, quantized here */
+  const void* bias;        /* bf16 N, or NULL */
+} svdq_parts_desc;
+
+/* Calibration statistic for the smoothing factor (Sec. 4.2):
+ * absmax[k] = max(absmax[k], max_m |X[m, k]|) if accumulate != 0, else
+ * absmax[k] = max_m |X[m, k]|.  X: device bf16 M x K; absmax: device float K.
+ * Asynchronous on `stream`. */
+SVDQ_API int svdq_calib_absmax(const void* X, int M, int K, float* absmax, int accumulate,
+                               void* stream);
+
+/* Offline preparation (Sec. 4.2 and Sec. 5.2): lambda_j = sqrt(max|X_j| /
+ * max|W_j|) (fp64, rounded to fp32); W_hat = diag(lambda) W; the optimal
+ * rank-r factors from the eigen-decomposition of the fp64 Gram matrix of
+ * W_hat (cuSOLVER), rounded to bf16; R = W_hat - L1 L2; Q(R); optional LoRA
+ * folded into the branch without requantizing R.  Allocates device memory
+ * (SVDQ_ERR_ALLOC) and synchronizes `stream`.  *out receives a new handle. */
+SVDQ_API int svdq_prepare_weights(const svdq_prepare_desc* desc, void* stream,
+                                  svdq_weights** out);
+
+/* Build a handle from given factors (e.g. a layer prepared offline elsewhere):
+ * copies 1/lambda, lambda, L1, L2 and the bias, and quantizes R on the device
+ * with the same quantizer as svdq_prepare_weights.  Synchronizes `stream`. */
+SVDQ_API int svdq_load_weights(const svdq_parts_desc* desc, void* stream, svdq_weights** out);
+
+/* Fold a LoRA (A: bf16 K x lora_rank, B: bf16 lora_rank x N, device) into the
+ * low-rank branch (Sec. 5.2): L1 <- [L1 | bf16(diag(lambda) A)], L2 <- [L2 ; B].
+ * The 4-bit residual codes are not touched.  Synchronizes `stream`. */
+SVDQ_API int svdq_append_lora(svdq_weights* w, const void* lora_A, const void* lora_B,
+                              int lora_rank, void* stream);
+
+/* Shape of a handle; any output pointer may be NULL. */
+SVDQ_API int svdq_weights_info(const svdq_weights* w, int* fmt, int* K, int* N, int* rank,
+                               int* rank_padded);
+
+/* Bytes of the activation workspace svdq_quantize_act fills for M tokens
+ * (codes, scales and X_hat L1).  The caller allocates it (device, 256-byte
+ * aligned) and may reuse it across calls with the same or smaller M. */
+SVDQ_API int svdq_act_workspace_bytes(const svdq_weights* w, int M, size_t* bytes);
+
+/* Fused activation kernel (Sec. 4.3, "quantize + down-projection"): one pass
+ * over X (device bf16 M x K) writes Q(X diag(lambda)^-1) codes and scales and
+ * bf16(X_hat) L1 into `workspace`.  Asynchronous on `stream`. */
+SVDQ_API int svdq_quantize_act(const svdq_weights* w, const void* X, int M, void* workspace,
+                               void* stream);
+
+/* Fused 4-bit GEMM + up-projection + bias (Sec. 4.3): Y (device bf16 M x N) =
+ * Q(X_hat) Q(R) + (X_hat L1) L2 + bias, from a workspace that
+ * svdq_quantize_act filled for the same M.  Asynchronous on `stream`. */
+SVDQ_API int svdq_linear(const svdq_weights* w, const void* workspace, int M, void* Y,
+                         void* stream);
+
+/* svdq_quantize_act followed by svdq_linear. */
+SVDQ_API int svdq_forward(const svdq_weights* w, const void* X, int M, void* Y, void* workspace,
+                          void* stream);
+
+/* Debug export of a filled workspace in plain layouts (host outputs, any may
+ * be NULL; synchronizes the device):
+ *   codes  M x K/2 bytes, element 2i in the low nibble (INT4: two's complement);
+ *   scales M x K/16 E4M3 bytes (NVFP4) or M x K/64 fp16 (INT4);
+ *   xl1    M x rank bf16. */
+SVDQ_API int svdq_export_act(const svdq_weights* w, const void* workspace, int M,
+                             uint8_t* codes, void* scales, void* xl1);
+
+/* Debug export of a handle in plain layouts (host outputs, any may be NULL):
+ *   codes N x K/2 (per output column, along K), scales N x K/16 or N x K/64,
+ *   L1 K x rank bf16, L2 rank x N bf16, inv_lambda K floats, lambda K floats. */
+SVDQ_API int svdq_export_weights(const svdq_weights* w, uint8_t* codes, void* scales, void* L1,
+                                 void* L2, float* inv_lambda, float* lambda);
+
+/* Sticky device error word of the current device: bit 0 = a bounded wait ran
+ * out in the activation kernel, bit 1 = in a GEMM kernel.  Reading clears it.
+ * Returns the word (>= 0) or -SVDQ_ERR_CUDA.  Synchronizes the device. */
+SVDQ_API int svdq_get_error(void);
+
+/* Clock-cycle budget of every bounded device wait (default 2^31, about one
+ * second; the environment variable SVDQ_WAIT_BUDGET_CYCLES also sets it). */
+SVDQ_API int svdq_set_wait_budget(long long cycles);
+
+SVDQ_API const char* svdq_status_string(int status);
+
+SVDQ_API void svdq_weights_destroy(svdq_weights* w);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SVDQ_H_ */

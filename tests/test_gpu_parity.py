@@ -1,0 +1,176 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle.
+
+Codes and scales must be bit-exact; X_hat L1 and Y must be within
+|d| <= 2^-7 |y| + 1e-3 rms(Y).  Both sides get the same seeded inputs; the
+library gets the oracle's prepared factors (so both quantize the same R),
+except in the tests of the library's own preparation, which are checked
+against invariants of the SVD instead.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import workloads as WL
+from gpu_common import (bits, load_from_oracle, oracle_layer, require_gpu, svdq, to_dev_bits,
+                        to_dev_f32, y_within_tol)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def S():
+    require_gpu()
+    return svdq()
+
+
+def _run_layer(S, w, X_bits):
+    X = to_dev_bits(X_bits)
+    M = X.shape[0]
+    ws = S.alloc_workspace(w, M)
+    Y = torch.empty(M, w.N, dtype=torch.bfloat16, device="cuda")
+    S.svdq_quantize_act(w, X, ws)
+    S.svdq_linear(w, ws, M, Y)
+    torch.cuda.synchronize()
+    assert S.svdq_get_error() == 0
+    return ws, Y
+
+
+def test_weight_quantizer_edge_values(S):
+    """Ties, subnormal and saturating scales, negative values rounding to zero."""
+    groups = [
+        [6, 3, -1.5, 0.25] + [0] * 12,
+        [1, 0.75, -0.5, 0.1] + [0] * 12,
+        [6, 5, 2.5, 0.75, 1.25, 1.75, 3.5, -5, -0.25, 0.5] + [0] * 6,
+        [0.003, -0.002, 0.001] + [0] * 13,
+        [0.006, -0.0012] + [0] * 14,
+        [3000, 2300, 2200, -1000] + [0] * 12,
+        [-0.01, 1, -0.2, 0.12] + [0] * 12,
+        [0.0] * 16,
+    ]
+    rng = np.random.default_rng(11)
+    K = 256
+    cols = []
+    for g in groups:
+        c = np.zeros(K, dtype=np.float32)
+        c[:16] = g
+        c[16:] = rng.standard_normal(K - 16) * 10.0 ** rng.uniform(-3, 3)
+        cols.append(c)
+    while len(cols) < 32:
+        cols.append((rng.standard_normal(K) * 10.0 ** rng.uniform(-4, 3)).astype(np.float32))
+    R = np.stack(cols, axis=1).astype(np.float32)     # K x 32
+    for fmt in ("nvfp4", "int4"):
+        w = S.svdq_load_weights(to_dev_f32(R), fmt=fmt)
+        got = S.svdq_export_weights(w)
+        codes, scales = O.weight_quant(fmt, R)
+        assert np.array_equal(got["scales"], scales), fmt
+        assert np.array_equal(got["codes"], codes), (fmt, np.argwhere(got["codes"] != codes)[:8])
+
+
+SHAPES = [
+    # M, K, N, rank, fmt, bias
+    (1, 256, 256, 32, "nvfp4", False),
+    (77, 512, 384, 32, "nvfp4", True),
+    (200, 1024, 512, 16, "nvfp4", False),
+    (256, 320, 272, 32, "nvfp4", True),      # K % 256 != 0, N % 256 != 0
+    (300, 768, 256, 64, "nvfp4", False),
+    (129, 512, 256, 0, "nvfp4", True),       # plain W4A4
+    (130, 512, 256, 48, "nvfp4", False),     # rank padded to 64
+    (96, 512, 256, 32, "int4", True),
+    (200, 1024, 512, 48, "int4", False),
+    (64, 256, 272, 0, "int4", False),
+]
+
+
+@pytest.mark.parametrize("M,K,N,rank,fmt,bias", SHAPES)
+def test_layer_parity_small(S, M, K, N, rank, fmt, bias):
+    data = WL.make_small(M, K, N, rank=rank, fmt=fmt, bias=bias, seed=M + K + N)
+    ref = oracle_layer(fmt, data, rank)
+    prep = ref["prep"]
+    bias_bits = WL.bf16_bits(data["bias"]) if bias else None
+    w = load_from_oracle(S, fmt, prep, bias_bits)
+    wexp = S.svdq_export_weights(w)
+    assert np.array_equal(wexp["codes"], ref["wq"][0]) and np.array_equal(wexp["scales"], ref["wq"][1])
+    ws, Y = _run_layer(S, w, WL.bf16_bits(data["X"]))
+    codes, scales, xl1 = S.svdq_export_act(w, ws, M)
+    assert np.array_equal(scales, ref["act"][1]), "activation scales differ"
+    assert np.array_equal(codes, ref["act"][0]), "activation codes differ"
+    if rank:
+        ok, info = y_within_tol(xl1, ref["act"][2])
+        assert ok, ("XL1", info)
+    ok, info = y_within_tol(bits(Y), ref["Y"])
+    assert ok, ("Y", info)
+
+
+def test_prepare_weights_invariants(S):
+    """The library's own preparation (cuSOLVER on the fp64 Gram matrix):
+    1/lambda bit-exact, the branch spans the oracle's optimal rank-r subspace,
+    and the residual carries the Eckart-Young energy."""
+    M, K, N, r = 256, 512, 384, 32
+    data = WL.make_small(M, K, N, w_outlier_rows=4, seed=5)
+    Xb, Wb = WL.bf16_bits(data["X"]), WL.bf16_bits(data["W"])
+    xm = O.calib_absmax(Xb)
+    prep = O.prepare(Wb, xm, r)
+    X = data["X"].cuda()
+    W = data["W"].cuda()
+    xabs = S.svdq_calib_absmax(X)
+    torch.cuda.synchronize()
+    assert np.array_equal(xabs.cpu().numpy(), xm)
+    w = S.svdq_prepare_weights(W, r, "nvfp4", x_absmax=xabs)
+    e = S.svdq_export_weights(w)
+    assert np.array_equal(e["inv_lambda"], prep["inv_lambda"])
+    assert np.array_equal(e["lambda"], prep["lam"])
+    L1L2_lib = O.bf16_decode(e["L1"]).astype(np.float64) @ O.bf16_decode(e["L2"]).astype(np.float64)
+    L1L2_ora = prep["L1_exact"] @ prep["L2_exact"]
+    assert np.linalg.norm(L1L2_lib - L1L2_ora) <= 0.02 * np.linalg.norm(L1L2_ora)
+    resid = np.linalg.norm(prep["W_hat"] - L1L2_lib) ** 2
+    eym = np.sum(prep["sigma"][r:] ** 2)
+    assert eym <= resid <= eym * 1.02 + 1e-4 * np.linalg.norm(prep["W_hat"]) ** 2
+    # the whole library path approximates X W as well as the oracle's layer does
+    ws, Y = _run_layer(S, w, Xb)
+    ref = O.layer("nvfp4", Xb, Wb, r)
+    exact = O.bf16_decode(Xb).astype(np.float64) @ O.bf16_decode(Wb).astype(np.float64)
+    e_lib = np.linalg.norm(O.bf16_decode(bits(Y)) - exact) / np.linalg.norm(exact)
+    e_ora = np.linalg.norm(O.bf16_decode(ref["Y"]) - exact) / np.linalg.norm(exact)
+    assert e_lib <= 1.1 * e_ora + 1e-3, (e_lib, e_ora)
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4"])
+def test_lora_fold_parity(S, fmt):
+    M, K, N, r, rl = 160, 512, 384, 32, 16
+    data = WL.make_small(M, K, N, rank=r, fmt=fmt, lora_rank=rl, seed=9)
+    ref = oracle_layer(fmt, data, r, lora=True)
+    base = O.prepare(WL.bf16_bits(data["W"]), O.calib_absmax(WL.bf16_bits(data["X"])), r)
+    w = load_from_oracle(S, fmt, base)
+    before = S.svdq_export_weights(w)
+    S.svdq_append_lora(w, data["lora_A"].cuda(), data["lora_B"].cuda())
+    assert w.rank == r + rl
+    after = S.svdq_export_weights(w)
+    assert np.array_equal(before["codes"], after["codes"]) and np.array_equal(before["scales"], after["scales"])
+    assert np.array_equal(after["L1"], ref["prep"]["L1"]) and np.array_equal(after["L2"], ref["prep"]["L2"])
+    ws, Y = _run_layer(S, w, WL.bf16_bits(data["X"]))
+    codes, scales, xl1 = S.svdq_export_act(w, ws, M)
+    assert np.array_equal(codes, ref["act"][0]) and np.array_equal(scales, ref["act"][1])
+    ok, info = y_within_tol(bits(Y), ref["Y"])
+    assert ok, info
+
+
+def test_forward_matches_two_calls_and_is_deterministic(S):
+    data = WL.make_small(333, 512, 256, seed=3)
+    prep = O.prepare(WL.bf16_bits(data["W"]), O.calib_absmax(WL.bf16_bits(data["X"])), 32)
+    w = load_from_oracle(S, "nvfp4", prep)
+    X = data["X"].cuda()
+    Y1 = S.svdq_forward(w, X)
+    Y2 = S.svdq_forward(w, X)
+    ws, Y3 = _run_layer(S, w, WL.bf16_bits(data["X"]))
+    torch.cuda.synchronize()
+    assert torch.equal(Y1, Y2) and torch.equal(Y1, Y3)
+
+
+def test_empty_batch_is_a_noop(S):
+    data = WL.make_small(16, 256, 256, seed=1)
+    prep = O.prepare(WL.bf16_bits(data["W"]), None, 16)
+    w = load_from_oracle(S, "nvfp4", prep)
+    X = torch.empty(0, 256, dtype=torch.bfloat16, device="cuda")
+    Y = S.svdq_forward(w, X)
+    assert Y.shape == (0, 256)

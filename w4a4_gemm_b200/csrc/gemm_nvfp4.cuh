@@ -1,0 +1,306 @@
+// gemm_nvfp4.cuh -- the fused 4-bit GEMM + low-rank up-projection + bias.
+//
+// SVDQuant Sec. 4.2 (Eq. 5) and Sec. 4.3 (Nunchaku, Fig. 6b):
+//   Y = Q(X_hat) Q(R) + (X_hat L1) L2 + b
+// The up-projection shares its output with the 4-bit GEMM, so its rank-r
+// product is accumulated by the tensor core into the same TMEM accumulator
+// right after the main K loop; the epilogue adds the bias and writes bf16 Y.
+//
+// Persistent kernel, one 128 x 256 output tile at a time per CTA:
+//   warp 0    : TMA producer.  Per 256-wide K step: A codes (128 x 128 B),
+//               B codes (256 x 128 B), the A / B scale atoms (bulk copies);
+//               then the low-rank operands XL1 (128 x r) and L2^T (256 x r).
+//   warp 1    : TMEM owner; one lane moves scales smem -> TMEM (tcgen05.cp)
+//               and issues tcgen05.mma kind::mxf4nvf4 (E2M1 x E2M1, UE4M3
+//               scale per 16) and, for the low-rank tail, kind::f16.
+//   warps 2-5 : epilogue, TMEM -> registers -> +bias -> bf16 -> global.
+#pragma once
+
+#include "svdq_formats.cuh"
+#include "svdq_ptx.cuh"
+
+namespace svdq {
+
+constexpr int kGemmBM = 128;
+constexpr int kGemmBN = 256;
+constexpr int kGemmBKB = 128;                  // K step in bytes of packed codes = 256 values
+constexpr int kGemmStages = 4;
+constexpr int kGemmThreads = 192;
+constexpr uint32_t kGemmAccCols = 256;
+constexpr uint32_t kGemmSfaCol = 256;          // 4 MMAs x 4 columns
+constexpr uint32_t kGemmSfbCol = 272;          // 4 MMAs x 8 columns
+constexpr uint32_t kGemmTmemCols = 512;
+
+constexpr uint32_t kGemmAOff = 0;
+constexpr uint32_t kGemmBOff = kGemmBM * kGemmBKB;                 // 16384
+constexpr uint32_t kGemmSfaOff = kGemmBOff + kGemmBN * kGemmBKB;   // 49152
+constexpr uint32_t kGemmSfbOff = kGemmSfaOff + 4 * 512;            // 51200
+constexpr uint32_t kGemmStageBytes = kGemmSfbOff + 8 * 512;        // 55296
+constexpr uint32_t kGemmBarOff = kGemmStageBytes * kGemmStages;
+constexpr uint32_t kGemmSmemBytes = kGemmBarOff + 256 + 1024;
+
+struct GemmParams {
+  int M, N, K;
+  int kt_total;        // ceil(K / 256)
+  int m_tiles, n_tiles, num_tiles;
+  int r_pad;           // 0, 16, 32, 64, 128, 192, 256
+  const uint8_t* sfa;  // activation scale atoms [M_pad/128][sf_kcols][512]
+  const uint8_t* sfb;  // weight scale atoms     [N_pad/128][sf_kcols][512]
+  int sf_kcols;        // K_pad / 64, K_pad = K rounded up to 256
+  const __nv_bfloat16* bias;  // N or nullptr
+  __nv_bfloat16* Y;    // M x N row-major
+  long long budget;
+};
+
+// Low-rank tail: r_pad is split into chunks of at most 64 bf16 (128 bytes).
+__host__ __device__ inline int lr_chunk_cols(int r_pad) { return r_pad < 64 ? r_pad : 64; }
+__host__ __device__ inline int lr_num_chunks(int r_pad) {
+  return r_pad == 0 ? 0 : (r_pad + 63) / 64;
+}
+
+__device__ __forceinline__ void gemm_tile_coords(const GemmParams& p, int tile, int& m_blk,
+                                                 int& n_blk) {
+  // consecutive tiles walk down M for a fixed column block of the weights
+  m_blk = tile % p.m_tiles;
+  n_blk = tile / p.m_tiles;
+}
+
+__device__ __forceinline__ uint64_t sf_desc(uint32_t saddr) {
+  // 32 rows x 16 bytes, rows 16 bytes apart, 8-row groups 128 bytes apart
+  return make_sdesc(saddr, 0, 128, kSwizzleNone);
+}
+
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a,
+                      const __grid_constant__ CUtensorMap tm_b,
+                      const __grid_constant__ CUtensorMap tm_xl1,
+                      const __grid_constant__ CUtensorMap tm_l2t, const GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kGemmBarOff);
+  uint64_t* empty = full + kGemmStages;
+  uint64_t* acc_full = empty + kGemmStages;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* mma_done = acc_empty + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const uint32_t warp = warp_id();
+  const uint32_t lane = lane_id();
+  const int n_lr = lr_num_chunks(p.r_pad);
+  const int lr_cols = lr_chunk_cols(p.r_pad);
+  const int steps_per_tile = p.kt_total + n_lr;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kGemmStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 4);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, kGemmTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    if (elect_one()) {
+      prefetch_tmap(&tm_a);
+      prefetch_tmap(&tm_b);
+      if (n_lr) {
+        prefetch_tmap(&tm_xl1);
+        prefetch_tmap(&tm_l2t);
+      }
+      const uint32_t main_tx = kGemmStageBytes;
+      const uint32_t lr_tx = (kGemmBM + kGemmBN) * lr_cols * 2;
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
+        int m_blk, n_blk;
+        gemm_tile_coords(p, tile, m_blk, n_blk);
+        const int m0 = m_blk * kGemmBM, n0 = n_blk * kGemmBN;
+        for (int step = 0; step < steps_per_tile; ++step, ++it) {
+          const int s = it % kGemmStages;
+          const uint32_t ph = (it / kGemmStages) & 1;
+          if (!mbar_wait(&empty[s], ph ^ 1, p.budget, abort_flag)) {
+            raise_error(kErrWaitGemm);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + s * kGemmStageBytes;
+          if (step < p.kt_total) {
+            const int kt = step;
+            mbar_arrive_expect_tx(&full[s], main_tx);
+            tma_load_2d(st + kGemmAOff, &tm_a, &full[s], kt * kGemmBKB, m0);
+            tma_load_2d(st + kGemmBOff, &tm_b, &full[s], kt * kGemmBKB, n0);
+            bulk_load(st + kGemmSfaOff,
+                      p.sfa + (static_cast<size_t>(m_blk) * p.sf_kcols + kt * 4) * 512, 2048,
+                      &full[s]);
+            bulk_load(st + kGemmSfbOff,
+                      p.sfb + (static_cast<size_t>(2 * n_blk) * p.sf_kcols + kt * 4) * 512, 2048,
+                      &full[s]);
+            bulk_load(st + kGemmSfbOff + 2048,
+                      p.sfb + (static_cast<size_t>(2 * n_blk + 1) * p.sf_kcols + kt * 4) * 512,
+                      2048, &full[s]);
+          } else {
+            const int c = step - p.kt_total;
+            mbar_arrive_expect_tx(&full[s], lr_tx);
+            tma_load_2d(st + kGemmAOff, &tm_xl1, &full[s], c * 64, m0);
+            tma_load_2d(st + kGemmBOff, &tm_l2t, &full[s], c * 64, n0);
+          }
+        }
+      }
+      if (*abort_flag) {
+        for (int i = (it > kGemmStages ? it - kGemmStages : 0); i < it; ++i)
+          mbar_wait(&full[i % kGemmStages], (i / kGemmStages) & 1, p.budget, nullptr);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (elect_one()) {
+      const uint32_t idesc_main = idesc_e2m1_ue4m3(kGemmBM, kGemmBN);
+      const uint32_t idesc_lr = idesc_bf16_f32(kGemmBM, kGemmBN);
+      const uint32_t lr_row_bytes = static_cast<uint32_t>(lr_cols) * 2;
+      const uint32_t d_tmem = tmem_base;
+      int it = 0, t_local = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x, ++t_local) {
+        if (!mbar_wait(acc_empty, (t_local & 1) ^ 1, p.budget, abort_flag)) {
+          raise_error(kErrWaitGemm);
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        for (int step = 0; step < steps_per_tile; ++step, ++it) {
+          const int s = it % kGemmStages;
+          const uint32_t ph = (it / kGemmStages) & 1;
+          if (!mbar_wait(&full[s], ph, p.budget, abort_flag)) {
+            raise_error(kErrWaitGemm);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          uint8_t* st = smem + s * kGemmStageBytes;
+          const uint32_t a0 = smem_u32(st + kGemmAOff);
+          const uint32_t b0 = smem_u32(st + kGemmBOff);
+          if (step < p.kt_total) {
+            const uint32_t sfa_s = smem_u32(st + kGemmSfaOff);
+            const uint32_t sfb_s = smem_u32(st + kGemmSfbOff);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              tmem_cp_32x128b_x4(tmem_base + kGemmSfaCol + 4 * j, sf_desc(sfa_s + 512 * j));
+              tmem_cp_32x128b_x4(tmem_base + kGemmSfbCol + 8 * j, sf_desc(sfb_s + 512 * j));
+              tmem_cp_32x128b_x4(tmem_base + kGemmSfbCol + 8 * j + 4,
+                                 sf_desc(sfb_s + 2048 + 512 * j));
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              mma_nvf4(d_tmem, make_kmajor_desc(a0 + 32 * j, 128), make_kmajor_desc(b0 + 32 * j, 128),
+                       idesc_main, tmem_base + kGemmSfaCol + 4 * j, tmem_base + kGemmSfbCol + 8 * j,
+                       (step > 0 || j > 0) ? 1u : 0u);
+            }
+          } else {
+            for (int j = 0; j < lr_cols / 16; ++j) {
+              mma_bf16(d_tmem, make_kmajor_desc(a0 + 32 * j, lr_row_bytes),
+                       make_kmajor_desc(b0 + 32 * j, lr_row_bytes), idesc_lr, 1u);
+            }
+          }
+          tc_commit(&empty[s]);
+        }
+        tc_commit(acc_full);
+      }
+      tc_commit(mma_done);  // retires once every MMA and copy issued above has completed
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const uint32_t q = warp & 3u;
+    const uint32_t row = q * 32 + lane;
+    int t_local = 0;
+    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++t_local) {
+      int m_blk, n_blk;
+      gemm_tile_coords(p, tile, m_blk, n_blk);
+      if (!warp_wait(acc_full, t_local & 1, p.budget, abort_flag)) {
+        if (lane == 0) raise_error(kErrWaitGemm);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const int m = m_blk * kGemmBM + static_cast<int>(row);
+      const int n0 = n_blk * kGemmBN;
+      const bool row_ok = m < p.M;
+      __nv_bfloat16* yrow = p.Y + static_cast<size_t>(m) * p.N;
+      for (int c = 0; c < kGemmBN; c += 32) {
+        uint32_t r[32];
+        tmem_ld32(tmem_base + ((q * 32u) << 16) + c, r);
+        tmem_wait_ld();
+        if (c + 32 == kGemmBN) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(acc_empty);
+        }
+        const int n = n0 + c;
+        if (row_ok && n < p.N) {
+          const int valid = min(32, p.N - n);   // multiple of 16 (N % 16 == 0)
+          float b[32];
+          if (p.bias != nullptr) {
+            const uint4* bp = reinterpret_cast<const uint4*>(p.bias + n);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint4 w = 8 * j < valid ? __ldg(bp + j) : make_uint4(0u, 0u, 0u, 0u);
+              const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+              for (int t = 0; t < 4; ++t) {
+                b[8 * j + 2 * t] = bf16_lo(w4[t]);
+                b[8 * j + 2 * t + 1] = bf16_hi(w4[t]);
+              }
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) b[j] = 0.0f;
+          }
+          uint4* dst = reinterpret_cast<uint4*>(yrow + n);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            if (8 * j < valid) {
+              uint4 o;
+              o.x = pack_bf16x2(__uint_as_float(r[8 * j + 0]) + b[8 * j + 0],
+                                __uint_as_float(r[8 * j + 1]) + b[8 * j + 1]);
+              o.y = pack_bf16x2(__uint_as_float(r[8 * j + 2]) + b[8 * j + 2],
+                                __uint_as_float(r[8 * j + 3]) + b[8 * j + 3]);
+              o.z = pack_bf16x2(__uint_as_float(r[8 * j + 4]) + b[8 * j + 4],
+                                __uint_as_float(r[8 * j + 5]) + b[8 * j + 5]);
+              o.w = pack_bf16x2(__uint_as_float(r[8 * j + 6]) + b[8 * j + 6],
+                                __uint_as_float(r[8 * j + 7]) + b[8 * j + 7]);
+              dst[j] = o;
+            }
+          }
+        }
+      }
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    // every MMA issued by this CTA has retired before its TMEM is released
+    mbar_wait(mma_done, 0, p.budget, nullptr);
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kGemmTmemCols);
+  }
+}
+
+}  // namespace svdq

@@ -1,0 +1,254 @@
+// prepare.cuh -- one-time weight preparation kernels (not on the timed path).
+//
+// SVDQuant Sec. 4.2: smoothing W_hat = diag(lambda) W, the optimal rank-r
+// factors of W_hat from its SVD (Eckart-Young-Mirsky), the residual
+// R = W_hat - L1 L2 and its 4-bit per-group quantization; Sec. 5.2: a LoRA
+// joins the low-rank branch (L1' = [L1 | diag(lambda) A], L2' = [L2 ; B])
+// with R left as it is.
+#pragma once
+
+#include "svdq_formats.cuh"
+#include "svdq_ptx.cuh"
+
+namespace svdq {
+
+// ------------------------------------------------------------ calibration ---
+// absmax[k] = max(absmax[k], max_m |X[m, k]|): one thread per column pair,
+// rows split across blockIdx.y; non-negative floats order like their bits.
+__global__ void calib_absmax_kernel(const __nv_bfloat16* __restrict__ X, int M, int K,
+                                    float* __restrict__ absmax) {
+  const int k2 = blockIdx.x * blockDim.x + threadIdx.x;   // column pair
+  if (2 * k2 >= K) return;
+  const int rows_per = (M + gridDim.y - 1) / gridDim.y;
+  const int r0 = blockIdx.y * rows_per, r1 = min(M, r0 + rows_per);
+  float a0 = 0.f, a1 = 0.f;
+  const uint32_t* x = reinterpret_cast<const uint32_t*>(X);
+  for (int m = r0; m < r1; ++m) {
+    const uint32_t w = __ldg(x + (static_cast<size_t>(m) * K) / 2 + k2);
+    a0 = fmaxf(a0, fabsf(bf16_lo(w)));
+    a1 = fmaxf(a1, fabsf(bf16_hi(w)));
+  }
+  atomicMax(reinterpret_cast<unsigned int*>(absmax) + 2 * k2, __float_as_uint(a0));
+  atomicMax(reinterpret_cast<unsigned int*>(absmax) + 2 * k2 + 1, __float_as_uint(a1));
+}
+
+// wmax[k] = max_n |W[k, n]| (one block per input channel k).
+__global__ void row_absmax_kernel(const __nv_bfloat16* __restrict__ W, int K, int N,
+                                  float* __restrict__ wmax) {
+  const int k = blockIdx.x;
+  float a = 0.f;
+  for (int n = threadIdx.x; n < N; n += blockDim.x)
+    a = fmaxf(a, fabsf(__bfloat162float(W[static_cast<size_t>(k) * N + n])));
+  for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+  __shared__ float red[32];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    a = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    if (threadIdx.x == 0) wmax[k] = a;
+  }
+}
+
+// lambda_k = sqrt(max|X_k| / max|W_k|) in fp64, rounded to fp32 (1 where either
+// maximum is 0 or no calibration is given); inv_lambda = fp32 1 / lambda.
+__global__ void smoothing_kernel(const float* __restrict__ xmax, const float* __restrict__ wmax,
+                                 int K, float* __restrict__ lam, float* __restrict__ inv) {
+  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  if (k >= K) return;
+  float l = 1.0f;
+  if (xmax != nullptr) {
+    const double xm = xmax[k], wm = wmax[k];
+    if (xm > 0.0 && wm > 0.0) l = static_cast<float>(sqrt(xm / wm));
+  }
+  lam[k] = l;
+  inv[k] = __fdiv_rn(1.0f, l);
+}
+
+// W_hat[k, n] = lambda_k * W[k, n] in fp64 (exact).
+__global__ void smooth_weight_kernel(const __nv_bfloat16* __restrict__ W,
+                                     const float* __restrict__ lam, int K, int N,
+                                     double* __restrict__ What) {
+  const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= static_cast<size_t>(K) * N) return;
+  const int k = static_cast<int>(i / N);
+  What[i] = static_cast<double>(lam[k]) * static_cast<double>(__bfloat162float(W[i]));
+}
+
+// Nearest bf16 of a finite double (ties to even), from the bit fields: keep 8
+// significant bits of the 53, rounding the dropped 45 to nearest even.
+__device__ __forceinline__ __nv_bfloat16 bf16_from_f64(double x) {
+  if (x == 0.0) return __float2bfloat16_rn(static_cast<float>(x));
+  const unsigned long long b = static_cast<unsigned long long>(__double_as_longlong(x));
+  const unsigned long long sign = b >> 63;
+  int e = static_cast<int>((b >> 52) & 0x7FF) - 1023;
+  unsigned long long mant = (b & ((1ull << 52) - 1)) | (1ull << 52);
+  if (e < -126) {
+    // below the normal bf16 range: fall back to the float path (values that
+    // small never occur in these factors)
+    return __float2bfloat16_rn(static_cast<float>(x));
+  }
+  unsigned long long kept = mant >> 45;
+  const unsigned long long rem = mant & ((1ull << 45) - 1), half = 1ull << 44;
+  if (rem > half || (rem == half && (kept & 1ull))) ++kept;
+  if (kept == (1ull << 8)) {
+    kept >>= 1;
+    ++e;
+  }
+  const uint32_t fbits = static_cast<uint32_t>(sign << 31) |
+                         (static_cast<uint32_t>(e + 127) << 23) |
+                         (static_cast<uint32_t>(kept & 0x7Full) << 16);
+  return __float2bfloat16_rn(__uint_as_float(fbits));   // exact: already 8 significant bits
+}
+
+// Low-rank factors from the eigenvectors of the Gram matrix (column-major,
+// ascending eigenvalues), written straight into the kernel layouts
+//   L1t[j][k] = bf16(L1[k, j])  (r_pad x K),   L2t[n][j] = bf16(L2[j, n])  (N x r_pad).
+// gram_left: G = W_hat W_hat^T (K x K), eigenvectors u_j; L1 = u_j sigma_j,
+//            L2 = u_j^T W_hat / sigma_j.
+// else     : G = W_hat^T W_hat (N x N), eigenvectors v_j; L2 = v_j^T, L1 = W_hat v_j.
+__global__ void lowrank_l1_kernel(const double* __restrict__ evec, const double* __restrict__ eval,
+                                  const double* __restrict__ What, int K, int N, int r, int r_pad,
+                                  int gram_left, __nv_bfloat16* __restrict__ l1t,
+                                  double* __restrict__ l1_f64) {
+  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  const int j = blockIdx.y;
+  if (k >= K) return;
+  double v = 0.0;
+  if (j < r) {
+    if (gram_left) {
+      const int col = K - 1 - j;
+      v = evec[static_cast<size_t>(col) * K + k] * sqrt(fmax(eval[col], 0.0));
+    } else {
+      const int col = N - 1 - j;
+      const double* vj = evec + static_cast<size_t>(col) * N;
+      const double* wr = What + static_cast<size_t>(k) * N;
+      for (int n = 0; n < N; ++n) v += wr[n] * vj[n];
+    }
+  }
+  l1t[static_cast<size_t>(j) * K + k] = j < r ? bf16_from_f64(v) : __float2bfloat16_rn(0.f);
+  if (l1_f64 != nullptr && j < r) l1_f64[static_cast<size_t>(k) * r + j] = v;
+}
+
+__global__ void lowrank_l2_kernel(const double* __restrict__ evec, const double* __restrict__ eval,
+                                  const double* __restrict__ What, int K, int N, int r, int r_pad,
+                                  int gram_left, __nv_bfloat16* __restrict__ l2t) {
+  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  const int j = blockIdx.y;
+  if (n >= N) return;
+  double v = 0.0;
+  if (j < r) {
+    if (gram_left) {
+      const int col = K - 1 - j;
+      const double sigma = sqrt(fmax(eval[col], 0.0));
+      const double* uj = evec + static_cast<size_t>(col) * K;
+      for (int k = 0; k < K; ++k) v += uj[k] * What[static_cast<size_t>(k) * N + n];
+      v = sigma > 0.0 ? v / sigma : 0.0;
+    } else {
+      v = evec[static_cast<size_t>(N - 1 - j) * N + n];
+    }
+  }
+  l2t[static_cast<size_t>(n) * r_pad + j] = j < r ? bf16_from_f64(v) : __float2bfloat16_rn(0.f);
+}
+
+// Re-layout caller-given factors: L1 (K x r, bf16 row-major) -> L1t (r_pad x K);
+// L2 (r x N) -> L2t (N x r_pad); padding is zero.  `col0` places them at
+// branch columns [col0, col0 + r) (used when a LoRA is appended).
+__global__ void layout_l1_kernel(const __nv_bfloat16* __restrict__ L1, int K, int r, int col0,
+                                 __nv_bfloat16* __restrict__ l1t) {
+  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  const int j = blockIdx.y;
+  if (k >= K || j >= r) return;
+  l1t[static_cast<size_t>(col0 + j) * K + k] = L1[static_cast<size_t>(k) * r + j];
+}
+
+__global__ void layout_l2_kernel(const __nv_bfloat16* __restrict__ L2, int N, int r, int col0,
+                                 int r_pad, __nv_bfloat16* __restrict__ l2t) {
+  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  const int j = blockIdx.y;
+  if (n >= N || j >= r) return;
+  l2t[static_cast<size_t>(n) * r_pad + col0 + j] = L2[static_cast<size_t>(j) * N + n];
+}
+
+// Copy branch columns [0, r_old) of the old layouts into wider ones.
+__global__ void widen_l1_kernel(const __nv_bfloat16* __restrict__ old_t, int K, int r_old,
+                                __nv_bfloat16* __restrict__ new_t) {
+  const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i < static_cast<size_t>(K) * r_old) new_t[i] = old_t[i];
+}
+
+__global__ void widen_l2_kernel(const __nv_bfloat16* __restrict__ old_t, int N, int r_old,
+                                int r_pad_old, int r_pad_new, __nv_bfloat16* __restrict__ new_t) {
+  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  if (n >= N) return;
+  for (int j = 0; j < r_old; ++j)
+    new_t[static_cast<size_t>(n) * r_pad_new + j] = old_t[static_cast<size_t>(n) * r_pad_old + j];
+}
+
+// LoRA A joins L1 as bf16(lambda_k * A[k, j]) (X A = X_hat diag(lambda) A).
+__global__ void lora_l1_kernel(const __nv_bfloat16* __restrict__ A, const float* __restrict__ lam,
+                               int K, int rl, int col0, __nv_bfloat16* __restrict__ l1t) {
+  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  const int j = blockIdx.y;
+  if (k >= K || j >= rl) return;
+  const double v = static_cast<double>(lam[k]) *
+                   static_cast<double>(__bfloat162float(A[static_cast<size_t>(k) * rl + j]));
+  l1t[static_cast<size_t>(col0 + j) * K + k] = bf16_from_f64(v);
+}
+
+// R[k, n] = W_hat[k, n] - sum_j L1[k, j] L2[j, n] with the bf16 factors, in fp64,
+// rounded to fp32.
+__global__ void residual_kernel(const double* __restrict__ What,
+                                const __nv_bfloat16* __restrict__ l1t,
+                                const __nv_bfloat16* __restrict__ l2t, int K, int N, int r,
+                                int r_pad, float* __restrict__ R) {
+  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  const int k = blockIdx.y;
+  if (n >= N) return;
+  double acc = What[static_cast<size_t>(k) * N + n];
+  for (int j = 0; j < r; ++j)
+    acc -= static_cast<double>(__bfloat162float(l1t[static_cast<size_t>(j) * K + k])) *
+           static_cast<double>(__bfloat162float(l2t[static_cast<size_t>(n) * r_pad + j]));
+  R[static_cast<size_t>(k) * N + n] = static_cast<float>(acc);
+}
+
+// Quantize R (K x N fp32) along K for each output column n.
+// NVFP4: one thread per (n, group of 16): codes N x K/2, scales in 512-byte atoms
+//        (128 columns x 4 groups; byte (n % 32) * 16 + (n % 128 / 32) * 4 + g % 4).
+// INT4 : one thread per (n, group of 64): int8 codes N x K, fp16 scales [K/64][N_pad].
+__global__ void quant_weight_nvfp4_kernel(const float* __restrict__ R, int K, int N, int sf_kcols,
+                                          uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
+  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  const int g = blockIdx.y;
+  if (n >= N) return;
+  float v[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = R[static_cast<size_t>(16 * g + i) * N + n];
+  uint32_t cw[2];
+  const uint32_t s8 = quant16_nvfp4(v, cw);
+  uint32_t* dst = reinterpret_cast<uint32_t*>(codes + static_cast<size_t>(n) * (K / 2) + 8 * g);
+  dst[0] = cw[0];
+  dst[1] = cw[1];
+  uint8_t* atom = sf + (static_cast<size_t>(n / 128) * sf_kcols + g / 4) * 512;
+  atom[(n & 31) * 16 + ((n & 127) >> 5) * 4 + (g & 3)] = static_cast<uint8_t>(s8);
+}
+
+__global__ void quant_weight_int4_kernel(const float* __restrict__ R, int K, int N, int N_pad,
+                                         int8_t* __restrict__ codes, uint16_t* __restrict__ sf) {
+  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  const int g = blockIdx.y;
+  if (n >= N) return;
+  float amax = 0.f;
+  for (int i = 0; i < 64; ++i) amax = fmaxf(amax, fabsf(R[static_cast<size_t>(64 * g + i) * N + n]));
+  const uint16_t sh = int4_scale_bits(amax);
+  const float sd = __half2float(__ushort_as_half(sh));
+  const float inv = sd == 0.f ? 0.f : __frcp_rn(sd);
+  for (int i = 0; i < 64; ++i) {
+    const float v = R[static_cast<size_t>(64 * g + i) * N + n];
+    codes[static_cast<size_t>(n) * K + 64 * g + i] =
+        static_cast<int8_t>(sd == 0.f ? 0 : int4_code(v, inv));
+  }
+  sf[static_cast<size_t>(g) * N_pad + n] = sh;
+}
+
+}  // namespace svdq

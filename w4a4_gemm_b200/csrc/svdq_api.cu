@@ -1,0 +1,832 @@
+// svdq_api.cu -- host side of the C ABI declared in include/svdq.h.
+//
+// One translation unit holds every kernel of the library (they share the
+// sticky device error word), the tensor-map set-up, argument checking,
+// launch configuration, weight preparation and the debug exports.
+#include <cublas_v2.h>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <cusolverDn.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/svdq.h"
+#include "gemm_int4.cuh"
+#include "gemm_nvfp4.cuh"
+#include "prepare.cuh"
+#include "quant_act.cuh"
+#include "svdq_formats.cuh"
+#include "svdq_ptx.cuh"
+
+using namespace svdq;
+
+struct svdq_weights {
+  int device = 0;
+  int fmt = 0, K = 0, N = 0, rank = 0, r_pad = 0;
+  int K_pad = 0;       // K rounded up to 256 (scale-atom columns)
+  int N_pad = 0;       // N rounded up to 256
+  int sf_kcols = 0;    // K_pad / 64
+  float* inv_lambda = nullptr;
+  float* lambda = nullptr;
+  uint8_t* wcodes = nullptr;  // NVFP4: N x K/2 packed; INT4: N x K int8
+  uint8_t* wsf = nullptr;     // NVFP4: atoms [N_pad/128][sf_kcols][512]; INT4: fp16 [K/64][N_pad]
+  __nv_bfloat16* l1t = nullptr;  // r_pad x K
+  __nv_bfloat16* l2t = nullptr;  // N x r_pad
+  __nv_bfloat16* bias = nullptr;
+  CUtensorMap tm_b, tm_l1t, tm_l2t;
+};
+
+namespace {
+
+long long g_budget = -1;
+std::mutex g_mutex;
+
+long long wait_budget() {
+  if (g_budget < 0) {
+    std::lock_guard<std::mutex> lk(g_mutex);
+    if (g_budget < 0) {
+      const char* env = std::getenv("SVDQ_WAIT_BUDGET_CYCLES");
+      long long v = env ? std::atoll(env) : 0;
+      g_budget = v > 0 ? v : (1LL << 31);
+    }
+  }
+  return g_budget;
+}
+
+inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+inline int round_up(int x, int m) { return (x + m - 1) / m * m; }
+
+int rank_padded(int r) {
+  if (r <= 0) return 0;
+  if (r <= 16) return 16;
+  if (r <= 32) return 32;
+  return round_up(r, 64);
+}
+
+#define SVDQ_CUDA(call)                                                                \
+  do {                                                                                 \
+    cudaError_t e_ = (call);                                                           \
+    if (e_ != cudaSuccess) {                                                           \
+      std::fprintf(stderr, "svdq: %s failed: %s (%s:%d)\n", #call, cudaGetErrorString(e_), \
+                   __FILE__, __LINE__);                                                \
+      return SVDQ_ERR_CUDA;                                                            \
+    }                                                                                  \
+  } while (0)
+
+#define SVDQ_CHECK_LAUNCH() SVDQ_CUDA(cudaGetLastError())
+
+// ------------------------------------------------------------ tensor maps ---
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+CUtensorMapSwizzle swizzle_for(uint32_t row_bytes) {
+  if (row_bytes >= 128) return CU_TENSOR_MAP_SWIZZLE_128B;
+  if (row_bytes == 64) return CU_TENSOR_MAP_SWIZZLE_64B;
+  return CU_TENSOR_MAP_SWIZZLE_32B;
+}
+
+// 2-D map over a row-major [rows][cols] array of `elem` bytes per element.
+int make_map(CUtensorMap* m, CUtensorMapDataType dt, size_t elem, const void* base, uint64_t cols,
+             uint64_t rows, uint32_t box_cols, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return SVDQ_ERR_CUDA;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * elem};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_for(static_cast<uint32_t>(box_cols * elem)),
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    std::fprintf(stderr, "svdq: cuTensorMapEncodeTiled failed (%d): cols=%llu rows=%llu box=%u x %u\n",
+                 static_cast<int>(r), static_cast<unsigned long long>(cols),
+                 static_cast<unsigned long long>(rows), box_cols, box_rows);
+    return SVDQ_ERR_CUDA;
+  }
+  return SVDQ_OK;
+}
+
+// ------------------------------------------------------------ device info ---
+struct DeviceInfo {
+  int sms = 0;
+  bool attrs_set = false;
+};
+DeviceInfo g_dev[64];
+
+int device_setup(int dev) {
+  if (dev < 0 || dev >= 64) return SVDQ_ERR_CUDA;
+  DeviceInfo& d = g_dev[dev];
+  if (d.attrs_set) return SVDQ_OK;
+  std::lock_guard<std::mutex> lk(g_mutex);
+  if (d.attrs_set) return SVDQ_OK;
+  SVDQ_CUDA(cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev));
+  SVDQ_CUDA(cudaFuncSetAttribute(quant_act_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 quant_smem_layout(256).total));
+  SVDQ_CUDA(cudaFuncSetAttribute(quant_act_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 quant_smem_layout(256).total));
+  SVDQ_CUDA(cudaFuncSetAttribute(gemm_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kGemmSmemBytes));
+  SVDQ_CUDA(cudaFuncSetAttribute(gemm_int4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kI4SmemBytes));
+  d.attrs_set = true;
+  return SVDQ_OK;
+}
+
+int current_device(int* dev) {
+  SVDQ_CUDA(cudaGetDevice(dev));
+  return device_setup(*dev);
+}
+
+// ------------------------------------------------------------ workspace ---
+struct ActLayout {
+  int M, M_pad;
+  size_t codes_off, codes_bytes, sf_off, sf_bytes, xl1_off, xl1_bytes, total;
+};
+
+ActLayout act_layout(const svdq_weights* w, int M) {
+  ActLayout L;
+  L.M = M;
+  L.M_pad = round_up(std::max(M, 1), 128);
+  L.codes_bytes = w->fmt == SVDQ_NVFP4 ? static_cast<size_t>(M) * w->K / 2
+                                       : static_cast<size_t>(M) * w->K;
+  L.sf_bytes = w->fmt == SVDQ_NVFP4 ? static_cast<size_t>(L.M_pad / 128) * w->sf_kcols * 512
+                                    : static_cast<size_t>(w->K / 64) * L.M_pad * 2;
+  L.xl1_bytes = static_cast<size_t>(M) * w->r_pad * 2;
+  L.codes_off = 0;
+  L.sf_off = align256(L.codes_bytes);
+  L.xl1_off = L.sf_off + align256(L.sf_bytes);
+  L.total = L.xl1_off + align256(L.xl1_bytes);
+  return L;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int encode_weight_maps(svdq_weights* w) {
+  int rc;
+  if (w->fmt == SVDQ_NVFP4)
+    rc = make_map(&w->tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->wcodes, w->K / 2, w->N, 128, kGemmBN);
+  else
+    rc = make_map(&w->tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->wcodes, w->K, w->N, 64, kI4BN);
+  if (rc) return rc;
+  if (w->r_pad > 0) {
+    rc = make_map(&w->tm_l1t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w->l1t, w->K, w->r_pad, 64, w->r_pad);
+    if (rc) return rc;
+    const int lc = lr_chunk_cols(w->r_pad);
+    rc = make_map(&w->tm_l2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w->l2t, w->r_pad, w->N, lc, kGemmBN);
+    if (rc) return rc;
+  } else {
+    w->tm_l1t = w->tm_b;
+    w->tm_l2t = w->tm_b;
+  }
+  return SVDQ_OK;
+}
+
+void free_weights(svdq_weights* w) {
+  if (!w) return;
+  cudaFree(w->inv_lambda);
+  cudaFree(w->lambda);
+  cudaFree(w->wcodes);
+  cudaFree(w->wsf);
+  cudaFree(w->l1t);
+  cudaFree(w->l2t);
+  cudaFree(w->bias);
+  delete w;
+}
+
+int check_shape(int fmt, int K, int N, int rank) {
+  if (fmt != SVDQ_NVFP4 && fmt != SVDQ_INT4) return SVDQ_ERR_INVALID_ARG;
+  if (K <= 0 || N <= 0 || K % 64 != 0 || N % 16 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  if (rank < 0 || rank > 256 || rank > std::min(K, N)) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  return SVDQ_OK;
+}
+
+// Allocate the quantized-weight buffers and the (zeroed) factor layouts.
+int alloc_weights(svdq_weights* w, cudaStream_t st) {
+  w->K_pad = round_up(w->K, 256);
+  w->N_pad = round_up(w->N, 256);
+  w->sf_kcols = w->K_pad / 64;
+  w->r_pad = rank_padded(w->rank);
+  const size_t codes = w->fmt == SVDQ_NVFP4 ? static_cast<size_t>(w->N) * w->K / 2
+                                            : static_cast<size_t>(w->N) * w->K;
+  const size_t sfb = w->fmt == SVDQ_NVFP4 ? static_cast<size_t>(w->N_pad / 128) * w->sf_kcols * 512
+                                          : static_cast<size_t>(w->K / 64) * w->N_pad * 2;
+  if (cudaMalloc(&w->inv_lambda, w->K * sizeof(float)) != cudaSuccess ||
+      cudaMalloc(&w->lambda, w->K * sizeof(float)) != cudaSuccess ||
+      cudaMalloc(&w->wcodes, codes) != cudaSuccess || cudaMalloc(&w->wsf, sfb) != cudaSuccess)
+    return SVDQ_ERR_ALLOC;
+  SVDQ_CUDA(cudaMemsetAsync(w->wsf, 0, sfb, st));
+  if (w->r_pad > 0) {
+    if (cudaMalloc(&w->l1t, static_cast<size_t>(w->r_pad) * w->K * 2) != cudaSuccess ||
+        cudaMalloc(&w->l2t, static_cast<size_t>(w->N) * w->r_pad * 2) != cudaSuccess)
+      return SVDQ_ERR_ALLOC;
+    SVDQ_CUDA(cudaMemsetAsync(w->l1t, 0, static_cast<size_t>(w->r_pad) * w->K * 2, st));
+    SVDQ_CUDA(cudaMemsetAsync(w->l2t, 0, static_cast<size_t>(w->N) * w->r_pad * 2, st));
+  }
+  return SVDQ_OK;
+}
+
+int quantize_residual(svdq_weights* w, const float* R, cudaStream_t st) {
+  const dim3 blk(128);
+  if (w->fmt == SVDQ_NVFP4) {
+    const dim3 grid((w->N + 127) / 128, w->K / 16);
+    quant_weight_nvfp4_kernel<<<grid, blk, 0, st>>>(R, w->K, w->N, w->sf_kcols, w->wcodes, w->wsf);
+  } else {
+    const dim3 grid((w->N + 127) / 128, w->K / 64);
+    quant_weight_int4_kernel<<<grid, blk, 0, st>>>(R, w->K, w->N, w->N_pad,
+                                                   reinterpret_cast<int8_t*>(w->wcodes),
+                                                   reinterpret_cast<uint16_t*>(w->wsf));
+  }
+  SVDQ_CHECK_LAUNCH();
+  return SVDQ_OK;
+}
+
+int copy_bias(svdq_weights* w, const void* bias, cudaStream_t st) {
+  if (bias == nullptr) return SVDQ_OK;
+  if (cudaMalloc(&w->bias, static_cast<size_t>(w->N) * 2) != cudaSuccess) return SVDQ_ERR_ALLOC;
+  SVDQ_CUDA(cudaMemcpyAsync(w->bias, bias, static_cast<size_t>(w->N) * 2, cudaMemcpyDeviceToDevice, st));
+  return SVDQ_OK;
+}
+
+struct DeviceBuf {
+  void* p = nullptr;
+  ~DeviceBuf() { if (p) cudaFree(p); }
+  bool alloc(size_t n) { return cudaMalloc(&p, n) == cudaSuccess; }
+  template <class T> T* as() const { return static_cast<T*>(p); }
+};
+
+int do_append_lora(svdq_weights* w, const void* A, const void* B, int rl, cudaStream_t st) {
+  if (rl <= 0) return SVDQ_OK;
+  const int r_old = w->rank, rp_old = w->r_pad;
+  const int r_new = r_old + rl;
+  if (r_new > 256 || r_new > std::min(w->K, w->N)) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  const int rp_new = rank_padded(r_new);
+  __nv_bfloat16 *l1t = nullptr, *l2t = nullptr;
+  if (cudaMalloc(&l1t, static_cast<size_t>(rp_new) * w->K * 2) != cudaSuccess) return SVDQ_ERR_ALLOC;
+  if (cudaMalloc(&l2t, static_cast<size_t>(w->N) * rp_new * 2) != cudaSuccess) {
+    cudaFree(l1t);
+    return SVDQ_ERR_ALLOC;
+  }
+  cudaMemsetAsync(l1t, 0, static_cast<size_t>(rp_new) * w->K * 2, st);
+  cudaMemsetAsync(l2t, 0, static_cast<size_t>(w->N) * rp_new * 2, st);
+  if (r_old > 0) {
+    const size_t n1 = static_cast<size_t>(r_old) * w->K;
+    widen_l1_kernel<<<static_cast<unsigned>((n1 + 255) / 256), 256, 0, st>>>(w->l1t, w->K, r_old, l1t);
+    widen_l2_kernel<<<(w->N + 255) / 256, 256, 0, st>>>(w->l2t, w->N, r_old, rp_old, rp_new, l2t);
+  }
+  lora_l1_kernel<<<dim3((w->K + 255) / 256, rl), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(A), w->lambda, w->K, rl, r_old, l1t);
+  layout_l2_kernel<<<dim3((w->N + 255) / 256, rl), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(B), w->N, rl, r_old, rp_new, l2t);
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) {
+    cudaFree(l1t);
+    cudaFree(l2t);
+    std::fprintf(stderr, "svdq: LoRA fold failed: %s\n", cudaGetErrorString(e));
+    return SVDQ_ERR_CUDA;
+  }
+  cudaFree(w->l1t);
+  cudaFree(w->l2t);
+  w->l1t = l1t;
+  w->l2t = l2t;
+  w->rank = r_new;
+  w->r_pad = rp_new;
+  return encode_weight_maps(w);
+}
+
+// Optimal rank-r factors of W_hat (fp64, K x N row-major) into w->l1t / w->l2t:
+// eigen-decomposition of the smaller Gram matrix (cuBLAS DSYRK + cuSOLVER DSYEVD).
+int lowrank_factors(svdq_weights* w, const double* What, cudaStream_t st) {
+  const int K = w->K, N = w->N, r = w->rank;
+  const bool left = K <= N;                 // G = W_hat W_hat^T (K x K), else W_hat^T W_hat
+  const int d = left ? K : N;
+  DeviceBuf G, ev, info, work;
+  if (!G.alloc(static_cast<size_t>(d) * d * 8) || !ev.alloc(static_cast<size_t>(d) * 8) ||
+      !info.alloc(sizeof(int)))
+    return SVDQ_ERR_ALLOC;
+  cublasHandle_t cb = nullptr;
+  cusolverDnHandle_t cs = nullptr;
+  int rc = SVDQ_OK;
+  if (cublasCreate(&cb) != CUBLAS_STATUS_SUCCESS) return SVDQ_ERR_LIBRARY;
+  if (cusolverDnCreate(&cs) != CUSOLVER_STATUS_SUCCESS) {
+    cublasDestroy(cb);
+    return SVDQ_ERR_LIBRARY;
+  }
+  cublasSetStream(cb, st);
+  cusolverDnSetStream(cs, st);
+  const double one = 1.0, zero = 0.0;
+  // W_hat (row-major K x N) is the column-major N x K matrix A = W_hat^T.
+  cublasStatus_t bs = left
+      ? cublasDsyrk(cb, CUBLAS_FILL_MODE_LOWER, CUBLAS_OP_T, K, N, &one, What, N, &zero, G.as<double>(), K)
+      : cublasDsyrk(cb, CUBLAS_FILL_MODE_LOWER, CUBLAS_OP_N, N, K, &one, What, N, &zero, G.as<double>(), N);
+  if (bs != CUBLAS_STATUS_SUCCESS) rc = SVDQ_ERR_LIBRARY;
+  int lwork = 0;
+  if (!rc && cusolverDnDsyevd_bufferSize(cs, CUSOLVER_EIG_MODE_VECTOR, CUBLAS_FILL_MODE_LOWER, d,
+                                         G.as<double>(), d, ev.as<double>(), &lwork) !=
+                 CUSOLVER_STATUS_SUCCESS)
+    rc = SVDQ_ERR_LIBRARY;
+  if (!rc && !work.alloc(static_cast<size_t>(std::max(lwork, 1)) * 8)) rc = SVDQ_ERR_ALLOC;
+  if (!rc && cusolverDnDsyevd(cs, CUSOLVER_EIG_MODE_VECTOR, CUBLAS_FILL_MODE_LOWER, d, G.as<double>(),
+                              d, ev.as<double>(), work.as<double>(), lwork, info.as<int>()) !=
+                 CUSOLVER_STATUS_SUCCESS)
+    rc = SVDQ_ERR_LIBRARY;
+  if (!rc) {
+    int h_info = 0;
+    if (cudaMemcpyAsync(&h_info, info.p, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+      rc = SVDQ_ERR_CUDA;
+    else if (h_info != 0)
+      rc = SVDQ_ERR_LIBRARY;
+  }
+  if (!rc) {
+    lowrank_l1_kernel<<<dim3((K + 127) / 128, w->r_pad), 128, 0, st>>>(
+        G.as<double>(), ev.as<double>(), What, K, N, r, w->r_pad, left ? 1 : 0, w->l1t, nullptr);
+    lowrank_l2_kernel<<<dim3((N + 127) / 128, w->r_pad), 128, 0, st>>>(
+        G.as<double>(), ev.as<double>(), What, K, N, r, w->r_pad, left ? 1 : 0, w->l2t);
+    if (cudaGetLastError() != cudaSuccess || cudaStreamSynchronize(st) != cudaSuccess)
+      rc = SVDQ_ERR_CUDA;
+  }
+  cusolverDnDestroy(cs);
+  cublasDestroy(cb);
+  return rc;
+}
+
+}  // namespace
+
+// =========================================================================
+extern "C" {
+
+SVDQ_API const char* svdq_status_string(int s) {
+  switch (s) {
+    case SVDQ_OK: return "ok";
+    case SVDQ_ERR_INVALID_ARG: return "invalid argument";
+    case SVDQ_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case SVDQ_ERR_ALLOC: return "device allocation failed";
+    case SVDQ_ERR_CUDA: return "CUDA error";
+    case SVDQ_ERR_TIMEOUT: return "device wait timed out";
+    case SVDQ_ERR_LIBRARY: return "cuSOLVER/cuBLAS error";
+    default: return "unknown status";
+  }
+}
+
+SVDQ_API int svdq_set_wait_budget(long long cycles) {
+  if (cycles <= 0) return SVDQ_ERR_INVALID_ARG;
+  g_budget = cycles;
+  return SVDQ_OK;
+}
+
+SVDQ_API int svdq_get_error(void) {
+  unsigned v = 0, z = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return -SVDQ_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(&v, g_error_word, sizeof v) != cudaSuccess) return -SVDQ_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_error_word, &z, sizeof z) != cudaSuccess) return -SVDQ_ERR_CUDA;
+  return static_cast<int>(v);
+}
+
+SVDQ_API int svdq_calib_absmax(const void* X, int M, int K, float* absmax, int accumulate,
+                               void* stream) {
+  if (X == nullptr || absmax == nullptr || M < 0 || K <= 0 || (K & 1)) return SVDQ_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!accumulate) SVDQ_CUDA(cudaMemsetAsync(absmax, 0, static_cast<size_t>(K) * 4, st));
+  if (M == 0) return SVDQ_OK;
+  const int pairs = K / 2;
+  const int splits = std::min(64, std::max(1, M / 64));
+  calib_absmax_kernel<<<dim3((pairs + 255) / 256, splits), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(X), M, K, absmax);
+  SVDQ_CHECK_LAUNCH();
+  return SVDQ_OK;
+}
+
+SVDQ_API int svdq_prepare_weights(const svdq_prepare_desc* d, void* stream, svdq_weights** out) {
+  if (d == nullptr || out == nullptr || d->W == nullptr) return SVDQ_ERR_INVALID_ARG;
+  *out = nullptr;
+  int rc = check_shape(d->fmt, d->K, d->N, d->rank);
+  if (rc) return rc;
+  if (d->lora_rank < 0 || (d->lora_rank > 0 && (d->lora_A == nullptr || d->lora_B == nullptr)))
+    return SVDQ_ERR_INVALID_ARG;
+  if (d->rank + d->lora_rank > 256 || d->rank + d->lora_rank > std::min(d->K, d->N))
+    return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  int dev;
+  if ((rc = current_device(&dev))) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  svdq_weights* w = new svdq_weights();
+  w->device = dev;
+  w->fmt = d->fmt;
+  w->K = d->K;
+  w->N = d->N;
+  w->rank = d->rank;
+  const int K = d->K, N = d->N;
+  do {
+    if ((rc = alloc_weights(w, st))) break;
+    DeviceBuf wmax, What, R;
+    if (!wmax.alloc(static_cast<size_t>(K) * 4) || !What.alloc(static_cast<size_t>(K) * N * 8) ||
+        !R.alloc(static_cast<size_t>(K) * N * 4)) {
+      rc = SVDQ_ERR_ALLOC;
+      break;
+    }
+    const __nv_bfloat16* W = static_cast<const __nv_bfloat16*>(d->W);
+    row_absmax_kernel<<<K, 256, 0, st>>>(W, K, N, wmax.as<float>());
+    smoothing_kernel<<<(K + 255) / 256, 256, 0, st>>>(d->x_absmax, wmax.as<float>(), K, w->lambda,
+                                                      w->inv_lambda);
+    const size_t KN = static_cast<size_t>(K) * N;
+    smooth_weight_kernel<<<static_cast<unsigned>((KN + 255) / 256), 256, 0, st>>>(
+        W, w->lambda, K, N, What.as<double>());
+    if (cudaGetLastError() != cudaSuccess) {
+      rc = SVDQ_ERR_CUDA;
+      break;
+    }
+    if (w->rank > 0 && (rc = lowrank_factors(w, What.as<double>(), st))) break;
+    residual_kernel<<<dim3((N + 255) / 256, K), 256, 0, st>>>(
+        What.as<double>(), w->l1t, w->l2t, K, N, w->rank, w->r_pad, R.as<float>());
+    if (cudaGetLastError() != cudaSuccess) {
+      rc = SVDQ_ERR_CUDA;
+      break;
+    }
+    if ((rc = quantize_residual(w, R.as<float>(), st))) break;
+    if ((rc = copy_bias(w, d->bias, st))) break;
+    if (cudaStreamSynchronize(st) != cudaSuccess) {
+      rc = SVDQ_ERR_CUDA;
+      break;
+    }
+    if ((rc = encode_weight_maps(w))) break;
+    if (d->lora_rank > 0 && (rc = do_append_lora(w, d->lora_A, d->lora_B, d->lora_rank, st))) break;
+  } while (false);
+  if (rc) {
+    free_weights(w);
+    return rc;
+  }
+  *out = w;
+  return SVDQ_OK;
+}
+
+SVDQ_API int svdq_load_weights(const svdq_parts_desc* d, void* stream, svdq_weights** out) {
+  if (d == nullptr || out == nullptr || d->R == nullptr) return SVDQ_ERR_INVALID_ARG;
+  *out = nullptr;
+  int rc = check_shape(d->fmt, d->K, d->N, d->rank);
+  if (rc) return rc;
+  if (d->rank > 0 && (d->L1 == nullptr || d->L2 == nullptr)) return SVDQ_ERR_INVALID_ARG;
+  int dev;
+  if ((rc = current_device(&dev))) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  svdq_weights* w = new svdq_weights();
+  w->device = dev;
+  w->fmt = d->fmt;
+  w->K = d->K;
+  w->N = d->N;
+  w->rank = d->rank;
+  const int K = d->K, N = d->N;
+  do {
+    if ((rc = alloc_weights(w, st))) break;
+    std::vector<float> ones;
+    if (d->inv_lambda) {
+      if (cudaMemcpyAsync(w->inv_lambda, d->inv_lambda, K * 4, cudaMemcpyDeviceToDevice, st)) {
+        rc = SVDQ_ERR_CUDA;
+        break;
+      }
+    }
+    if (d->lambda) {
+      if (cudaMemcpyAsync(w->lambda, d->lambda, K * 4, cudaMemcpyDeviceToDevice, st)) {
+        rc = SVDQ_ERR_CUDA;
+        break;
+      }
+    }
+    if (!d->inv_lambda || !d->lambda) {
+      // host-side fill: lambda = 1 / inv_lambda (or both 1)
+      std::vector<float> inv(K, 1.0f), lam(K, 1.0f);
+      if (d->inv_lambda &&
+          cudaMemcpy(inv.data(), d->inv_lambda, K * 4, cudaMemcpyDeviceToHost) != cudaSuccess) {
+        rc = SVDQ_ERR_CUDA;
+        break;
+      }
+      for (int k = 0; k < K; ++k) lam[k] = 1.0f / inv[k];
+      if (!d->inv_lambda && cudaMemcpy(w->inv_lambda, inv.data(), K * 4, cudaMemcpyHostToDevice)) {
+        rc = SVDQ_ERR_CUDA;
+        break;
+      }
+      if (!d->lambda && cudaMemcpy(w->lambda, lam.data(), K * 4, cudaMemcpyHostToDevice)) {
+        rc = SVDQ_ERR_CUDA;
+        break;
+      }
+    }
+    if (w->rank > 0) {
+      layout_l1_kernel<<<dim3((K + 255) / 256, w->rank), 256, 0, st>>>(
+          static_cast<const __nv_bfloat16*>(d->L1), K, w->rank, 0, w->l1t);
+      layout_l2_kernel<<<dim3((N + 255) / 256, w->rank), 256, 0, st>>>(
+          static_cast<const __nv_bfloat16*>(d->L2), N, w->rank, 0, w->r_pad, w->l2t);
+      if (cudaGetLastError() != cudaSuccess) {
+        rc = SVDQ_ERR_CUDA;
+        break;
+      }
+    }
+    if ((rc = quantize_residual(w, d->R, st))) break;
+    if ((rc = copy_bias(w, d->bias, st))) break;
+    if (cudaStreamSynchronize(st) != cudaSuccess) {
+      rc = SVDQ_ERR_CUDA;
+      break;
+    }
+    rc = encode_weight_maps(w);
+  } while (false);
+  if (rc) {
+    free_weights(w);
+    return rc;
+  }
+  *out = w;
+  return SVDQ_OK;
+}
+
+SVDQ_API int svdq_append_lora(svdq_weights* w, const void* A, const void* B, int rl, void* stream) {
+  if (w == nullptr || A == nullptr || B == nullptr || rl <= 0) return SVDQ_ERR_INVALID_ARG;
+  int dev;
+  int rc = current_device(&dev);
+  if (rc) return rc;
+  if (dev != w->device) return SVDQ_ERR_INVALID_ARG;
+  return do_append_lora(w, A, B, rl, static_cast<cudaStream_t>(stream));
+}
+
+SVDQ_API int svdq_weights_info(const svdq_weights* w, int* fmt, int* K, int* N, int* rank,
+                               int* rank_padded_out) {
+  if (w == nullptr) return SVDQ_ERR_INVALID_ARG;
+  if (fmt) *fmt = w->fmt;
+  if (K) *K = w->K;
+  if (N) *N = w->N;
+  if (rank) *rank = w->rank;
+  if (rank_padded_out) *rank_padded_out = w->r_pad;
+  return SVDQ_OK;
+}
+
+SVDQ_API int svdq_act_workspace_bytes(const svdq_weights* w, int M, size_t* bytes) {
+  if (w == nullptr || bytes == nullptr || M < 0) return SVDQ_ERR_INVALID_ARG;
+  *bytes = act_layout(w, M).total;
+  return SVDQ_OK;
+}
+
+SVDQ_API int svdq_quantize_act(const svdq_weights* w, const void* X, int M, void* ws, void* stream) {
+  if (w == nullptr || M < 0) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  if (X == nullptr || ws == nullptr || !aligned16(X) || (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return SVDQ_ERR_INVALID_ARG;
+  int dev;
+  int rc = current_device(&dev);
+  if (rc) return rc;
+  if (dev != w->device) return SVDQ_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const ActLayout L = act_layout(w, M);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  CUtensorMap tm_x;
+  if ((rc = make_map(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, w->K, M, kQuantBK, kQuantBM)))
+    return rc;
+  QuantParams p;
+  p.M = M;
+  p.K = w->K;
+  p.r_pad = w->r_pad;
+  p.kt_total = w->K / kQuantBK;
+  p.M_pad = L.M_pad;
+  p.sf_kcols = w->sf_kcols;
+  p.inv_lambda = w->inv_lambda;
+  p.codes = base + L.codes_off;
+  p.sf = base + L.sf_off;
+  p.xl1 = reinterpret_cast<__nv_bfloat16*>(base + L.xl1_off);
+  p.budget = wait_budget();
+  const int m_tiles = L.M_pad / kQuantBM;
+  // split K over a cluster when the row blocks alone leave the GPU idle
+  int ks = 1;
+  const int target = 2 * g_dev[dev].sms;
+  while (ks < 8 && m_tiles * ks < target && (ks * 2) <= p.kt_total) ks *= 2;
+  p.ksplit = ks;
+  if (w->fmt == SVDQ_NVFP4 && w->sf_kcols * 64 != w->K) {
+    // zero the scale atoms of the K padding (read by the GEMM's last K step)
+    const size_t pitch = static_cast<size_t>(w->sf_kcols) * 512;
+    const size_t off = static_cast<size_t>(w->K / 64) * 512;
+    SVDQ_CUDA(cudaMemset2DAsync(p.sf + off, pitch, 0, pitch - off, m_tiles, st));
+  }
+  const QuantSmem S = quant_smem_layout(w->r_pad);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(m_tiles, ks, 1);
+  cfg.blockDim = dim3(kQuantThreads, 1, 1);
+  cfg.dynamicSmemBytes = S.total;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = ks;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = ks > 1 ? 1 : 0;
+  const CUtensorMap& tm_l1t = w->r_pad > 0 ? w->tm_l1t : tm_x;
+  cudaError_t e = w->fmt == SVDQ_NVFP4 ? cudaLaunchKernelEx(&cfg, quant_act_kernel<0>, tm_x, tm_l1t, p)
+                                       : cudaLaunchKernelEx(&cfg, quant_act_kernel<1>, tm_x, tm_l1t, p);
+  if (e != cudaSuccess) {
+    std::fprintf(stderr, "svdq: activation kernel launch failed: %s\n", cudaGetErrorString(e));
+    return SVDQ_ERR_CUDA;
+  }
+  return SVDQ_OK;
+}
+
+SVDQ_API int svdq_linear(const svdq_weights* w, const void* ws, int M, void* Y, void* stream) {
+  if (w == nullptr || M < 0) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  if (ws == nullptr || Y == nullptr || !aligned16(Y) || (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return SVDQ_ERR_INVALID_ARG;
+  int dev;
+  int rc = current_device(&dev);
+  if (rc) return rc;
+  if (dev != w->device) return SVDQ_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const ActLayout L = act_layout(w, M);
+  const uint8_t* base = static_cast<const uint8_t*>(ws);
+  CUtensorMap tm_a, tm_xl1;
+  const int m_tiles = L.M_pad / 128;
+  const int n_tiles = (w->N + 255) / 256;
+  const int tiles = m_tiles * n_tiles;
+  const int grid = std::min(tiles, g_dev[dev].sms);
+  if (w->fmt == SVDQ_NVFP4) {
+    if ((rc = make_map(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base + L.codes_off, w->K / 2, M, 128,
+                       kGemmBM)))
+      return rc;
+  } else {
+    if ((rc = make_map(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base + L.codes_off, w->K, M, 64,
+                       kI4BM)))
+      return rc;
+  }
+  if (w->r_pad > 0) {
+    if ((rc = make_map(&tm_xl1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base + L.xl1_off, w->r_pad, M,
+                       lr_chunk_cols(w->r_pad), 128)))
+      return rc;
+  } else {
+    tm_xl1 = tm_a;
+  }
+  if (w->fmt == SVDQ_NVFP4) {
+    GemmParams p;
+    p.M = M;
+    p.N = w->N;
+    p.K = w->K;
+    p.kt_total = (w->K + 255) / 256;
+    p.m_tiles = m_tiles;
+    p.n_tiles = n_tiles;
+    p.num_tiles = tiles;
+    p.r_pad = w->r_pad;
+    p.sfa = base + L.sf_off;
+    p.sfb = w->wsf;
+    p.sf_kcols = w->sf_kcols;
+    p.bias = w->bias;
+    p.Y = static_cast<__nv_bfloat16*>(Y);
+    p.budget = wait_budget();
+    gemm_nvfp4_kernel<<<grid, kGemmThreads, kGemmSmemBytes, st>>>(tm_a, w->tm_b, tm_xl1, w->tm_l2t, p);
+  } else {
+    GemmI4Params p;
+    p.M = M;
+    p.N = w->N;
+    p.K = w->K;
+    p.groups = w->K / 64;
+    p.m_tiles = m_tiles;
+    p.n_tiles = n_tiles;
+    p.num_tiles = tiles;
+    p.r_pad = w->r_pad;
+    p.sx = reinterpret_cast<const uint16_t*>(base + L.sf_off);
+    p.sw = reinterpret_cast<const uint16_t*>(w->wsf);
+    p.M_pad = L.M_pad;
+    p.N_pad = w->N_pad;
+    p.bias = w->bias;
+    p.Y = static_cast<__nv_bfloat16*>(Y);
+    p.budget = wait_budget();
+    gemm_int4_kernel<<<grid, kI4Threads, kI4SmemBytes, st>>>(tm_a, w->tm_b, tm_xl1, w->tm_l2t, p);
+  }
+  SVDQ_CHECK_LAUNCH();
+  return SVDQ_OK;
+}
+
+SVDQ_API int svdq_forward(const svdq_weights* w, const void* X, int M, void* Y, void* ws, void* stream) {
+  int rc = svdq_quantize_act(w, X, M, ws, stream);
+  if (rc) return rc;
+  return svdq_linear(w, ws, M, Y, stream);
+}
+
+SVDQ_API int svdq_export_act(const svdq_weights* w, const void* ws, int M, uint8_t* codes,
+                             void* scales, void* xl1) {
+  if (w == nullptr || ws == nullptr || M < 0) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  SVDQ_CUDA(cudaDeviceSynchronize());
+  const ActLayout L = act_layout(w, M);
+  const uint8_t* base = static_cast<const uint8_t*>(ws);
+  const int K = w->K;
+  if (codes) {
+    if (w->fmt == SVDQ_NVFP4) {
+      SVDQ_CUDA(cudaMemcpy(codes, base + L.codes_off, L.codes_bytes, cudaMemcpyDeviceToHost));
+    } else {
+      std::vector<int8_t> tmp(L.codes_bytes);
+      SVDQ_CUDA(cudaMemcpy(tmp.data(), base + L.codes_off, L.codes_bytes, cudaMemcpyDeviceToHost));
+      for (size_t i = 0; i < tmp.size() / 2; ++i)
+        codes[i] = static_cast<uint8_t>((tmp[2 * i] & 0xF) | ((tmp[2 * i + 1] & 0xF) << 4));
+    }
+  }
+  if (scales) {
+    std::vector<uint8_t> tmp(L.sf_bytes);
+    SVDQ_CUDA(cudaMemcpy(tmp.data(), base + L.sf_off, L.sf_bytes, cudaMemcpyDeviceToHost));
+    if (w->fmt == SVDQ_NVFP4) {
+      uint8_t* out = static_cast<uint8_t*>(scales);
+      const int G = K / 16;
+      for (int m = 0; m < M; ++m)
+        for (int g = 0; g < G; ++g) {
+          const size_t atom = (static_cast<size_t>(m / 128) * w->sf_kcols + g / 4) * 512;
+          out[static_cast<size_t>(m) * G + g] = tmp[atom + (m % 32) * 16 + ((m % 128) / 32) * 4 + g % 4];
+        }
+    } else {
+      uint16_t* out = static_cast<uint16_t*>(scales);
+      const uint16_t* in = reinterpret_cast<const uint16_t*>(tmp.data());
+      const int G = K / 64;
+      for (int m = 0; m < M; ++m)
+        for (int g = 0; g < G; ++g) out[static_cast<size_t>(m) * G + g] = in[static_cast<size_t>(g) * L.M_pad + m];
+    }
+  }
+  if (xl1 && w->rank > 0) {
+    std::vector<uint16_t> tmp(static_cast<size_t>(M) * w->r_pad);
+    SVDQ_CUDA(cudaMemcpy(tmp.data(), base + L.xl1_off, tmp.size() * 2, cudaMemcpyDeviceToHost));
+    uint16_t* out = static_cast<uint16_t*>(xl1);
+    for (int m = 0; m < M; ++m)
+      for (int j = 0; j < w->rank; ++j)
+        out[static_cast<size_t>(m) * w->rank + j] = tmp[static_cast<size_t>(m) * w->r_pad + j];
+  }
+  return SVDQ_OK;
+}
+
+SVDQ_API int svdq_export_weights(const svdq_weights* w, uint8_t* codes, void* scales, void* L1,
+                                 void* L2, float* inv_lambda, float* lambda) {
+  if (w == nullptr) return SVDQ_ERR_INVALID_ARG;
+  SVDQ_CUDA(cudaDeviceSynchronize());
+  const int K = w->K, N = w->N;
+  if (codes) {
+    if (w->fmt == SVDQ_NVFP4) {
+      SVDQ_CUDA(cudaMemcpy(codes, w->wcodes, static_cast<size_t>(N) * K / 2, cudaMemcpyDeviceToHost));
+    } else {
+      std::vector<int8_t> tmp(static_cast<size_t>(N) * K);
+      SVDQ_CUDA(cudaMemcpy(tmp.data(), w->wcodes, tmp.size(), cudaMemcpyDeviceToHost));
+      for (size_t i = 0; i < tmp.size() / 2; ++i)
+        codes[i] = static_cast<uint8_t>((tmp[2 * i] & 0xF) | ((tmp[2 * i + 1] & 0xF) << 4));
+    }
+  }
+  if (scales) {
+    if (w->fmt == SVDQ_NVFP4) {
+      const size_t bytes = static_cast<size_t>(w->N_pad / 128) * w->sf_kcols * 512;
+      std::vector<uint8_t> tmp(bytes);
+      SVDQ_CUDA(cudaMemcpy(tmp.data(), w->wsf, bytes, cudaMemcpyDeviceToHost));
+      uint8_t* out = static_cast<uint8_t*>(scales);
+      const int G = K / 16;
+      for (int n = 0; n < N; ++n)
+        for (int g = 0; g < G; ++g) {
+          const size_t atom = (static_cast<size_t>(n / 128) * w->sf_kcols + g / 4) * 512;
+          out[static_cast<size_t>(n) * G + g] = tmp[atom + (n % 32) * 16 + ((n % 128) / 32) * 4 + g % 4];
+        }
+    } else {
+      const int G = K / 64;
+      std::vector<uint16_t> tmp(static_cast<size_t>(G) * w->N_pad);
+      SVDQ_CUDA(cudaMemcpy(tmp.data(), w->wsf, tmp.size() * 2, cudaMemcpyDeviceToHost));
+      uint16_t* out = static_cast<uint16_t*>(scales);
+      for (int n = 0; n < N; ++n)
+        for (int g = 0; g < G; ++g) out[static_cast<size_t>(n) * G + g] = tmp[static_cast<size_t>(g) * w->N_pad + n];
+    }
+  }
+  if (L1 && w->rank > 0) {
+    std::vector<uint16_t> tmp(static_cast<size_t>(w->r_pad) * K);
+    SVDQ_CUDA(cudaMemcpy(tmp.data(), w->l1t, tmp.size() * 2, cudaMemcpyDeviceToHost));
+    uint16_t* out = static_cast<uint16_t*>(L1);
+    for (int k = 0; k < K; ++k)
+      for (int j = 0; j < w->rank; ++j) out[static_cast<size_t>(k) * w->rank + j] = tmp[static_cast<size_t>(j) * K + k];
+  }
+  if (L2 && w->rank > 0) {
+    std::vector<uint16_t> tmp(static_cast<size_t>(N) * w->r_pad);
+    SVDQ_CUDA(cudaMemcpy(tmp.data(), w->l2t, tmp.size() * 2, cudaMemcpyDeviceToHost));
+    uint16_t* out = static_cast<uint16_t*>(L2);
+    for (int j = 0; j < w->rank; ++j)
+      for (int n = 0; n < N; ++n) out[static_cast<size_t>(j) * N + n] = tmp[static_cast<size_t>(n) * w->r_pad + j];
+  }
+  if (inv_lambda) SVDQ_CUDA(cudaMemcpy(inv_lambda, w->inv_lambda, K * 4, cudaMemcpyDeviceToHost));
+  if (lambda) SVDQ_CUDA(cudaMemcpy(lambda, w->lambda, K * 4, cudaMemcpyDeviceToHost));
+  return SVDQ_OK;
+}
+
+SVDQ_API void svdq_weights_destroy(svdq_weights* w) { free_weights(w); }
+
+}  // extern "C"
