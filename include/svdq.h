@@ -138,6 +138,24 @@ SVDQ_API int svdq_linear(const svdq_weights* w, const void* workspace, int M, vo
 SVDQ_API int svdq_forward(const svdq_weights* w, const void* X, int M, void* Y, void* workspace,
                           void* stream);
 
+/* Fixed size of the device workspace array behind svdq_forward_noalloc. */
+#define SVDQ_NOALLOC_WORKSPACE_BYTES (16u << 20)
+
+/* svdq_forward without a caller workspace and without any allocation.  The
+ * paper has no counterpart: this is for callers that cannot call cudaMalloc,
+ * e.g. a plugin whose host framework owns all device memory, or a serving
+ * loop that must not pay cudaMalloc's implicit device synchronization.  The
+ * activation workspace lives in a fixed __device__ array of
+ * SVDQ_NOALLOC_WORKSPACE_BYTES (16 MiB) that every GPU loading the library
+ * keeps until exit.  M is limited to what fits: svdq_act_workspace_bytes(w, M)
+ * must be <= SVDQ_NOALLOC_WORKSPACE_BYTES (for K = 3072, rank 32, NVFP4: about
+ * 9000 tokens), else SVDQ_ERR_UNSUPPORTED_SHAPE and nothing is launched.
+ * The first call on a device looks up the array's address (do it before any
+ * stream capture).  All calls on a device share the one array: calls that
+ * overlap on the GPU (other streams, other threads) race and must be
+ * serialized by the caller.  X, Y, stream: as for svdq_forward. */
+SVDQ_API int svdq_forward_noalloc(const svdq_weights* w, const void* X, int M, void* Y, void* stream);
+
 /* Debug export of a filled workspace in plain layouts (host outputs, any may
  * be NULL; synchronizes the device):
  *   codes  M x K/2 bytes, element 2i in the low nibble (INT4: two's complement);

@@ -28,7 +28,7 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "device all
 
 EXPORTED = ("svdq_calib_absmax", "svdq_prepare_weights", "svdq_load_weights", "svdq_append_lora",
             "svdq_weights_info", "svdq_act_workspace_bytes", "svdq_quantize_act", "svdq_linear",
-            "svdq_forward", "svdq_export_act", "svdq_export_weights", "svdq_get_error",
+            "svdq_forward", "svdq_forward_noalloc", "svdq_export_act", "svdq_export_weights", "svdq_get_error",
             "svdq_set_wait_budget", "svdq_status_string", "svdq_weights_destroy")
 
 
@@ -73,6 +73,7 @@ def lib() -> ctypes.CDLL:
     L.svdq_quantize_act.argtypes = [P, P, I, P, P]
     L.svdq_linear.argtypes = [P, P, I, P, P]
     L.svdq_forward.argtypes = [P, P, I, P, P, P]
+    L.svdq_forward_noalloc.argtypes = [P, P, I, P, P]
     L.svdq_export_act.argtypes = [P, P, I, P, P, P]
     L.svdq_export_weights.argtypes = [P, P, P, P, P, P, P]
     L.svdq_get_error.argtypes = []
@@ -253,6 +254,20 @@ def svdq_forward(w: Weights, X: torch.Tensor, Y: Optional[torch.Tensor] = None,
         workspace = alloc_workspace(w, M, X.device)
     _check(lib().svdq_forward(w.handle, _ptr(X), M, _ptr(Y), _ptr(workspace), _stream(stream)),
            "svdq_forward")
+    return Y
+
+
+def svdq_forward_noalloc(w: Weights, X: torch.Tensor, Y: Optional[torch.Tensor] = None,
+                         stream=None) -> torch.Tensor:
+    """svdq_forward with the library's fixed device workspace (no allocation
+    inside the call; see include/svdq.h for the size limit and the sharing rule)."""
+    _dev(X, torch.bfloat16, "X")
+    M = X.shape[0]
+    if Y is None:
+        Y = torch.empty(M, w.N, dtype=torch.bfloat16, device=X.device)
+    _dev(Y, torch.bfloat16, "Y", (M, w.N))
+    _check(lib().svdq_forward_noalloc(w.handle, _ptr(X), M, _ptr(Y), _stream(stream)),
+           "svdq_forward_noalloc")
     return Y
 
 

@@ -724,6 +724,51 @@ SVDQ_API int svdq_forward(const svdq_weights* w, const void* X, int M, void* Y, 
   return svdq_linear(w, ws, M, Y, stream);
 }
 
+// ------------------------------------------------------------ no-allocation forward ---
+// Some callers may not allocate device memory at all: a plugin inside a host
+// framework that owns every device byte, or a latency-critical serving loop
+// where cudaMalloc's implicit device-wide synchronization is not acceptable.
+// svdq_forward_noalloc keeps the activation workspace in this fixed array
+// instead.  Every GPU that loads the library holds it until the process exits.
+static __device__ __align__(256) uint8_t g_noalloc_workspace[SVDQ_NOALLOC_WORKSPACE_BYTES];
+
+SVDQ_API int svdq_forward_noalloc(const svdq_weights* w, const void* X, int M, void* Y, void* stream) {
+  static void* ws_ptr[64] = {};
+  if (w == nullptr || M < 0) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  const size_t need = act_layout(w, M).total;
+  if (need > SVDQ_NOALLOC_WORKSPACE_BYTES) {
+    std::fprintf(stderr,
+                 "svdq_forward_noalloc: M=%d K=%d rank_padded=%d needs a %zu-byte workspace, more than "
+                 "the %u-byte fixed one; use svdq_forward with a caller workspace\n",
+                 M, w->K, w->r_pad, need, static_cast<unsigned>(SVDQ_NOALLOC_WORKSPACE_BYTES));
+    return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  }
+  int dev;
+  int rc = current_device(&dev);
+  if (rc) return rc;
+  if (dev != w->device) return SVDQ_ERR_INVALID_ARG;
+  if (ws_ptr[dev] == nullptr) {
+    // first call on this device: look up the array's device address once
+    // (host code cannot use the symbol itself as a device pointer)
+    std::lock_guard<std::mutex> lk(g_mutex);
+    if (ws_ptr[dev] == nullptr) {
+      void* p = nullptr;
+      const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_workspace);
+      if (e != cudaSuccess) {
+        std::fprintf(stderr, "svdq_forward_noalloc: cudaGetSymbolAddress failed: %s\n",
+                     cudaGetErrorString(e));
+        return SVDQ_ERR_CUDA;
+      }
+      ws_ptr[dev] = p;
+    }
+  }
+  // The activation kernel rewrites every workspace byte the GEMM reads for this
+  // M (codes, scales including the K padding, XL1), so the array's previous
+  // contents never leak into the result.
+  return svdq_forward(w, X, M, Y, ws_ptr[dev], stream);
+}
+
 SVDQ_API int svdq_export_act(const svdq_weights* w, const void* ws, int M, uint8_t* codes,
                              void* scales, void* xl1) {
   if (w == nullptr || ws == nullptr || M < 0) return SVDQ_ERR_INVALID_ARG;
