@@ -124,7 +124,8 @@ SVDQ_API int svdq_act_workspace_bytes(const svdq_weights* w, int M, size_t* byte
 
 /* Fused activation kernel (Sec. 4.3, "quantize + down-projection"): one pass
  * over X (device bf16 M x K) writes Q(X diag(lambda)^-1) codes and scales and
- * bf16(X_hat) L1 into `workspace`.  Asynchronous on `stream`. */
+ * X_hat L1 = X (diag(lambda)^-1 L1) (fp32 precision, as a bf16 hi/lo pair)
+ * into `workspace`.  Asynchronous on `stream`. */
 SVDQ_API int svdq_quantize_act(const svdq_weights* w, const void* X, int M, void* workspace,
                                void* stream);
 
@@ -160,7 +161,7 @@ SVDQ_API int svdq_forward_noalloc(const svdq_weights* w, const void* X, int M, v
  * be NULL; synchronizes the device):
  *   codes  M x K/2 bytes, element 2i in the low nibble (INT4: two's complement);
  *   scales M x K/16 E4M3 bytes (NVFP4) or M x K/64 fp16 (INT4);
- *   xl1    M x rank bf16. */
+ *   xl1    M x rank fp32 (X_hat L1 at fp32 precision; stored as a bf16 pair). */
 SVDQ_API int svdq_export_act(const svdq_weights* w, const void* workspace, int M,
                              uint8_t* codes, void* scales, void* xl1);
 

@@ -79,6 +79,8 @@ def lib() -> ctypes.CDLL:
             getattr(_lib, name).argtypes = [P, L, P]
             getattr(_lib, name).restype = None
         _lib.oracle_act_quant.argtypes = [I, I, I, I, P, P, P, P, P, P]
+        _lib.oracle_fold_l1.argtypes = [I, I, P, P, P]
+        _lib.oracle_fold_l1.restype = None
         _lib.oracle_weight_quant.argtypes = [I, I, I, P, P, P]
         _lib.oracle_linear_rows.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, P, I, P]
         _lib.oracle_dequant.argtypes = [I, I, I, P, P, P]
@@ -248,8 +250,20 @@ def weight_quant(fmt, R: np.ndarray):
     return codes, scales
 
 
+def fold_l1(L1_bits: np.ndarray, inv_lambda: Optional[np.ndarray]) -> np.ndarray:
+    """The down-projection factor with the smoothing folded in:
+    L1s = bf16(diag(inv_lambda) L1), so that X_hat L1 = X L1s (Sec. 4.2)."""
+    L1 = np.ascontiguousarray(L1_bits, dtype=np.uint16)
+    K, r = L1.shape
+    out = np.zeros((K, r), dtype=np.uint16)
+    inv = None if inv_lambda is None else np.ascontiguousarray(inv_lambda, dtype=np.float32)
+    lib().oracle_fold_l1(K, r, _ptr(inv), _ptr(L1), _ptr(out))
+    return out
+
+
 def act_quant(fmt, X_bits: np.ndarray, inv_lambda: Optional[np.ndarray], L1_bits: Optional[np.ndarray]):
-    """Smooth, quantize and down-project X (M x K bf16) -> codes, scales, XL1 (M x r bf16)."""
+    """Smooth and quantize X (M x K bf16) -> codes, scales, and the down-projection
+    XL1 = X fold_l1(L1, inv_lambda) (M x r fp32, fp32 accumulation in increasing k)."""
     fmt = _FMT[fmt]
     X_bits = np.ascontiguousarray(X_bits, dtype=np.uint16)
     M, K = X_bits.shape
@@ -257,10 +271,10 @@ def act_quant(fmt, X_bits: np.ndarray, inv_lambda: Optional[np.ndarray], L1_bits
     r = 0 if L1_bits is None else L1_bits.shape[1]
     codes = np.zeros((M, K // 2), dtype=np.uint8)
     scales = np.zeros((M, K // g), dtype=np.uint8 if fmt == NVFP4 else np.uint16)
-    XL1 = np.zeros((M, r), dtype=np.uint16)
+    XL1 = np.zeros((M, r), dtype=np.float32)
     inv = None if inv_lambda is None else np.ascontiguousarray(inv_lambda, dtype=np.float32)
-    L1 = None if L1_bits is None else np.ascontiguousarray(L1_bits, dtype=np.uint16)
-    rc = lib().oracle_act_quant(fmt, M, K, r, _ptr(X_bits), _ptr(inv), _ptr(L1),
+    L1s = None if L1_bits is None else fold_l1(L1_bits, inv)
+    rc = lib().oracle_act_quant(fmt, M, K, r, _ptr(X_bits), _ptr(inv), _ptr(L1s),
                                 _ptr(codes), _ptr(scales), _ptr(XL1))
     assert rc == 0
     return codes, scales, XL1

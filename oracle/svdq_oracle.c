@@ -27,6 +27,10 @@
  *   - codes round to nearest, ties to the even code; a zero scale gives zero
  *     codes; the sign bit of an E2M1 code is the sign of X * RN(1/s);
  *   - INT4 codes are clamped to [-7, 7] (symmetric, q_max = 7);
+ *   - the down-projection folds the smoothing into its factor,
+ *     X_hat L1 = X (diag(lambda)^-1 L1), with the folded factor rounded to
+ *     bf16 once; X itself is already 16-bit; the branch's intermediate X_hat L1
+ *     stays at fp32 accumulator precision (only the factors are 16-bit);
  *   - the GEMM accumulates in fp32: exact per-group integer/E2M1 partial sums,
  *     scaled by s_x * s_w, summed over groups in increasing order, then the
  *     low-rank term sum_j XL1[m,j] L2[j,n] in increasing j, then the bias.
@@ -243,39 +247,53 @@ static void quantize_row(int fmt, const float *v, int K, uint8_t *codes_row, voi
 /* Activation side (the fused "quantize + down-projection" of Sec. 4.3).     */
 /*   x_hat[m,k] = fp32(x[m,k]) * inv_lambda[k]                                */
 /*   codes/scales = Q(x_hat) per group                                         */
-/*   XL1[m,j]   = bf16( sum_k bf16(x_hat[m,k]) * L1[k,j] ), fp32, increasing k */
-/* X: M x K bf16; L1: K x r bf16 (row-major); codes: M x K/2 bytes (element  */
-/* 2i in the low nibble); scales: M x K/g (uint8 E4M3 or uint16 fp16);        */
-/* XL1: M x r bf16.  inv_lambda may be NULL (lambda = 1).                     */
+/*   XL1[m,j]   = sum_k fp32(x[m,k]) * L1s[k,j], fp32, increasing k (kept fp32)*/
+/* where L1s = bf16(diag(inv_lambda) L1) is the down-projection factor with  */
+/* the smoothing folded in (X_hat L1 = X diag(lambda)^-1 L1), computed by     */
+/* oracle_fold_l1.  X: M x K bf16; L1s: K x r bf16 (row-major); codes:         */
+/* M x K/2 bytes (element 2i in the low nibble); scales: M x K/g (uint8 E4M3  */
+/* or uint16 fp16); XL1: M x r fp32.  inv_lambda may be NULL (lambda = 1).     */
 /* ------------------------------------------------------------------------- */
 int oracle_act_quant(int fmt, int M, int K, int r, const uint16_t *X, const float *inv_lambda,
-                     const uint16_t *L1, uint8_t *codes, void *scales, uint16_t *XL1) {
+                     const uint16_t *L1s, uint8_t *codes, void *scales, float *XL1) {
     int g = (fmt == ORACLE_NVFP4) ? 16 : 64;
     if (K % g) return 1;
     int ssz = (fmt == ORACLE_NVFP4) ? 1 : 2;
 #pragma omp parallel
     {
         float *xh = (float *)__builtin_alloca(sizeof(float) * (size_t)K);
-        float *xb = (float *)__builtin_alloca(sizeof(float) * (size_t)K);
+        float *xf = (float *)__builtin_alloca(sizeof(float) * (size_t)K);
 #pragma omp for schedule(static)
         for (int m = 0; m < M; ++m) {
             const uint16_t *xr = X + (long)m * K;
             for (int k = 0; k < K; ++k) {
-                float x = oracle_bf16_decode(xr[k]);
-                xh[k] = inv_lambda ? x * inv_lambda[k] : x;
-                xb[k] = oracle_bf16_decode(oracle_bf16_round((double)xh[k]));
+                xf[k] = oracle_bf16_decode(xr[k]);
+                xh[k] = inv_lambda ? xf[k] * inv_lambda[k] : xf[k];
             }
             quantize_row(fmt, xh, K, codes + (long)m * (K / 2),
                          (uint8_t *)scales + (long)m * (K / g) * ssz);
             for (int j = 0; j < r; ++j) {
                 float acc = 0.0f;
                 for (int k = 0; k < K; ++k)
-                    acc += xb[k] * oracle_bf16_decode(L1[(long)k * r + j]);
-                XL1[(long)m * r + j] = oracle_bf16_round((double)acc);
+                    acc += xf[k] * oracle_bf16_decode(L1s[(long)k * r + j]);
+                XL1[(long)m * r + j] = acc;
             }
         }
     }
     return 0;
+}
+
+/* The smoothing folded into the down-projection factor:
+ * L1s[k,j] = bf16( inv_lambda[k] * L1[k,j] ), the product exact in double and
+ * rounded once (nearest, ties to even).  L1: K x r bf16; inv_lambda may be
+ * NULL (then L1s = L1). */
+void oracle_fold_l1(int K, int r, const float *inv_lambda, const uint16_t *L1, uint16_t *L1s) {
+    for (long k = 0; k < K; ++k)
+        for (int j = 0; j < r; ++j) {
+            double v = (double)oracle_bf16_decode(L1[k * r + j]);
+            if (inv_lambda) v *= (double)inv_lambda[k];
+            L1s[k * r + j] = oracle_bf16_round(v);
+        }
 }
 
 /* ------------------------------------------------------------------------- */
@@ -302,12 +320,12 @@ int oracle_weight_quant(int fmt, int K, int N, const float *R, uint8_t *codes, v
 /* ------------------------------------------------------------------------- */
 /* The layer output (Eq. 5 of Sec. 4.2 plus bias):                            */
 /*   y[m,n] = bf16( sum_g s_x[m,g] s_w[n,g] sum_{k in g} deq(qx) deq(qw)      */
-/*                  + sum_j XL1[m,j] L2[j,n] + bias[n] )                      */
+/*                  + sum_j XL1[m,j] L2[j,n] + bias[n] )   (XL1 fp32)         */
 /* for the rows listed in `rows` (all rows if rows == NULL, n_rows = M) and   */
 /* all N columns; Y is n_rows x N bf16.  L2: r x N bf16; bias may be NULL.   */
 /* ------------------------------------------------------------------------- */
 int oracle_linear_rows(int fmt, int M, int N, int K, int r, const uint8_t *codes_x,
-                       const void *scales_x, const uint16_t *XL1, const uint8_t *codes_w,
+                       const void *scales_x, const float *XL1, const uint8_t *codes_w,
                        const void *scales_w, const uint16_t *L2, const uint16_t *bias,
                        const int *rows, int n_rows, uint16_t *Y) {
     int g = (fmt == ORACLE_NVFP4) ? 16 : 64;
@@ -336,8 +354,7 @@ int oracle_linear_rows(int fmt, int M, int N, int K, int r, const uint8_t *codes
                 acc += (sx * sw) * part;
             }
             for (int j = 0; j < r; ++j)
-                acc += oracle_bf16_decode(XL1[(long)m * r + j]) *
-                       oracle_bf16_decode(L2[(long)j * N + n]);
+                acc += XL1[(long)m * r + j] * oracle_bf16_decode(L2[(long)j * N + n]);
             if (bias) acc += oracle_bf16_decode(bias[n]);
             Y[(long)i * N + n] = oracle_bf16_round((double)acc);
         }

@@ -43,6 +43,15 @@ def y_within_tol(y_gpu_bits, y_ora_bits):
                              "n_bad": int(bad.sum()), "n": int(o.size)}
 
 
+def close_f32(got: np.ndarray, want: np.ndarray, rel=2.0 ** -12):
+    """fp32 intermediates (X_hat L1): |d| <= rel |want| + rel rms(want)."""
+    g, o = got.astype(np.float64), want.astype(np.float64)
+    rms = np.sqrt(np.mean(o ** 2)) if o.size else 0.0
+    err = np.abs(g - o)
+    tol = rel * np.abs(o) + rel * rms
+    return bool(np.all(err <= tol)), {"max_err_over_tol": float(np.max(err / np.maximum(tol, 1e-30))) if o.size else 0.0}
+
+
 def to_dev_bits(a: np.ndarray) -> torch.Tensor:
     """uint16 bf16 bit patterns -> device bf16 tensor."""
     return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()

@@ -111,7 +111,8 @@ def test_quantization_error_bound():
 
 
 def test_act_quant_packing_and_xl1():
-    """Element 2i sits in the low nibble; XL1 = bf16(bf16(x_hat) @ L1) in fp32."""
+    """Element 2i sits in the low nibble; XL1 = X @ bf16(diag(1/lambda) L1) in fp32,
+    which equals X_hat L1 up to the rounding of the folded factor."""
     M, K, r = 3, 32, 4
     rng = np.random.default_rng(7)
     X = torch.from_numpy(rng.standard_normal((M, K)).astype(np.float32)).to(torch.bfloat16)
@@ -126,7 +127,15 @@ def test_act_quant_packing_and_xl1():
             assert s == scales[m, g]
             packed = codes[m, 8 * g:8 * g + 8]
             assert np.array_equal(packed & 0xF, c[0::2]) and np.array_equal(packed >> 4, c[1::2])
-    xb = O.bf16_decode(O.bf16_round(xh.astype(np.float64))).astype(np.float64)
-    ref = xb @ O.bf16_decode(L1).astype(np.float64)
-    got = O.bf16_decode(XL1)
-    assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -8 + 1e-6)
+    # the folded factor is one nearest rounding of the exact product inv * L1
+    L1s = O.fold_l1(L1, inv)
+    prod = inv.astype(np.float64)[:, None] * O.bf16_decode(L1).astype(np.float64)
+    assert np.all(np.abs(O.bf16_decode(L1s) - prod) <= np.abs(prod) * 2.0 ** -8)
+    x = O.bf16_decode(Xb).astype(np.float64)
+    ref = x @ O.bf16_decode(L1s).astype(np.float64)
+    got = XL1.astype(np.float64)
+    assert XL1.dtype == np.float32
+    assert np.all(np.abs(got - ref) <= 1e-5 * np.abs(x) @ np.abs(O.bf16_decode(L1s)).astype(np.float64))
+    # and it is X_hat L1 up to the rounding of the folded factor
+    exact = xh.astype(np.float64) @ O.bf16_decode(L1).astype(np.float64)
+    assert np.all(np.abs(got - exact) <= np.abs(xh) @ np.abs(O.bf16_decode(L1)) * 2.0 ** -8 + 1e-6)

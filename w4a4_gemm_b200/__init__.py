@@ -272,11 +272,11 @@ def svdq_forward_noalloc(w: Weights, X: torch.Tensor, Y: Optional[torch.Tensor] 
 
 
 def svdq_export_act(w: Weights, workspace: torch.Tensor, M: int):
-    """(codes M x K/2 uint8, scales M x K/g, xl1 M x rank uint16 bf16 bits) on the host."""
+    """(codes M x K/2 uint8, scales M x K/g, xl1 M x rank float32) on the host."""
     g = GROUP[w.fmt]
     codes = np.zeros((M, w.K // 2), dtype=np.uint8)
     scales = np.zeros((M, w.K // g), dtype=np.uint8 if w.fmt == NVFP4 else np.uint16)
-    xl1 = np.zeros((M, w.rank), dtype=np.uint16)
+    xl1 = np.zeros((M, w.rank), dtype=np.float32)
     _check(lib().svdq_export_act(w.handle, _ptr(workspace), int(M), codes.ctypes.data_as(ctypes.c_void_p),
                                  scales.ctypes.data_as(ctypes.c_void_p),
                                  xl1.ctypes.data_as(ctypes.c_void_p) if w.rank else None),

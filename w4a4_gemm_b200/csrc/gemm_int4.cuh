@@ -25,23 +25,21 @@ namespace svdq {
 constexpr int kI4BM = 128;
 constexpr int kI4BN = 256;
 constexpr int kI4BK = 64;                 // one group
-constexpr int kI4Stages = 6;
 constexpr int kI4Threads = 320;
 constexpr int kI4EpiWarps = 8;
 constexpr uint32_t kI4AOff = 0;
-constexpr uint32_t kI4BOff = kI4BM * 128;                  // 16384 (room for a 128 B-row tail chunk)
-constexpr uint32_t kI4SxOff = kI4BOff + kI4BN * 128;       // 49152
+constexpr uint32_t kI4BOff = kI4BM * 128;                  // 16384 (A region fits a 128 B-row tail chunk)
+constexpr uint32_t kI4SxOff = kI4BOff + kI4BN * 128;       // 49152 (so does the B region)
 constexpr uint32_t kI4SwOff = kI4SxOff + kI4BM * 2;        // 49408
 constexpr uint32_t kI4StageBytes = 50176;                  // 49 KB, multiple of 1024
-constexpr uint32_t kI4BarOff = kI4StageBytes * 4;
-constexpr int kI4StagesUsed = 4;
-constexpr uint32_t kI4SmemBytes = kI4BarOff + 256 + 1024;
+constexpr int kI4Stages = 4;
+constexpr uint32_t kI4SmemBytes = kI4StageBytes * kI4Stages + 256 + 1024;
 
 struct GemmI4Params {
   int M, N, K;
   int groups;          // K / 64
   int m_tiles, n_tiles, num_tiles;
-  int r_pad;
+  int r_tail;          // tail K: 2 r_pad (X_hat L1 as hi | lo against L2^T | L2^T), 0 = none
   const uint16_t* sx;  // fp16 [K/64][M_pad]
   const uint16_t* sw;  // fp16 [K/64][N_pad]
   int M_pad, N_pad;
@@ -57,8 +55,8 @@ __global__ void __launch_bounds__(kI4Threads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  constexpr int S = kI4StagesUsed;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kI4BarOff);
+  constexpr int S = kI4Stages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kI4StageBytes * S);
   uint64_t* empty = full + S;
   uint64_t* pfull = empty + S;      // [2]
   uint64_t* pempty = pfull + 2;     // [2]
@@ -68,8 +66,8 @@ __global__ void __launch_bounds__(kI4Threads, 1)
 
   const uint32_t warp = warp_id();
   const uint32_t lane = lane_id();
-  const int n_lr = lr_num_chunks(p.r_pad);
-  const int lr_cols = lr_chunk_cols(p.r_pad);
+  const int n_lr = lr_num_chunks(p.r_tail);
+  const int lr_cols = lr_chunk_cols(p.r_tail);
   const int steps_per_tile = p.groups + n_lr;
 
   if (threadIdx.x == 0) {
@@ -98,6 +96,10 @@ __global__ void __launch_bounds__(kI4Threads, 1)
     if (elect_one()) {
       prefetch_tmap(&tm_a);
       prefetch_tmap(&tm_b);
+      if (n_lr) {
+        prefetch_tmap(&tm_xl1);
+        prefetch_tmap(&tm_l2t);
+      }
       const uint32_t main_tx = kI4BM * 64 + kI4BN * 64 + kI4BM * 2 + kI4BN * 2;
       const uint32_t lr_tx = (kI4BM + kI4BN) * lr_cols * 2;
       int it = 0;
@@ -148,6 +150,7 @@ __global__ void __launch_bounds__(kI4Threads, 1)
           const uint32_t ph = (it / S) & 1;
           const int b = it & 1;
           const uint32_t pph = (it >> 1) & 1;
+          const bool tail = step >= p.groups;
           if (!mbar_wait(&pempty[b], pph ^ 1, p.budget, abort_flag) ||
               !mbar_wait(&full[s], ph, p.budget, abort_flag)) {
             raise_error(kErrWaitGemm);
@@ -159,7 +162,7 @@ __global__ void __launch_bounds__(kI4Threads, 1)
           uint8_t* st = smem + s * kI4StageBytes;
           const uint32_t a0 = smem_u32(st + kI4AOff), b0 = smem_u32(st + kI4BOff);
           const uint32_t d = tmem_base + 256u * b;
-          if (step < p.groups) {
+          if (!tail) {
 #pragma unroll
             for (int j = 0; j < 2; ++j)
               mma_i8(d, make_kmajor_desc(a0 + 32 * j, 64), make_kmajor_desc(b0 + 32 * j, 64),
@@ -184,6 +187,7 @@ __global__ void __launch_bounds__(kI4Threads, 1)
     bool ok = true;
     for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
       const int m_blk = tile % p.m_tiles, n_blk = tile / p.m_tiles;
+      const int m = m_blk * kI4BM + static_cast<int>(row);
       float acc[128];
 #pragma unroll
       for (int j = 0; j < 128; ++j) acc[j] = 0.f;
@@ -239,7 +243,6 @@ __global__ void __launch_bounds__(kI4Threads, 1)
       }
       if (!ok) break;
       // bias, bf16, store
-      const int m = m_blk * kI4BM + static_cast<int>(row);
       const int n_base = n_blk * kI4BN + 128 * static_cast<int>(h);
       if (m < p.M) {
         __nv_bfloat16* yrow = p.Y + static_cast<size_t>(m) * p.N;

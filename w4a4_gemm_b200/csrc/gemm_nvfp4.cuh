@@ -9,11 +9,17 @@
 // Persistent kernel, one 128 x 256 output tile at a time per CTA:
 //   warp 0    : TMA producer.  Per 256-wide K step: A codes (128 x 128 B),
 //               B codes (256 x 128 B), the A / B scale atoms (bulk copies);
-//               then the low-rank operands XL1 (128 x r) and L2^T (256 x r).
+//               then the low-rank operands, XL1 (128 x 2r: the fp32 values as
+//               bf16 hi | lo) and [L2^T | L2^T] (256 x 2r), so the tail MMA adds
+//               (hi + lo) L2 with fp32 accuracy.
 //   warp 1    : TMEM owner; one lane moves scales smem -> TMEM (tcgen05.cp)
 //               and issues tcgen05.mma kind::mxf4nvf4 (E2M1 x E2M1, UE4M3
 //               scale per 16) and, for the low-rank tail, kind::f16.
-//   warps 2-5 : epilogue, TMEM -> registers -> +bias -> bf16 -> global.
+//   warps 2-9 : epilogue.  Warp w serves TMEM lane quarter w % 4 (rows) and
+//               columns [128 h, 128 h + 128), h = (w - 2) / 4.  Per tile they
+//               copy their accumulator columns to registers and hand the TMEM
+//               back at once, so the next tile's MMAs overlap the bias, bf16
+//               conversion and stores.
 #pragma once
 
 #include "svdq_formats.cuh"
@@ -24,9 +30,8 @@ namespace svdq {
 constexpr int kGemmBM = 128;
 constexpr int kGemmBN = 256;
 constexpr int kGemmBKB = 128;                  // K step in bytes of packed codes = 256 values
-constexpr int kGemmStages = 4;
-constexpr int kGemmThreads = 192;
-constexpr uint32_t kGemmAccCols = 256;
+constexpr int kGemmThreads = 320;
+constexpr int kGemmEpiWarps = 8;
 constexpr uint32_t kGemmSfaCol = 256;          // 4 MMAs x 4 columns
 constexpr uint32_t kGemmSfbCol = 272;          // 4 MMAs x 8 columns
 constexpr uint32_t kGemmTmemCols = 512;
@@ -36,14 +41,20 @@ constexpr uint32_t kGemmBOff = kGemmBM * kGemmBKB;                 // 16384
 constexpr uint32_t kGemmSfaOff = kGemmBOff + kGemmBN * kGemmBKB;   // 49152
 constexpr uint32_t kGemmSfbOff = kGemmSfaOff + 4 * 512;            // 51200
 constexpr uint32_t kGemmStageBytes = kGemmSfbOff + 8 * 512;        // 55296
-constexpr uint32_t kGemmBarOff = kGemmStageBytes * kGemmStages;
-constexpr uint32_t kGemmSmemBytes = kGemmBarOff + 256 + 1024;
+
+// Low-rank tail: its K (2 r_pad) is split into chunks of at most 64 bf16 (128 bytes).
+__host__ __device__ inline int lr_chunk_cols(int k_tail) { return k_tail < 64 ? k_tail : 64; }
+__host__ __device__ inline int lr_num_chunks(int k_tail) {
+  return k_tail == 0 ? 0 : (k_tail + 63) / 64;
+}
+constexpr int kGemmStages = 4;
+constexpr uint32_t kGemmSmemBytes = kGemmStageBytes * kGemmStages + 256 + 1024;
 
 struct GemmParams {
   int M, N, K;
   int kt_total;        // ceil(K / 256)
   int m_tiles, n_tiles, num_tiles;
-  int r_pad;           // 0, 16, 32, 64, 128, 192, 256
+  int r_tail;          // tail K: 2 r_pad (X_hat L1 as hi | lo against L2^T | L2^T), 0 = none
   const uint8_t* sfa;  // activation scale atoms [M_pad/128][sf_kcols][512]
   const uint8_t* sfb;  // weight scale atoms     [N_pad/128][sf_kcols][512]
   int sf_kcols;        // K_pad / 64, K_pad = K rounded up to 256
@@ -52,17 +63,10 @@ struct GemmParams {
   long long budget;
 };
 
-// Low-rank tail: r_pad is split into chunks of at most 64 bf16 (128 bytes).
-__host__ __device__ inline int lr_chunk_cols(int r_pad) { return r_pad < 64 ? r_pad : 64; }
-__host__ __device__ inline int lr_num_chunks(int r_pad) {
-  return r_pad == 0 ? 0 : (r_pad + 63) / 64;
-}
-
-__device__ __forceinline__ void gemm_tile_coords(const GemmParams& p, int tile, int& m_blk,
-                                                 int& n_blk) {
+__device__ __forceinline__ void gemm_tile_coords(int m_tiles, int tile, int& m_blk, int& n_blk) {
   // consecutive tiles walk down M for a fixed column block of the weights
-  m_blk = tile % p.m_tiles;
-  n_blk = tile / p.m_tiles;
+  m_blk = tile % m_tiles;
+  n_blk = tile / m_tiles;
 }
 
 __device__ __forceinline__ uint64_t sf_desc(uint32_t saddr) {
@@ -70,17 +74,46 @@ __device__ __forceinline__ uint64_t sf_desc(uint32_t saddr) {
   return make_sdesc(saddr, 0, 128, kSwizzleNone);
 }
 
+// Epilogue: 32 fp32 accumulators of one row (columns n0 .. n0 + 31) + bias ->
+// bf16 -> global.  Columns at or past N are skipped (N % 16 == 0).
+__device__ __forceinline__ void store_row_chunk(const uint32_t (&r)[32], __nv_bfloat16* yrow, int n0,
+                                                int N, const __nv_bfloat16* __restrict__ bias) {
+#pragma unroll
+  for (int j = 0; j < 32; j += 8) {
+    const int n = n0 + j;
+    if (n < N) {
+      float bb[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      if (bias != nullptr) {
+        const uint4 w = __ldg(reinterpret_cast<const uint4*>(bias + n));
+        const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          bb[2 * t] = bf16_lo(w4[t]);
+          bb[2 * t + 1] = bf16_hi(w4[t]);
+        }
+      }
+      uint4 o;
+      o.x = pack_bf16x2(__uint_as_float(r[j + 0]) + bb[0], __uint_as_float(r[j + 1]) + bb[1]);
+      o.y = pack_bf16x2(__uint_as_float(r[j + 2]) + bb[2], __uint_as_float(r[j + 3]) + bb[3]);
+      o.z = pack_bf16x2(__uint_as_float(r[j + 4]) + bb[4], __uint_as_float(r[j + 5]) + bb[5]);
+      o.w = pack_bf16x2(__uint_as_float(r[j + 6]) + bb[6], __uint_as_float(r[j + 7]) + bb[7]);
+      *reinterpret_cast<uint4*>(yrow + n) = o;
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a,
                       const __grid_constant__ CUtensorMap tm_b,
                       const __grid_constant__ CUtensorMap tm_xl1,
                       const __grid_constant__ CUtensorMap tm_l2t, const GemmParams p) {
+  constexpr int STAGES = kGemmStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kGemmBarOff);
-  uint64_t* empty = full + kGemmStages;
-  uint64_t* acc_full = empty + kGemmStages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kGemmStageBytes * STAGES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* acc_full = empty + STAGES;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* mma_done = acc_empty + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
@@ -88,17 +121,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   const uint32_t warp = warp_id();
   const uint32_t lane = lane_id();
-  const int n_lr = lr_num_chunks(p.r_pad);
-  const int lr_cols = lr_chunk_cols(p.r_pad);
+  const int n_lr = lr_num_chunks(p.r_tail);
+  const int lr_cols = lr_chunk_cols(p.r_tail);
   const int steps_per_tile = p.kt_total + n_lr;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kGemmStages; ++s) {
+    for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 4);
+    mbar_init(acc_empty, kGemmEpiWarps);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -121,17 +154,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         prefetch_tmap(&tm_xl1);
         prefetch_tmap(&tm_l2t);
       }
-      const uint32_t main_tx = kGemmStageBytes;
       const uint32_t lr_tx = (kGemmBM + kGemmBN) * lr_cols * 2;
       int it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
         int m_blk, n_blk;
-        gemm_tile_coords(p, tile, m_blk, n_blk);
+        gemm_tile_coords(p.m_tiles, tile, m_blk, n_blk);
         const int m0 = m_blk * kGemmBM, n0 = n_blk * kGemmBN;
         for (int step = 0; step < steps_per_tile; ++step, ++it) {
-          const int s = it % kGemmStages;
-          const uint32_t ph = (it / kGemmStages) & 1;
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
           if (!mbar_wait(&empty[s], ph ^ 1, p.budget, abort_flag)) {
             raise_error(kErrWaitGemm);
             *abort_flag = 1;
@@ -141,7 +173,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           uint8_t* st = smem + s * kGemmStageBytes;
           if (step < p.kt_total) {
             const int kt = step;
-            mbar_arrive_expect_tx(&full[s], main_tx);
+            mbar_arrive_expect_tx(&full[s], kGemmStageBytes);
             tma_load_2d(st + kGemmAOff, &tm_a, &full[s], kt * kGemmBKB, m0);
             tma_load_2d(st + kGemmBOff, &tm_b, &full[s], kt * kGemmBKB, n0);
             bulk_load(st + kGemmSfaOff,
@@ -162,8 +194,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
       }
       if (*abort_flag) {
-        for (int i = (it > kGemmStages ? it - kGemmStages : 0); i < it; ++i)
-          mbar_wait(&full[i % kGemmStages], (i / kGemmStages) & 1, p.budget, nullptr);
+        for (int i = (it > STAGES ? it - STAGES : 0); i < it; ++i)
+          mbar_wait(&full[i % STAGES], (i / STAGES) & 1, p.budget, nullptr);
       }
     }
   } else if (warp == 1) {
@@ -183,8 +215,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         tc_fence_after();
         for (int step = 0; step < steps_per_tile; ++step, ++it) {
-          const int s = it % kGemmStages;
-          const uint32_t ph = (it / kGemmStages) & 1;
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          const bool tail = step >= p.kt_total;
           if (!mbar_wait(&full[s], ph, p.budget, abort_flag)) {
             raise_error(kErrWaitGemm);
             *abort_flag = 1;
@@ -195,7 +228,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           uint8_t* st = smem + s * kGemmStageBytes;
           const uint32_t a0 = smem_u32(st + kGemmAOff);
           const uint32_t b0 = smem_u32(st + kGemmBOff);
-          if (step < p.kt_total) {
+          if (!tail) {
             const uint32_t sfa_s = smem_u32(st + kGemmSfaOff);
             const uint32_t sfb_s = smem_u32(st + kGemmSfbOff);
 #pragma unroll
@@ -219,6 +252,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           tc_commit(&empty[s]);
         }
+        if (!ok) break;
         tc_commit(acc_full);
       }
       tc_commit(mma_done);  // retires once every MMA and copy issued above has completed
@@ -226,67 +260,38 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else {
     // ---------------------------------------------------------------- epilogue
     const uint32_t q = warp & 3u;
+    const uint32_t h = (warp - 2) >> 2;
     const uint32_t row = q * 32 + lane;
     int t_local = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++t_local) {
       int m_blk, n_blk;
-      gemm_tile_coords(p, tile, m_blk, n_blk);
+      gemm_tile_coords(p.m_tiles, tile, m_blk, n_blk);
+      const int m = m_blk * kGemmBM + static_cast<int>(row);
+      // accumulator columns [128 h, 128 h + 128) of this row -> registers
       if (!warp_wait(acc_full, t_local & 1, p.budget, abort_flag)) {
         if (lane == 0) raise_error(kErrWaitGemm);
         *abort_flag = 1;
         break;
       }
       tc_fence_after();
-      const int m = m_blk * kGemmBM + static_cast<int>(row);
-      const int n0 = n_blk * kGemmBN;
-      const bool row_ok = m < p.M;
-      __nv_bfloat16* yrow = p.Y + static_cast<size_t>(m) * p.N;
-      for (int c = 0; c < kGemmBN; c += 32) {
-        uint32_t r[32];
-        tmem_ld32(tmem_base + ((q * 32u) << 16) + c, r);
-        tmem_wait_ld();
-        if (c + 32 == kGemmBN) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(acc_empty);
-        }
-        const int n = n0 + c;
-        if (row_ok && n < p.N) {
-          const int valid = min(32, p.N - n);   // multiple of 16 (N % 16 == 0)
-          float b[32];
-          if (p.bias != nullptr) {
-            const uint4* bp = reinterpret_cast<const uint4*>(p.bias + n);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const uint4 w = 8 * j < valid ? __ldg(bp + j) : make_uint4(0u, 0u, 0u, 0u);
-              const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-              for (int t = 0; t < 4; ++t) {
-                b[8 * j + 2 * t] = bf16_lo(w4[t]);
-                b[8 * j + 2 * t + 1] = bf16_hi(w4[t]);
-              }
-            }
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) b[j] = 0.0f;
-          }
-          uint4* dst = reinterpret_cast<uint4*>(yrow + n);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            if (8 * j < valid) {
-              uint4 o;
-              o.x = pack_bf16x2(__uint_as_float(r[8 * j + 0]) + b[8 * j + 0],
-                                __uint_as_float(r[8 * j + 1]) + b[8 * j + 1]);
-              o.y = pack_bf16x2(__uint_as_float(r[8 * j + 2]) + b[8 * j + 2],
-                                __uint_as_float(r[8 * j + 3]) + b[8 * j + 3]);
-              o.z = pack_bf16x2(__uint_as_float(r[8 * j + 4]) + b[8 * j + 4],
-                                __uint_as_float(r[8 * j + 5]) + b[8 * j + 5]);
-              o.w = pack_bf16x2(__uint_as_float(r[8 * j + 6]) + b[8 * j + 6],
-                                __uint_as_float(r[8 * j + 7]) + b[8 * j + 7]);
-              dst[j] = o;
-            }
-          }
-        }
+      uint32_t v0[32], v1[32], v2[32], v3[32];
+      const uint32_t taddr = tmem_base + ((q * 32u) << 16) + 128u * h;
+      tmem_ld32(taddr, v0);
+      tmem_ld32(taddr + 32, v1);
+      tmem_ld32(taddr + 64, v2);
+      tmem_ld32(taddr + 96, v3);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
+      // bias, bf16, store
+      const int nb = n_blk * kGemmBN + 128 * static_cast<int>(h);
+      if (m < p.M) {
+        __nv_bfloat16* yrow = p.Y + static_cast<size_t>(m) * p.N;
+        store_row_chunk(v0, yrow, nb, p.N, p.bias);
+        store_row_chunk(v1, yrow, nb + 32, p.N, p.bias);
+        store_row_chunk(v2, yrow, nb + 64, p.N, p.bias);
+        store_row_chunk(v3, yrow, nb + 96, p.N, p.bias);
       }
     }
   }

@@ -196,6 +196,32 @@ __global__ void lora_l1_kernel(const __nv_bfloat16* __restrict__ A, const float*
   l1t[static_cast<size_t>(col0 + j) * K + k] = bf16_from_f64(v);
 }
 
+// The smoothing folded into the down-projection factor:
+// l1st[j][k] = bf16(inv_lambda[k] * l1t[j][k]) (exact product, one rounding),
+// so that X_hat L1 = X (diag(lambda)^-1 L1) reads X as it is.
+__global__ void fold_l1_kernel(const __nv_bfloat16* __restrict__ l1t, const float* __restrict__ inv,
+                               int K, int r, __nv_bfloat16* __restrict__ l1st) {
+  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  const int j = blockIdx.y;
+  if (k >= K || j >= r) return;
+  const double v = static_cast<double>(inv[k]) *
+                   static_cast<double>(__bfloat162float(l1t[static_cast<size_t>(j) * K + k]));
+  l1st[static_cast<size_t>(j) * K + k] = bf16_from_f64(v);
+}
+
+// The up-projection operand of the GEMM's tail: [L2^T | L2^T] (N x 2 r_pad), so
+// that one MMA over K = 2 r_pad adds (hi + lo) L2 for X_hat L1 = hi + lo.
+__global__ void dup_l2_kernel(const __nv_bfloat16* __restrict__ l2t, int N, int r_pad,
+                              __nv_bfloat16* __restrict__ l2t2) {
+  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  if (n >= N) return;
+  for (int j = 0; j < r_pad; ++j) {
+    const __nv_bfloat16 v = l2t[static_cast<size_t>(n) * r_pad + j];
+    l2t2[static_cast<size_t>(n) * 2 * r_pad + j] = v;
+    l2t2[static_cast<size_t>(n) * 2 * r_pad + r_pad + j] = v;
+  }
+}
+
 // R[k, n] = W_hat[k, n] - sum_j L1[k, j] L2[j, n] with the bf16 factors, in fp64,
 // rounded to fp32.
 __global__ void residual_kernel(const double* __restrict__ What,
@@ -218,6 +244,9 @@ __global__ void residual_kernel(const double* __restrict__ What,
 // INT4 : one thread per (n, group of 64): int8 codes N x K, fp16 scales [K/64][N_pad].
 __global__ void quant_weight_nvfp4_kernel(const float* __restrict__ R, int K, int N, int sf_kcols,
                                           uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
+  __shared__ float rcp_tab[128];
+  fill_e4m3_rcp_table(rcp_tab, threadIdx.x, blockDim.x);
+  __syncthreads();
   const int n = blockIdx.x * blockDim.x + threadIdx.x;
   const int g = blockIdx.y;
   if (n >= N) return;
@@ -225,7 +254,7 @@ __global__ void quant_weight_nvfp4_kernel(const float* __restrict__ R, int K, in
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = R[static_cast<size_t>(16 * g + i) * N + n];
   uint32_t cw[2];
-  const uint32_t s8 = quant16_nvfp4(v, cw);
+  const uint32_t s8 = quant16_nvfp4(v, cw, rcp_tab);
   uint32_t* dst = reinterpret_cast<uint32_t*>(codes + static_cast<size_t>(n) * (K / 2) + 8 * g);
   dst[0] = cw[0];
   dst[1] = cw[1];

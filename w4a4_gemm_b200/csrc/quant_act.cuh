@@ -2,19 +2,28 @@
 // quantization and the low-rank down-projection in one pass over X.
 //
 // SVDQuant Sec. 4.3 (Nunchaku, Fig. 6b): the down-projection X_hat L1 shares
-// its input with the quantizer, so both are computed from one read of X.
+// its input with the quantizer, so both are computed from one read of X.  The
+// smoothing is folded into the factor, X_hat L1 = X (diag(lambda)^-1 L1), so
+// the tensor core reads the TMA-loaded X tile as it is, in parallel with the
+// quantizer warps.
 //
-// CTA = 128 rows x a contiguous range of 64-wide K tiles.  Row blocks with
-// too few CTAs to fill the GPU are split along K across a thread-block
-// cluster; the rank-r partial products are then summed in fixed rank order
-// through distributed shared memory.
-//   warp 0      : TMA producer (X tile 128x64 bf16, L1^T tile r_pad x 64, 1/lambda)
-//   warp 1      : TMEM owner; one lane issues the tcgen05 bf16 MMAs
-//                 XL1 += bf16(x_hat) (128 x 64) * L1^T(64 x r_pad)
-//   warps 2..9  : quantizers; warp w serves TMEM lane quarter w % 4 (rows)
-//                 and K half (w - 2) / 4 of every tile.  They smooth X,
-//                 quantize it, store codes and scales, and write bf16(x_hat)
-//                 back in place as the MMA's A operand.
+// One CTA owns BM = 128 / S token rows over the whole of K, so no partial sum
+// ever leaves the CTA.  Each pipeline stage holds S consecutive 64-wide K
+// sub-tiles of those rows stacked on top of each other as the 128-row A
+// operand of one tcgen05 MMA, and the S matching 64 x r_pad slices of the
+// folded factor L1s side by side as its N = S * r_pad wide B operand:
+//   D[j*BM + i, j'*r_pad + c] += sum_k x[i, sub-tile j, k] * L1s[sub-tile j', k, c]
+// Only the diagonal blocks j == j' are wanted; summing them over j gives
+// X L1s = X_hat L1 for row i.  The host picks the smallest S (1, 2, 4 or 8, at most
+// 256 / r_pad) that gives about one CTA per SM.
+//   warp 0      : TMA producer (S X boxes BM x 64, S L1s^T boxes r_pad x 64, 1/lambda)
+//   warp 1      : TMEM owner; one lane issues the kind::f16 MMAs
+//   warps 2..17 : quantizers; warp w serves A-tile rows 32 (w % 4) .. + 31 and
+//                 K quarter (w - 2) / 4 (one NVFP4 group of 16) of each 64-wide
+//                 sub-tile.  They smooth X, quantize it, release the stage and
+//                 then store codes and scales.  At the end warps 2..5 read the
+//                 diagonal blocks and the CTA sums them into XL1, kept at fp32
+//                 precision as a bf16 pair hi + lo for the GEMM's tail MMA.
 #pragma once
 
 #include "svdq_formats.cuh"
@@ -22,42 +31,49 @@
 
 namespace svdq {
 
-constexpr int kQuantBM = 128;
-constexpr int kQuantBK = 64;
-constexpr int kQuantStages = 4;
-constexpr int kQuantThreads = 320;
-constexpr int kQuantWarps = 8;  // quantizer warps
+constexpr int kQuantTileRows = 128;   // rows of the MMA A operand
+constexpr int kQuantBK = 64;          // K width of one sub-tile
+constexpr int kQuantMaxStages = 8;
+constexpr int kQuantThreads = 576;
+constexpr int kQuantWarps = 16;       // quantizer warps
+constexpr uint32_t kQuantStageBudget = 200u * 1024u;   // shared memory for the pipeline
 
 struct QuantParams {
   int M, K;
   int r_pad;        // 0 = no low-rank branch; else 16, 32, 64, 128, 192 or 256
-  int kt_total;     // K / 64
-  int ksplit;       // CTAs per 128-row block (cluster extent along y)
-  int M_pad;        // M rounded up to 128
+  int S;            // stacked K sub-tiles per stage (BM = 128 / S rows per CTA)
+  int M_pad;        // M rounded up to 128 (scale atoms)
   int sf_kcols;     // NVFP4: K_pad / 64 scale atoms per 128-row block
-  const float* inv_lambda;
+  const float* inv_lambda;  // K rounded up to 512 (zero padded)
   uint8_t* codes;   // NVFP4: M x K/2 packed E2M1; INT4: M x K int8
   uint8_t* sf;      // NVFP4: 512-byte atoms; INT4: fp16 [K/64][M_pad]
-  __nv_bfloat16* xl1;  // M x r_pad
+  __nv_bfloat16* xl1;  // M x 2 r_pad: X_hat L1 as a bf16 pair, hi | lo (hi + lo = fp32 value)
   long long budget;
 };
 
+// Most sub-tiles that can be stacked for a given padded rank (N = S * r_pad <= 256).
+__host__ __device__ inline int quant_stack_max(int r_pad) {
+  if (r_pad <= 32) return 8;
+  if (r_pad <= 64) return 4;
+  if (r_pad <= 128) return 2;
+  return 1;
+}
+
 struct QuantSmem {
-  uint32_t x_off, l1_off, il_off, stage_bytes, red_off, bar_off, total;
+  uint32_t x_off, l1_off, il_off, stage_bytes, stages, bar_off, total;
 };
 
-__host__ __device__ inline QuantSmem quant_smem_layout(int r_pad) {
+__host__ __device__ inline QuantSmem quant_smem_layout(int r_pad, int S) {
   QuantSmem L;
   L.x_off = 0;
-  L.l1_off = kQuantBM * kQuantBK * 2;                      // 16384
-  L.il_off = L.l1_off + r_pad * 128;
-  uint32_t sb = L.il_off + kQuantBK * 4;
+  L.l1_off = kQuantTileRows * kQuantBK * 2;                // 16384
+  L.il_off = L.l1_off + S * r_pad * 128;                   // S * r_pad rows of 128 bytes
+  uint32_t sb = L.il_off + S * kQuantBK * 4;
   L.stage_bytes = (sb + 1023u) & ~1023u;
-  // the K-split partial sums reuse the stage buffers once the K loop is over
-  // (128 x r_pad fp32 never exceeds the four stages)
-  L.red_off = 0;
-  L.bar_off = L.stage_bytes * kQuantStages;
-  L.total = L.bar_off + 256 + 1024;                        // barriers + alignment slack
+  L.stages = kQuantStageBudget / L.stage_bytes;
+  if (L.stages > static_cast<uint32_t>(kQuantMaxStages)) L.stages = kQuantMaxStages;
+  L.bar_off = L.stage_bytes * L.stages;
+  L.total = L.bar_off + 256 + 512 + 1024;                  // barriers, 1/scale table, alignment
   return L;
 }
 
@@ -66,37 +82,39 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
     quant_act_kernel(const __grid_constant__ CUtensorMap tm_x,
                      const __grid_constant__ CUtensorMap tm_l1t, const QuantParams p) {
   extern __shared__ uint8_t smem_raw[];
-  const QuantSmem L = quant_smem_layout(p.r_pad);
+  const QuantSmem L = quant_smem_layout(p.r_pad, p.S);
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
+  const int NS = static_cast<int>(L.stages);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bar_off);
-  uint64_t* xready = full + kQuantStages;
-  uint64_t* empty = xready + kQuantStages;
-  uint64_t* acc_full = empty + kQuantStages;
+  uint64_t* empty = full + kQuantMaxStages;
+  uint64_t* acc_full = empty + kQuantMaxStages;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_full + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  float* rcp_tab = reinterpret_cast<float*>(smem + L.bar_off + 256);   // 1/E4M3 value, 128 entries
 
   const uint32_t warp = warp_id();
   const uint32_t lane = lane_id();
   const bool has_lr = p.r_pad > 0;
-  const int m_blk = blockIdx.x;
-  const int m0 = m_blk * kQuantBM;
-  const int ks = blockIdx.y;
-  const int kt_begin = (ks * p.kt_total) / p.ksplit;
-  const int kt_end = ((ks + 1) * p.kt_total) / p.ksplit;
-  const int nkt = kt_end - kt_begin;
-  const uint32_t tmem_cols = p.r_pad <= 32 ? 32u : (p.r_pad <= 64 ? 64u : (p.r_pad <= 128 ? 128u : 256u));
+  const int S = p.S;
+  const int BM = kQuantTileRows / S;
+  const int m0 = blockIdx.x * BM;
+  const int kstep = S * kQuantBK;                       // K columns per stage
+  const int nkt = (p.K + kstep - 1) / kstep;
+  const int n_mma = S * p.r_pad;                        // MMA N
+  const uint32_t tmem_cols = n_mma <= 32 ? 32u : (n_mma <= 64 ? 64u : (n_mma <= 128 ? 128u : 256u));
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kQuantStages; ++s) {
+    for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&xready[s], kQuantWarps);
-      mbar_init(&empty[s], has_lr ? 1 : kQuantWarps);
+      // released by the quantizer warps and, with a low-rank branch, the MMAs
+      mbar_init(&empty[s], kQuantWarps + (has_lr ? 1 : 0));
     }
     mbar_init(acc_full, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
+  if (FMT == 0 && warp >= 2 && warp < 6) fill_e4m3_rcp_table(rcp_tab, threadIdx.x - 64, 128);
   if (warp == 1 && has_lr) {
     tmem_alloc(tmem_holder, tmem_cols);
     tmem_relinquish();
@@ -111,42 +129,42 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
     if (elect_one()) {
       prefetch_tmap(&tm_x);
       if (has_lr) prefetch_tmap(&tm_l1t);
-      const uint32_t tx = kQuantBM * kQuantBK * 2 + (has_lr ? p.r_pad * 128 : 0) + kQuantBK * 4;
+      const uint32_t tx = S * (BM * kQuantBK * 2 + (has_lr ? p.r_pad * 128 : 0) + kQuantBK * 4);
       int issued = 0;
       for (int i = 0; i < nkt; ++i) {
-        const int s = i % kQuantStages;
-        const uint32_t ph = (i / kQuantStages) & 1;
+        const int s = i % NS;
+        const uint32_t ph = (i / NS) & 1;
         if (!mbar_wait(&empty[s], ph ^ 1, p.budget, abort_flag)) {
           raise_error(kErrWaitQuant);
           *abort_flag = 1;
           break;
         }
         uint8_t* st = smem + s * L.stage_bytes;
-        const int kt = kt_begin + i;
         mbar_arrive_expect_tx(&full[s], tx);
-        tma_load_2d(st + L.x_off, &tm_x, &full[s], kt * kQuantBK, m0);
-        if (has_lr) tma_load_2d(st + L.l1_off, &tm_l1t, &full[s], kt * kQuantBK, 0);
-        bulk_load(st + L.il_off, p.inv_lambda + kt * kQuantBK, kQuantBK * 4, &full[s]);
+        for (int j = 0; j < S; ++j) {
+          const int k = (i * S + j) * kQuantBK;   // may lie past K: the box is zero-filled
+          tma_load_2d(st + L.x_off + j * BM * 128, &tm_x, &full[s], k, m0);
+          if (has_lr) tma_load_2d(st + L.l1_off + j * p.r_pad * 128, &tm_l1t, &full[s], k, 0);
+        }
+        bulk_load(st + L.il_off, p.inv_lambda + i * kstep, S * kQuantBK * 4, &full[s]);
         issued = i + 1;
       }
       // never leave while a copy into this CTA's shared memory is still in flight
       if (*abort_flag) {
-        for (int i = (issued > kQuantStages ? issued - kQuantStages : 0); i < issued; ++i)
-          mbar_wait(&full[i % kQuantStages], (i / kQuantStages) & 1, p.budget, nullptr);
+        for (int i = (issued > NS ? issued - NS : 0); i < issued; ++i)
+          mbar_wait(&full[i % NS], (i / NS) & 1, p.budget, nullptr);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (has_lr && elect_one()) {
-      const uint32_t idesc = idesc_bf16_f32(kQuantBM, p.r_pad);
-      bool ok = true;
+      const uint32_t idesc = idesc_bf16_f32(kQuantTileRows, n_mma);
       for (int i = 0; i < nkt; ++i) {
-        const int s = i % kQuantStages;
-        const uint32_t ph = (i / kQuantStages) & 1;
-        if (!mbar_wait(&xready[s], ph, p.budget, abort_flag)) {
+        const int s = i % NS;
+        const uint32_t ph = (i / NS) & 1;
+        if (!mbar_wait(&full[s], ph, p.budget, abort_flag)) {
           raise_error(kErrWaitQuant);
           *abort_flag = 1;
-          ok = false;
           break;
         }
         tc_fence_after();
@@ -159,183 +177,165 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
         }
         tc_commit(&empty[s]);
       }
-      (void)ok;
       tc_commit(acc_full);  // also covers an early exit: waits for every issued MMA
     }
   } else {
     // ------------------------------------------------------------ quantizers
-    // NVFP4: warp half h quantizes K columns [32h, 32h + 32) of every tile (two
-    // groups of 16).  INT4: a group spans the whole 64-wide tile, so the h = 0
-    // warps quantize it alone and the h = 1 warps only take part in the
-    // hand-off to the MMA.
-    const uint32_t q = warp & 3u;             // TMEM lane quarter = row group
-    const uint32_t h = (warp - 2) >> 2;       // K half of each 64-wide tile
-    const uint32_t row = q * 32 + lane;
-    const int m = m0 + static_cast<int>(row);
+    // NVFP4: warp quarter g quantizes K columns [16g, 16g + 16) of each
+    // sub-tile row (one group).  INT4: a group spans the whole 64-wide
+    // sub-tile, so the g = 0 warps quantize it alone and the others only
+    // release the stage.
+    const uint32_t q = warp & 3u;
+    const uint32_t g = (warp - 2) >> 2;
+    const uint32_t R = q * 32 + lane;          // row of the stacked A tile
+    const int j = static_cast<int>(R) / BM;    // K sub-tile
+    const int m = m0 + static_cast<int>(R) % BM;
     const bool row_ok = m < p.M;
-    constexpr int kChunks = FMT == 0 ? 4 : 8;   // 16-byte chunks (8 bf16) per thread
-    const bool active = FMT == 0 || h == 0;
-    const uint32_t c0 = FMT == 0 ? 4 * h : 0;
+    constexpr int kChunks = FMT == 0 ? 2 : 8;  // 16-byte chunks (8 bf16) per thread
+    const bool active = FMT == 0 || g == 0;
+    const uint32_t c0 = FMT == 0 ? 2 * g : 0;
     for (int i = 0; i < nkt; ++i) {
-      const int s = i % kQuantStages;
-      const uint32_t ph = (i / kQuantStages) & 1;
+      const int s = i % NS;
+      const uint32_t ph = (i / NS) & 1;
       if (!warp_wait(&full[s], ph, p.budget, abort_flag)) {
         if (lane == 0) raise_error(kErrWaitQuant);
         *abort_flag = 1;
         break;
       }
+      const int kcol = i * S + j;              // 64-wide column group of X
+      const bool col_ok = kcol * kQuantBK < p.K;
+      uint32_t out[FMT == 0 ? 2 : 16];         // codes to store once the stage is released
+      uint32_t sfv = 0;
       if (active) {
-        uint8_t* st = smem + s * L.stage_bytes;
-        const float* il = reinterpret_cast<const float*>(st + L.il_off) + 8 * c0;
-        uint8_t* xrow = st + L.x_off + row * 128;
-        const int kt = kt_begin + i;
+        const uint8_t* st = smem + s * L.stage_bytes;
+        const float4* il = reinterpret_cast<const float4*>(st + L.il_off + (j * kQuantBK + 8 * c0) * 4);
+        const uint8_t* xrow = st + L.x_off + R * 128;
         float v[8 * kChunks];
 #pragma unroll
         for (int c = 0; c < kChunks; ++c) {
-          const uint32_t chunk = ((c0 + c) ^ (row & 7u)) << 4;   // 128-byte swizzle
+          const uint32_t chunk = ((c0 + c) ^ (R & 7u)) << 4;   // 128-byte swizzle
           const uint4 raw = *reinterpret_cast<const uint4*>(xrow + chunk);
-          const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            v[8 * c + 2 * j] = __fmul_rn(bf16_lo(w4[j]), il[8 * c + 2 * j]);
-            v[8 * c + 2 * j + 1] = __fmul_rn(bf16_hi(w4[j]), il[8 * c + 2 * j + 1]);
-          }
+          const float4 l0 = il[2 * c], l1 = il[2 * c + 1];
+          float2 t;
+          t = fmul2_rn(make_float2(bf16_lo(raw.x), bf16_hi(raw.x)), make_float2(l0.x, l0.y));
+          v[8 * c + 0] = t.x; v[8 * c + 1] = t.y;
+          t = fmul2_rn(make_float2(bf16_lo(raw.y), bf16_hi(raw.y)), make_float2(l0.z, l0.w));
+          v[8 * c + 2] = t.x; v[8 * c + 3] = t.y;
+          t = fmul2_rn(make_float2(bf16_lo(raw.z), bf16_hi(raw.z)), make_float2(l1.x, l1.y));
+          v[8 * c + 4] = t.x; v[8 * c + 5] = t.y;
+          t = fmul2_rn(make_float2(bf16_lo(raw.w), bf16_hi(raw.w)), make_float2(l1.z, l1.w));
+          v[8 * c + 6] = t.x; v[8 * c + 7] = t.y;
         }
         if constexpr (FMT == 0) {
-          uint32_t cw[4];
-          const uint32_t s0 = quant16_nvfp4(v, cw);
-          const uint32_t s1 = quant16_nvfp4(v + 16, cw + 2);
-          if (row_ok) {
-            uint8_t* dst = p.codes + static_cast<size_t>(m) * (p.K / 2) + kt * (kQuantBK / 2) + 16 * h;
-            *reinterpret_cast<uint4*>(dst) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-          }
-          // scale atom: 128 rows x 4 scales, byte (row % 32) * 16 + (row / 32) * 4 + k4
-          uint8_t* atom = p.sf + (static_cast<size_t>(m_blk) * p.sf_kcols + kt) * 512;
-          *reinterpret_cast<uint16_t*>(atom + (row & 31u) * 16 + (row >> 5) * 4 + 2 * h) =
-              static_cast<uint16_t>(row_ok ? (s0 | (s1 << 8)) : 0u);
+          sfv = quant16_nvfp4(v, out, rcp_tab);
         } else {
           float amax = 0.0f;
 #pragma unroll
-          for (int j = 0; j < 64; ++j) amax = fmaxf(amax, fabsf(v[j]));
+          for (int e = 0; e < 64; e += 16) amax = fmaxf(amax, absmax16(v + e));
           const uint16_t sh = int4_scale_bits(amax);
           const float sd = __half2float(__ushort_as_half(sh));
-          uint32_t packed[16];
+          sfv = sh;
           if (sd == 0.0f) {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) packed[j] = 0u;
+            for (int e = 0; e < 16; ++e) out[e] = 0u;
           } else {
             const float inv = __frcp_rn(sd);
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
+            for (int e = 0; e < 16; ++e) {
               uint32_t w = 0;
 #pragma unroll
               for (int b = 0; b < 4; ++b)
-                w |= (static_cast<uint32_t>(int4_code(v[4 * j + b], inv)) & 0xFFu) << (8 * b);
-              packed[j] = w;
+                w |= (static_cast<uint32_t>(int4_code(v[4 * e + b], inv)) & 0xFFu) << (8 * b);
+              out[e] = w;
             }
           }
-          if (row_ok) {
-            uint4* dst = reinterpret_cast<uint4*>(p.codes + static_cast<size_t>(m) * p.K + kt * kQuantBK);
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              dst[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
-          }
-          reinterpret_cast<uint16_t*>(p.sf)[static_cast<size_t>(kt) * p.M_pad + m0 + row] =
-              row_ok ? sh : static_cast<uint16_t>(0);
-        }
-        if (has_lr) {
-          // bf16(x_hat) back into the tile at the same swizzled positions: the MMA's A operand
-#pragma unroll
-          for (int c = 0; c < kChunks; ++c) {
-            const uint32_t chunk = ((c0 + c) ^ (row & 7u)) << 4;
-            uint4 o;
-            o.x = pack_bf16x2(v[8 * c + 0], v[8 * c + 1]);
-            o.y = pack_bf16x2(v[8 * c + 2], v[8 * c + 3]);
-            o.z = pack_bf16x2(v[8 * c + 4], v[8 * c + 5]);
-            o.w = pack_bf16x2(v[8 * c + 6], v[8 * c + 7]);
-            *reinterpret_cast<uint4*>(xrow + chunk) = o;
-          }
-          fence_proxy_async_smem();
         }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(has_lr ? &xready[s] : &empty[s]);
+      if (lane == 0) mbar_arrive(&empty[s]);
+      if (active && col_ok) {
+        if constexpr (FMT == 0) {
+          if (row_ok) {
+            uint8_t* dst = p.codes + static_cast<size_t>(m) * (p.K / 2) + kcol * (kQuantBK / 2) + 8 * g;
+            *reinterpret_cast<uint2*>(dst) = make_uint2(out[0], out[1]);
+          }
+          // scale atom: 128 rows x 4 scales, byte (m % 32) * 16 + (m % 128 / 32) * 4 + k4
+          uint8_t* atom = p.sf + (static_cast<size_t>(m / 128) * p.sf_kcols + kcol) * 512;
+          atom[(m & 31) * 16 + ((m & 127) >> 5) * 4 + g] = static_cast<uint8_t>(row_ok ? sfv : 0u);
+        } else {
+          if (row_ok) {
+            uint4* dst = reinterpret_cast<uint4*>(p.codes + static_cast<size_t>(m) * p.K + kcol * kQuantBK);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) dst[e] = make_uint4(out[4 * e], out[4 * e + 1], out[4 * e + 2], out[4 * e + 3]);
+          }
+          reinterpret_cast<uint16_t*>(p.sf)[static_cast<size_t>(kcol) * p.M_pad + m] =
+              row_ok ? static_cast<uint16_t>(sfv) : static_cast<uint16_t>(0);
+        }
+      }
     }
   }
-
   __syncwarp();
 
   // ---------------------------------------------------------------- XL1 out
-  float* red = reinterpret_cast<float*>(smem + L.red_off);
-  const bool epi = has_lr && warp >= 2 && warp < 6;
-  if (epi) {
+  // Diagonal block j of the accumulator = the K sub-tiles j (mod S); warps
+  // 2..5 park them in shared memory (the stage buffers are free by now) and
+  // the CTA sums them over j in fixed order and rounds to bf16.
+  float* red = reinterpret_cast<float*>(smem);   // [128][r_pad] fp32
+  if (has_lr && warp >= 2 && warp < 6) {
     const uint32_t q = warp & 3u;
-    const uint32_t row = q * 32 + lane;
-    const bool got = warp_wait(acc_full, 0, p.budget, abort_flag);
-    if (!got) {
+    const uint32_t R = q * 32 + lane;
+    const int j = static_cast<int>(R) / BM;
+    if (!warp_wait(acc_full, 0, p.budget, abort_flag)) {
       if (lane == 0) raise_error(kErrWaitQuant);
       *abort_flag = 1;
     }
     tc_fence_after();
-    for (int c = 0; c < p.r_pad; c += 16) {
-      uint32_t r[16];
-      tmem_ld16(tmem_base + ((q * 32u) << 16) + c, r);
-      tmem_wait_ld();
-      if (p.ksplit == 1) {
-        const int m = m0 + static_cast<int>(row);
-        if (m < p.M) {
-          uint4 o0, o1;
-          o0.x = pack_bf16x2(__uint_as_float(r[0]), __uint_as_float(r[1]));
-          o0.y = pack_bf16x2(__uint_as_float(r[2]), __uint_as_float(r[3]));
-          o0.z = pack_bf16x2(__uint_as_float(r[4]), __uint_as_float(r[5]));
-          o0.w = pack_bf16x2(__uint_as_float(r[6]), __uint_as_float(r[7]));
-          o1.x = pack_bf16x2(__uint_as_float(r[8]), __uint_as_float(r[9]));
-          o1.y = pack_bf16x2(__uint_as_float(r[10]), __uint_as_float(r[11]));
-          o1.z = pack_bf16x2(__uint_as_float(r[12]), __uint_as_float(r[13]));
-          o1.w = pack_bf16x2(__uint_as_float(r[14]), __uint_as_float(r[15]));
-          uint4* dst = reinterpret_cast<uint4*>(p.xl1 + static_cast<size_t>(m) * p.r_pad + c);
-          dst[0] = o0;
-          dst[1] = o1;
-        }
-      } else {
-        float* dst = red + row * p.r_pad + c;
+    // a TMEM load reads the same columns for all 32 lanes: when a warp's rows
+    // span two sub-tiles (BM = 16), read both diagonal blocks, keep the own one
+    const int j_first = static_cast<int>(q * 32) / BM, j_last = static_cast<int>(q * 32 + 31) / BM;
+    for (int jj = j_first; jj <= j_last; ++jj) {
+      for (int c = 0; c < p.r_pad; c += 16) {
+        uint32_t r[16];
+        tmem_ld16(tmem_base + ((q * 32u) << 16) + jj * p.r_pad + c, r);
+        tmem_wait_ld();
+        if (jj == j) {
 #pragma unroll
-        for (int j = 0; j < 16; j += 4)
-          *reinterpret_cast<float4*>(dst + j) =
-              make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]),
-                          __uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
-      }
-    }
-  }
-  if (has_lr && p.ksplit > 1) {
-    cluster_sync();  // every partial is in its CTA's shared memory
-    if (ks == 0 && epi) {
-      const uint32_t row = (warp & 3u) * 32 + lane;
-      const int m = m0 + static_cast<int>(row);
-      const uint32_t base = smem_u32(red + row * p.r_pad);
-      for (int c = 0; c < p.r_pad; c += 8) {
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int rk = 0; rk < p.ksplit; ++rk) {
-          const uint32_t a = map_shared_rank(base + 4 * c, rk);
-          const float4 x0 = ld_shared_cluster_f32x4(a);
-          const float4 x1 = ld_shared_cluster_f32x4(a + 16);
-          acc[0] += x0.x; acc[1] += x0.y; acc[2] += x0.z; acc[3] += x0.w;
-          acc[4] += x1.x; acc[5] += x1.y; acc[6] += x1.z; acc[7] += x1.w;
-        }
-        if (m < p.M) {
-          uint4 o;
-          o.x = pack_bf16x2(acc[0], acc[1]);
-          o.y = pack_bf16x2(acc[2], acc[3]);
-          o.z = pack_bf16x2(acc[4], acc[5]);
-          o.w = pack_bf16x2(acc[6], acc[7]);
-          *reinterpret_cast<uint4*>(p.xl1 + static_cast<size_t>(m) * p.r_pad + c) = o;
+          for (int e = 0; e < 16; e += 4)
+            *reinterpret_cast<float4*>(red + R * p.r_pad + c + e) =
+                make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]),
+                            __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
         }
       }
     }
-    cluster_sync();  // keep every CTA's partial alive until rank 0 has read it
   }
   tc_fence_before();
   __syncthreads();
+  if (has_lr) {
+    // BM rows x r_pad columns, 8 columns per thread over all 320 threads
+    const int units = BM * (p.r_pad / 8);
+    for (int u = threadIdx.x; u < units; u += kQuantThreads) {
+      const int i = u / (p.r_pad / 8);
+      const int c = (u % (p.r_pad / 8)) * 8;
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      for (int jj = 0; jj < S; ++jj) {
+        const float* src = red + (jj * BM + i) * p.r_pad + c;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = __fadd_rn(acc[e], src[e]);
+      }
+      if (m0 + i < p.M) {
+        // hi = bf16(acc), lo = bf16(acc - hi): hi + lo carries acc to ~2^-17
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          hi[e] = pack_bf16x2(acc[2 * e], acc[2 * e + 1]);
+          lo[e] = pack_bf16x2(acc[2 * e] - bf16_lo(hi[e]), acc[2 * e + 1] - bf16_hi(hi[e]));
+        }
+        __nv_bfloat16* dst = p.xl1 + static_cast<size_t>(m0 + i) * (2 * p.r_pad) + c;
+        *reinterpret_cast<uint4*>(dst) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4*>(dst + p.r_pad) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      }
+    }
+  }
   if (warp == 1 && has_lr) {
     // every MMA this CTA issued has retired before its TMEM is released
     mbar_wait(acc_full, 0, p.budget, nullptr);

@@ -38,7 +38,9 @@ struct svdq_weights {
   uint8_t* wcodes = nullptr;  // NVFP4: N x K/2 packed; INT4: N x K int8
   uint8_t* wsf = nullptr;     // NVFP4: atoms [N_pad/128][sf_kcols][512]; INT4: fp16 [K/64][N_pad]
   __nv_bfloat16* l1t = nullptr;  // r_pad x K
+  __nv_bfloat16* l1st = nullptr; // r_pad x K: bf16(diag(1/lambda) L1)^T, read by the activation kernel
   __nv_bfloat16* l2t = nullptr;  // N x r_pad
+  __nv_bfloat16* l2t2 = nullptr; // N x 2 r_pad: [L2^T | L2^T], the tail MMA's B operand
   __nv_bfloat16* bias = nullptr;
   CUtensorMap tm_b, tm_l1t, tm_l2t;
 };
@@ -143,10 +145,11 @@ int device_setup(int dev) {
   std::lock_guard<std::mutex> lk(g_mutex);
   if (d.attrs_set) return SVDQ_OK;
   SVDQ_CUDA(cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev));
-  SVDQ_CUDA(cudaFuncSetAttribute(quant_act_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 quant_smem_layout(256).total));
-  SVDQ_CUDA(cudaFuncSetAttribute(quant_act_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 quant_smem_layout(256).total));
+  uint32_t qmax = 0;
+  for (int rp : {0, 16, 32, 64, 128, 192, 256})
+    for (int S = 1; S <= quant_stack_max(rp); S *= 2) qmax = std::max(qmax, quant_smem_layout(rp, S).total);
+  SVDQ_CUDA(cudaFuncSetAttribute(quant_act_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, qmax));
+  SVDQ_CUDA(cudaFuncSetAttribute(quant_act_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, qmax));
   SVDQ_CUDA(cudaFuncSetAttribute(gemm_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kGemmSmemBytes));
   SVDQ_CUDA(cudaFuncSetAttribute(gemm_int4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -161,6 +164,15 @@ int current_device(int* dev) {
 }
 
 // ------------------------------------------------------------ workspace ---
+// Stacked K sub-tiles of the activation kernel (rows per CTA = 128 / S): the
+// smallest S that gives about one CTA per SM, as far as the rank allows.
+int quant_stack_for(int M, int r_pad, int sms) {
+  const int smax = r_pad > 0 ? quant_stack_max(r_pad) : 8;
+  int S = 1;
+  while (S < smax && (M + 128 / S - 1) / (128 / S) < (9 * sms) / 10) S *= 2;
+  return S;
+}
+
 struct ActLayout {
   int M, M_pad;
   size_t codes_off, codes_bytes, sf_off, sf_bytes, xl1_off, xl1_bytes, total;
@@ -174,7 +186,7 @@ ActLayout act_layout(const svdq_weights* w, int M) {
                                        : static_cast<size_t>(M) * w->K;
   L.sf_bytes = w->fmt == SVDQ_NVFP4 ? static_cast<size_t>(L.M_pad / 128) * w->sf_kcols * 512
                                     : static_cast<size_t>(w->K / 64) * L.M_pad * 2;
-  L.xl1_bytes = static_cast<size_t>(M) * w->r_pad * 2;
+  L.xl1_bytes = static_cast<size_t>(M) * 2 * w->r_pad * 2;   // bf16 hi | lo
   L.codes_off = 0;
   L.sf_off = align256(L.codes_bytes);
   L.xl1_off = L.sf_off + align256(L.sf_bytes);
@@ -192,10 +204,10 @@ int encode_weight_maps(svdq_weights* w) {
     rc = make_map(&w->tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->wcodes, w->K, w->N, 64, kI4BN);
   if (rc) return rc;
   if (w->r_pad > 0) {
-    rc = make_map(&w->tm_l1t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w->l1t, w->K, w->r_pad, 64, w->r_pad);
+    rc = make_map(&w->tm_l1t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w->l1st, w->K, w->r_pad, 64, w->r_pad);
     if (rc) return rc;
-    const int lc = lr_chunk_cols(w->r_pad);
-    rc = make_map(&w->tm_l2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w->l2t, w->r_pad, w->N, lc, kGemmBN);
+    const int lc = lr_chunk_cols(2 * w->r_pad);
+    rc = make_map(&w->tm_l2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w->l2t2, 2 * w->r_pad, w->N, lc, kGemmBN);
     if (rc) return rc;
   } else {
     w->tm_l1t = w->tm_b;
@@ -211,7 +223,9 @@ void free_weights(svdq_weights* w) {
   cudaFree(w->wcodes);
   cudaFree(w->wsf);
   cudaFree(w->l1t);
+  cudaFree(w->l1st);
   cudaFree(w->l2t);
+  cudaFree(w->l2t2);
   cudaFree(w->bias);
   delete w;
 }
@@ -233,16 +247,21 @@ int alloc_weights(svdq_weights* w, cudaStream_t st) {
                                             : static_cast<size_t>(w->N) * w->K;
   const size_t sfb = w->fmt == SVDQ_NVFP4 ? static_cast<size_t>(w->N_pad / 128) * w->sf_kcols * 512
                                           : static_cast<size_t>(w->K / 64) * w->N_pad * 2;
-  if (cudaMalloc(&w->inv_lambda, w->K * sizeof(float)) != cudaSuccess ||
+  // 1/lambda is read in 512-value blocks by the activation kernel: zero-pad it
+  const size_t il_bytes = static_cast<size_t>(round_up(w->K, 512)) * sizeof(float);
+  if (cudaMalloc(&w->inv_lambda, il_bytes) != cudaSuccess ||
       cudaMalloc(&w->lambda, w->K * sizeof(float)) != cudaSuccess ||
       cudaMalloc(&w->wcodes, codes) != cudaSuccess || cudaMalloc(&w->wsf, sfb) != cudaSuccess)
     return SVDQ_ERR_ALLOC;
+  SVDQ_CUDA(cudaMemsetAsync(w->inv_lambda, 0, il_bytes, st));
   SVDQ_CUDA(cudaMemsetAsync(w->wsf, 0, sfb, st));
   if (w->r_pad > 0) {
     if (cudaMalloc(&w->l1t, static_cast<size_t>(w->r_pad) * w->K * 2) != cudaSuccess ||
+        cudaMalloc(&w->l1st, static_cast<size_t>(w->r_pad) * w->K * 2) != cudaSuccess ||
         cudaMalloc(&w->l2t, static_cast<size_t>(w->N) * w->r_pad * 2) != cudaSuccess)
       return SVDQ_ERR_ALLOC;
     SVDQ_CUDA(cudaMemsetAsync(w->l1t, 0, static_cast<size_t>(w->r_pad) * w->K * 2, st));
+    SVDQ_CUDA(cudaMemsetAsync(w->l1st, 0, static_cast<size_t>(w->r_pad) * w->K * 2, st));
     SVDQ_CUDA(cudaMemsetAsync(w->l2t, 0, static_cast<size_t>(w->N) * w->r_pad * 2, st));
   }
   return SVDQ_OK;
@@ -259,6 +278,21 @@ int quantize_residual(svdq_weights* w, const float* R, cudaStream_t st) {
                                                    reinterpret_cast<int8_t*>(w->wcodes),
                                                    reinterpret_cast<uint16_t*>(w->wsf));
   }
+  SVDQ_CHECK_LAUNCH();
+  return SVDQ_OK;
+}
+
+// The derived operands the kernels read: l1st = bf16(diag(1/lambda) L1)^T and
+// l2t2 = [L2^T | L2^T], from the current l1t, l2t and inv_lambda.
+int refold_l1(svdq_weights* w, cudaStream_t st) {
+  if (w->rank == 0) return SVDQ_OK;
+  cudaFree(w->l2t2);
+  w->l2t2 = nullptr;
+  if (cudaMalloc(&w->l2t2, static_cast<size_t>(w->N) * 2 * w->r_pad * 2) != cudaSuccess)
+    return SVDQ_ERR_ALLOC;
+  dup_l2_kernel<<<(w->N + 255) / 256, 256, 0, st>>>(w->l2t, w->N, w->r_pad, w->l2t2);
+  fold_l1_kernel<<<dim3((w->K + 255) / 256, w->rank), 256, 0, st>>>(w->l1t, w->inv_lambda, w->K,
+                                                                     w->rank, w->l1st);
   SVDQ_CHECK_LAUNCH();
   return SVDQ_OK;
 }
@@ -283,13 +317,19 @@ int do_append_lora(svdq_weights* w, const void* A, const void* B, int rl, cudaSt
   const int r_new = r_old + rl;
   if (r_new > 256 || r_new > std::min(w->K, w->N)) return SVDQ_ERR_UNSUPPORTED_SHAPE;
   const int rp_new = rank_padded(r_new);
-  __nv_bfloat16 *l1t = nullptr, *l2t = nullptr;
+  __nv_bfloat16 *l1t = nullptr, *l1st = nullptr, *l2t = nullptr;
   if (cudaMalloc(&l1t, static_cast<size_t>(rp_new) * w->K * 2) != cudaSuccess) return SVDQ_ERR_ALLOC;
-  if (cudaMalloc(&l2t, static_cast<size_t>(w->N) * rp_new * 2) != cudaSuccess) {
+  if (cudaMalloc(&l1st, static_cast<size_t>(rp_new) * w->K * 2) != cudaSuccess) {
     cudaFree(l1t);
     return SVDQ_ERR_ALLOC;
   }
+  if (cudaMalloc(&l2t, static_cast<size_t>(w->N) * rp_new * 2) != cudaSuccess) {
+    cudaFree(l1t);
+    cudaFree(l1st);
+    return SVDQ_ERR_ALLOC;
+  }
   cudaMemsetAsync(l1t, 0, static_cast<size_t>(rp_new) * w->K * 2, st);
+  cudaMemsetAsync(l1st, 0, static_cast<size_t>(rp_new) * w->K * 2, st);
   cudaMemsetAsync(l2t, 0, static_cast<size_t>(w->N) * rp_new * 2, st);
   if (r_old > 0) {
     const size_t n1 = static_cast<size_t>(r_old) * w->K;
@@ -304,16 +344,22 @@ int do_append_lora(svdq_weights* w, const void* A, const void* B, int rl, cudaSt
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) {
     cudaFree(l1t);
+    cudaFree(l1st);
     cudaFree(l2t);
     std::fprintf(stderr, "svdq: LoRA fold failed: %s\n", cudaGetErrorString(e));
     return SVDQ_ERR_CUDA;
   }
   cudaFree(w->l1t);
+  cudaFree(w->l1st);
   cudaFree(w->l2t);
   w->l1t = l1t;
+  w->l1st = l1st;
   w->l2t = l2t;
   w->rank = r_new;
   w->r_pad = rp_new;
+  int rc = refold_l1(w, st);
+  if (rc == SVDQ_OK && cudaStreamSynchronize(st) != cudaSuccess) rc = SVDQ_ERR_CUDA;
+  if (rc) return rc;
   return encode_weight_maps(w);
 }
 
@@ -459,6 +505,7 @@ SVDQ_API int svdq_prepare_weights(const svdq_prepare_desc* d, void* stream, svdq
       break;
     }
     if (w->rank > 0 && (rc = lowrank_factors(w, What.as<double>(), st))) break;
+    if ((rc = refold_l1(w, st))) break;
     residual_kernel<<<dim3((N + 255) / 256, K), 256, 0, st>>>(
         What.as<double>(), w->l1t, w->l2t, K, N, w->rank, w->r_pad, R.as<float>());
     if (cudaGetLastError() != cudaSuccess) {
@@ -541,6 +588,7 @@ SVDQ_API int svdq_load_weights(const svdq_parts_desc* d, void* stream, svdq_weig
         break;
       }
     }
+    if ((rc = refold_l1(w, st))) break;
     if ((rc = quantize_residual(w, d->R, st))) break;
     if ((rc = copy_bias(w, d->bias, st))) break;
     if (cudaStreamSynchronize(st) != cudaSuccess) {
@@ -595,14 +643,16 @@ SVDQ_API int svdq_quantize_act(const svdq_weights* w, const void* X, int M, void
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const ActLayout L = act_layout(w, M);
   uint8_t* base = static_cast<uint8_t*>(ws);
+  const int S = quant_stack_for(M, w->r_pad, g_dev[dev].sms);
+  const int BM = kQuantTileRows / S;
   CUtensorMap tm_x;
-  if ((rc = make_map(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, w->K, M, kQuantBK, kQuantBM)))
+  if ((rc = make_map(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, w->K, M, kQuantBK, BM)))
     return rc;
   QuantParams p;
   p.M = M;
   p.K = w->K;
   p.r_pad = w->r_pad;
-  p.kt_total = w->K / kQuantBK;
+  p.S = S;
   p.M_pad = L.M_pad;
   p.sf_kcols = w->sf_kcols;
   p.inv_lambda = w->inv_lambda;
@@ -610,38 +660,20 @@ SVDQ_API int svdq_quantize_act(const svdq_weights* w, const void* X, int M, void
   p.sf = base + L.sf_off;
   p.xl1 = reinterpret_cast<__nv_bfloat16*>(base + L.xl1_off);
   p.budget = wait_budget();
-  const int m_tiles = L.M_pad / kQuantBM;
-  // split K over a cluster when the row blocks alone leave the GPU idle
-  int ks = 1;
-  const int target = 2 * g_dev[dev].sms;
-  while (ks < 8 && m_tiles * ks < target && (ks * 2) <= p.kt_total) ks *= 2;
-  p.ksplit = ks;
   if (w->fmt == SVDQ_NVFP4 && w->sf_kcols * 64 != w->K) {
     // zero the scale atoms of the K padding (read by the GEMM's last K step)
     const size_t pitch = static_cast<size_t>(w->sf_kcols) * 512;
     const size_t off = static_cast<size_t>(w->K / 64) * 512;
-    SVDQ_CUDA(cudaMemset2DAsync(p.sf + off, pitch, 0, pitch - off, m_tiles, st));
+    SVDQ_CUDA(cudaMemset2DAsync(p.sf + off, pitch, 0, pitch - off, L.M_pad / 128, st));
   }
-  const QuantSmem S = quant_smem_layout(w->r_pad);
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(m_tiles, ks, 1);
-  cfg.blockDim = dim3(kQuantThreads, 1, 1);
-  cfg.dynamicSmemBytes = S.total;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = ks;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = ks > 1 ? 1 : 0;
+  const QuantSmem Q = quant_smem_layout(w->r_pad, S);
+  const dim3 grid((M + BM - 1) / BM);
   const CUtensorMap& tm_l1t = w->r_pad > 0 ? w->tm_l1t : tm_x;
-  cudaError_t e = w->fmt == SVDQ_NVFP4 ? cudaLaunchKernelEx(&cfg, quant_act_kernel<0>, tm_x, tm_l1t, p)
-                                       : cudaLaunchKernelEx(&cfg, quant_act_kernel<1>, tm_x, tm_l1t, p);
-  if (e != cudaSuccess) {
-    std::fprintf(stderr, "svdq: activation kernel launch failed: %s\n", cudaGetErrorString(e));
-    return SVDQ_ERR_CUDA;
-  }
+  if (w->fmt == SVDQ_NVFP4)
+    quant_act_kernel<0><<<grid, kQuantThreads, Q.total, st>>>(tm_x, tm_l1t, p);
+  else
+    quant_act_kernel<1><<<grid, kQuantThreads, Q.total, st>>>(tm_x, tm_l1t, p);
+  SVDQ_CHECK_LAUNCH();
   return SVDQ_OK;
 }
 
@@ -662,18 +694,14 @@ SVDQ_API int svdq_linear(const svdq_weights* w, const void* ws, int M, void* Y, 
   const int n_tiles = (w->N + 255) / 256;
   const int tiles = m_tiles * n_tiles;
   const int grid = std::min(tiles, g_dev[dev].sms);
-  if (w->fmt == SVDQ_NVFP4) {
-    if ((rc = make_map(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base + L.codes_off, w->K / 2, M, 128,
-                       kGemmBM)))
-      return rc;
-  } else {
-    if ((rc = make_map(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base + L.codes_off, w->K, M, 64,
-                       kI4BM)))
-      return rc;
-  }
+  if (w->fmt == SVDQ_NVFP4)
+    rc = make_map(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base + L.codes_off, w->K / 2, M, 128, kGemmBM);
+  else
+    rc = make_map(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base + L.codes_off, w->K, M, 64, kI4BM);
+  if (rc) return rc;
   if (w->r_pad > 0) {
-    if ((rc = make_map(&tm_xl1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base + L.xl1_off, w->r_pad, M,
-                       lr_chunk_cols(w->r_pad), 128)))
+    if ((rc = make_map(&tm_xl1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base + L.xl1_off, 2 * w->r_pad, M,
+                       lr_chunk_cols(2 * w->r_pad), 128)))
       return rc;
   } else {
     tm_xl1 = tm_a;
@@ -687,7 +715,7 @@ SVDQ_API int svdq_linear(const svdq_weights* w, const void* ws, int M, void* Y, 
     p.m_tiles = m_tiles;
     p.n_tiles = n_tiles;
     p.num_tiles = tiles;
-    p.r_pad = w->r_pad;
+    p.r_tail = 2 * w->r_pad;
     p.sfa = base + L.sf_off;
     p.sfb = w->wsf;
     p.sf_kcols = w->sf_kcols;
@@ -704,7 +732,7 @@ SVDQ_API int svdq_linear(const svdq_weights* w, const void* ws, int M, void* Y, 
     p.m_tiles = m_tiles;
     p.n_tiles = n_tiles;
     p.num_tiles = tiles;
-    p.r_pad = w->r_pad;
+    p.r_tail = 2 * w->r_pad;
     p.sx = reinterpret_cast<const uint16_t*>(base + L.sf_off);
     p.sw = reinterpret_cast<const uint16_t*>(w->wsf);
     p.M_pad = L.M_pad;
@@ -807,12 +835,21 @@ SVDQ_API int svdq_export_act(const svdq_weights* w, const void* ws, int M, uint8
     }
   }
   if (xl1 && w->rank > 0) {
-    std::vector<uint16_t> tmp(static_cast<size_t>(M) * w->r_pad);
+    // fp32 value = hi + lo (exact in fp32)
+    std::vector<uint16_t> tmp(static_cast<size_t>(M) * 2 * w->r_pad);
     SVDQ_CUDA(cudaMemcpy(tmp.data(), base + L.xl1_off, tmp.size() * 2, cudaMemcpyDeviceToHost));
-    uint16_t* out = static_cast<uint16_t*>(xl1);
+    float* out = static_cast<float*>(xl1);
+    auto bf = [](uint16_t h) {
+      const uint32_t u = static_cast<uint32_t>(h) << 16;
+      float f;
+      std::memcpy(&f, &u, 4);
+      return f;
+    };
     for (int m = 0; m < M; ++m)
-      for (int j = 0; j < w->rank; ++j)
-        out[static_cast<size_t>(m) * w->rank + j] = tmp[static_cast<size_t>(m) * w->r_pad + j];
+      for (int j = 0; j < w->rank; ++j) {
+        const size_t row = static_cast<size_t>(m) * 2 * w->r_pad;
+        out[static_cast<size_t>(m) * w->rank + j] = bf(tmp[row + j]) + bf(tmp[row + w->r_pad + j]);
+      }
   }
   return SVDQ_OK;
 }

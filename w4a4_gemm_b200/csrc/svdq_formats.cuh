@@ -4,7 +4,7 @@
 //
 // The quantizer decisions are taken in fp32 exactly as follows:
 //   amax  = max |v|                         (exact)
-//   s32   = amax / q_max                    (IEEE fp32 division, q_max = 6 or 7)
+//   s32   = amax / q_max                    (IEEE fp32 quotient, q_max = 6 or 7)
 //   scale = E4M3(s32) saturating at 448     (NVFP4, round to nearest even)
 //         | fp16(min(s32, 65504))           (INT4, round to nearest even)
 //   q     = v * RN(1 / scale)               (IEEE reciprocal, one RN multiply)
@@ -50,32 +50,91 @@ __device__ __forceinline__ uint32_t e2m1_pack8(const float* q) {
   return out;
 }
 
+// IEEE fp32 x / 6 and x / 7 without a division: q0 = x * RN(1/d),
+// r = fma(-d, q0, x) (exact remainder), q = fma(r, RN(1/d), q0) -- the FMA
+// division by a constant of Markstein and of Brisebarre & Muller ("Accelerating
+// correctly rounded floating-point division when the divisor is known in
+// advance", IEEE TC 2004).  Checked over every significand of a normal binade
+// (and, by power-of-two scaling, every normal x) against IEEE division: equal
+// for d = 7 everywhere and for d = 6 whenever x >= 2^-125; below that x / 6
+// is subnormal and both round to the E4M3 scale 0.
+__device__ __forceinline__ float div_by_const_rn(float x, float d, float rcp_d) {
+  const float q0 = __fmul_rn(x, rcp_d);
+  const float r = __fmaf_rn(-d, q0, x);
+  return __fmaf_rn(r, rcp_d, q0);
+}
+__device__ __forceinline__ float div6_rn(float x) {
+  return div_by_const_rn(x, 6.0f, __uint_as_float(0x3E2AAAABu));   // RN(1/6)
+}
+__device__ __forceinline__ float div7_rn(float x) {
+  return div_by_const_rn(x, 7.0f, __uint_as_float(0x3E124925u));   // RN(1/7)
+}
+
+// Two fp32 products in one instruction (IEEE round-to-nearest per lane).
+__device__ __forceinline__ float2 fmul2_rn(float2 a, float2 b) {
+  unsigned long long x, y, z;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(a.x), "f"(a.y));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(y) : "f"(b.x), "f"(b.y));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(z) : "l"(x), "l"(y));
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(z));
+  return r;
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float m;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(a), "f"(b), "f"(c));
+  return m;
+}
+
+// max |v_i| over 16 values
+__device__ __forceinline__ float absmax16(const float* v) {
+  const float a = fmax3(fabsf(v[0]), fabsf(v[1]), fabsf(v[2]));
+  const float b = fmax3(fabsf(v[3]), fabsf(v[4]), fabsf(v[5]));
+  const float c = fmax3(fabsf(v[6]), fabsf(v[7]), fabsf(v[8]));
+  const float d = fmax3(fabsf(v[9]), fabsf(v[10]), fabsf(v[11]));
+  const float e = fmax3(fabsf(v[12]), fabsf(v[13]), fabsf(v[14]));
+  return fmax3(fmax3(a, b, c), fmax3(d, e, fabsf(v[15])), 0.0f);
+}
+
 // NVFP4 group of 16 values (already smoothed): writes the 8 code bytes into
-// codes[0..1] (two 32-bit words) and returns the E4M3 scale code.
-__device__ __forceinline__ uint32_t quant16_nvfp4(const float* v, uint32_t* codes) {
-  float amax = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
-  const float s32 = __fdiv_rn(amax, 6.0f);
+// codes[0..1] (two 32-bit words) and returns the E4M3 scale code.  `rcp_tab`
+// holds RN(1 / value) of every finite E4M3 code (0 for code 0).
+__device__ __forceinline__ uint32_t quant16_nvfp4(const float* v, uint32_t* codes,
+                                                  const float* rcp_tab) {
+  const float s32 = div6_rn(absmax16(v));
   const uint32_t s8 = e4m3_code(s32);
-  const float sd = e4m3_value(s8);
-  if (sd == 0.0f) {
+  const float inv = rcp_tab[s8];
+  if (inv == 0.0f) {               // zero scale: all codes 0
     codes[0] = 0u;
     codes[1] = 0u;
     return s8;
   }
-  const float inv = __frcp_rn(sd);
   float q[16];
+  const float2 i2 = make_float2(inv, inv);
 #pragma unroll
-  for (int i = 0; i < 16; ++i) q[i] = __fmul_rn(v[i], inv);
+  for (int i = 0; i < 16; i += 2) {
+    const float2 r = fmul2_rn(make_float2(v[i], v[i + 1]), i2);
+    q[i] = r.x;
+    q[i + 1] = r.y;
+  }
   codes[0] = e2m1_pack8(q);
   codes[1] = e2m1_pack8(q + 8);
   return s8;
 }
 
+// Fill a 128-entry table with RN(1 / E4M3 value) for codes 0..127 (code 0 -> 0,
+// NaN code 0x7F -> 0; scales never take it: they saturate at 448).
+__device__ __forceinline__ void fill_e4m3_rcp_table(float* tab, int tid, int nthreads) {
+  for (int c = tid; c < 128; c += nthreads) {
+    const float v = e4m3_value(static_cast<uint32_t>(c));
+    tab[c] = (c == 0 || c == 0x7F) ? 0.0f : __frcp_rn(v);
+  }
+}
+
 // INT4 scale of a group whose absolute maximum is `amax`: fp16 bits.
 __device__ __forceinline__ uint16_t int4_scale_bits(float amax) {
-  const float s32 = __fdiv_rn(amax, 7.0f);
+  const float s32 = div7_rn(amax);
   return __half_as_ushort(__float2half_rn(fminf(s32, 65504.0f)));
 }
 
