@@ -4,16 +4,26 @@
 // SVDQuant Sec. 5.1: INT4 quantization uses groups of 64 with 16-bit scales.
 // Per-group scales s_x[m,g] s_w[g,n] do not factor out of a K sum, so each
 // 64-wide group is one tcgen05 kind::i8 product (two K=32 MMAs, codes held as
-// int8) into one of two TMEM partial buffers; the epilogue warps drain every
-// partial, scale it and accumulate it in fp32 registers while the tensor core
-// fills the other buffer.  The low-rank tail (kind::f16, fp32) goes through
-// the same buffers with scale 1.
+// int8) into one of four TMEM partial buffers; the drain warps scale every
+// partial and accumulate it in fp32 registers while the tensor core fills the
+// other buffers.  The low-rank tail (kind::f16, fp32) goes through the same
+// buffers with scale 1.
 //
-//   warp 0    : TMA producer (A 128 x 64 int8, B 256 x 64 int8, the group's
-//               activation and weight scales; then XL1 / L2^T chunks)
+// The integer partial P (|P| <= 64 * 49 < 2^22) reaches the drain already as
+// fp32: each buffer is pre-filled with the bit pattern of 1.5 * 2^23 and the
+// MMAs accumulate onto it, so the bits read back are those of 1.5 * 2^23 + P
+// exactly, and one subtraction recovers P.  After reading a buffer the drain
+// refills it.  The drain then costs three packed fp32x2 operations per two
+// outputs (subtract, scale product, fused multiply-add).
+//
+//   warp 0    : TMA producer (A 128 x 64 int8, B 128 x 64 int8, the group's
+//               activation scales (fp16) and weight scales (fp32); then the
+//               XL1 / L2^T chunks of the low-rank tail)
 //   warp 1    : TMEM owner, MMA issuer
-//   warps 2-9 : epilogue; warp w drains TMEM lane quarter w % 4 and output
-//               columns [128 * ((w - 2) / 4), +128) of the 128 x 256 tile.
+//   warps 2-9 : drain + epilogue; warp w serves TMEM lane quarter w % 4 and
+//               output columns [64 * ((w - 2) / 4), +64) of the 128 x 128 tile,
+//               read from TMEM in two halves of 32 columns to stay within
+//               168 registers (10 warps share four 16K-register sub-partitions).
 #pragma once
 
 #include "gemm_nvfp4.cuh"
@@ -23,17 +33,20 @@
 namespace svdq {
 
 constexpr int kI4BM = 128;
-constexpr int kI4BN = 256;
+constexpr int kI4BN = 128;
 constexpr int kI4BK = 64;                 // one group
 constexpr int kI4Threads = 320;
 constexpr int kI4EpiWarps = 8;
+constexpr int kI4Bufs = 4;                // TMEM partial buffers of kI4BN columns
 constexpr uint32_t kI4AOff = 0;
 constexpr uint32_t kI4BOff = kI4BM * 128;                  // 16384 (A region fits a 128 B-row tail chunk)
-constexpr uint32_t kI4SxOff = kI4BOff + kI4BN * 128;       // 49152 (so does the B region)
-constexpr uint32_t kI4SwOff = kI4SxOff + kI4BM * 2;        // 49408
-constexpr uint32_t kI4StageBytes = 50176;                  // 49 KB, multiple of 1024
-constexpr int kI4Stages = 4;
+constexpr uint32_t kI4SxOff = kI4BOff + kI4BN * 128;       // 32768 (so does the B region)
+constexpr uint32_t kI4SwOff = kI4SxOff + kI4BM * 2;        // 33024
+constexpr uint32_t kI4StageBytes = 33792;                  // 33 KB, multiple of 1024
+constexpr int kI4Stages = 6;
 constexpr uint32_t kI4SmemBytes = kI4StageBytes * kI4Stages + 256 + 1024;
+constexpr uint32_t kI4Magic = 0x4B400000u;                 // bits of 1.5 * 2^23
+constexpr float kI4MagicF = 12582912.0f;
 
 struct GemmI4Params {
   int M, N, K;
@@ -41,12 +54,64 @@ struct GemmI4Params {
   int m_tiles, n_tiles, num_tiles;
   int r_tail;          // tail K: 2 r_pad (X_hat L1 as hi | lo against L2^T | L2^T), 0 = none
   const uint16_t* sx;  // fp16 [K/64][M_pad]
-  const uint16_t* sw;  // fp16 [K/64][N_pad]
+  const float* sw;     // fp32 [K/64][N_pad] (exact copies of the fp16 weight scales)
   int M_pad, N_pad;
   const __nv_bfloat16* bias;
   __nv_bfloat16* Y;
   long long budget;
 };
+
+__device__ __forceinline__ void tmem_st32_const(uint32_t taddr, uint32_t v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, "
+      "%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1};" ::"r"(taddr),
+      "r"(v)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ unsigned long long f2_pack(float a, float b) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+
+__device__ __forceinline__ unsigned long long u2_pack(uint32_t a, uint32_t b) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+__device__ __forceinline__ float2 f2_unpack(unsigned long long v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+
+// acc + s * (x - c), each lane of the pair rounded as sub, then fused multiply-add.
+__device__ __forceinline__ unsigned long long f2_scale_acc(unsigned long long acc, unsigned long long x,
+                                                           unsigned long long c, unsigned long long s) {
+  unsigned long long p, r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(p) : "l"(x), "l"(c));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(p), "l"(s), "l"(acc));
+  return r;
+}
+
+__device__ __forceinline__ unsigned long long f2_mul(unsigned long long a, unsigned long long b) {
+  unsigned long long r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+__device__ __forceinline__ unsigned long long f2_add(unsigned long long a, unsigned long long b) {
+  unsigned long long r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
 
 __global__ void __launch_bounds__(kI4Threads, 1)
     gemm_int4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
@@ -56,11 +121,12 @@ __global__ void __launch_bounds__(kI4Threads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   constexpr int S = kI4Stages;
+  constexpr int NB = kI4Bufs;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kI4StageBytes * S);
   uint64_t* empty = full + S;
-  uint64_t* pfull = empty + S;      // [2]
-  uint64_t* pempty = pfull + 2;     // [2]
-  uint64_t* mma_done = pempty + 2;
+  uint64_t* pfull = empty + S;      // [NB]
+  uint64_t* pempty = pfull + NB;    // [NB]
+  uint64_t* mma_done = pempty + NB;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
@@ -75,7 +141,7 @@ __global__ void __launch_bounds__(kI4Threads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1 + kI4EpiWarps);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NB; ++b) {
       mbar_init(&pfull[b], 1);
       mbar_init(&pempty[b], kI4EpiWarps);
     }
@@ -91,6 +157,17 @@ __global__ void __launch_bounds__(kI4Threads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  if (warp >= 2) {
+    // every partial buffer starts out holding the conversion offset
+    const uint32_t q = warp & 3u, h = (warp - 2) >> 2;
+    for (int b = 0; b < NB; ++b)
+      for (int c = 0; c < 2; ++c)
+        tmem_st32_const(tmem_base + ((q * 32u) << 16) + kI4BN * b + 64u * h + 32u * c, kI4Magic);
+    tmem_wait_st();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
 
   if (warp == 0) {
     if (elect_one()) {
@@ -100,7 +177,7 @@ __global__ void __launch_bounds__(kI4Threads, 1)
         prefetch_tmap(&tm_xl1);
         prefetch_tmap(&tm_l2t);
       }
-      const uint32_t main_tx = kI4BM * 64 + kI4BN * 64 + kI4BM * 2 + kI4BN * 2;
+      const uint32_t main_tx = kI4BM * 64 + kI4BN * 64 + kI4BM * 2 + kI4BN * 4;
       const uint32_t lr_tx = (kI4BM + kI4BN) * lr_cols * 2;
       int it = 0;
       bool ok = true;
@@ -123,7 +200,7 @@ __global__ void __launch_bounds__(kI4Threads, 1)
             tma_load_2d(st + kI4AOff, &tm_a, &full[s], g * kI4BK, m0);
             tma_load_2d(st + kI4BOff, &tm_b, &full[s], g * kI4BK, n0);
             bulk_load(st + kI4SxOff, p.sx + static_cast<size_t>(g) * p.M_pad + m0, kI4BM * 2, &full[s]);
-            bulk_load(st + kI4SwOff, p.sw + static_cast<size_t>(g) * p.N_pad + n0, kI4BN * 2, &full[s]);
+            bulk_load(st + kI4SwOff, p.sw + static_cast<size_t>(g) * p.N_pad + n0, kI4BN * 4, &full[s]);
           } else {
             const int c = step - p.groups;
             mbar_arrive_expect_tx(&full[s], lr_tx);
@@ -148,8 +225,8 @@ __global__ void __launch_bounds__(kI4Threads, 1)
         for (int step = 0; step < steps_per_tile; ++step, ++it) {
           const int s = it % S;
           const uint32_t ph = (it / S) & 1;
-          const int b = it & 1;
-          const uint32_t pph = (it >> 1) & 1;
+          const int b = it % NB;
+          const uint32_t pph = (it / NB) & 1;
           const bool tail = step >= p.groups;
           if (!mbar_wait(&pempty[b], pph ^ 1, p.budget, abort_flag) ||
               !mbar_wait(&full[s], ph, p.budget, abort_flag)) {
@@ -161,12 +238,13 @@ __global__ void __launch_bounds__(kI4Threads, 1)
           tc_fence_after();
           uint8_t* st = smem + s * kI4StageBytes;
           const uint32_t a0 = smem_u32(st + kI4AOff), b0 = smem_u32(st + kI4BOff);
-          const uint32_t d = tmem_base + 256u * b;
+          const uint32_t d = tmem_base + kI4BN * b;
           if (!tail) {
+            // accumulate onto the buffer's conversion offset
 #pragma unroll
             for (int j = 0; j < 2; ++j)
               mma_i8(d, make_kmajor_desc(a0 + 32 * j, 64), make_kmajor_desc(b0 + 32 * j, 64),
-                     idesc_main, j > 0 ? 1u : 0u);
+                     idesc_main, 1u);
           } else {
             for (int j = 0; j < lr_cols / 16; ++j)
               mma_bf16(d, make_kmajor_desc(a0 + 32 * j, lr_row_bytes),
@@ -183,18 +261,19 @@ __global__ void __launch_bounds__(kI4Threads, 1)
     const uint32_t q = warp & 3u;
     const uint32_t h = (warp - 2) >> 2;
     const uint32_t row = q * 32 + lane;
+    const unsigned long long magic2 = f2_pack(kI4MagicF, kI4MagicF);
     int it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
       const int m_blk = tile % p.m_tiles, n_blk = tile / p.m_tiles;
       const int m = m_blk * kI4BM + static_cast<int>(row);
-      float acc[128];
+      unsigned long long acc[32];   // 64 fp32 accumulators, pairs of adjacent columns
 #pragma unroll
-      for (int j = 0; j < 128; ++j) acc[j] = 0.f;
+      for (int j = 0; j < 32; ++j) acc[j] = 0ull;
       for (int step = 0; step < steps_per_tile; ++step, ++it) {
         const int s = it % S;
-        const int b = it & 1;
-        const uint32_t pph = (it >> 1) & 1;
+        const int b = it % NB;
+        const uint32_t pph = (it / NB) & 1;
         if (!warp_wait(&pfull[b], pph, p.budget, abort_flag)) {
           if (lane == 0) raise_error(kErrWaitGemm);
           *abort_flag = 1;
@@ -202,52 +281,50 @@ __global__ void __launch_bounds__(kI4Threads, 1)
           break;
         }
         tc_fence_after();
-        const uint8_t* st = smem + s * kI4StageBytes;
         const bool main_step = step < p.groups;
+        const uint8_t* st = smem + s * kI4StageBytes;
         const float sx = main_step
             ? __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(st + kI4SxOff)[row]))
             : 1.0f;
-        const uint16_t* swp = reinterpret_cast<const uint16_t*>(st + kI4SwOff) + 128 * h;
-        const uint32_t taddr = tmem_base + 256u * b + ((q * 32u) << 16) + 128u * h;
+        const unsigned long long sx2 = f2_pack(sx, sx);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
+          const uint32_t taddr = tmem_base + ((q * 32u) << 16) + kI4BN * b + 64u * h + 32u * c;
           uint32_t r[32];
-          tmem_ld32(taddr + 32 * c, r);
+          tmem_ld32(taddr, r);
           tmem_wait_ld();
+          tmem_st32_const(taddr, kI4Magic);
+          unsigned long long* a = acc + 16 * c;
           if (main_step) {
+            const float4* swp = reinterpret_cast<const float4*>(st + kI4SwOff) + 16 * h + 8 * c;
 #pragma unroll
-            for (int j = 0; j < 32; j += 8) {
-              const uint4 w = *reinterpret_cast<const uint4*>(swp + 32 * c + j);
-              const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-              for (int t = 0; t < 4; ++t) {
-                const float2 s2 = __half22float2(*reinterpret_cast<const __half2*>(&w4[t]));
-                // exact int32 -> fp32 for |P| < 2^22: add the bits of 1.5 * 2^23, subtract
-                const float p0 = __int_as_float(static_cast<int>(r[j + 2 * t]) + 0x4B400000) - 12582912.0f;
-                const float p1 = __int_as_float(static_cast<int>(r[j + 2 * t + 1]) + 0x4B400000) - 12582912.0f;
-                acc[32 * c + j + 2 * t] = fmaf(sx * s2.x, p0, acc[32 * c + j + 2 * t]);
-                acc[32 * c + j + 2 * t + 1] = fmaf(sx * s2.y, p1, acc[32 * c + j + 2 * t + 1]);
-              }
+            for (int j = 0; j < 8; ++j) {
+              const float4 w = swp[j];
+              a[2 * j] = f2_scale_acc(a[2 * j], u2_pack(r[4 * j], r[4 * j + 1]), magic2,
+                                      f2_mul(sx2, f2_pack(w.x, w.y)));
+              a[2 * j + 1] = f2_scale_acc(a[2 * j + 1], u2_pack(r[4 * j + 2], r[4 * j + 3]), magic2,
+                                          f2_mul(sx2, f2_pack(w.z, w.w)));
             }
           } else {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) acc[32 * c + j] += __uint_as_float(r[j]);
+            for (int j = 0; j < 16; ++j) a[j] = f2_add(a[j], u2_pack(r[2 * j], r[2 * j + 1]));
           }
         }
+        tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(&pempty[b]);
-          mbar_arrive(&empty[s]);
+          mbar_arrive(&pempty[b]);   // the buffer holds the offset again
+          mbar_arrive(&empty[s]);    // done with this stage's scales
         }
       }
       if (!ok) break;
       // bias, bf16, store
-      const int n_base = n_blk * kI4BN + 128 * static_cast<int>(h);
+      const int n_base = n_blk * kI4BN + 64 * static_cast<int>(h);
       if (m < p.M) {
         __nv_bfloat16* yrow = p.Y + static_cast<size_t>(m) * p.N;
 #pragma unroll
-        for (int j = 0; j < 128; j += 8) {
+        for (int j = 0; j < 64; j += 8) {
           const int n = n_base + j;
           if (n < p.N) {
             float bb[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -260,11 +337,18 @@ __global__ void __launch_bounds__(kI4Threads, 1)
                 bb[2 * t + 1] = bf16_hi(w4[t]);
               }
             }
+            float v[8];
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+              const float2 a = f2_unpack(acc[j / 2 + t]);
+              v[2 * t] = a.x + bb[2 * t];
+              v[2 * t + 1] = a.y + bb[2 * t + 1];
+            }
             uint4 o;
-            o.x = pack_bf16x2(acc[j + 0] + bb[0], acc[j + 1] + bb[1]);
-            o.y = pack_bf16x2(acc[j + 2] + bb[2], acc[j + 3] + bb[3]);
-            o.z = pack_bf16x2(acc[j + 4] + bb[4], acc[j + 5] + bb[5]);
-            o.w = pack_bf16x2(acc[j + 6] + bb[6], acc[j + 7] + bb[7]);
+            o.x = pack_bf16x2(v[0], v[1]);
+            o.y = pack_bf16x2(v[2], v[3]);
+            o.z = pack_bf16x2(v[4], v[5]);
+            o.w = pack_bf16x2(v[6], v[7]);
             *reinterpret_cast<uint4*>(yrow + n) = o;
           }
         }

@@ -263,7 +263,8 @@ __global__ void quant_weight_nvfp4_kernel(const float* __restrict__ R, int K, in
 }
 
 __global__ void quant_weight_int4_kernel(const float* __restrict__ R, int K, int N, int N_pad,
-                                         int8_t* __restrict__ codes, uint16_t* __restrict__ sf) {
+                                         int8_t* __restrict__ codes, uint16_t* __restrict__ sf,
+                                         float* __restrict__ sf32) {
   const int n = blockIdx.x * blockDim.x + threadIdx.x;
   const int g = blockIdx.y;
   if (n >= N) return;
@@ -278,6 +279,7 @@ __global__ void quant_weight_int4_kernel(const float* __restrict__ R, int K, int
         static_cast<int8_t>(sd == 0.f ? 0 : int4_code(v, inv));
   }
   sf[static_cast<size_t>(g) * N_pad + n] = sh;
+  sf32[static_cast<size_t>(g) * N_pad + n] = sd;   // exact: every fp16 value is an fp32 value
 }
 
 }  // namespace svdq

@@ -37,6 +37,7 @@ struct svdq_weights {
   float* lambda = nullptr;
   uint8_t* wcodes = nullptr;  // NVFP4: N x K/2 packed; INT4: N x K int8
   uint8_t* wsf = nullptr;     // NVFP4: atoms [N_pad/128][sf_kcols][512]; INT4: fp16 [K/64][N_pad]
+  float* wsf32 = nullptr;     // INT4: the same scales as fp32, read by the GEMM
   __nv_bfloat16* l1t = nullptr;  // r_pad x K
   __nv_bfloat16* l1st = nullptr; // r_pad x K: bf16(diag(1/lambda) L1)^T, read by the activation kernel
   __nv_bfloat16* l2t = nullptr;  // N x r_pad
@@ -207,7 +208,8 @@ int encode_weight_maps(svdq_weights* w) {
     rc = make_map(&w->tm_l1t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w->l1st, w->K, w->r_pad, 64, w->r_pad);
     if (rc) return rc;
     const int lc = lr_chunk_cols(2 * w->r_pad);
-    rc = make_map(&w->tm_l2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w->l2t2, 2 * w->r_pad, w->N, lc, kGemmBN);
+    rc = make_map(&w->tm_l2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w->l2t2, 2 * w->r_pad, w->N, lc,
+                  w->fmt == SVDQ_NVFP4 ? kGemmBN : kI4BN);
     if (rc) return rc;
   } else {
     w->tm_l1t = w->tm_b;
@@ -222,6 +224,7 @@ void free_weights(svdq_weights* w) {
   cudaFree(w->lambda);
   cudaFree(w->wcodes);
   cudaFree(w->wsf);
+  cudaFree(w->wsf32);
   cudaFree(w->l1t);
   cudaFree(w->l1st);
   cudaFree(w->l2t);
@@ -255,6 +258,11 @@ int alloc_weights(svdq_weights* w, cudaStream_t st) {
     return SVDQ_ERR_ALLOC;
   SVDQ_CUDA(cudaMemsetAsync(w->inv_lambda, 0, il_bytes, st));
   SVDQ_CUDA(cudaMemsetAsync(w->wsf, 0, sfb, st));
+  if (w->fmt == SVDQ_INT4) {
+    const size_t sf32 = static_cast<size_t>(w->K / 64) * w->N_pad * sizeof(float);
+    if (cudaMalloc(&w->wsf32, sf32) != cudaSuccess) return SVDQ_ERR_ALLOC;
+    SVDQ_CUDA(cudaMemsetAsync(w->wsf32, 0, sf32, st));
+  }
   if (w->r_pad > 0) {
     if (cudaMalloc(&w->l1t, static_cast<size_t>(w->r_pad) * w->K * 2) != cudaSuccess ||
         cudaMalloc(&w->l1st, static_cast<size_t>(w->r_pad) * w->K * 2) != cudaSuccess ||
@@ -276,7 +284,7 @@ int quantize_residual(svdq_weights* w, const float* R, cudaStream_t st) {
     const dim3 grid((w->N + 127) / 128, w->K / 64);
     quant_weight_int4_kernel<<<grid, blk, 0, st>>>(R, w->K, w->N, w->N_pad,
                                                    reinterpret_cast<int8_t*>(w->wcodes),
-                                                   reinterpret_cast<uint16_t*>(w->wsf));
+                                                   reinterpret_cast<uint16_t*>(w->wsf), w->wsf32);
   }
   SVDQ_CHECK_LAUNCH();
   return SVDQ_OK;
@@ -691,7 +699,7 @@ SVDQ_API int svdq_linear(const svdq_weights* w, const void* ws, int M, void* Y, 
   const uint8_t* base = static_cast<const uint8_t*>(ws);
   CUtensorMap tm_a, tm_xl1;
   const int m_tiles = L.M_pad / 128;
-  const int n_tiles = (w->N + 255) / 256;
+  const int n_tiles = w->fmt == SVDQ_NVFP4 ? (w->N + kGemmBN - 1) / kGemmBN : (w->N + kI4BN - 1) / kI4BN;
   const int tiles = m_tiles * n_tiles;
   const int grid = std::min(tiles, g_dev[dev].sms);
   if (w->fmt == SVDQ_NVFP4)
@@ -734,7 +742,7 @@ SVDQ_API int svdq_linear(const svdq_weights* w, const void* ws, int M, void* Y, 
     p.num_tiles = tiles;
     p.r_tail = 2 * w->r_pad;
     p.sx = reinterpret_cast<const uint16_t*>(base + L.sf_off);
-    p.sw = reinterpret_cast<const uint16_t*>(w->wsf);
+    p.sw = w->wsf32;
     p.M_pad = L.M_pad;
     p.N_pad = w->N_pad;
     p.bias = w->bias;
