@@ -128,6 +128,69 @@ def layer_inputs(args):
 
 
 # ----------------------------------------------------------------------------- ours
+def time_layer(S, w, X, ws, Y, M, flush, stream, steps, warmup, world, sampler=None):
+    """Per-step seconds of the activation kernel and of the GEMM (CUDA events on
+    the launching stream), with the 126 MB L2 flushed before every step."""
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        S.svdq_quantize_act(w, X, ws)
+        if ev:
+            ev[1].record(stream)
+        S.svdq_linear(w, ws, M, Y)
+        if ev:
+            ev[2].record(stream)
+
+    for _ in range(warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if S.svdq_get_error():
+        raise RuntimeError("device wait timed out during warm-up")
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+    for i in range(steps):
+        flush.zero_()          # L2 flush between steps, outside the timed events
+        step(events[i])
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler else None
+    if world > 1:
+        torch.distributed.barrier()
+    t_q = np.array([e[0].elapsed_time(e[1]) for e in events]) * 1e-3   # s
+    t_g = np.array([e[1].elapsed_time(e[2]) for e in events]) * 1e-3
+    return t_q, t_g, clocks
+
+
+def tensor_ceiling(S, fmt, stream):
+    """The tensor cores' own ceiling for the GEMM's instruction (no global
+    traffic): a ~5 ms burst and a ~1 s sustained run, in TFLOP/s."""
+    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    flop_step = sms * 4 * 2 * 128 * 256 * (64 if fmt == "nvfp4" else 32)
+
+    def run(steps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        S.svdq_tensor_peak(fmt, steps, stream)
+        b.record(stream)
+        torch.cuda.synchronize()
+        if S.svdq_get_error():
+            raise RuntimeError("device wait timed out in the tensor ceiling kernel")
+        return a.elapsed_time(b) * 1e-3
+
+    t = run(2000)
+    steps_burst = max(2000, int(2000 * 0.005 / t))
+    burst = max(flop_step * steps_burst / run(steps_burst) for _ in range(3)) / 1e12
+    steps_long = max(2000, int(2000 * 1.0 / t))
+    sustained = flop_step * steps_long / run(steps_long) / 1e12
+    return {"burst": round(burst, 1), "sustained": round(sustained, 1), "unit": "TFLOP/s",
+            "what": "tcgen05 " + ("kind::mxf4nvf4 128x256x64" if fmt == "nvfp4" else "kind::i8 128x256x32")
+                    + " back to back from shared memory on every SM, no global loads"}
+
+
 def run_ours(args):
     import w4a4_gemm_b200 as S
 
@@ -149,45 +212,14 @@ def run_ours(args):
                                bias=bias.to(dev) if bias is not None else None,
                                lora_A=A.to(dev) if A is not None else None,
                                lora_B=B.to(dev) if B is not None else None)
-    del W
     ws = S.alloc_workspace(w, M, dev)
     Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
     launches_per_step = 2 + (1 if (spec.fmt == "nvfp4" and K % 256) else 0)
 
-    def step(ev=None):
-        if ev:
-            ev[0].record(stream)
-        S.svdq_quantize_act(w, X, ws)
-        if ev:
-            ev[1].record(stream)
-        S.svdq_linear(w, ws, M, Y)
-        if ev:
-            ev[2].record(stream)
-
-    for _ in range(args.warmup):
-        flush.zero_()
-        step()
-    torch.cuda.synchronize()
-    if S.svdq_get_error():
-        raise RuntimeError("device wait timed out during warm-up")
-
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     sampler = ClockSampler(local)
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    sampler.start()
-    for i in range(args.steps):
-        flush.zero_()          # L2 flush between steps, outside the timed events
-        step(events[i])
-    torch.cuda.synchronize()
-    clocks = sampler.stop()
-    if world > 1:
-        torch.distributed.barrier()
-    t_q = np.array([e[0].elapsed_time(e[1]) for e in events]) * 1e-3   # s
-    t_g = np.array([e[1].elapsed_time(e[2]) for e in events]) * 1e-3
+    t_q, t_g, clocks = time_layer(S, w, X, ws, Y, M, flush, stream, args.steps, args.warmup, world, sampler)
     t_layer = t_q + t_g
     total = float(t_layer.sum())
     if world > 1:
@@ -256,6 +288,24 @@ def run_ours(args):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
+    if world == 1 and not args.no_extras:
+        # the same layer without the low-rank branch (plain W4A4, same smoothing)
+        w0 = S.svdq_prepare_weights(W, 0, spec.fmt, x_absmax=xabs,
+                                    bias=bias.to(dev) if bias is not None else None)
+        q0, g0, _ = time_layer(S, w0, X, ws, Y, M, flush, stream, args.steps, args.warmup, world)
+        w0.close()
+        l0 = float(q0.mean() + g0.mean())
+        line["lowrank_overhead"] = {
+            "us_layer_r0": round(l0 * 1e6, 2), "us_quant_r0": round(float(q0.mean()) * 1e6, 2),
+            "us_gemm_r0": round(float(g0.mean()) * 1e6, 2),
+            "layer": round(total / args.steps / l0 - 1.0, 4),
+            "gemm": round(tg_mean / float(g0.mean()) - 1.0, 4), "target": 0.15,
+            "what": f"us(rank {r}) / us(rank 0) - 1, same format, shapes, smoothing and bias"}
+        ceil = tensor_ceiling(S, spec.fmt, stream)
+        ceil["gemm_frac_of_burst"] = round(achieved / ceil["burst"], 4)
+        ceil["gemm_frac_of_sustained"] = round(achieved / ceil["sustained"], 4)
+        line["tensor_ceiling"] = ceil
+    del W
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(spec, M, args.cpu_rows)
     if rank == 0:
@@ -337,6 +387,8 @@ def main():
     ap.add_argument("--M", type=int, default=None)
     ap.add_argument("--cpu-rows", type=int, default=64)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the rank-0 comparison and the tensor-ceiling measurement")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

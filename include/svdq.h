@@ -182,6 +182,15 @@ SVDQ_API int svdq_set_wait_budget(long long cycles);
 
 SVDQ_API const char* svdq_status_string(int status);
 
+/* Measurement helper, not a step of the layer: every SM of the current device
+ * issues `steps` 256-wide K steps of the GEMM's own tensor-core instruction
+ * (NVFP4: 4 x tcgen05.mma kind::mxf4nvf4 M=128 N=256 K=64; INT4: 4 x kind::i8
+ * M=128 N=256 K=32) back to back from shared memory, with no global-memory
+ * traffic.  Timing it with events on `stream` gives the tensor-core ceiling:
+ *   FLOP = SMs * steps * 4 * 2 * 128 * 256 * (64 for NVFP4, 32 for INT4).
+ * Asynchronous; returns SVDQ_ERR_INVALID_ARG for a bad format or steps < 1. */
+SVDQ_API int svdq_tensor_peak(int fmt, long long steps, void* stream);
+
 SVDQ_API void svdq_weights_destroy(svdq_weights* w);
 
 #ifdef __cplusplus

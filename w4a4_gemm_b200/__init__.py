@@ -29,7 +29,7 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "device all
 EXPORTED = ("svdq_calib_absmax", "svdq_prepare_weights", "svdq_load_weights", "svdq_append_lora",
             "svdq_weights_info", "svdq_act_workspace_bytes", "svdq_quantize_act", "svdq_linear",
             "svdq_forward", "svdq_forward_noalloc", "svdq_export_act", "svdq_export_weights", "svdq_get_error",
-            "svdq_set_wait_budget", "svdq_status_string", "svdq_weights_destroy")
+            "svdq_set_wait_budget", "svdq_status_string", "svdq_tensor_peak", "svdq_weights_destroy")
 
 
 class SvdqError(RuntimeError):
@@ -80,6 +80,7 @@ def lib() -> ctypes.CDLL:
     L.svdq_set_wait_budget.argtypes = [LL]
     L.svdq_status_string.argtypes = [I]
     L.svdq_status_string.restype = ctypes.c_char_p
+    L.svdq_tensor_peak.argtypes = [I, LL, P]
     L.svdq_weights_destroy.argtypes = [P]
     L.svdq_weights_destroy.restype = None
     _lib = L
@@ -300,6 +301,12 @@ def svdq_export_weights(w: Weights) -> dict:
 
 def svdq_get_error() -> int:
     return int(lib().svdq_get_error())
+
+
+def svdq_tensor_peak(fmt: str, steps: int, stream=None):
+    """Launch the tensor-core ceiling kernel (see include/svdq.h); time it with
+    CUDA events.  FLOP = SMs * steps * 4 * 2 * 128 * 256 * (64 NVFP4 | 32 INT4)."""
+    _check(lib().svdq_tensor_peak(_FMT[fmt], int(steps), _stream(stream)), "svdq_tensor_peak")
 
 
 def svdq_set_wait_budget(cycles: int):

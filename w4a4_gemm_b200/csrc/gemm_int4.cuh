@@ -48,6 +48,12 @@ constexpr uint32_t kI4SmemBytes = kI4StageBytes * kI4Stages + 256 + 1024;
 constexpr uint32_t kI4Magic = 0x4B400000u;                 // bits of 1.5 * 2^23
 constexpr float kI4MagicF = 12582912.0f;
 
+// Low-rank tail chunks of at most 64 bf16 columns (128-byte rows).
+__host__ __device__ inline int i4_lr_chunk_cols(int k_tail) { return k_tail < 64 ? k_tail : 64; }
+__host__ __device__ inline int i4_lr_num_chunks(int k_tail) {
+  return k_tail == 0 ? 0 : (k_tail + 63) / 64;
+}
+
 struct GemmI4Params {
   int M, N, K;
   int groups;          // K / 64
@@ -132,8 +138,8 @@ __global__ void __launch_bounds__(kI4Threads, 1)
 
   const uint32_t warp = warp_id();
   const uint32_t lane = lane_id();
-  const int n_lr = lr_num_chunks(p.r_tail);
-  const int lr_cols = lr_chunk_cols(p.r_tail);
+  const int n_lr = i4_lr_num_chunks(p.r_tail);
+  const int lr_cols = i4_lr_chunk_cols(p.r_tail);
   const int steps_per_tile = p.groups + n_lr;
 
   if (threadIdx.x == 0) {

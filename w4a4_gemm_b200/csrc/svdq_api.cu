@@ -20,6 +20,7 @@
 #include "../../include/svdq.h"
 #include "gemm_int4.cuh"
 #include "gemm_nvfp4.cuh"
+#include "peak.cuh"
 #include "prepare.cuh"
 #include "quant_act.cuh"
 #include "svdq_formats.cuh"
@@ -155,6 +156,10 @@ int device_setup(int dev) {
                                  kGemmSmemBytes));
   SVDQ_CUDA(cudaFuncSetAttribute(gemm_int4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kI4SmemBytes));
+  SVDQ_CUDA(cudaFuncSetAttribute(tensor_peak_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kPeakSmemBytes));
+  SVDQ_CUDA(cudaFuncSetAttribute(tensor_peak_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kPeakSmemBytes));
   d.attrs_set = true;
   return SVDQ_OK;
 }
@@ -207,7 +212,7 @@ int encode_weight_maps(svdq_weights* w) {
   if (w->r_pad > 0) {
     rc = make_map(&w->tm_l1t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w->l1st, w->K, w->r_pad, 64, w->r_pad);
     if (rc) return rc;
-    const int lc = lr_chunk_cols(2 * w->r_pad);
+    const int lc = w->fmt == SVDQ_NVFP4 ? lr_chunk_cols(2 * w->r_pad) : i4_lr_chunk_cols(2 * w->r_pad);
     rc = make_map(&w->tm_l2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w->l2t2, 2 * w->r_pad, w->N, lc,
                   w->fmt == SVDQ_NVFP4 ? kGemmBN : kI4BN);
     if (rc) return rc;
@@ -444,6 +449,20 @@ SVDQ_API const char* svdq_status_string(int s) {
     case SVDQ_ERR_LIBRARY: return "cuSOLVER/cuBLAS error";
     default: return "unknown status";
   }
+}
+
+SVDQ_API int svdq_tensor_peak(int fmt, long long steps, void* stream) {
+  if ((fmt != SVDQ_NVFP4 && fmt != SVDQ_INT4) || steps < 1) return SVDQ_ERR_INVALID_ARG;
+  int dev;
+  int rc = current_device(&dev);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (fmt == SVDQ_NVFP4)
+    tensor_peak_kernel<0><<<g_dev[dev].sms, kPeakThreads, kPeakSmemBytes, st>>>(steps, wait_budget());
+  else
+    tensor_peak_kernel<1><<<g_dev[dev].sms, kPeakThreads, kPeakSmemBytes, st>>>(steps, wait_budget());
+  SVDQ_CHECK_LAUNCH();
+  return SVDQ_OK;
 }
 
 SVDQ_API int svdq_set_wait_budget(long long cycles) {
@@ -709,7 +728,8 @@ SVDQ_API int svdq_linear(const svdq_weights* w, const void* ws, int M, void* Y, 
   if (rc) return rc;
   if (w->r_pad > 0) {
     if ((rc = make_map(&tm_xl1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base + L.xl1_off, 2 * w->r_pad, M,
-                       lr_chunk_cols(2 * w->r_pad), 128)))
+                       w->fmt == SVDQ_NVFP4 ? lr_chunk_cols(2 * w->r_pad) : i4_lr_chunk_cols(2 * w->r_pad),
+                       128)))
       return rc;
   } else {
     tm_xl1 = tm_a;
