@@ -19,7 +19,11 @@
 //               columns [128 h, 128 h + 128), h = (w - 2) / 4.  Per tile they
 //               copy their accumulator columns to registers and hand the TMEM
 //               back at once, so the next tile's MMAs overlap the bias, bf16
-//               conversion and stores.
+//               conversion and stores.  Each warp writes Y through its own 1 KB
+//               shared-memory buffer (32 rows x 16 columns) and TMA stores:
+//               whole 32-byte row segments instead of one scattered 16-byte
+//               store per row and instruction, which kept the shared-memory
+//               pipe busy while the tensor core was reading its operands.
 #pragma once
 
 #include "svdq_formats.cuh"
@@ -48,7 +52,10 @@ __host__ __device__ inline int lr_num_chunks(int k_tail) {
   return k_tail == 0 ? 0 : (k_tail + 63) / 64;
 }
 constexpr int kGemmStages = 4;
-constexpr uint32_t kGemmSmemBytes = kGemmStageBytes * kGemmStages + 256 + 1024;
+constexpr uint32_t kGemmEpiBufBytes = 32 * 32;                              // 32 rows x 16 bf16
+constexpr uint32_t kGemmEpiOff = kGemmStageBytes * kGemmStages;
+constexpr uint32_t kGemmBarOff = kGemmEpiOff + kGemmEpiWarps * kGemmEpiBufBytes;
+constexpr uint32_t kGemmSmemBytes = kGemmBarOff + 256 + 1024;
 
 struct GemmParams {
   int M, N, K;
@@ -59,7 +66,6 @@ struct GemmParams {
   const uint8_t* sfb;  // weight scale atoms     [N_pad/128][sf_kcols][512]
   int sf_kcols;        // K_pad / 64, K_pad = K rounded up to 256
   const __nv_bfloat16* bias;  // N or nullptr
-  __nv_bfloat16* Y;    // M x N row-major
   long long budget;
 };
 
@@ -74,31 +80,47 @@ __device__ __forceinline__ uint64_t sf_desc(uint32_t saddr) {
   return make_sdesc(saddr, 0, 128, kSwizzleNone);
 }
 
-// Epilogue: 32 fp32 accumulators of one row (columns n0 .. n0 + 31) + bias ->
-// bf16 -> global.  Columns at or past N are skipped (N % 16 == 0).
-__device__ __forceinline__ void store_row_chunk(const uint32_t (&r)[32], __nv_bfloat16* yrow, int n0,
-                                                int N, const __nv_bfloat16* __restrict__ bias) {
+// Epilogue: 16 fp32 accumulators of this lane's row (columns n0 .. n0 + 15)
+// + bias -> bf16 -> the warp's buffer (32 rows of 32 bytes in the TMA 32-byte
+// swizzle: the 16-byte half c of row r sits at half c ^ ((r >> 2) & 1)) ->
+// one TMA store of the 32 x 16 box at (n0, row0).  The store clips rows past M
+// and columns past N; the bias is read only below N (N % 16 == 0).
+__device__ __forceinline__ void epi_store_16(const uint32_t* r, uint8_t* buf, const CUtensorMap* tm_y,
+                                             int n0, int row0, int N,
+                                             const __nv_bfloat16* __restrict__ bias, uint32_t lane) {
+  float bb[16];
 #pragma unroll
-  for (int j = 0; j < 32; j += 8) {
-    const int n = n0 + j;
-    if (n < N) {
-      float bb[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      if (bias != nullptr) {
-        const uint4 w = __ldg(reinterpret_cast<const uint4*>(bias + n));
-        const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
+  for (int j = 0; j < 16; ++j) bb[j] = 0.f;
+  if (bias != nullptr && n0 < N) {
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          bb[2 * t] = bf16_lo(w4[t]);
-          bb[2 * t + 1] = bf16_hi(w4[t]);
-        }
+    for (int h = 0; h < 2; ++h) {
+      const uint4 b = __ldg(reinterpret_cast<const uint4*>(bias + n0 + 8 * h));
+      const uint32_t b4[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        bb[8 * h + 2 * t] = bf16_lo(b4[t]);
+        bb[8 * h + 2 * t + 1] = bf16_hi(b4[t]);
       }
-      uint4 o;
-      o.x = pack_bf16x2(__uint_as_float(r[j + 0]) + bb[0], __uint_as_float(r[j + 1]) + bb[1]);
-      o.y = pack_bf16x2(__uint_as_float(r[j + 2]) + bb[2], __uint_as_float(r[j + 3]) + bb[3]);
-      o.z = pack_bf16x2(__uint_as_float(r[j + 4]) + bb[4], __uint_as_float(r[j + 5]) + bb[5]);
-      o.w = pack_bf16x2(__uint_as_float(r[j + 6]) + bb[6], __uint_as_float(r[j + 7]) + bb[7]);
-      *reinterpret_cast<uint4*>(yrow + n) = o;
     }
+  }
+  uint32_t w[8];
+#pragma unroll
+  for (int t = 0; t < 8; ++t)
+    w[t] = pack_bf16x2(__uint_as_float(r[2 * t]) + bb[2 * t], __uint_as_float(r[2 * t + 1]) + bb[2 * t + 1]);
+  if (lane == 0) bulk_wait_group_read<0>();   // the previous store has read the buffer
+  __syncwarp();
+  const uint32_t row_addr = smem_u32(buf) + lane * 32u;
+  const uint32_t sw = (lane >> 2) & 1u;
+#pragma unroll
+  for (uint32_t c = 0; c < 2; ++c)
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row_addr + ((c ^ sw) << 4)),
+                 "r"(w[4 * c]), "r"(w[4 * c + 1]), "r"(w[4 * c + 2]), "r"(w[4 * c + 3])
+                 : "memory");
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(tm_y, buf, n0, row0);
+    bulk_commit_group();
   }
 }
 
@@ -106,12 +128,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a,
                       const __grid_constant__ CUtensorMap tm_b,
                       const __grid_constant__ CUtensorMap tm_xl1,
-                      const __grid_constant__ CUtensorMap tm_l2t, const GemmParams p) {
+                      const __grid_constant__ CUtensorMap tm_l2t,
+                      const __grid_constant__ CUtensorMap tm_y, const GemmParams p) {
   constexpr int STAGES = kGemmStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kGemmStageBytes * STAGES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kGemmBarOff);
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;
   uint64_t* acc_empty = acc_full + 1;
@@ -261,39 +284,37 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ---------------------------------------------------------------- epilogue
     const uint32_t q = warp & 3u;
     const uint32_t h = (warp - 2) >> 2;
-    const uint32_t row = q * 32 + lane;
+    uint8_t* ebuf = smem + kGemmEpiOff + (warp - 2) * kGemmEpiBufBytes;
     int t_local = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++t_local) {
       int m_blk, n_blk;
       gemm_tile_coords(p.m_tiles, tile, m_blk, n_blk);
-      const int m = m_blk * kGemmBM + static_cast<int>(row);
-      // accumulator columns [128 h, 128 h + 128) of this row -> registers
+      // accumulator columns [128 h, 128 h + 128) of this warp's 32 rows -> registers
       if (!warp_wait(acc_full, t_local & 1, p.budget, abort_flag)) {
         if (lane == 0) raise_error(kErrWaitGemm);
         *abort_flag = 1;
         break;
       }
       tc_fence_after();
-      uint32_t v0[32], v1[32], v2[32], v3[32];
+      uint32_t v[4][32];
       const uint32_t taddr = tmem_base + ((q * 32u) << 16) + 128u * h;
-      tmem_ld32(taddr, v0);
-      tmem_ld32(taddr + 32, v1);
-      tmem_ld32(taddr + 64, v2);
-      tmem_ld32(taddr + 96, v3);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(taddr + 32 * c, v[c]);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_empty);
-      // bias, bf16, store
+      // bias, bf16, staged TMA stores
+      const int row0 = m_blk * kGemmBM + static_cast<int>(q) * 32;
       const int nb = n_blk * kGemmBN + 128 * static_cast<int>(h);
-      if (m < p.M) {
-        __nv_bfloat16* yrow = p.Y + static_cast<size_t>(m) * p.N;
-        store_row_chunk(v0, yrow, nb, p.N, p.bias);
-        store_row_chunk(v1, yrow, nb + 32, p.N, p.bias);
-        store_row_chunk(v2, yrow, nb + 64, p.N, p.bias);
-        store_row_chunk(v3, yrow, nb + 96, p.N, p.bias);
+      if (row0 < p.M) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          if (nb + 16 * c < p.N)
+            epi_store_16(&v[c / 2][16 * (c % 2)], ebuf, &tm_y, nb + 16 * c, row0, p.N, p.bias, lane);
       }
     }
+    if (lane == 0) bulk_wait_group_all();
   }
 
   __syncwarp();

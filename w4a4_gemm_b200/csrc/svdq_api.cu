@@ -735,6 +735,8 @@ SVDQ_API int svdq_linear(const svdq_weights* w, const void* ws, int M, void* Y, 
     tm_xl1 = tm_a;
   }
   if (w->fmt == SVDQ_NVFP4) {
+    CUtensorMap tm_y;
+    if ((rc = make_map(&tm_y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Y, w->N, M, 16, 32))) return rc;
     GemmParams p;
     p.M = M;
     p.N = w->N;
@@ -748,9 +750,9 @@ SVDQ_API int svdq_linear(const svdq_weights* w, const void* ws, int M, void* Y, 
     p.sfb = w->wsf;
     p.sf_kcols = w->sf_kcols;
     p.bias = w->bias;
-    p.Y = static_cast<__nv_bfloat16*>(Y);
     p.budget = wait_budget();
-    gemm_nvfp4_kernel<<<grid, kGemmThreads, kGemmSmemBytes, st>>>(tm_a, w->tm_b, tm_xl1, w->tm_l2t, p);
+    gemm_nvfp4_kernel<<<grid, kGemmThreads, kGemmSmemBytes, st>>>(tm_a, w->tm_b, tm_xl1, w->tm_l2t,
+                                                                  tm_y, p);
   } else {
     GemmI4Params p;
     p.M = M;
