@@ -18,12 +18,13 @@
 // 256 / r_pad) that gives about one CTA per SM.
 //   warp 0      : TMA producer (S X boxes BM x 64, S L1s^T boxes r_pad x 64, 1/lambda)
 //   warp 1      : TMEM owner; one lane issues the kind::f16 MMAs
-//   warps 2..17 : quantizers; warp w serves A-tile rows 32 (w % 4) .. + 31 and
-//                 K quarter (w - 2) / 4 (one NVFP4 group of 16) of each 64-wide
-//                 sub-tile.  They smooth X, quantize it, release the stage and
-//                 then store codes and scales.  At the end warps 2..5 read the
-//                 diagonal blocks and the CTA sums them into XL1, kept at fp32
-//                 precision as a bf16 pair hi + lo for the GEMM's tail MMA.
+//   warps 2..13 : quantizers in three groups of four; group k takes every
+//                 third stage, and its warp w serves A-tile rows 32 (w % 4) .. + 31,
+//                 one lane per row over the whole 64-wide sub-tile.  They smooth
+//                 X, quantize it, release the stage and store codes and scales.
+//                 At the end warps 2..5 read the diagonal blocks and the CTA
+//                 sums them into XL1, kept at fp32 precision as a bf16 pair
+//                 hi + lo for the GEMM's tail MMA.
 #pragma once
 
 #include "svdq_formats.cuh"
@@ -34,8 +35,9 @@ namespace svdq {
 constexpr int kQuantTileRows = 128;   // rows of the MMA A operand
 constexpr int kQuantBK = 64;          // K width of one sub-tile
 constexpr int kQuantMaxStages = 8;
-constexpr int kQuantThreads = 576;
-constexpr int kQuantWarps = 16;       // quantizer warps
+constexpr int kQuantGroups = 3;       // quantizer groups working on consecutive stages
+constexpr int kQuantWarps = 4 * kQuantGroups;   // quantizer warps (one per lane quarter per group)
+constexpr int kQuantThreads = 32 * (2 + kQuantWarps);
 constexpr uint32_t kQuantStageBudget = 200u * 1024u;   // shared memory for the pipeline
 
 struct QuantParams {
@@ -108,7 +110,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 1);
       // released by the quantizer warps and, with a low-rank branch, the MMAs
-      mbar_init(&empty[s], kQuantWarps + (has_lr ? 1 : 0));
+      mbar_init(&empty[s], 4 + (has_lr ? 1 : 0));
     }
     mbar_init(acc_full, 1);
     *abort_flag = 0;
@@ -181,20 +183,19 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ quantizers
-    // NVFP4: warp quarter g quantizes K columns [16g, 16g + 16) of each
-    // sub-tile row (one group).  INT4: a group spans the whole 64-wide
-    // sub-tile, so the g = 0 warps quantize it alone and the others only
-    // release the stage.
+    // Group k = (warp - 2) / 4 takes the stages k, k + G, k + 2G, ... (G groups);
+    // its warp of lane quarter q quantizes rows 32 q .. 32 q + 31 of the
+    // stacked tile, one lane per row over the whole 64-wide sub-tile: four
+    // independent NVFP4 groups of 16 (or one INT4 group of 64) per lane, so
+    // each lane has four chains of work in flight and writes its row's codes
+    // (32 or 64 contiguous bytes) and scales (one 4-byte word or one fp16).
     const uint32_t q = warp & 3u;
-    const uint32_t g = (warp - 2) >> 2;
+    const int grp = static_cast<int>(warp - 2) >> 2;
     const uint32_t R = q * 32 + lane;          // row of the stacked A tile
     const int j = static_cast<int>(R) / BM;    // K sub-tile
     const int m = m0 + static_cast<int>(R) % BM;
     const bool row_ok = m < p.M;
-    constexpr int kChunks = FMT == 0 ? 2 : 8;  // 16-byte chunks (8 bf16) per thread
-    const bool active = FMT == 0 || g == 0;
-    const uint32_t c0 = FMT == 0 ? 2 * g : 0;
-    for (int i = 0; i < nkt; ++i) {
+    for (int i = grp; i < nkt; i += kQuantGroups) {
       const int s = i % NS;
       const uint32_t ph = (i / NS) & 1;
       if (!warp_wait(&full[s], ph, p.budget, abort_flag)) {
@@ -204,72 +205,72 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
       }
       const int kcol = i * S + j;              // 64-wide column group of X
       const bool col_ok = kcol * kQuantBK < p.K;
-      uint32_t out[FMT == 0 ? 2 : 16];         // codes to store once the stage is released
-      uint32_t sfv = 0;
-      if (active) {
-        const uint8_t* st = smem + s * L.stage_bytes;
-        const float4* il = reinterpret_cast<const float4*>(st + L.il_off + (j * kQuantBK + 8 * c0) * 4);
-        const uint8_t* xrow = st + L.x_off + R * 128;
-        float v[8 * kChunks];
+      const uint8_t* st = smem + s * L.stage_bytes;
+      const float4* il = reinterpret_cast<const float4*>(st + L.il_off + j * kQuantBK * 4);
+      const uint8_t* xrow = st + L.x_off + R * 128;
+      float v[64];
 #pragma unroll
-        for (int c = 0; c < kChunks; ++c) {
-          const uint32_t chunk = ((c0 + c) ^ (R & 7u)) << 4;   // 128-byte swizzle
-          const uint4 raw = *reinterpret_cast<const uint4*>(xrow + chunk);
-          const float4 l0 = il[2 * c], l1 = il[2 * c + 1];
-          float2 t;
-          t = fmul2_rn(make_float2(bf16_lo(raw.x), bf16_hi(raw.x)), make_float2(l0.x, l0.y));
-          v[8 * c + 0] = t.x; v[8 * c + 1] = t.y;
-          t = fmul2_rn(make_float2(bf16_lo(raw.y), bf16_hi(raw.y)), make_float2(l0.z, l0.w));
-          v[8 * c + 2] = t.x; v[8 * c + 3] = t.y;
-          t = fmul2_rn(make_float2(bf16_lo(raw.z), bf16_hi(raw.z)), make_float2(l1.x, l1.y));
-          v[8 * c + 4] = t.x; v[8 * c + 5] = t.y;
-          t = fmul2_rn(make_float2(bf16_lo(raw.w), bf16_hi(raw.w)), make_float2(l1.z, l1.w));
-          v[8 * c + 6] = t.x; v[8 * c + 7] = t.y;
-        }
-        if constexpr (FMT == 0) {
-          sfv = quant16_nvfp4(v, out, rcp_tab);
-        } else {
-          float amax = 0.0f;
-#pragma unroll
-          for (int e = 0; e < 64; e += 16) amax = fmaxf(amax, absmax16(v + e));
-          const uint16_t sh = int4_scale_bits(amax);
-          const float sd = __half2float(__ushort_as_half(sh));
-          sfv = sh;
-          if (sd == 0.0f) {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) out[e] = 0u;
-          } else {
-            const float inv = __frcp_rn(sd);
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              uint32_t w = 0;
-#pragma unroll
-              for (int b = 0; b < 4; ++b)
-                w |= (static_cast<uint32_t>(int4_code(v[4 * e + b], inv)) & 0xFFu) << (8 * b);
-              out[e] = w;
-            }
-          }
-        }
+      for (int c = 0; c < 8; ++c) {
+        const uint32_t chunk = (static_cast<uint32_t>(c) ^ (R & 7u)) << 4;   // 128-byte swizzle
+        const uint4 raw = *reinterpret_cast<const uint4*>(xrow + chunk);
+        const float4 l0 = il[2 * c], l1 = il[2 * c + 1];
+        float2 t;
+        t = fmul2_rn(make_float2(bf16_lo(raw.x), bf16_hi(raw.x)), make_float2(l0.x, l0.y));
+        v[8 * c + 0] = t.x; v[8 * c + 1] = t.y;
+        t = fmul2_rn(make_float2(bf16_lo(raw.y), bf16_hi(raw.y)), make_float2(l0.z, l0.w));
+        v[8 * c + 2] = t.x; v[8 * c + 3] = t.y;
+        t = fmul2_rn(make_float2(bf16_lo(raw.z), bf16_hi(raw.z)), make_float2(l1.x, l1.y));
+        v[8 * c + 4] = t.x; v[8 * c + 5] = t.y;
+        t = fmul2_rn(make_float2(bf16_lo(raw.w), bf16_hi(raw.w)), make_float2(l1.z, l1.w));
+        v[8 * c + 6] = t.x; v[8 * c + 7] = t.y;
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
-      if (active && col_ok) {
-        if constexpr (FMT == 0) {
+      if constexpr (FMT == 0) {
+        uint32_t out[8];
+        uint32_t sfw = 0;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) sfw |= quant16_nvfp4(v + 16 * g, out + 2 * g, rcp_tab) << (8 * g);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+        if (col_ok) {
           if (row_ok) {
-            uint8_t* dst = p.codes + static_cast<size_t>(m) * (p.K / 2) + kcol * (kQuantBK / 2) + 8 * g;
-            *reinterpret_cast<uint2*>(dst) = make_uint2(out[0], out[1]);
+            uint4* dst = reinterpret_cast<uint4*>(p.codes + static_cast<size_t>(m) * (p.K / 2) +
+                                                  kcol * (kQuantBK / 2));
+            dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
+            dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
           }
           // scale atom: 128 rows x 4 scales, byte (m % 32) * 16 + (m % 128 / 32) * 4 + k4
           uint8_t* atom = p.sf + (static_cast<size_t>(m / 128) * p.sf_kcols + kcol) * 512;
-          atom[(m & 31) * 16 + ((m & 127) >> 5) * 4 + g] = static_cast<uint8_t>(row_ok ? sfv : 0u);
-        } else {
+          *reinterpret_cast<uint32_t*>(atom + (m & 31) * 16 + ((m & 127) >> 5) * 4) = row_ok ? sfw : 0u;
+        }
+      } else {
+        float amax = 0.0f;
+#pragma unroll
+        for (int e = 0; e < 64; e += 16) amax = fmaxf(amax, absmax16(v + e));
+        const uint16_t sh = int4_scale_bits(amax);
+        const float sd = __half2float(__ushort_as_half(sh));
+        const float inv = sd == 0.0f ? 0.0f : __frcp_rn(sd);
+        uint32_t out[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          uint32_t w = 0;
+          if (sd != 0.0f) {
+#pragma unroll
+            for (int b = 0; b < 4; ++b)
+              w |= (static_cast<uint32_t>(int4_code(v[4 * e + b], inv)) & 0xFFu) << (8 * b);
+          }
+          out[e] = w;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+        if (col_ok) {
           if (row_ok) {
             uint4* dst = reinterpret_cast<uint4*>(p.codes + static_cast<size_t>(m) * p.K + kcol * kQuantBK);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) dst[e] = make_uint4(out[4 * e], out[4 * e + 1], out[4 * e + 2], out[4 * e + 3]);
+            for (int e = 0; e < 4; ++e)
+              dst[e] = make_uint4(out[4 * e], out[4 * e + 1], out[4 * e + 2], out[4 * e + 3]);
           }
           reinterpret_cast<uint16_t*>(p.sf)[static_cast<size_t>(kcol) * p.M_pad + m] =
-              row_ok ? static_cast<uint16_t>(sfv) : static_cast<uint16_t>(0);
+              row_ok ? sh : static_cast<uint16_t>(0);
         }
       }
     }
@@ -311,7 +312,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
   tc_fence_before();
   __syncthreads();
   if (has_lr) {
-    // BM rows x r_pad columns, 8 columns per thread over all 320 threads
+    // BM rows x r_pad columns, 8 columns per thread over all threads
     const int units = BM * (p.r_pad / 8);
     for (int u = threadIdx.x; u < units; u += kQuantThreads) {
       const int i = u / (p.r_pad / 8);
