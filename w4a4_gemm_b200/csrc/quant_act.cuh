@@ -38,7 +38,10 @@ constexpr int kQuantMaxStages = 8;
 constexpr int kQuantGroups = 3;       // quantizer groups working on consecutive stages
 constexpr int kQuantWarps = 4 * kQuantGroups;   // quantizer warps (one per lane quarter per group)
 constexpr int kQuantThreads = 32 * (2 + kQuantWarps);
-constexpr uint32_t kQuantStageBudget = 200u * 1024u;   // shared memory for the pipeline
+constexpr uint32_t kQuantSmemBudget = 220u * 1024u;    // shared memory for stages + code staging
+
+// Bytes of codes one row of a 64-wide sub-tile produces: 64 E2M1 (NVFP4) or 64 int8 (INT4).
+__host__ __device__ constexpr uint32_t quant_code_row_bytes(int fmt) { return fmt == 0 ? 32u : 64u; }
 
 struct QuantParams {
   int M, K;
@@ -47,7 +50,6 @@ struct QuantParams {
   int M_pad;        // M rounded up to 128 (scale atoms)
   int sf_kcols;     // NVFP4: K_pad / 64 scale atoms per 128-row block
   const float* inv_lambda;  // K rounded up to 512 (zero padded)
-  uint8_t* codes;   // NVFP4: M x K/2 packed E2M1; INT4: M x K int8
   uint8_t* sf;      // NVFP4: 512-byte atoms; INT4: fp16 [K/64][M_pad]
   __nv_bfloat16* xl1;  // M x 2 r_pad: X_hat L1 as a bf16 pair, hi | lo (hi + lo = fp32 value)
   long long budget;
@@ -62,19 +64,24 @@ __host__ __device__ inline int quant_stack_max(int r_pad) {
 }
 
 struct QuantSmem {
-  uint32_t x_off, l1_off, il_off, stage_bytes, stages, bar_off, total;
+  uint32_t x_off, l1_off, il_off, stage_bytes, stages, stg_off, stg_bytes, bar_off, total;
 };
 
-__host__ __device__ inline QuantSmem quant_smem_layout(int r_pad, int S) {
+// Per stage: the stacked X tile, S slices of L1s^T and 1/lambda.  After the
+// stages: two code staging buffers (128 rows of codes) per quantizer group.
+__host__ __device__ inline QuantSmem quant_smem_layout(int fmt, int r_pad, int S) {
   QuantSmem L;
   L.x_off = 0;
   L.l1_off = kQuantTileRows * kQuantBK * 2;                // 16384
   L.il_off = L.l1_off + S * r_pad * 128;                   // S * r_pad rows of 128 bytes
   uint32_t sb = L.il_off + S * kQuantBK * 4;
   L.stage_bytes = (sb + 1023u) & ~1023u;
-  L.stages = kQuantStageBudget / L.stage_bytes;
+  L.stg_bytes = kQuantTileRows * quant_code_row_bytes(fmt);   // one staging buffer
+  const uint32_t stg_total = 2u * kQuantGroups * L.stg_bytes;
+  L.stages = (kQuantSmemBudget - stg_total) / L.stage_bytes;
   if (L.stages > static_cast<uint32_t>(kQuantMaxStages)) L.stages = kQuantMaxStages;
-  L.bar_off = L.stage_bytes * L.stages;
+  L.stg_off = L.stage_bytes * L.stages;
+  L.bar_off = L.stg_off + stg_total;
   L.total = L.bar_off + 256 + 512 + 1024;                  // barriers, 1/scale table, alignment
   return L;
 }
@@ -82,9 +89,10 @@ __host__ __device__ inline QuantSmem quant_smem_layout(int r_pad, int S) {
 template <int FMT>  // 0 = NVFP4 (groups of 16), 1 = INT4 (groups of 64)
 __global__ void __launch_bounds__(kQuantThreads, 1)
     quant_act_kernel(const __grid_constant__ CUtensorMap tm_x,
-                     const __grid_constant__ CUtensorMap tm_l1t, const QuantParams p) {
+                     const __grid_constant__ CUtensorMap tm_l1t,
+                     const __grid_constant__ CUtensorMap tm_codes, const QuantParams p) {
   extern __shared__ uint8_t smem_raw[];
-  const QuantSmem L = quant_smem_layout(p.r_pad, p.S);
+  const QuantSmem L = quant_smem_layout(FMT, p.r_pad, p.S);
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   const int NS = static_cast<int>(L.stages);
@@ -186,62 +194,63 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
     // Group k = (warp - 2) / 4 takes the stages k, k + G, k + 2G, ... (G groups);
     // its warp of lane quarter q quantizes rows 32 q .. 32 q + 31 of the
     // stacked tile, one lane per row over the whole 64-wide sub-tile: four
-    // independent NVFP4 groups of 16 (or one INT4 group of 64) per lane, so
-    // each lane has four chains of work in flight and writes its row's codes
-    // (32 or 64 contiguous bytes) and scales (one 4-byte word or one fp16).
+    // independent NVFP4 groups of 16 (or one INT4 group of 64) per lane.  The
+    // group stages its 128 rows of codes in shared memory and one of its
+    // threads writes them with a TMA store per sub-tile; each lane writes its
+    // row's scales itself (one 4-byte word or one fp16).  A failed wait does
+    // not leave the loop: the group's named barriers stay matched.
+    constexpr uint32_t RB = quant_code_row_bytes(FMT);   // code bytes per row
     const uint32_t q = warp & 3u;
     const int grp = static_cast<int>(warp - 2) >> 2;
+    const bool leader = warp == static_cast<uint32_t>(2 + 4 * grp) && lane == 0;
+    const uint32_t bar_free = 1 + 2 * grp, bar_full = 2 + 2 * grp;   // named barriers of the group
     const uint32_t R = q * 32 + lane;          // row of the stacked A tile
     const int j = static_cast<int>(R) / BM;    // K sub-tile
     const int m = m0 + static_cast<int>(R) % BM;
     const bool row_ok = m < p.M;
-    for (int i = grp; i < nkt; i += kQuantGroups) {
+    int use = 0;
+    for (int i = grp; i < nkt; i += kQuantGroups, ++use) {
       const int s = i % NS;
       const uint32_t ph = (i / NS) & 1;
-      if (!warp_wait(&full[s], ph, p.budget, abort_flag)) {
+      const bool ok = warp_wait(&full[s], ph, p.budget, abort_flag);
+      if (!ok) {
         if (lane == 0) raise_error(kErrWaitQuant);
         *abort_flag = 1;
-        break;
       }
       const int kcol = i * S + j;              // 64-wide column group of X
       const bool col_ok = kcol * kQuantBK < p.K;
       const uint8_t* st = smem + s * L.stage_bytes;
-      const float4* il = reinterpret_cast<const float4*>(st + L.il_off + j * kQuantBK * 4);
-      const uint8_t* xrow = st + L.x_off + R * 128;
       float v[64];
+      if (ok) {
+        const float4* il = reinterpret_cast<const float4*>(st + L.il_off + j * kQuantBK * 4);
+        const uint8_t* xrow = st + L.x_off + R * 128;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint32_t chunk = (static_cast<uint32_t>(c) ^ (R & 7u)) << 4;   // 128-byte swizzle
-        const uint4 raw = *reinterpret_cast<const uint4*>(xrow + chunk);
-        const float4 l0 = il[2 * c], l1 = il[2 * c + 1];
-        float2 t;
-        t = fmul2_rn(make_float2(bf16_lo(raw.x), bf16_hi(raw.x)), make_float2(l0.x, l0.y));
-        v[8 * c + 0] = t.x; v[8 * c + 1] = t.y;
-        t = fmul2_rn(make_float2(bf16_lo(raw.y), bf16_hi(raw.y)), make_float2(l0.z, l0.w));
-        v[8 * c + 2] = t.x; v[8 * c + 3] = t.y;
-        t = fmul2_rn(make_float2(bf16_lo(raw.z), bf16_hi(raw.z)), make_float2(l1.x, l1.y));
-        v[8 * c + 4] = t.x; v[8 * c + 5] = t.y;
-        t = fmul2_rn(make_float2(bf16_lo(raw.w), bf16_hi(raw.w)), make_float2(l1.z, l1.w));
-        v[8 * c + 6] = t.x; v[8 * c + 7] = t.y;
+        for (int c = 0; c < 8; ++c) {
+          const uint32_t chunk = (static_cast<uint32_t>(c) ^ (R & 7u)) << 4;   // 128-byte swizzle
+          const uint4 raw = *reinterpret_cast<const uint4*>(xrow + chunk);
+          const float4 l0 = il[2 * c], l1 = il[2 * c + 1];
+          float2 t;
+          t = fmul2_rn(make_float2(bf16_lo(raw.x), bf16_hi(raw.x)), make_float2(l0.x, l0.y));
+          v[8 * c + 0] = t.x; v[8 * c + 1] = t.y;
+          t = fmul2_rn(make_float2(bf16_lo(raw.y), bf16_hi(raw.y)), make_float2(l0.z, l0.w));
+          v[8 * c + 2] = t.x; v[8 * c + 3] = t.y;
+          t = fmul2_rn(make_float2(bf16_lo(raw.z), bf16_hi(raw.z)), make_float2(l1.x, l1.y));
+          v[8 * c + 4] = t.x; v[8 * c + 5] = t.y;
+          t = fmul2_rn(make_float2(bf16_lo(raw.w), bf16_hi(raw.w)), make_float2(l1.z, l1.w));
+          v[8 * c + 6] = t.x; v[8 * c + 7] = t.y;
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 64; ++e) v[e] = 0.0f;
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);   // X of this stage is in registers
+      uint32_t out[RB / 4];
+      uint32_t sfw;
       if constexpr (FMT == 0) {
-        uint32_t out[8];
-        uint32_t sfw = 0;
+        sfw = 0;
 #pragma unroll
         for (int g = 0; g < 4; ++g) sfw |= quant16_nvfp4(v + 16 * g, out + 2 * g, rcp_tab) << (8 * g);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
-        if (col_ok) {
-          if (row_ok) {
-            uint4* dst = reinterpret_cast<uint4*>(p.codes + static_cast<size_t>(m) * (p.K / 2) +
-                                                  kcol * (kQuantBK / 2));
-            dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
-            dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
-          }
-          // scale atom: 128 rows x 4 scales, byte (m % 32) * 16 + (m % 128 / 32) * 4 + k4
-          uint8_t* atom = p.sf + (static_cast<size_t>(m / 128) * p.sf_kcols + kcol) * 512;
-          *reinterpret_cast<uint32_t*>(atom + (m & 31) * 16 + ((m & 127) >> 5) * 4) = row_ok ? sfw : 0u;
-        }
       } else {
         float amax = 0.0f;
 #pragma unroll
@@ -249,31 +258,51 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
         const uint16_t sh = int4_scale_bits(amax);
         const float sd = __half2float(__ushort_as_half(sh));
         const float inv = sd == 0.0f ? 0.0f : __frcp_rn(sd);
-        uint32_t out[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           uint32_t w = 0;
-          if (sd != 0.0f) {
 #pragma unroll
-            for (int b = 0; b < 4; ++b)
-              w |= (static_cast<uint32_t>(int4_code(v[4 * e + b], inv)) & 0xFFu) << (8 * b);
-          }
-          out[e] = w;
+          for (int b = 0; b < 4; ++b)
+            w |= (static_cast<uint32_t>(int4_code(v[4 * e + b], inv)) & 0xFFu) << (8 * b);
+          out[e] = sd == 0.0f ? 0u : w;
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
-        if (col_ok) {
-          if (row_ok) {
-            uint4* dst = reinterpret_cast<uint4*>(p.codes + static_cast<size_t>(m) * p.K + kcol * kQuantBK);
+        sfw = sh;
+      }
+      // codes -> this group's staging buffer (rows of RB bytes in the TMA swizzle
+      // of that row length: 16-byte chunk c of row R sits at c ^ ((R >> sh) & mask))
+      uint8_t* buf = smem + L.stg_off + (2 * grp + (use & 1)) * L.stg_bytes;
+      if (leader) bulk_wait_group_read<1>();   // its store from two uses ago has read it
+      named_bar_sync(bar_free, 128);
+      {
+        const uint32_t row_addr = smem_u32(buf) + R * RB;
+        const uint32_t sw = FMT == 0 ? ((R >> 2) & 1u) : ((R >> 1) & 3u);
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-              dst[e] = make_uint4(out[4 * e], out[4 * e + 1], out[4 * e + 2], out[4 * e + 3]);
-          }
+        for (uint32_t c = 0; c < RB / 16; ++c)
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row_addr + ((c ^ sw) << 4)),
+                       "r"(out[4 * c]), "r"(out[4 * c + 1]), "r"(out[4 * c + 2]), "r"(out[4 * c + 3])
+                       : "memory");
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(bar_full, 128);
+      if (leader && ok) {
+        for (int jj = 0; jj < S; ++jj) {
+          const int kc = i * S + jj;
+          if (kc * kQuantBK < p.K) tma_store_2d(&tm_codes, buf + jj * BM * RB, kc * RB, m0);
+        }
+        bulk_commit_group();
+      }
+      if (ok && col_ok) {
+        if constexpr (FMT == 0) {
+          // scale atom: 128 rows x 4 scales, byte (m % 32) * 16 + (m % 128 / 32) * 4 + k4
+          uint8_t* atom = p.sf + (static_cast<size_t>(m / 128) * p.sf_kcols + kcol) * 512;
+          *reinterpret_cast<uint32_t*>(atom + (m & 31) * 16 + ((m & 127) >> 5) * 4) = row_ok ? sfw : 0u;
+        } else {
           reinterpret_cast<uint16_t*>(p.sf)[static_cast<size_t>(kcol) * p.M_pad + m] =
-              row_ok ? sh : static_cast<uint16_t>(0);
+              row_ok ? static_cast<uint16_t>(sfw) : static_cast<uint16_t>(0);
         }
       }
     }
+    if (leader) bulk_wait_group_all();
   }
   __syncwarp();
 

@@ -149,7 +149,8 @@ int device_setup(int dev) {
   SVDQ_CUDA(cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev));
   uint32_t qmax = 0;
   for (int rp : {0, 16, 32, 64, 128, 192, 256})
-    for (int S = 1; S <= quant_stack_max(rp); S *= 2) qmax = std::max(qmax, quant_smem_layout(rp, S).total);
+    for (int S = 1; S <= quant_stack_max(rp); S *= 2)
+      for (int f = 0; f < 2; ++f) qmax = std::max(qmax, quant_smem_layout(f, rp, S).total);
   SVDQ_CUDA(cudaFuncSetAttribute(quant_act_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, qmax));
   SVDQ_CUDA(cudaFuncSetAttribute(quant_act_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, qmax));
   SVDQ_CUDA(cudaFuncSetAttribute(gemm_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -672,8 +673,13 @@ SVDQ_API int svdq_quantize_act(const svdq_weights* w, const void* X, int M, void
   uint8_t* base = static_cast<uint8_t*>(ws);
   const int S = quant_stack_for(M, w->r_pad, g_dev[dev].sms);
   const int BM = kQuantTileRows / S;
-  CUtensorMap tm_x;
+  CUtensorMap tm_x, tm_codes;
   if ((rc = make_map(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, w->K, M, kQuantBK, BM)))
+    return rc;
+  // codes: NVFP4 M x K/2 packed E2M1, INT4 M x K int8; one box = one sub-tile's BM rows
+  const uint32_t rb = quant_code_row_bytes(w->fmt == SVDQ_NVFP4 ? 0 : 1);
+  if ((rc = make_map(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base + L.codes_off,
+                     w->fmt == SVDQ_NVFP4 ? w->K / 2 : w->K, M, rb, BM)))
     return rc;
   QuantParams p;
   p.M = M;
@@ -683,7 +689,6 @@ SVDQ_API int svdq_quantize_act(const svdq_weights* w, const void* X, int M, void
   p.M_pad = L.M_pad;
   p.sf_kcols = w->sf_kcols;
   p.inv_lambda = w->inv_lambda;
-  p.codes = base + L.codes_off;
   p.sf = base + L.sf_off;
   p.xl1 = reinterpret_cast<__nv_bfloat16*>(base + L.xl1_off);
   p.budget = wait_budget();
@@ -693,13 +698,13 @@ SVDQ_API int svdq_quantize_act(const svdq_weights* w, const void* X, int M, void
     const size_t off = static_cast<size_t>(w->K / 64) * 512;
     SVDQ_CUDA(cudaMemset2DAsync(p.sf + off, pitch, 0, pitch - off, L.M_pad / 128, st));
   }
-  const QuantSmem Q = quant_smem_layout(w->r_pad, S);
+  const QuantSmem Q = quant_smem_layout(w->fmt == SVDQ_NVFP4 ? 0 : 1, w->r_pad, S);
   const dim3 grid((M + BM - 1) / BM);
   const CUtensorMap& tm_l1t = w->r_pad > 0 ? w->tm_l1t : tm_x;
   if (w->fmt == SVDQ_NVFP4)
-    quant_act_kernel<0><<<grid, kQuantThreads, Q.total, st>>>(tm_x, tm_l1t, p);
+    quant_act_kernel<0><<<grid, kQuantThreads, Q.total, st>>>(tm_x, tm_l1t, tm_codes, p);
   else
-    quant_act_kernel<1><<<grid, kQuantThreads, Q.total, st>>>(tm_x, tm_l1t, p);
+    quant_act_kernel<1><<<grid, kQuantThreads, Q.total, st>>>(tm_x, tm_l1t, tm_codes, p);
   SVDQ_CHECK_LAUNCH();
   return SVDQ_OK;
 }

@@ -284,6 +284,11 @@ __host__ __device__ constexpr uint32_t idesc_e2m1_ue4m3(int M, int N) {
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// Barrier `id` (1..15) among `count` threads (whole warps) of the CTA.
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // ------------------------------------------------------------- TMA store ---
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int x, int y) {
   asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
