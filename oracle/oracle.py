@@ -197,9 +197,31 @@ def calib_absmax(X_bits: np.ndarray) -> np.ndarray:
     return np.max(np.abs(bf16_decode(X_bits)), axis=0).astype(np.float32)
 
 
+def _top_factors_gram(W_hat: np.ndarray, r: int):
+    """The top-r singular triplets of W_hat from the fp64 eigendecomposition of
+    its smaller Gram matrix (W_hat W_hat^T or W_hat^T W_hat): the same rank-r
+    subspace as the SVD, at O(min(K, N)^3) instead of a full SVD."""
+    K, N = W_hat.shape
+    if K <= N:
+        ev, U = np.linalg.eigh(W_hat @ W_hat.T)
+        order = np.argsort(ev)[::-1]
+        S = np.sqrt(np.maximum(ev[order], 0.0))
+        U = U[:, order]
+        L1 = U[:, :r] * S[:r]
+        L2 = np.divide(U[:, :r].T @ W_hat, S[:r, None], out=np.zeros((r, N)), where=S[:r, None] > 0)
+    else:
+        ev, V = np.linalg.eigh(W_hat.T @ W_hat)
+        order = np.argsort(ev)[::-1]
+        S = np.sqrt(np.maximum(ev[order], 0.0))
+        V = V[:, order]
+        L2 = V[:, :r].T
+        L1 = W_hat @ V[:, :r]
+    return L1, L2, S
+
+
 def prepare(W_bits: np.ndarray, x_absmax: Optional[np.ndarray], rank: int,
             lora_A_bits: Optional[np.ndarray] = None,
-            lora_B_bits: Optional[np.ndarray] = None) -> dict:
+            lora_B_bits: Optional[np.ndarray] = None, svd: str = "full") -> dict:
     """Smoothing, truncated SVD, residual and optional LoRA fold, in fp64.
 
     W_hat = diag(lambda) W; W_hat = U S V^T (numpy/LAPACK fp64);
@@ -208,15 +230,22 @@ def prepare(W_bits: np.ndarray, x_absmax: Optional[np.ndarray], rank: int,
     taken against the factors the layer actually uses.  A LoRA (A: K x rl,
     B: rl x N) joins the branch as L1' = [L1 | bf16(diag(lambda) A)],
     L2' = [L2 ; B] without touching R (no requantization).
+
+    svd="gram" takes the top-r factors from the Gram matrix instead of a full
+    SVD (for layers of FLUX size, where the full SVD takes minutes); "sigma"
+    then holds the square roots of the Gram eigenvalues.
     """
     W = bf16_decode(W_bits).astype(np.float64)
     K, N = W.shape
     lam, inv = smoothing(x_absmax, W_bits)
     W_hat = lam.astype(np.float64)[:, None] * W
-    U, S, Vt = np.linalg.svd(W_hat, full_matrices=False)
     r = int(rank)
-    L1_exact = U[:, :r] * S[:r]
-    L2_exact = Vt[:r, :]
+    if svd == "gram":
+        L1_exact, L2_exact, S = _top_factors_gram(W_hat, r)
+    else:
+        U, S, Vt = np.linalg.svd(W_hat, full_matrices=False)
+        L1_exact = U[:, :r] * S[:r]
+        L2_exact = Vt[:r, :]
     L1 = bf16_round(L1_exact)
     L2 = bf16_round(L2_exact)
     R64 = W_hat - bf16_decode(L1).astype(np.float64) @ bf16_decode(L2).astype(np.float64)

@@ -228,3 +228,25 @@ def test_row_subset_matches_full():
     Ys = O.linear("nvfp4", full["act"], full["wq"], full["prep"]["L2"], WL.bf16_bits(d["bias"]),
                   48, rows=rows)
     assert np.array_equal(Ys, full["Y"][rows])
+
+
+@pytest.mark.parametrize("K,N", [(96, 160), (160, 96)])
+def test_gram_route_spans_the_svd_subspace(K, N):
+    """prepare(svd="gram") (top-r factors from the smaller Gram matrix, used for
+    the full-size GPU parity tests) gives the same rank-r product, singular
+    values and, where the bf16 rounding of the factors agrees, the same residual
+    as the full SVD; a dropped Sigma or a transposed Gram matrix would not."""
+    d = WL.make_small(32, K, N, w_outlier_rows=3, seed=K + N)
+    Wb = WL.bf16_bits(d["W"])
+    xm = O.calib_absmax(WL.bf16_bits(d["X"]))
+    a = O.prepare(Wb, xm, 24)
+    b = O.prepare(Wb, xm, 24, svd="gram")
+    pa = a["L1_exact"] @ a["L2_exact"]
+    pb = b["L1_exact"] @ b["L2_exact"]
+    assert np.linalg.norm(pa - pb) <= 1e-9 * np.linalg.norm(pa)
+    assert np.allclose(a["sigma"][:24], b["sigma"][:24], rtol=1e-9)
+    assert np.array_equal(a["lam"], b["lam"]) and np.array_equal(a["inv_lambda"], b["inv_lambda"])
+    # the residuals differ only through the bf16 rounding of sign-flipped factors
+    Ra = a["R"].astype(np.float64)
+    Rb = b["R"].astype(np.float64)
+    assert np.linalg.norm(Ra - Rb) <= 2.0 ** -7 * np.linalg.norm(pa)
