@@ -128,6 +128,21 @@ def layer_inputs(args):
 
 
 # ----------------------------------------------------------------------------- ours
+def max_over_ranks(values, world, device):
+    """Element-wise maximum over all ranks (the slowest rank sets the time)."""
+    if world <= 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_throughput(world, flops_per_rank_step, steps, seconds):
+    """Whole-job TFLOP/s: every rank runs its own batch of the layer (weak
+    scaling), so the work of all ranks over the slowest rank's time."""
+    return world * flops_per_rank_step * steps / seconds / 1e12
+
+
 def time_layer(S, w, X, ws, Y, M, flush, stream, steps, warmup, world, sampler=None):
     """Per-step seconds of the activation kernel and of the GEMM (CUDA events on
     the launching stream), with the 126 MB L2 flushed before every step."""
@@ -222,12 +237,7 @@ def run_ours(args):
     t_q, t_g, clocks = time_layer(S, w, X, ws, Y, M, flush, stream, args.steps, args.warmup, world, sampler)
     t_layer = t_q + t_g
     total = float(t_layer.sum())
-    if world > 1:
-        t = torch.tensor([total, float(t_q.mean()), float(t_g.mean())], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total, tq_mean, tg_mean = (float(v) for v in t.tolist())
-    else:
-        tq_mean, tg_mean = float(t_q.mean()), float(t_g.mean())
+    total, tq_mean, tg_mean = max_over_ranks([total, float(t_q.mean()), float(t_g.mean())], world, dev)
 
     # end to end through the public API: pinned host X in, host Y out, every step
     X_host = X.cpu().pin_memory()
@@ -262,7 +272,7 @@ def run_ours(args):
     scale_bytes = M * K / 16 if spec.fmt == "nvfp4" else M * K / 64 * 2
     q_bytes = 2.0 * M * K + code_bytes + scale_bytes + 2.0 * M * w.rank_padded
     q_gbs = q_bytes / tq_mean / 1e9
-    value = world * flops * args.steps / total / 1e12
+    value = job_throughput(world, flops, args.steps, total)
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
