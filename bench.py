@@ -59,6 +59,42 @@ def peaks():
         return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
 
 
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
+# one ncu capture of `bench.py --steps 3 --warmup 3 --no-cpu-baseline
+# --no-extras` (the summaries under profiles/), keyed by kernel, workload and a
+# fingerprint of the kernel's sources: a kernel changed since the capture
+# reports null.  Y of the QKV layer (85 MB) is still mostly dirty in the
+# 126 MB L2 when the GEMM ends, so its write traffic is below Y's size.
+NCU_TRAFFIC = {
+    ("gemm_nvfp4_kernel", "c2_qkv/qkv", 4608): (60281344, "454e3f84fc5c6294"),
+    ("quant_act_kernel", "c2_qkv/qkv", 4608): (28556544, "bf98e5d72b08526b"),
+    ("gemm_int4_kernel", "c4_int4_lora/proj", 4608): (26704640, "330358d37af68794"),
+}
+KERNEL_SOURCES = {
+    "gemm_nvfp4_kernel": ("gemm_nvfp4.cuh", "svdq_ptx.cuh", "svdq_formats.cuh"),
+    "quant_act_kernel": ("quant_act.cuh", "svdq_ptx.cuh", "svdq_formats.cuh"),
+    "gemm_int4_kernel": ("gemm_int4.cuh", "gemm_nvfp4.cuh", "svdq_ptx.cuh", "svdq_formats.cuh"),
+}
+
+
+def kernel_fingerprint(kernel):
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "w4a4_gemm_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel, workload, M):
+    """Measured DRAM bytes per launch, or None if not captured for this
+    workload or the kernel changed since."""
+    entry = NCU_TRAFFIC.get((kernel, workload, M))
+    if entry is None or kernel_fingerprint(kernel) != entry[1]:
+        return None
+    return entry[0]
+
+
 def dist_env():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -273,6 +309,7 @@ def run_ours(args):
     q_bytes = 2.0 * M * K + code_bytes + scale_bytes + 2.0 * M * w.rank_padded
     q_gbs = q_bytes / tq_mean / 1e9
     value = job_throughput(world, flops, args.steps, total)
+    gemm_kernel = "gemm_nvfp4_kernel" if spec.fmt == "nvfp4" else "gemm_int4_kernel"
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
@@ -286,13 +323,15 @@ def run_ours(args):
         "us_per_layer": round(total / args.steps * 1e6, 2),
         "us_quant": round(tq_mean * 1e6, 2), "us_gemm": round(tg_mean * 1e6, 2),
         "pct_fp4_peak_layer": round(100.0 * flops / (total / args.steps) / 1e12 / fp_peak, 2),
-        "roofline": {"bound": "tensor", "kernel": "gemm_nvfp4_kernel" if spec.fmt == "nvfp4" else "gemm_int4_kernel",
+        "roofline": {"bound": "tensor", "kernel": gemm_kernel,
                      "achieved": round(achieved, 1), "peak": round(fp_peak, 1), "unit": "TFLOP/s",
-                     "frac": round(achieved / fp_peak, 4), "traffic": None,
+                     "frac": round(achieved / fp_peak, 4),
+                     "traffic": ncu_traffic(gemm_kernel, f"{args.config}/{spec.name}", M),
                      "peak_note": f"{pk['source']}: bf16 {pk['bf16']} TF/s x {'4 (FP4)' if spec.fmt == 'nvfp4' else '2 (INT8)'}"},
         "roofline_quant": {"bound": "hbm", "kernel": "quant_act_kernel", "achieved": round(q_gbs, 1),
                            "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": round(q_gbs / pk["hbm_gbs"], 4),
-                           "algorithmic_bytes": int(q_bytes)},
+                           "algorithmic_bytes": int(q_bytes),
+                           "traffic": ncu_traffic("quant_act_kernel", f"{args.config}/{spec.name}", M)},
         "e2e": {"value": round(flops / t_e2e / 1e12, 3), "unit": UNIT,
                 "h2d_bytes_per_step": int(X.numel() * 2), "d2h_bytes_per_step": int(Y.numel() * 2)},
         "gpu_launches": launches_per_step * args.steps,
