@@ -25,9 +25,9 @@ from typing import Optional
 
 import numpy as np
 
-NVFP4, INT4 = 0, 1
-_FMT = {"nvfp4": NVFP4, "int4": INT4, NVFP4: NVFP4, INT4: INT4}
-GROUP = {NVFP4: 16, INT4: 64}
+NVFP4, INT4, FP4G32 = 0, 1, 2
+_FMT = {"nvfp4": NVFP4, "int4": INT4, "fp4g32": FP4G32, NVFP4: NVFP4, INT4: INT4, FP4G32: FP4G32}
+GROUP = {NVFP4: 16, INT4: 64, FP4G32: 32}
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "svdq_oracle.c")
@@ -73,6 +73,7 @@ def lib() -> ctypes.CDLL:
         _lib.oracle_fp16_round_sat.restype = ctypes.c_uint16
         _lib.oracle_fp16_round_sat.argtypes = [ctypes.c_float]
         _lib.oracle_quant_group_nvfp4.argtypes = [P, P, P]
+        _lib.oracle_quant_group_fp4g32.argtypes = [P, P, P]
         _lib.oracle_quant_group_int4.argtypes = [P, P, P]
         for name in ("oracle_bf16_round_array", "oracle_e4m3_round_array",
                      "oracle_e2m1_round_array", "oracle_fp16_round_array"):
@@ -151,7 +152,7 @@ def fp16_decode(codes) -> np.ndarray:
 
 
 def quant_group(fmt, v) -> tuple:
-    """One group (16 values NVFP4 / 64 values INT4) -> (codes one per byte, scale code)."""
+    """One group (16 values NVFP4 / 32 FP4 g32 / 64 INT4) -> (codes one per byte, scale code)."""
     fmt = _FMT[fmt]
     v = np.ascontiguousarray(v, dtype=np.float32)
     assert v.size == GROUP[fmt]
@@ -159,6 +160,9 @@ def quant_group(fmt, v) -> tuple:
     if fmt == NVFP4:
         sc = np.zeros(1, dtype=np.uint8)
         lib().oracle_quant_group_nvfp4(_ptr(v), _ptr(codes), _ptr(sc))
+    elif fmt == FP4G32:
+        sc = np.zeros(1, dtype=np.uint8)
+        lib().oracle_quant_group_fp4g32(_ptr(v), _ptr(codes), _ptr(sc))
     else:
         sc = np.zeros(1, dtype=np.uint16)
         lib().oracle_quant_group_int4(_ptr(v), _ptr(codes), _ptr(sc))
@@ -273,7 +277,7 @@ def weight_quant(fmt, R: np.ndarray):
     K, N = R.shape
     g = GROUP[fmt]
     codes = np.zeros((N, K // 2), dtype=np.uint8)
-    scales = np.zeros((N, K // g), dtype=np.uint8 if fmt == NVFP4 else np.uint16)
+    scales = np.zeros((N, K // g), dtype=np.uint16 if fmt == INT4 else np.uint8)
     rc = lib().oracle_weight_quant(fmt, K, N, _ptr(R), _ptr(codes), _ptr(scales))
     assert rc == 0
     return codes, scales
@@ -299,7 +303,7 @@ def act_quant(fmt, X_bits: np.ndarray, inv_lambda: Optional[np.ndarray], L1_bits
     g = GROUP[fmt]
     r = 0 if L1_bits is None else L1_bits.shape[1]
     codes = np.zeros((M, K // 2), dtype=np.uint8)
-    scales = np.zeros((M, K // g), dtype=np.uint8 if fmt == NVFP4 else np.uint16)
+    scales = np.zeros((M, K // g), dtype=np.uint16 if fmt == INT4 else np.uint8)
     XL1 = np.zeros((M, r), dtype=np.float32)
     inv = None if inv_lambda is None else np.ascontiguousarray(inv_lambda, dtype=np.float32)
     L1s = None if L1_bits is None else fold_l1(L1_bits, inv)

@@ -16,8 +16,10 @@
  *   Sec. 4.2 "SVDQuant": X_hat = X diag(lambda)^-1, W_hat = diag(lambda) W,
  *        X W ~ X_hat L1 L2 + Q(X_hat) Q(R), low-rank branch in 16 bits.
  *   Sec. 5.1 "Implementation details": per-group symmetric quantization of both
- *        operands; INT4 uses groups of 64 with 16-bit scales.  The NVFP4
- *        variant built here uses E2M1 codes with one E4M3 scale per 16 values.
+ *        operands; INT4 uses groups of 64 with 16-bit scales; FP4 uses groups of
+ *        32 with an FP8 scale.  Three formats are built: NVFP4 (E2M1 codes, one
+ *        E4M3 scale per 16 values), FP4 g32 (E2M1 codes, one E4M3 scale per 32
+ *        values: the paper's FP4, FP8 read as E4M3) and INT4 (groups of 64).
  *
  * Readings of steps the paper leaves open:
  *   - groups run along K, the reduction dimension, for both operands;
@@ -41,6 +43,11 @@
 
 #define ORACLE_NVFP4 0
 #define ORACLE_INT4 1
+#define ORACLE_FP4G32 2
+
+/* Group size along K and bytes per scale of each format. */
+static int fmt_group(int fmt) { return fmt == ORACLE_NVFP4 ? 16 : (fmt == ORACLE_FP4G32 ? 32 : 64); }
+static int fmt_scale_bytes(int fmt) { return fmt == ORACLE_INT4 ? 2 : 1; }
 
 /* ------------------------------------------------------------------------- */
 /* bf16: the upper half of an IEEE binary32.                                 */
@@ -181,20 +188,28 @@ static float round_half_even(float x) {
 /* Codes come out one per byte (low nibble); callers pack.                   */
 /* ------------------------------------------------------------------------- */
 
-/* NVFP4: 16 values -> 16 E2M1 codes + one E4M3 scale. */
-void oracle_quant_group_nvfp4(const float *v, uint8_t *codes, uint8_t *scale) {
+/* FP4: g values -> g E2M1 codes + one E4M3 scale (g = 16 NVFP4, 32 FP4 g32). */
+static void quant_group_fp4(int g, const float *v, uint8_t *codes, uint8_t *scale) {
     float amax = 0.0f;
-    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    for (int i = 0; i < g; ++i) amax = fmaxf(amax, fabsf(v[i]));
     float s32 = amax / 6.0f;                       /* q_max = 6 for E2M1 */
     uint8_t s8 = oracle_e4m3_round_sat(s32);
     float sd = oracle_e4m3_decode(s8);
     *scale = s8;
     if (sd == 0.0f) {
-        for (int i = 0; i < 16; ++i) codes[i] = 0;
+        for (int i = 0; i < g; ++i) codes[i] = 0;
         return;
     }
     float inv = 1.0f / sd;
-    for (int i = 0; i < 16; ++i) codes[i] = oracle_e2m1_round(v[i] * inv);
+    for (int i = 0; i < g; ++i) codes[i] = oracle_e2m1_round(v[i] * inv);
+}
+
+void oracle_quant_group_nvfp4(const float *v, uint8_t *codes, uint8_t *scale) {
+    quant_group_fp4(16, v, codes, scale);
+}
+
+void oracle_quant_group_fp4g32(const float *v, uint8_t *codes, uint8_t *scale) {
+    quant_group_fp4(32, v, codes, scale);
 }
 
 /* INT4: 64 values -> 64 signed codes in [-7, 7] (4-bit two's complement in the
@@ -220,7 +235,7 @@ void oracle_quant_group_int4(const float *v, uint8_t *codes, uint16_t *scale) {
 }
 
 static float deq_code(int fmt, uint8_t code) {
-    if (fmt == ORACLE_NVFP4) return oracle_e2m1_decode(code & 0xF);
+    if (fmt != ORACLE_INT4) return oracle_e2m1_decode(code & 0xF);
     int q = code & 0xF;
     return (float)(q >= 8 ? q - 16 : q);
 }
@@ -231,11 +246,11 @@ static uint8_t get_nibble(const uint8_t *packed, long i) {
 }
 
 static void quantize_row(int fmt, const float *v, int K, uint8_t *codes_row, void *scales_row) {
-    int g = (fmt == ORACLE_NVFP4) ? 16 : 64;
+    int g = fmt_group(fmt);
     uint8_t c[64];
     for (int k0 = 0; k0 < K; k0 += g) {
-        if (fmt == ORACLE_NVFP4)
-            oracle_quant_group_nvfp4(v + k0, c, (uint8_t *)scales_row + k0 / g);
+        if (fmt != ORACLE_INT4)
+            quant_group_fp4(g, v + k0, c, (uint8_t *)scales_row + k0 / g);
         else
             oracle_quant_group_int4(v + k0, c, (uint16_t *)scales_row + k0 / g);
         for (int i = 0; i < g; i += 2)
@@ -256,9 +271,9 @@ static void quantize_row(int fmt, const float *v, int K, uint8_t *codes_row, voi
 /* ------------------------------------------------------------------------- */
 int oracle_act_quant(int fmt, int M, int K, int r, const uint16_t *X, const float *inv_lambda,
                      const uint16_t *L1s, uint8_t *codes, void *scales, float *XL1) {
-    int g = (fmt == ORACLE_NVFP4) ? 16 : 64;
+    int g = fmt_group(fmt);
     if (K % g) return 1;
-    int ssz = (fmt == ORACLE_NVFP4) ? 1 : 2;
+    int ssz = fmt_scale_bytes(fmt);
 #pragma omp parallel
     {
         float *xh = (float *)__builtin_alloca(sizeof(float) * (size_t)K);
@@ -301,9 +316,9 @@ void oracle_fold_l1(int K, int r, const float *inv_lambda, const uint16_t *L1, u
 /* each output column n.  codes: N x K/2, scales: N x K/g.                    */
 /* ------------------------------------------------------------------------- */
 int oracle_weight_quant(int fmt, int K, int N, const float *R, uint8_t *codes, void *scales) {
-    int g = (fmt == ORACLE_NVFP4) ? 16 : 64;
+    int g = fmt_group(fmt);
     if (K % g) return 1;
-    int ssz = (fmt == ORACLE_NVFP4) ? 1 : 2;
+    int ssz = fmt_scale_bytes(fmt);
 #pragma omp parallel
     {
         float *col = (float *)__builtin_alloca(sizeof(float) * (size_t)K);
@@ -328,7 +343,7 @@ int oracle_linear_rows(int fmt, int M, int N, int K, int r, const uint8_t *codes
                        const void *scales_x, const float *XL1, const uint8_t *codes_w,
                        const void *scales_w, const uint16_t *L2, const uint16_t *bias,
                        const int *rows, int n_rows, uint16_t *Y) {
-    int g = (fmt == ORACLE_NVFP4) ? 16 : 64;
+    int g = fmt_group(fmt);
     if (K % g) return 1;
     int G = K / g;
 #pragma omp parallel for schedule(dynamic, 1)
@@ -341,14 +356,14 @@ int oracle_linear_rows(int fmt, int M, int N, int K, int r, const uint8_t *codes
             float acc = 0.0f;
             for (int gi = 0; gi < G; ++gi) {
                 float sx, sw;
-                if (fmt == ORACLE_NVFP4) {
+                if (fmt != ORACLE_INT4) {
                     sx = oracle_e4m3_decode(((const uint8_t *)scales_x)[(long)m * G + gi]);
                     sw = oracle_e4m3_decode(((const uint8_t *)scales_w)[(long)n * G + gi]);
                 } else {
                     sx = oracle_fp16_decode(((const uint16_t *)scales_x)[(long)m * G + gi]);
                     sw = oracle_fp16_decode(((const uint16_t *)scales_w)[(long)n * G + gi]);
                 }
-                float part = 0.0f;          /* exact: small multiples of 1/4 or integers */
+                float part = 0.0f;  /* exact: multiples of 1/4 below 2^12, or integers below 2^12 */
                 for (int k = gi * g; k < (gi + 1) * g; ++k)
                     part += deq_code(fmt, get_nibble(cx, k)) * deq_code(fmt, get_nibble(cw, k));
                 acc += (sx * sw) * part;
@@ -364,12 +379,12 @@ int oracle_linear_rows(int fmt, int M, int N, int K, int r, const uint8_t *codes
 
 /* Dequantize packed codes + scales (rows x K) to fp32: s * deq(q). */
 int oracle_dequant(int fmt, int rows, int K, const uint8_t *codes, const void *scales, float *out) {
-    int g = (fmt == ORACLE_NVFP4) ? 16 : 64;
+    int g = fmt_group(fmt);
     if (K % g) return 1;
     int G = K / g;
     for (long i = 0; i < rows; ++i)
         for (int k = 0; k < K; ++k) {
-            float s = (fmt == ORACLE_NVFP4)
+            float s = (fmt != ORACLE_INT4)
                           ? oracle_e4m3_decode(((const uint8_t *)scales)[i * G + k / g])
                           : oracle_fp16_decode(((const uint16_t *)scales)[i * G + k / g]);
             out[i * K + k] = s * deq_code(fmt, get_nibble(codes + i * (K / 2), k));
