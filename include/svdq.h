@@ -12,7 +12,10 @@
  * per-group 4-bit quantizer of Sec. 3.  Two 4-bit formats are supported:
  *   SVDQ_NVFP4: E2M1 codes with one E4M3 scale per 16 values along K;
  *   SVDQ_INT4 : signed 4-bit integers in [-7, 7] with one fp16 scale per 64
- *               values along K (Sec. 5.1).
+ *               values along K (Sec. 5.1);
+ *   SVDQ_FP4G32: E2M1 codes with one E4M3 scale per 32 values along K (the
+ *               paper's FP4 setting of Sec. 5.1: groups of 32, an FP8 scale).
+ *               It runs on the NVFP4 kernels with each scale stored twice.
  *
  * Conventions for every call:
  *   - "device" pointers are CUDA global-memory pointers on the current device;
@@ -56,7 +59,7 @@ typedef enum {
   SVDQ_ERR_LIBRARY = 6            /* cuSOLVER / cuBLAS failed during preparation */
 } svdq_status;
 
-typedef enum { SVDQ_NVFP4 = 0, SVDQ_INT4 = 1 } svdq_format;
+typedef enum { SVDQ_NVFP4 = 0, SVDQ_INT4 = 1, SVDQ_FP4G32 = 2 } svdq_format;
 
 /* Opaque prepared layer: 4-bit residual codes and scales, the bf16 low-rank
  * factors, 1/lambda and the bias, all in device memory owned by the handle. */

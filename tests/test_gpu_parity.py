@@ -59,7 +59,7 @@ def test_weight_quantizer_edge_values(S):
     while len(cols) < 32:
         cols.append((rng.standard_normal(K) * 10.0 ** rng.uniform(-4, 3)).astype(np.float32))
     R = np.stack(cols, axis=1).astype(np.float32)     # K x 32
-    for fmt in ("nvfp4", "int4"):
+    for fmt in ("nvfp4", "int4", "fp4g32"):
         w = S.svdq_load_weights(to_dev_f32(R), fmt=fmt)
         got = S.svdq_export_weights(w)
         codes, scales = O.weight_quant(fmt, R)
@@ -79,6 +79,8 @@ SHAPES = [
     (96, 512, 256, 32, "int4", True),
     (200, 1024, 512, 48, "int4", False),
     (64, 256, 272, 0, "int4", False),
+    (77, 512, 384, 32, "fp4g32", True),      # one E4M3 scale per 32 values, stored per 16
+    (300, 320, 272, 48, "fp4g32", False),
 ]
 
 
@@ -135,7 +137,7 @@ def test_prepare_weights_invariants(S):
     assert e_lib <= 1.1 * e_ora + 1e-3, (e_lib, e_ora)
 
 
-@pytest.mark.parametrize("fmt", ["nvfp4", "int4"])
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4", "fp4g32"])
 def test_lora_fold_parity(S, fmt):
     M, K, N, r, rl = 160, 512, 384, 32, 16
     data = WL.make_small(M, K, N, rank=r, fmt=fmt, lora_rank=rl, seed=9)

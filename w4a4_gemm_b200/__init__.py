@@ -19,9 +19,9 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libsvdq.so")
 
-NVFP4, INT4 = 0, 1
-_FMT = {"nvfp4": NVFP4, "int4": INT4, NVFP4: NVFP4, INT4: INT4}
-GROUP = {NVFP4: 16, INT4: 64}
+NVFP4, INT4, FP4G32 = 0, 1, 2
+_FMT = {"nvfp4": NVFP4, "int4": INT4, "fp4g32": FP4G32, NVFP4: NVFP4, INT4: INT4, FP4G32: FP4G32}
+GROUP = {NVFP4: 16, INT4: 64, FP4G32: 32}
 
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "device allocation failed",
           4: "CUDA error", 5: "device wait timed out", 6: "cuSOLVER/cuBLAS error"}
@@ -276,7 +276,7 @@ def svdq_export_act(w: Weights, workspace: torch.Tensor, M: int):
     """(codes M x K/2 uint8, scales M x K/g, xl1 M x rank float32) on the host."""
     g = GROUP[w.fmt]
     codes = np.zeros((M, w.K // 2), dtype=np.uint8)
-    scales = np.zeros((M, w.K // g), dtype=np.uint8 if w.fmt == NVFP4 else np.uint16)
+    scales = np.zeros((M, w.K // g), dtype=np.uint16 if w.fmt == INT4 else np.uint8)
     xl1 = np.zeros((M, w.rank), dtype=np.float32)
     _check(lib().svdq_export_act(w.handle, _ptr(workspace), int(M), codes.ctypes.data_as(ctypes.c_void_p),
                                  scales.ctypes.data_as(ctypes.c_void_p),
@@ -288,7 +288,7 @@ def svdq_export_act(w: Weights, workspace: torch.Tensor, M: int):
 def svdq_export_weights(w: Weights) -> dict:
     g = GROUP[w.fmt]
     codes = np.zeros((w.N, w.K // 2), dtype=np.uint8)
-    scales = np.zeros((w.N, w.K // g), dtype=np.uint8 if w.fmt == NVFP4 else np.uint16)
+    scales = np.zeros((w.N, w.K // g), dtype=np.uint16 if w.fmt == INT4 else np.uint8)
     L1 = np.zeros((w.K, w.rank), dtype=np.uint16)
     L2 = np.zeros((w.rank, w.N), dtype=np.uint16)
     inv = np.zeros(w.K, dtype=np.float32)
@@ -305,7 +305,7 @@ def svdq_get_error() -> int:
 
 def svdq_tensor_peak(fmt: str, steps: int, stream=None):
     """Launch the tensor-core ceiling kernel (see include/svdq.h); time it with
-    CUDA events.  FLOP = SMs * steps * 4 * 2 * 128 * 256 * (64 NVFP4 | 32 INT4)."""
+    CUDA events.  FLOP = SMs * steps * 4 * 2 * 128 * 256 * (64 NVFP4 / FP4 g32 | 32 INT4)."""
     _check(lib().svdq_tensor_peak(_FMT[fmt], int(steps), _stream(stream)), "svdq_tensor_peak")
 
 

@@ -242,6 +242,29 @@ __global__ void residual_kernel(const double* __restrict__ What,
 // NVFP4: one thread per (n, group of 16): codes N x K/2, scales in 512-byte atoms
 //        (128 columns x 4 groups; byte (n % 32) * 16 + (n % 128 / 32) * 4 + g % 4).
 // INT4 : one thread per (n, group of 64): int8 codes N x K, fp16 scales [K/64][N_pad].
+// FP4 g32: one E4M3 scale per 32 values of K, stored in both 16-value slots of
+// the scale atom so the NVFP4 GEMM (block16) applies it to both halves.
+__global__ void quant_weight_fp4g32_kernel(const float* __restrict__ R, int K, int N, int sf_kcols,
+                                           uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
+  __shared__ float rcp_tab[128];
+  fill_e4m3_rcp_table(rcp_tab, threadIdx.x, blockDim.x);
+  __syncthreads();
+  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  const int g = blockIdx.y;                  // group of 32
+  if (n >= N) return;
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = R[static_cast<size_t>(32 * g + i) * N + n];
+  uint32_t cw[4];
+  const uint32_t s8 = quant32_fp4(v, cw, rcp_tab);
+  uint4* dst = reinterpret_cast<uint4*>(codes + static_cast<size_t>(n) * (K / 2) + 16 * g);
+  *dst = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+  uint8_t* atom = sf + (static_cast<size_t>(n / 128) * sf_kcols + g / 2) * 512;
+  uint8_t* slot = atom + (n & 31) * 16 + ((n & 127) >> 5) * 4 + 2 * (g & 1);
+  slot[0] = static_cast<uint8_t>(s8);
+  slot[1] = static_cast<uint8_t>(s8);
+}
+
 __global__ void quant_weight_nvfp4_kernel(const float* __restrict__ R, int K, int N, int sf_kcols,
                                           uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
   __shared__ float rcp_tab[128];

@@ -40,8 +40,8 @@ constexpr int kQuantWarps = 4 * kQuantGroups;   // quantizer warps (one per lane
 constexpr int kQuantThreads = 32 * (2 + kQuantWarps);
 constexpr uint32_t kQuantSmemBudget = 220u * 1024u;    // shared memory for stages + code staging
 
-// Bytes of codes one row of a 64-wide sub-tile produces: 64 E2M1 (NVFP4) or 64 int8 (INT4).
-__host__ __device__ constexpr uint32_t quant_code_row_bytes(int fmt) { return fmt == 0 ? 32u : 64u; }
+// Bytes of codes one row of a 64-wide sub-tile produces: 64 E2M1 (NVFP4, FP4 g32) or 64 int8 (INT4).
+__host__ __device__ constexpr uint32_t quant_code_row_bytes(int fmt) { return fmt == 1 ? 64u : 32u; }
 
 struct QuantParams {
   int M, K;
@@ -86,7 +86,7 @@ __host__ __device__ inline QuantSmem quant_smem_layout(int fmt, int r_pad, int S
   return L;
 }
 
-template <int FMT>  // 0 = NVFP4 (groups of 16), 1 = INT4 (groups of 64)
+template <int FMT>  // 0 = NVFP4 (groups of 16), 1 = INT4 (groups of 64), 2 = FP4 g32 (groups of 32)
 __global__ void __launch_bounds__(kQuantThreads, 1)
     quant_act_kernel(const __grid_constant__ CUtensorMap tm_x,
                      const __grid_constant__ CUtensorMap tm_l1t,
@@ -124,7 +124,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (FMT == 0 && warp >= 2 && warp < 6) fill_e4m3_rcp_table(rcp_tab, threadIdx.x - 64, 128);
+  if (FMT != 1 && warp >= 2 && warp < 6) fill_e4m3_rcp_table(rcp_tab, threadIdx.x - 64, 128);
   if (warp == 1 && has_lr) {
     tmem_alloc(tmem_holder, tmem_cols);
     tmem_relinquish();
@@ -251,6 +251,11 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
         sfw = 0;
 #pragma unroll
         for (int g = 0; g < 4; ++g) sfw |= quant16_nvfp4(v + 16 * g, out + 2 * g, rcp_tab) << (8 * g);
+      } else if constexpr (FMT == 2) {
+        // one scale per 32 values, stored in both 16-value slots of the atom
+        const uint32_t s0 = quant32_fp4(v, out, rcp_tab);
+        const uint32_t s1 = quant32_fp4(v + 32, out + 4, rcp_tab);
+        sfw = s0 * 0x0101u | (s1 * 0x0101u) << 16;
       } else {
         float amax = 0.0f;
 #pragma unroll
@@ -275,7 +280,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
       named_bar_sync(bar_free, 128);
       {
         const uint32_t row_addr = smem_u32(buf) + R * RB;
-        const uint32_t sw = FMT == 0 ? ((R >> 2) & 1u) : ((R >> 1) & 3u);
+        const uint32_t sw = FMT != 1 ? ((R >> 2) & 1u) : ((R >> 1) & 3u);
 #pragma unroll
         for (uint32_t c = 0; c < RB / 16; ++c)
           asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row_addr + ((c ^ sw) << 4)),
@@ -292,7 +297,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
         bulk_commit_group();
       }
       if (ok && col_ok) {
-        if constexpr (FMT == 0) {
+        if constexpr (FMT != 1) {
           // scale atom: 128 rows x 4 scales, byte (m % 32) * 16 + (m % 128 / 32) * 4 + k4
           uint8_t* atom = p.sf + (static_cast<size_t>(m / 128) * p.sf_kcols + kcol) * 512;
           *reinterpret_cast<uint32_t*>(atom + (m & 31) * 16 + ((m & 127) >> 5) * 4) = row_ok ? sfw : 0u;

@@ -28,6 +28,10 @@
 
 using namespace svdq;
 
+// E2M1 codes with E4M3 scales in the tcgen05 atom layout: NVFP4 (a scale per
+// 16 values) and FP4 g32 (a scale per 32, stored twice, once per 16).
+inline bool is_fp4(int fmt) { return fmt == SVDQ_NVFP4 || fmt == SVDQ_FP4G32; }
+
 struct svdq_weights {
   int device = 0;
   int fmt = 0, K = 0, N = 0, rank = 0, r_pad = 0;
@@ -153,6 +157,7 @@ int device_setup(int dev) {
       for (int f = 0; f < 2; ++f) qmax = std::max(qmax, quant_smem_layout(f, rp, S).total);
   SVDQ_CUDA(cudaFuncSetAttribute(quant_act_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, qmax));
   SVDQ_CUDA(cudaFuncSetAttribute(quant_act_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, qmax));
+  SVDQ_CUDA(cudaFuncSetAttribute(quant_act_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, qmax));
   SVDQ_CUDA(cudaFuncSetAttribute(gemm_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kGemmSmemBytes));
   SVDQ_CUDA(cudaFuncSetAttribute(gemm_int4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -189,9 +194,9 @@ ActLayout act_layout(const svdq_weights* w, int M) {
   ActLayout L;
   L.M = M;
   L.M_pad = round_up(std::max(M, 1), 128);
-  L.codes_bytes = w->fmt == SVDQ_NVFP4 ? static_cast<size_t>(M) * w->K / 2
+  L.codes_bytes = is_fp4(w->fmt) ? static_cast<size_t>(M) * w->K / 2
                                        : static_cast<size_t>(M) * w->K;
-  L.sf_bytes = w->fmt == SVDQ_NVFP4 ? static_cast<size_t>(L.M_pad / 128) * w->sf_kcols * 512
+  L.sf_bytes = is_fp4(w->fmt) ? static_cast<size_t>(L.M_pad / 128) * w->sf_kcols * 512
                                     : static_cast<size_t>(w->K / 64) * L.M_pad * 2;
   L.xl1_bytes = static_cast<size_t>(M) * 2 * w->r_pad * 2;   // bf16 hi | lo
   L.codes_off = 0;
@@ -205,7 +210,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 int encode_weight_maps(svdq_weights* w) {
   int rc;
-  if (w->fmt == SVDQ_NVFP4)
+  if (is_fp4(w->fmt))
     rc = make_map(&w->tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->wcodes, w->K / 2, w->N, 128, kGemmBN);
   else
     rc = make_map(&w->tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->wcodes, w->K, w->N, 64, kI4BN);
@@ -213,9 +218,9 @@ int encode_weight_maps(svdq_weights* w) {
   if (w->r_pad > 0) {
     rc = make_map(&w->tm_l1t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w->l1st, w->K, w->r_pad, 64, w->r_pad);
     if (rc) return rc;
-    const int lc = w->fmt == SVDQ_NVFP4 ? lr_chunk_cols(2 * w->r_pad) : i4_lr_chunk_cols(2 * w->r_pad);
+    const int lc = is_fp4(w->fmt) ? lr_chunk_cols(2 * w->r_pad) : i4_lr_chunk_cols(2 * w->r_pad);
     rc = make_map(&w->tm_l2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w->l2t2, 2 * w->r_pad, w->N, lc,
-                  w->fmt == SVDQ_NVFP4 ? kGemmBN : kI4BN);
+                  is_fp4(w->fmt) ? kGemmBN : kI4BN);
     if (rc) return rc;
   } else {
     w->tm_l1t = w->tm_b;
@@ -240,7 +245,7 @@ void free_weights(svdq_weights* w) {
 }
 
 int check_shape(int fmt, int K, int N, int rank) {
-  if (fmt != SVDQ_NVFP4 && fmt != SVDQ_INT4) return SVDQ_ERR_INVALID_ARG;
+  if (fmt != SVDQ_NVFP4 && fmt != SVDQ_INT4 && fmt != SVDQ_FP4G32) return SVDQ_ERR_INVALID_ARG;
   if (K <= 0 || N <= 0 || K % 64 != 0 || N % 16 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
   if (rank < 0 || rank > 256 || rank > std::min(K, N)) return SVDQ_ERR_UNSUPPORTED_SHAPE;
   return SVDQ_OK;
@@ -252,9 +257,9 @@ int alloc_weights(svdq_weights* w, cudaStream_t st) {
   w->N_pad = round_up(w->N, 256);
   w->sf_kcols = w->K_pad / 64;
   w->r_pad = rank_padded(w->rank);
-  const size_t codes = w->fmt == SVDQ_NVFP4 ? static_cast<size_t>(w->N) * w->K / 2
+  const size_t codes = is_fp4(w->fmt) ? static_cast<size_t>(w->N) * w->K / 2
                                             : static_cast<size_t>(w->N) * w->K;
-  const size_t sfb = w->fmt == SVDQ_NVFP4 ? static_cast<size_t>(w->N_pad / 128) * w->sf_kcols * 512
+  const size_t sfb = is_fp4(w->fmt) ? static_cast<size_t>(w->N_pad / 128) * w->sf_kcols * 512
                                           : static_cast<size_t>(w->K / 64) * w->N_pad * 2;
   // 1/lambda is read in 512-value blocks by the activation kernel: zero-pad it
   const size_t il_bytes = static_cast<size_t>(round_up(w->K, 512)) * sizeof(float);
@@ -286,6 +291,9 @@ int quantize_residual(svdq_weights* w, const float* R, cudaStream_t st) {
   if (w->fmt == SVDQ_NVFP4) {
     const dim3 grid((w->N + 127) / 128, w->K / 16);
     quant_weight_nvfp4_kernel<<<grid, blk, 0, st>>>(R, w->K, w->N, w->sf_kcols, w->wcodes, w->wsf);
+  } else if (w->fmt == SVDQ_FP4G32) {
+    const dim3 grid((w->N + 127) / 128, w->K / 32);
+    quant_weight_fp4g32_kernel<<<grid, blk, 0, st>>>(R, w->K, w->N, w->sf_kcols, w->wcodes, w->wsf);
   } else {
     const dim3 grid((w->N + 127) / 128, w->K / 64);
     quant_weight_int4_kernel<<<grid, blk, 0, st>>>(R, w->K, w->N, w->N_pad,
@@ -453,12 +461,12 @@ SVDQ_API const char* svdq_status_string(int s) {
 }
 
 SVDQ_API int svdq_tensor_peak(int fmt, long long steps, void* stream) {
-  if ((fmt != SVDQ_NVFP4 && fmt != SVDQ_INT4) || steps < 1) return SVDQ_ERR_INVALID_ARG;
+  if ((fmt != SVDQ_NVFP4 && fmt != SVDQ_INT4 && fmt != SVDQ_FP4G32) || steps < 1) return SVDQ_ERR_INVALID_ARG;
   int dev;
   int rc = current_device(&dev);
   if (rc) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (fmt == SVDQ_NVFP4)
+  if (is_fp4(fmt))
     tensor_peak_kernel<0><<<g_dev[dev].sms, kPeakThreads, kPeakSmemBytes, st>>>(steps, wait_budget());
   else
     tensor_peak_kernel<1><<<g_dev[dev].sms, kPeakThreads, kPeakSmemBytes, st>>>(steps, wait_budget());
@@ -677,9 +685,9 @@ SVDQ_API int svdq_quantize_act(const svdq_weights* w, const void* X, int M, void
   if ((rc = make_map(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, w->K, M, kQuantBK, BM)))
     return rc;
   // codes: NVFP4 M x K/2 packed E2M1, INT4 M x K int8; one box = one sub-tile's BM rows
-  const uint32_t rb = quant_code_row_bytes(w->fmt == SVDQ_NVFP4 ? 0 : 1);
+  const uint32_t rb = quant_code_row_bytes(is_fp4(w->fmt) ? 0 : 1);
   if ((rc = make_map(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base + L.codes_off,
-                     w->fmt == SVDQ_NVFP4 ? w->K / 2 : w->K, M, rb, BM)))
+                     is_fp4(w->fmt) ? w->K / 2 : w->K, M, rb, BM)))
     return rc;
   QuantParams p;
   p.M = M;
@@ -692,17 +700,19 @@ SVDQ_API int svdq_quantize_act(const svdq_weights* w, const void* X, int M, void
   p.sf = base + L.sf_off;
   p.xl1 = reinterpret_cast<__nv_bfloat16*>(base + L.xl1_off);
   p.budget = wait_budget();
-  if (w->fmt == SVDQ_NVFP4 && w->sf_kcols * 64 != w->K) {
+  if (is_fp4(w->fmt) && w->sf_kcols * 64 != w->K) {
     // zero the scale atoms of the K padding (read by the GEMM's last K step)
     const size_t pitch = static_cast<size_t>(w->sf_kcols) * 512;
     const size_t off = static_cast<size_t>(w->K / 64) * 512;
     SVDQ_CUDA(cudaMemset2DAsync(p.sf + off, pitch, 0, pitch - off, L.M_pad / 128, st));
   }
-  const QuantSmem Q = quant_smem_layout(w->fmt == SVDQ_NVFP4 ? 0 : 1, w->r_pad, S);
+  const QuantSmem Q = quant_smem_layout(is_fp4(w->fmt) ? 0 : 1, w->r_pad, S);
   const dim3 grid((M + BM - 1) / BM);
   const CUtensorMap& tm_l1t = w->r_pad > 0 ? w->tm_l1t : tm_x;
   if (w->fmt == SVDQ_NVFP4)
     quant_act_kernel<0><<<grid, kQuantThreads, Q.total, st>>>(tm_x, tm_l1t, tm_codes, p);
+  else if (w->fmt == SVDQ_FP4G32)
+    quant_act_kernel<2><<<grid, kQuantThreads, Q.total, st>>>(tm_x, tm_l1t, tm_codes, p);
   else
     quant_act_kernel<1><<<grid, kQuantThreads, Q.total, st>>>(tm_x, tm_l1t, tm_codes, p);
   SVDQ_CHECK_LAUNCH();
@@ -723,23 +733,23 @@ SVDQ_API int svdq_linear(const svdq_weights* w, const void* ws, int M, void* Y, 
   const uint8_t* base = static_cast<const uint8_t*>(ws);
   CUtensorMap tm_a, tm_xl1;
   const int m_tiles = L.M_pad / 128;
-  const int n_tiles = w->fmt == SVDQ_NVFP4 ? (w->N + kGemmBN - 1) / kGemmBN : (w->N + kI4BN - 1) / kI4BN;
+  const int n_tiles = is_fp4(w->fmt) ? (w->N + kGemmBN - 1) / kGemmBN : (w->N + kI4BN - 1) / kI4BN;
   const int tiles = m_tiles * n_tiles;
   const int grid = std::min(tiles, g_dev[dev].sms);
-  if (w->fmt == SVDQ_NVFP4)
+  if (is_fp4(w->fmt))
     rc = make_map(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base + L.codes_off, w->K / 2, M, 128, kGemmBM);
   else
     rc = make_map(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base + L.codes_off, w->K, M, 64, kI4BM);
   if (rc) return rc;
   if (w->r_pad > 0) {
     if ((rc = make_map(&tm_xl1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base + L.xl1_off, 2 * w->r_pad, M,
-                       w->fmt == SVDQ_NVFP4 ? lr_chunk_cols(2 * w->r_pad) : i4_lr_chunk_cols(2 * w->r_pad),
+                       is_fp4(w->fmt) ? lr_chunk_cols(2 * w->r_pad) : i4_lr_chunk_cols(2 * w->r_pad),
                        128)))
       return rc;
   } else {
     tm_xl1 = tm_a;
   }
-  if (w->fmt == SVDQ_NVFP4) {
+  if (is_fp4(w->fmt)) {
     CUtensorMap tm_y;
     if ((rc = make_map(&tm_y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Y, w->N, M, 16, 32))) return rc;
     GemmParams p;
@@ -841,7 +851,7 @@ SVDQ_API int svdq_export_act(const svdq_weights* w, const void* ws, int M, uint8
   const uint8_t* base = static_cast<const uint8_t*>(ws);
   const int K = w->K;
   if (codes) {
-    if (w->fmt == SVDQ_NVFP4) {
+    if (is_fp4(w->fmt)) {
       SVDQ_CUDA(cudaMemcpy(codes, base + L.codes_off, L.codes_bytes, cudaMemcpyDeviceToHost));
     } else {
       std::vector<int8_t> tmp(L.codes_bytes);
@@ -853,13 +863,16 @@ SVDQ_API int svdq_export_act(const svdq_weights* w, const void* ws, int M, uint8
   if (scales) {
     std::vector<uint8_t> tmp(L.sf_bytes);
     SVDQ_CUDA(cudaMemcpy(tmp.data(), base + L.sf_off, L.sf_bytes, cudaMemcpyDeviceToHost));
-    if (w->fmt == SVDQ_NVFP4) {
+    if (is_fp4(w->fmt)) {
+      // plain [M][K/g] from the atoms (FP4 g32: the first of each stored pair)
       uint8_t* out = static_cast<uint8_t*>(scales);
-      const int G = K / 16;
+      const int step = w->fmt == SVDQ_FP4G32 ? 2 : 1;
+      const int G = K / (16 * step);
       for (int m = 0; m < M; ++m)
         for (int g = 0; g < G; ++g) {
-          const size_t atom = (static_cast<size_t>(m / 128) * w->sf_kcols + g / 4) * 512;
-          out[static_cast<size_t>(m) * G + g] = tmp[atom + (m % 32) * 16 + ((m % 128) / 32) * 4 + g % 4];
+          const int b = g * step;   // block of 16
+          const size_t atom = (static_cast<size_t>(m / 128) * w->sf_kcols + b / 4) * 512;
+          out[static_cast<size_t>(m) * G + g] = tmp[atom + (m % 32) * 16 + ((m % 128) / 32) * 4 + b % 4];
         }
     } else {
       uint16_t* out = static_cast<uint16_t*>(scales);
@@ -895,7 +908,7 @@ SVDQ_API int svdq_export_weights(const svdq_weights* w, uint8_t* codes, void* sc
   SVDQ_CUDA(cudaDeviceSynchronize());
   const int K = w->K, N = w->N;
   if (codes) {
-    if (w->fmt == SVDQ_NVFP4) {
+    if (is_fp4(w->fmt)) {
       SVDQ_CUDA(cudaMemcpy(codes, w->wcodes, static_cast<size_t>(N) * K / 2, cudaMemcpyDeviceToHost));
     } else {
       std::vector<int8_t> tmp(static_cast<size_t>(N) * K);
@@ -905,16 +918,18 @@ SVDQ_API int svdq_export_weights(const svdq_weights* w, uint8_t* codes, void* sc
     }
   }
   if (scales) {
-    if (w->fmt == SVDQ_NVFP4) {
+    if (is_fp4(w->fmt)) {
       const size_t bytes = static_cast<size_t>(w->N_pad / 128) * w->sf_kcols * 512;
       std::vector<uint8_t> tmp(bytes);
       SVDQ_CUDA(cudaMemcpy(tmp.data(), w->wsf, bytes, cudaMemcpyDeviceToHost));
       uint8_t* out = static_cast<uint8_t*>(scales);
-      const int G = K / 16;
+      const int step = w->fmt == SVDQ_FP4G32 ? 2 : 1;
+      const int G = K / (16 * step);
       for (int n = 0; n < N; ++n)
         for (int g = 0; g < G; ++g) {
-          const size_t atom = (static_cast<size_t>(n / 128) * w->sf_kcols + g / 4) * 512;
-          out[static_cast<size_t>(n) * G + g] = tmp[atom + (n % 32) * 16 + ((n % 128) / 32) * 4 + g % 4];
+          const int b = g * step;   // block of 16
+          const size_t atom = (static_cast<size_t>(n / 128) * w->sf_kcols + b / 4) * 512;
+          out[static_cast<size_t>(n) * G + g] = tmp[atom + (n % 32) * 16 + ((n % 128) / 32) * 4 + b % 4];
         }
     } else {
       const int G = K / 64;

@@ -123,6 +123,26 @@ __device__ __forceinline__ uint32_t quant16_nvfp4(const float* v, uint32_t* code
   return s8;
 }
 
+// FP4 group of 32 values (one E4M3 scale for all 32): writes 16 code bytes
+// into codes[0..3] and returns the E4M3 scale code.
+__device__ __forceinline__ uint32_t quant32_fp4(const float* v, uint32_t* codes,
+                                                const float* rcp_tab) {
+  const float s32 = div6_rn(fmaxf(absmax16(v), absmax16(v + 16)));
+  const uint32_t s8 = e4m3_code(s32);
+  const float inv = rcp_tab[s8];
+  float q[32];
+  const float2 i2 = make_float2(inv, inv);
+#pragma unroll
+  for (int i = 0; i < 32; i += 2) {
+    const float2 r = fmul2_rn(make_float2(v[i], v[i + 1]), i2);
+    q[i] = r.x;
+    q[i + 1] = r.y;
+  }
+#pragma unroll
+  for (int w = 0; w < 4; ++w) codes[w] = inv == 0.0f ? 0u : e2m1_pack8(q + 8 * w);   // zero scale: zero codes
+  return s8;
+}
+
 // Fill a 128-entry table with RN(1 / E4M3 value) for codes 0..127 (code 0 -> 0,
 // NaN code 0x7F -> 0; scales never take it: they saturate at 448).
 __device__ __forceinline__ void fill_e4m3_rcp_table(float* tab, int tid, int nthreads) {
