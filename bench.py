@@ -219,6 +219,40 @@ def time_layer(S, w, X, ws, Y, M, flush, stream, steps, warmup, world, sampler=N
     return t_q, t_g, clocks
 
 
+def unfused_foil(S, w, w0, X, ws, Y, M, flush, stream, steps, warmup):
+    """Seconds per step of the low-rank branch run unfused: the 4-bit layer at
+    rank 0 (w0), then the smoothing pass X_hat = X / lambda, X_hat L1 and
+    (X_hat L1) L2 as separate cuBLAS bf16 GEMMs and an addition into Y.  A
+    comparison point for the fused kernels, not part of the product."""
+    e = S.svdq_export_weights(w)
+    dev = X.device
+    bf = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+    L1 = bf(e["L1"])                              # K x r
+    L2 = bf(e["L2"])                              # r x N
+    inv = torch.from_numpy(e["inv_lambda"]).to(dev).to(torch.bfloat16)
+
+    def step():
+        S.svdq_quantize_act(w0, X, ws)
+        S.svdq_linear(w0, ws, M, Y)
+        xh = X * inv                                # one bf16 pass over X
+        Y.addmm_(torch.matmul(xh, L1), L2)          # Y += (X_hat L1) L2, one pass over Y
+
+    for _ in range(warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        step()
+        b.record(stream)
+        ts.append((a, b))
+    torch.cuda.synchronize()
+    return float(np.mean([a.elapsed_time(b) for a, b in ts])) * 1e-3
+
+
 def tensor_ceiling(S, fmt, stream):
     """The tensor cores' own ceiling for the GEMM's instruction (no global
     traffic): a ~5 ms burst and a ~1 s sustained run, in TFLOP/s."""
@@ -345,6 +379,7 @@ def run_ours(args):
         w0 = S.svdq_prepare_weights(W, 0, spec.fmt, x_absmax=xabs,
                                     bias=bias.to(dev) if bias is not None else None)
         q0, g0, _ = time_layer(S, w0, X, ws, Y, M, flush, stream, args.steps, args.warmup, world)
+        t_unf = unfused_foil(S, w, w0, X, ws, Y, M, flush, stream, args.steps, args.warmup) if r else None
         w0.close()
         l0 = float(q0.mean() + g0.mean())
         line["lowrank_overhead"] = {
@@ -353,6 +388,24 @@ def run_ours(args):
             "layer": round(total / args.steps / l0 - 1.0, 4),
             "gemm": round(tg_mean / float(g0.mean()) - 1.0, 4), "target": 0.15,
             "what": f"us(rank {r}) / us(rank 0) - 1, same format, shapes, smoothing and bias"}
+        if t_unf is not None:
+            line["lowrank_overhead"]["unfused_foil"] = {
+                "us_layer": round(t_unf * 1e6, 2), "layer": round(t_unf / l0 - 1.0, 4),
+                "what": "rank-0 layer, then smoothing, X_hat L1 and (X_hat L1) L2 as separate cuBLAS bf16 "
+                        "GEMMs and an addition into Y (the unfused design the fused kernels replace)"}
+        if args.rank_sweep:
+            sweep = []
+            for rr in args.rank_sweep:
+                wr = S.svdq_prepare_weights(W, rr, spec.fmt, x_absmax=xabs,
+                                            bias=bias.to(dev) if bias is not None else None)
+                wsr = S.alloc_workspace(wr, M, dev)   # X_hat L1 grows with the rank
+                qr, gr, _ = time_layer(S, wr, X, wsr, Y, M, flush, stream, args.steps, args.warmup, world)
+                del wsr
+                wr.close()
+                lr = float(qr.mean() + gr.mean())
+                sweep.append({"rank": rr, "us_layer": round(lr * 1e6, 2), "us_quant": round(float(qr.mean()) * 1e6, 2),
+                              "us_gemm": round(float(gr.mean()) * 1e6, 2), "overhead": round(lr / l0 - 1.0, 4)})
+            line["rank_sweep"] = sweep
         ceil = tensor_ceiling(S, spec.fmt, stream)
         ceil["gemm_frac_of_burst"] = round(achieved / ceil["burst"], 4)
         ceil["gemm_frac_of_sustained"] = round(achieved / ceil["sustained"], 4)
@@ -441,6 +494,8 @@ def main():
                     help="override the workload's 4-bit format")
     ap.add_argument("--cpu-rows", type=int, default=64)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--rank-sweep", type=lambda v: [int(x) for x in v.split(",")], default=None,
+                    help="also time the layer at these ranks, e.g. 16,32,48,64")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the rank-0 comparison and the tensor-ceiling measurement")
     args = ap.parse_args()
