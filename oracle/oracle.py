@@ -223,9 +223,19 @@ def _top_factors_gram(W_hat: np.ndarray, r: int):
     return L1, L2, S
 
 
+def weight_error(fmt, W_hat: np.ndarray, L1_bits: np.ndarray, L2_bits: np.ndarray, R: np.ndarray):
+    """||W_hat - L1 L2 - deq(Q(R))||_F in fp64 for bf16 factors and the fp32
+    residual R (K x N), and the dequantized Q(R) (K x N)."""
+    codes, scales = weight_quant(fmt, R)
+    Rq = dequant(fmt, codes, scales).T.astype(np.float64)
+    LL = bf16_decode(L1_bits).astype(np.float64) @ bf16_decode(L2_bits).astype(np.float64)
+    return float(np.linalg.norm(W_hat - LL - Rq)), Rq
+
+
 def prepare(W_bits: np.ndarray, x_absmax: Optional[np.ndarray], rank: int,
             lora_A_bits: Optional[np.ndarray] = None,
-            lora_B_bits: Optional[np.ndarray] = None, svd: str = "full") -> dict:
+            lora_B_bits: Optional[np.ndarray] = None, svd: str = "full",
+            refine_fmt=None, refine_iters: int = 0) -> dict:
     """Smoothing, truncated SVD, residual and optional LoRA fold, in fp64.
 
     W_hat = diag(lambda) W; W_hat = U S V^T (numpy/LAPACK fp64);
@@ -238,6 +248,13 @@ def prepare(W_bits: np.ndarray, x_absmax: Optional[np.ndarray], rank: int,
     svd="gram" takes the top-r factors from the Gram matrix instead of a full
     SVD (for layers of FLUX size, where the full SVD takes minutes); "sigma"
     then holds the square roots of the Gram eigenvalues.
+
+    refine_iters > 0 runs the iterative update of the low-rank branch (Sec. 4.2,
+    last paragraph): decompose the part of W_hat the quantized residual misses,
+    E = W_hat - deq(Q(R)), into its rank-r factors, take R = W_hat - L1 L2 again,
+    quantize it in `refine_fmt`, repeat, and keep the iterate (the SVD start
+    included) with the smallest ||W_hat - L1 L2 - deq(Q(R))||_F; the errors of
+    all iterates are returned in "refine_errors".
     """
     W = bf16_decode(W_bits).astype(np.float64)
     K, N = W.shape
@@ -254,9 +271,28 @@ def prepare(W_bits: np.ndarray, x_absmax: Optional[np.ndarray], rank: int,
     L2 = bf16_round(L2_exact)
     R64 = W_hat - bf16_decode(L1).astype(np.float64) @ bf16_decode(L2).astype(np.float64)
     R = R64.astype(np.float32)
+    refine_errors = None
+    if refine_iters and r:
+        err, Rq = weight_error(refine_fmt, W_hat, L1, L2, R)
+        refine_errors = [err]
+        best = (err, L1, L2, R, L1_exact, L2_exact)
+        for _ in range(int(refine_iters)):
+            E = W_hat - Rq
+            if svd == "gram":
+                L1_exact, L2_exact, _ = _top_factors_gram(E, r)
+            else:
+                U, Se, Vt = np.linalg.svd(E, full_matrices=False)
+                L1_exact, L2_exact = U[:, :r] * Se[:r], Vt[:r, :]
+            L1, L2 = bf16_round(L1_exact), bf16_round(L2_exact)
+            R = (W_hat - bf16_decode(L1).astype(np.float64) @ bf16_decode(L2).astype(np.float64)).astype(np.float32)
+            err, Rq = weight_error(refine_fmt, W_hat, L1, L2, R)
+            refine_errors.append(err)
+            if err < best[0]:
+                best = (err, L1, L2, R, L1_exact, L2_exact)
+        _, L1, L2, R, L1_exact, L2_exact = best
     out = {"lam": lam, "inv_lambda": inv, "W_hat": W_hat, "sigma": S,
            "L1_exact": L1_exact, "L2_exact": L2_exact, "L1": L1, "L2": L2, "R": R,
-           "rank": r}
+           "rank": r, "refine_errors": refine_errors}
     if lora_A_bits is not None:
         A = bf16_decode(lora_A_bits).astype(np.float64)
         L1_lora = bf16_round(lam.astype(np.float64)[:, None] * A)

@@ -250,3 +250,27 @@ def test_gram_route_spans_the_svd_subspace(K, N):
     Ra = a["R"].astype(np.float64)
     Rb = b["R"].astype(np.float64)
     assert np.linalg.norm(Ra - Rb) <= 2.0 ** -7 * np.linalg.norm(pa)
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4", "fp4g32"])
+def test_iterative_refinement_keeps_the_best_iterate(fmt):
+    """Sec. 4.2, last paragraph: re-decomposing W_hat - deq(Q(R)) and requantizing
+    lowers the weight error on outlier-heavy weights; the returned parts are the
+    iterate with the smallest error, and they keep the residual convention."""
+    d = WL.make_small(64, 256, 192, w_outlier_rows=6, seed=11)
+    Wb = WL.bf16_bits(d["W"])
+    xm = O.calib_absmax(WL.bf16_bits(d["X"]))
+    plain = O.prepare(Wb, xm, 16)
+    none = O.prepare(Wb, xm, 16, refine_fmt=fmt, refine_iters=0)
+    assert none["refine_errors"] is None
+    assert np.array_equal(none["L1"], plain["L1"]) and np.array_equal(none["R"], plain["R"])
+    ref = O.prepare(Wb, xm, 16, refine_fmt=fmt, refine_iters=4)
+    errs = ref["refine_errors"]
+    assert len(errs) == 5
+    e0, _ = O.weight_error(fmt, plain["W_hat"], plain["L1"], plain["L2"], plain["R"])
+    assert errs[0] == pytest.approx(e0, rel=1e-12)
+    got, _ = O.weight_error(fmt, ref["W_hat"], ref["L1"], ref["L2"], ref["R"])
+    assert got == pytest.approx(min(errs), rel=1e-12)
+    assert min(errs) < 0.97 * errs[0]
+    R64 = ref["W_hat"] - O.bf16_decode(ref["L1"]).astype(np.float64) @ O.bf16_decode(ref["L2"]).astype(np.float64)
+    assert np.array_equal(ref["R"], R64.astype(np.float32))
