@@ -76,6 +76,7 @@ typedef struct {
   const void* lora_A;      /* bf16 K x lora_rank, or NULL */
   const void* lora_B;      /* bf16 lora_rank x N, or NULL */
   int lora_rank;           /* 0 = no LoRA */
+  int refine_iters;        /* iterative updates of the low-rank branch (Sec. 4.2), 0 = none */
 } svdq_prepare_desc;
 
 /* Inputs of svdq_load_weights: an already decomposed layer (device pointers). */
@@ -100,8 +101,13 @@ SVDQ_API int svdq_calib_absmax(const void* X, int M, int K, float* absmax, int a
  * max|W_j|) (fp64, rounded to fp32); W_hat = diag(lambda) W; the optimal
  * rank-r factors from the eigen-decomposition of the fp64 Gram matrix of
  * W_hat (cuSOLVER), rounded to bf16; R = W_hat - L1 L2; Q(R); optional LoRA
- * folded into the branch without requantizing R.  Allocates device memory
- * (SVDQ_ERR_ALLOC) and synchronizes `stream`.  *out receives a new handle. */
+ * folded into the branch without requantizing R.  With refine_iters = T > 0
+ * the branch is updated T times (Sec. 4.2, last paragraph): the rank-r factors
+ * of E = W_hat - deq(Q(R)) replace L1, L2, R = W_hat - L1 L2 is requantized,
+ * and the iterate (the SVD start included) with the smallest
+ * ||W_hat - L1 L2 - deq(Q(R))||_F is kept (before any LoRA is folded in).
+ * Allocates device memory (SVDQ_ERR_ALLOC) and synchronizes `stream`.
+ * *out receives a new handle. */
 SVDQ_API int svdq_prepare_weights(const svdq_prepare_desc* desc, void* stream,
                                   svdq_weights** out);
 
@@ -115,6 +121,10 @@ SVDQ_API int svdq_load_weights(const svdq_parts_desc* desc, void* stream, svdq_w
  * The 4-bit residual codes are not touched.  Synchronizes `stream`. */
 SVDQ_API int svdq_append_lora(svdq_weights* w, const void* lora_A, const void* lora_B,
                               int lora_rank, void* stream);
+
+/* Weight error ||W_hat - L1 L2 - deq(Q(R))||_F of the SVD start and of the
+ * kept iterate of svdq_prepare_weights' refinement (both -1 without it). */
+SVDQ_API int svdq_weights_refine_error(const svdq_weights* w, double* initial, double* kept);
 
 /* Shape of a handle; any output pointer may be NULL. */
 SVDQ_API int svdq_weights_info(const svdq_weights* w, int* fmt, int* K, int* N, int* rank,

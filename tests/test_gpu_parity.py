@@ -176,3 +176,32 @@ def test_empty_batch_is_a_noop(S):
     X = torch.empty(0, 256, dtype=torch.bfloat16, device="cuda")
     Y = S.svdq_forward(w, X)
     assert Y.shape == (0, 256)
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4", "fp4g32"])
+def test_prepare_refinement(S, fmt):
+    """Iterative refinement of the branch in svdq_prepare_weights: the kept
+    error is what the exported parts give, it drops below the SVD start, and
+    both ends agree with the oracle's refinement of the same layer."""
+    M, K, N, r = 128, 256, 192, 16
+    data = WL.make_small(M, K, N, w_outlier_rows=6, seed=11)
+    Xb, Wb = WL.bf16_bits(data["X"]), WL.bf16_bits(data["W"])
+    xm = O.calib_absmax(Xb)
+    ora = O.prepare(Wb, xm, r, refine_fmt=fmt, refine_iters=4)
+    w = S.svdq_prepare_weights(data["W"].cuda(), r, fmt, x_absmax=S.svdq_calib_absmax(data["X"].cuda()),
+                               refine_iters=4)
+    e0, kept = S.svdq_weights_refine_error(w)
+    e = S.svdq_export_weights(w)
+    What = ora["W_hat"]
+    LL = O.bf16_decode(e["L1"]).astype(np.float64) @ O.bf16_decode(e["L2"]).astype(np.float64)
+    Rq = O.dequant(fmt, e["codes"], e["scales"]).T.astype(np.float64)
+    assert np.linalg.norm(What - LL - Rq) == pytest.approx(kept, rel=1e-9)
+    assert kept <= e0 and kept < 0.97 * e0
+    errs = ora["refine_errors"]
+    assert e0 == pytest.approx(errs[0], rel=0.02)
+    assert kept == pytest.approx(min(errs), rel=0.03)
+    # the exported codes are the oracle quantizer's codes of the kept residual
+    R = (What - LL).astype(np.float32)
+    codes, scales = O.weight_quant(fmt, R)
+    assert np.array_equal(scales, e["scales"]) and np.array_equal(codes, e["codes"])
+    w.close()

@@ -27,7 +27,7 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "device all
           4: "CUDA error", 5: "device wait timed out", 6: "cuSOLVER/cuBLAS error"}
 
 EXPORTED = ("svdq_calib_absmax", "svdq_prepare_weights", "svdq_load_weights", "svdq_append_lora",
-            "svdq_weights_info", "svdq_act_workspace_bytes", "svdq_quantize_act", "svdq_linear",
+            "svdq_weights_info", "svdq_weights_refine_error", "svdq_act_workspace_bytes", "svdq_quantize_act", "svdq_linear",
             "svdq_forward", "svdq_forward_noalloc", "svdq_export_act", "svdq_export_weights", "svdq_get_error",
             "svdq_set_wait_budget", "svdq_status_string", "svdq_tensor_peak", "svdq_weights_destroy")
 
@@ -42,7 +42,8 @@ class _PrepareDesc(ctypes.Structure):
     _fields_ = [("fmt", ctypes.c_int), ("K", ctypes.c_int), ("N", ctypes.c_int),
                 ("rank", ctypes.c_int), ("W", ctypes.c_void_p), ("x_absmax", ctypes.c_void_p),
                 ("bias", ctypes.c_void_p), ("lora_A", ctypes.c_void_p),
-                ("lora_B", ctypes.c_void_p), ("lora_rank", ctypes.c_int)]
+                ("lora_B", ctypes.c_void_p), ("lora_rank", ctypes.c_int),
+                ("refine_iters", ctypes.c_int)]
 
 
 class _PartsDesc(ctypes.Structure):
@@ -69,6 +70,7 @@ def lib() -> ctypes.CDLL:
     L.svdq_load_weights.argtypes = [ctypes.POINTER(_PartsDesc), P, ctypes.POINTER(P)]
     L.svdq_append_lora.argtypes = [P, P, P, I, P]
     L.svdq_weights_info.argtypes = [P] + [ctypes.POINTER(I)] * 5
+    L.svdq_weights_refine_error.argtypes = [P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)]
     L.svdq_act_workspace_bytes.argtypes = [P, I, ctypes.POINTER(ctypes.c_size_t)]
     L.svdq_quantize_act.argtypes = [P, P, I, P, P]
     L.svdq_linear.argtypes = [P, P, I, P, P]
@@ -160,7 +162,8 @@ def svdq_calib_absmax(X: torch.Tensor, out: Optional[torch.Tensor] = None, accum
 
 def svdq_prepare_weights(W: torch.Tensor, rank: int, fmt="nvfp4", x_absmax: Optional[torch.Tensor] = None,
                          bias: Optional[torch.Tensor] = None, lora_A: Optional[torch.Tensor] = None,
-                         lora_B: Optional[torch.Tensor] = None, stream=None) -> Weights:
+                         lora_B: Optional[torch.Tensor] = None, refine_iters: int = 0,
+                         stream=None) -> Weights:
     _dev(W, torch.bfloat16, "W")
     K, N = W.shape
     if x_absmax is not None:
@@ -176,7 +179,7 @@ def svdq_prepare_weights(W: torch.Tensor, rank: int, fmt="nvfp4", x_absmax: Opti
                      x_absmax.data_ptr() if x_absmax is not None else None,
                      bias.data_ptr() if bias is not None else None,
                      lora_A.data_ptr() if lora_A is not None else None,
-                     lora_B.data_ptr() if lora_B is not None else None, rl)
+                     lora_B.data_ptr() if lora_B is not None else None, rl, int(refine_iters))
     h = ctypes.c_void_p()
     _check(lib().svdq_prepare_weights(ctypes.byref(d), _stream(stream), ctypes.byref(h)),
            "svdq_prepare_weights")
@@ -301,6 +304,14 @@ def svdq_export_weights(w: Weights) -> dict:
 
 def svdq_get_error() -> int:
     return int(lib().svdq_get_error())
+
+
+def svdq_weights_refine_error(w: "Weights"):
+    """(initial, kept) weight error of the refinement, -1 where none ran."""
+    a, b = ctypes.c_double(), ctypes.c_double()
+    _check(lib().svdq_weights_refine_error(w.handle, ctypes.byref(a), ctypes.byref(b)),
+           "svdq_weights_refine_error")
+    return a.value, b.value
 
 
 def svdq_tensor_peak(fmt: str, steps: int, stream=None):

@@ -242,29 +242,6 @@ __global__ void residual_kernel(const double* __restrict__ What,
 // NVFP4: one thread per (n, group of 16): codes N x K/2, scales in 512-byte atoms
 //        (128 columns x 4 groups; byte (n % 32) * 16 + (n % 128 / 32) * 4 + g % 4).
 // INT4 : one thread per (n, group of 64): int8 codes N x K, fp16 scales [K/64][N_pad].
-// FP4 g32: one E4M3 scale per 32 values of K, stored in both 16-value slots of
-// the scale atom so the NVFP4 GEMM (block16) applies it to both halves.
-__global__ void quant_weight_fp4g32_kernel(const float* __restrict__ R, int K, int N, int sf_kcols,
-                                           uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
-  __shared__ float rcp_tab[128];
-  fill_e4m3_rcp_table(rcp_tab, threadIdx.x, blockDim.x);
-  __syncthreads();
-  const int n = blockIdx.x * blockDim.x + threadIdx.x;
-  const int g = blockIdx.y;                  // group of 32
-  if (n >= N) return;
-  float v[32];
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = R[static_cast<size_t>(32 * g + i) * N + n];
-  uint32_t cw[4];
-  const uint32_t s8 = quant32_fp4(v, cw, rcp_tab);
-  uint4* dst = reinterpret_cast<uint4*>(codes + static_cast<size_t>(n) * (K / 2) + 16 * g);
-  *dst = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-  uint8_t* atom = sf + (static_cast<size_t>(n / 128) * sf_kcols + g / 2) * 512;
-  uint8_t* slot = atom + (n & 31) * 16 + ((n & 127) >> 5) * 4 + 2 * (g & 1);
-  slot[0] = static_cast<uint8_t>(s8);
-  slot[1] = static_cast<uint8_t>(s8);
-}
-
 __global__ void quant_weight_nvfp4_kernel(const float* __restrict__ R, int K, int N, int sf_kcols,
                                           uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
   __shared__ float rcp_tab[128];
@@ -303,6 +280,95 @@ __global__ void quant_weight_int4_kernel(const float* __restrict__ R, int K, int
   }
   sf[static_cast<size_t>(g) * N_pad + n] = sh;
   sf32[static_cast<size_t>(g) * N_pad + n] = sd;   // exact: every fp16 value is an fp32 value
+}
+
+// FP4 g32: one E4M3 scale per 32 values of K, stored in both 16-value slots of
+// the scale atom so the NVFP4 GEMM (block16) applies it to both halves.
+__global__ void quant_weight_fp4g32_kernel(const float* __restrict__ R, int K, int N, int sf_kcols,
+                                           uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
+  __shared__ float rcp_tab[128];
+  fill_e4m3_rcp_table(rcp_tab, threadIdx.x, blockDim.x);
+  __syncthreads();
+  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  const int g = blockIdx.y;                  // group of 32
+  if (n >= N) return;
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = R[static_cast<size_t>(32 * g + i) * N + n];
+  uint32_t cw[4];
+  const uint32_t s8 = quant32_fp4(v, cw, rcp_tab);
+  uint4* dst = reinterpret_cast<uint4*>(codes + static_cast<size_t>(n) * (K / 2) + 16 * g);
+  *dst = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+  uint8_t* atom = sf + (static_cast<size_t>(n / 128) * sf_kcols + g / 2) * 512;
+  uint8_t* slot = atom + (n & 31) * 16 + ((n & 127) >> 5) * 4 + 2 * (g & 1);
+  slot[0] = static_cast<uint8_t>(s8);
+  slot[1] = static_cast<uint8_t>(s8);
+}
+
+// ------------------------------------------------------------ refinement ---
+// Iterative update of the low-rank branch (SVDQuant paper, Sec. 4.2, last
+// paragraph): the part of W_hat the quantized residual misses,
+// E = W_hat - deq(Q(R)), is decomposed again, and the iterate with the
+// smallest ||W_hat - L1 L2 - deq(Q(R))||_F is kept.
+
+// deq(Q(R))[k, n] from the handle's codes and scales (fmt: 0 NVFP4, 1 INT4,
+// 2 FP4 g32 -- whose scale sits in both 16-value slots, so the block-of-16
+// lookup serves it too).
+__device__ __forceinline__ double deq_weight(int fmt, const uint8_t* __restrict__ codes,
+                                             const uint8_t* __restrict__ sf,
+                                             const float* __restrict__ sf32, int K, int N_pad,
+                                             int sf_kcols, int k, int n) {
+  if (fmt == 1) {
+    const int8_t q = reinterpret_cast<const int8_t*>(codes)[static_cast<size_t>(n) * K + k];
+    return static_cast<double>(q) * static_cast<double>(sf32[static_cast<size_t>(k / 64) * N_pad + n]);
+  }
+  const uint8_t b = codes[static_cast<size_t>(n) * (K / 2) + k / 2];
+  const uint32_t c = (k & 1) ? (b >> 4) : (b & 15u);
+  const int g = k / 16;
+  const uint8_t s8 = sf[(static_cast<size_t>(n / 128) * sf_kcols + g / 4) * 512 + (n & 31) * 16 +
+                        ((n & 127) >> 5) * 4 + (g & 3)];
+  return static_cast<double>(e2m1_value(c)) * static_cast<double>(e4m3_value(s8));
+}
+
+// E = W_hat - deq(Q(R)), fp64 K x N.
+__global__ void refine_target_kernel(const double* __restrict__ What, int fmt,
+                                     const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sf,
+                                     const float* __restrict__ sf32, int K, int N, int N_pad,
+                                     int sf_kcols, double* __restrict__ E) {
+  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  const int k = blockIdx.y;
+  if (n >= N) return;
+  const size_t i = static_cast<size_t>(k) * N + n;
+  E[i] = What[i] - deq_weight(fmt, codes, sf, sf32, K, N_pad, sf_kcols, k, n);
+}
+
+// *sum += sum over the block's elements of (W_hat - L1 L2 - deq(Q(R)))^2, fp64.
+__global__ void refine_error_kernel(const double* __restrict__ What,
+                                    const __nv_bfloat16* __restrict__ l1t,
+                                    const __nv_bfloat16* __restrict__ l2t, int r, int r_pad, int fmt,
+                                    const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sf,
+                                    const float* __restrict__ sf32, int K, int N, int N_pad,
+                                    int sf_kcols, double* __restrict__ sum) {
+  __shared__ double part[8];
+  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  const int k = blockIdx.y;
+  double d2 = 0.0;
+  if (n < N) {
+    double acc = What[static_cast<size_t>(k) * N + n];
+    for (int j = 0; j < r; ++j)
+      acc -= static_cast<double>(__bfloat162float(l1t[static_cast<size_t>(j) * K + k])) *
+             static_cast<double>(__bfloat162float(l2t[static_cast<size_t>(n) * r_pad + j]));
+    acc -= deq_weight(fmt, codes, sf, sf32, K, N_pad, sf_kcols, k, n);
+    d2 = acc * acc;
+  }
+  for (int o = 16; o > 0; o >>= 1) d2 += __shfl_xor_sync(0xffffffffu, d2, o);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = d2;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) t += part[w];
+    atomicAdd(sum, t);
+  }
 }
 
 }  // namespace svdq

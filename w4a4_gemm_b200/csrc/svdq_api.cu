@@ -49,6 +49,7 @@ struct svdq_weights {
   __nv_bfloat16* l2t2 = nullptr; // N x 2 r_pad: [L2^T | L2^T], the tail MMA's B operand
   __nv_bfloat16* bias = nullptr;
   CUtensorMap tm_b, tm_l1t, tm_l2t;
+  double refine_err0 = -1.0, refine_err = -1.0;   // weight error: SVD start, kept iterate
 };
 
 namespace {
@@ -442,6 +443,71 @@ int lowrank_factors(svdq_weights* w, const double* What, cudaStream_t st) {
   return rc;
 }
 
+// ||W_hat - L1 L2 - deq(Q(R))||_F of the handle's current branch and codes.
+int weight_error(svdq_weights* w, const double* What, double* err_dev, double* out, cudaStream_t st) {
+  SVDQ_CUDA(cudaMemsetAsync(err_dev, 0, sizeof(double), st));
+  refine_error_kernel<<<dim3((w->N + 255) / 256, w->K), 256, 0, st>>>(
+      What, w->l1t, w->l2t, w->rank, w->r_pad, w->fmt, w->wcodes, w->wsf, w->wsf32, w->K, w->N,
+      w->N_pad, w->sf_kcols, err_dev);
+  SVDQ_CHECK_LAUNCH();
+  double h = 0.0;
+  SVDQ_CUDA(cudaMemcpyAsync(&h, err_dev, sizeof(double), cudaMemcpyDeviceToHost, st));
+  SVDQ_CUDA(cudaStreamSynchronize(st));
+  *out = std::sqrt(h);
+  return SVDQ_OK;
+}
+
+// Iterative update of the low-rank branch (SVDQuant paper, Sec. 4.2, last
+// paragraph): iters times, factor E = W_hat - deq(Q(R)), R = W_hat - L1 L2,
+// requantize; keep the iterate with the smallest weight error.  R is scratch.
+int refine_branch(svdq_weights* w, const double* What, float* R, int iters, cudaStream_t st) {
+  const size_t KN = static_cast<size_t>(w->K) * w->N;
+  const size_t l1b = static_cast<size_t>(w->r_pad) * w->K * 2, l2b = static_cast<size_t>(w->N) * w->r_pad * 2;
+  const size_t cb = w->fmt == SVDQ_INT4 ? KN : KN / 2;
+  const size_t sfb = w->fmt == SVDQ_INT4 ? static_cast<size_t>(w->K / 64) * w->N_pad * 2
+                                         : static_cast<size_t>(w->N_pad / 128) * w->sf_kcols * 512;
+  const size_t sf32b = w->fmt == SVDQ_INT4 ? static_cast<size_t>(w->K / 64) * w->N_pad * 4 : 0;
+  DeviceBuf E, err, b_l1, b_l2, b_codes, b_sf, b_sf32;
+  if (!E.alloc(KN * 8) || !err.alloc(sizeof(double)) || !b_l1.alloc(l1b) || !b_l2.alloc(l2b) ||
+      !b_codes.alloc(cb) || !b_sf.alloc(sfb) || (sf32b && !b_sf32.alloc(sf32b)))
+    return SVDQ_ERR_ALLOC;
+  auto save = [&](bool to_best) -> int {
+    auto cp = [&](void* best, void* cur, size_t n) {
+      return to_best ? cudaMemcpyAsync(best, cur, n, cudaMemcpyDeviceToDevice, st)
+                     : cudaMemcpyAsync(cur, best, n, cudaMemcpyDeviceToDevice, st);
+    };
+    if (cp(b_l1.p, w->l1t, l1b) != cudaSuccess || cp(b_l2.p, w->l2t, l2b) != cudaSuccess ||
+        cp(b_codes.p, w->wcodes, cb) != cudaSuccess || cp(b_sf.p, w->wsf, sfb) != cudaSuccess ||
+        (sf32b && cp(b_sf32.p, w->wsf32, sf32b) != cudaSuccess))
+      return SVDQ_ERR_CUDA;
+    return SVDQ_OK;
+  };
+  int rc;
+  double best = 0.0, e = 0.0;
+  if ((rc = weight_error(w, What, err.as<double>(), &best, st))) return rc;
+  w->refine_err0 = best;
+  if ((rc = save(true))) return rc;
+  for (int t = 0; t < iters; ++t) {
+    refine_target_kernel<<<dim3((w->N + 255) / 256, w->K), 256, 0, st>>>(
+        What, w->fmt, w->wcodes, w->wsf, w->wsf32, w->K, w->N, w->N_pad, w->sf_kcols, E.as<double>());
+    SVDQ_CHECK_LAUNCH();
+    if ((rc = lowrank_factors(w, E.as<double>(), st))) return rc;
+    residual_kernel<<<dim3((w->N + 255) / 256, w->K), 256, 0, st>>>(What, w->l1t, w->l2t, w->K, w->N,
+                                                                       w->rank, w->r_pad, R);
+    SVDQ_CHECK_LAUNCH();
+    if ((rc = quantize_residual(w, R, st))) return rc;
+    if ((rc = weight_error(w, What, err.as<double>(), &e, st))) return rc;
+    if (e < best) {
+      best = e;
+      if ((rc = save(true))) return rc;
+    }
+  }
+  if ((rc = save(false))) return rc;
+  w->refine_err = best;
+  SVDQ_CUDA(cudaStreamSynchronize(st));
+  return SVDQ_OK;
+}
+
 }  // namespace
 
 // =========================================================================
@@ -511,6 +577,7 @@ SVDQ_API int svdq_prepare_weights(const svdq_prepare_desc* d, void* stream, svdq
     return SVDQ_ERR_INVALID_ARG;
   if (d->rank + d->lora_rank > 256 || d->rank + d->lora_rank > std::min(d->K, d->N))
     return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  if (d->refine_iters < 0 || d->refine_iters > 64) return SVDQ_ERR_INVALID_ARG;
   int dev;
   if ((rc = current_device(&dev))) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -549,6 +616,10 @@ SVDQ_API int svdq_prepare_weights(const svdq_prepare_desc* d, void* stream, svdq
       break;
     }
     if ((rc = quantize_residual(w, R.as<float>(), st))) break;
+    if (d->refine_iters > 0 && w->rank > 0) {
+      if ((rc = refine_branch(w, What.as<double>(), R.as<float>(), d->refine_iters, st))) break;
+      if ((rc = refold_l1(w, st))) break;   // the folded factors of the kept iterate
+    }
     if ((rc = copy_bias(w, d->bias, st))) break;
     if (cudaStreamSynchronize(st) != cudaSuccess) {
       rc = SVDQ_ERR_CUDA;
@@ -648,6 +719,13 @@ SVDQ_API int svdq_append_lora(svdq_weights* w, const void* A, const void* B, int
   if (rc) return rc;
   if (dev != w->device) return SVDQ_ERR_INVALID_ARG;
   return do_append_lora(w, A, B, rl, static_cast<cudaStream_t>(stream));
+}
+
+SVDQ_API int svdq_weights_refine_error(const svdq_weights* w, double* initial, double* kept) {
+  if (w == nullptr) return SVDQ_ERR_INVALID_ARG;
+  if (initial) *initial = w->refine_err0;
+  if (kept) *kept = w->refine_err;
+  return SVDQ_OK;
 }
 
 SVDQ_API int svdq_weights_info(const svdq_weights* w, int* fmt, int* K, int* N, int* rank,

@@ -35,6 +35,15 @@ __device__ __forceinline__ float e4m3_value(uint32_t code) {
   return __uint_as_float(((e + 120u) << 23) | (m << 20));
 }
 
+// Value of an E2M1 code from its bit fields: sign bit 3, exponent bits 2..1
+// (bias 1), mantissa bit 0; exponent field 0 = subnormal m * 0.5.
+__device__ __forceinline__ float e2m1_value(uint32_t code) {
+  const uint32_t e = (code >> 1) & 3u, m = code & 1u;
+  const float mag = e == 0 ? 0.5f * static_cast<float>(m)
+                           : static_cast<float>(1u << (e - 1)) * (1.0f + 0.5f * static_cast<float>(m));
+  return (code & 8u) ? -mag : mag;
+}
+
 // Eight fp32 values -> eight packed E2M1 codes (value 2i in the low nibble of
 // byte i), nearest even, saturating at +-6.
 __device__ __forceinline__ uint32_t e2m1_pack8(const float* q) {
