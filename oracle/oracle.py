@@ -25,9 +25,10 @@ from typing import Optional
 
 import numpy as np
 
-NVFP4, INT4, FP4G32 = 0, 1, 2
-_FMT = {"nvfp4": NVFP4, "int4": INT4, "fp4g32": FP4G32, NVFP4: NVFP4, INT4: INT4, FP4G32: FP4G32}
-GROUP = {NVFP4: 16, INT4: 64, FP4G32: 32}
+NVFP4, INT4, FP4G32, W8A8 = 0, 1, 2, 3
+_FMT = {"nvfp4": NVFP4, "int4": INT4, "fp4g32": FP4G32, "w8a8": W8A8,
+        NVFP4: NVFP4, INT4: INT4, FP4G32: FP4G32, W8A8: W8A8}
+GROUP = {NVFP4: 16, INT4: 64, FP4G32: 32}   # W8A8: one scale per row over all of K
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "svdq_oracle.c")
@@ -74,6 +75,9 @@ def lib() -> ctypes.CDLL:
         _lib.oracle_fp16_round_sat.argtypes = [ctypes.c_float]
         _lib.oracle_quant_group_nvfp4.argtypes = [P, P, P]
         _lib.oracle_quant_group_fp4g32.argtypes = [P, P, P]
+        _lib.oracle_act_quant_w8.argtypes = [I, I, I, P, P, P, P, P, P]
+        _lib.oracle_weight_quant_w8.argtypes = [I, I, P, P, P]
+        _lib.oracle_linear_rows_w8.argtypes = [I, I, I, I, P, P, P, P, P, P, P, P, I, P]
         _lib.oracle_quant_group_int4.argtypes = [P, P, P]
         for name in ("oracle_bf16_round_array", "oracle_e4m3_round_array",
                      "oracle_e2m1_round_array", "oracle_fp16_round_array"):
@@ -307,10 +311,16 @@ def prepare(W_bits: np.ndarray, x_absmax: Optional[np.ndarray], rank: int,
 # --------------------------------------------------------------------------
 
 def weight_quant(fmt, R: np.ndarray):
-    """Quantize R (K x N fp32) along K per output column -> codes (N x K/2), scales (N x K/g)."""
+    """Quantize R (K x N fp32) along K per output column -> codes (N x K/2), scales (N x K/g);
+    W8A8: codes N x K int8, scales N fp32 (one per output channel)."""
     fmt = _FMT[fmt]
     R = np.ascontiguousarray(R, dtype=np.float32)
     K, N = R.shape
+    if fmt == W8A8:
+        codes = np.zeros((N, K), dtype=np.int8)
+        scales = np.zeros(N, dtype=np.float32)
+        assert lib().oracle_weight_quant_w8(K, N, _ptr(R), _ptr(codes), _ptr(scales)) == 0
+        return codes, scales
     g = GROUP[fmt]
     codes = np.zeros((N, K // 2), dtype=np.uint8)
     scales = np.zeros((N, K // g), dtype=np.uint16 if fmt == INT4 else np.uint8)
@@ -336,12 +346,21 @@ def act_quant(fmt, X_bits: np.ndarray, inv_lambda: Optional[np.ndarray], L1_bits
     fmt = _FMT[fmt]
     X_bits = np.ascontiguousarray(X_bits, dtype=np.uint16)
     M, K = X_bits.shape
-    g = GROUP[fmt]
     r = 0 if L1_bits is None else L1_bits.shape[1]
+    inv = None if inv_lambda is None else np.ascontiguousarray(inv_lambda, dtype=np.float32)
+    if fmt == W8A8:
+        # per-token: codes M x K int8, scales M fp32
+        codes = np.zeros((M, K), dtype=np.int8)
+        scales = np.zeros(M, dtype=np.float32)
+        XL1 = np.zeros((M, r), dtype=np.float32)
+        L1s = None if L1_bits is None else fold_l1(L1_bits, inv)
+        assert lib().oracle_act_quant_w8(M, K, r, _ptr(X_bits), _ptr(inv), _ptr(L1s), _ptr(codes),
+                                         _ptr(scales), _ptr(XL1)) == 0
+        return codes, scales, XL1
+    g = GROUP[fmt]
     codes = np.zeros((M, K // 2), dtype=np.uint8)
     scales = np.zeros((M, K // g), dtype=np.uint16 if fmt == INT4 else np.uint8)
     XL1 = np.zeros((M, r), dtype=np.float32)
-    inv = None if inv_lambda is None else np.ascontiguousarray(inv_lambda, dtype=np.float32)
     L1s = None if L1_bits is None else fold_l1(L1_bits, inv)
     rc = lib().oracle_act_quant(fmt, M, K, r, _ptr(X_bits), _ptr(inv), _ptr(L1s),
                                 _ptr(codes), _ptr(scales), _ptr(XL1))
@@ -356,7 +375,7 @@ def linear(fmt, act, wq, L2_bits: Optional[np.ndarray], bias_bits: Optional[np.n
     cx, sx, XL1 = act
     cw, sw = wq
     M = cx.shape[0]
-    K = cx.shape[1] * 2
+    K = cx.shape[1] * (1 if fmt == W8A8 else 2)
     r = XL1.shape[1]
     if r:
         assert L2_bits is not None and L2_bits.shape == (r, N)
@@ -365,15 +384,22 @@ def linear(fmt, act, wq, L2_bits: Optional[np.ndarray], bias_bits: Optional[np.n
     Y = np.zeros((n_rows, N), dtype=np.uint16)
     L2 = None if not r else np.ascontiguousarray(L2_bits, dtype=np.uint16)
     bias = None if bias_bits is None else np.ascontiguousarray(bias_bits, dtype=np.uint16)
-    rc = lib().oracle_linear_rows(fmt, M, N, K, r, _ptr(cx), _ptr(sx), _ptr(XL1), _ptr(cw),
-                                  _ptr(sw), _ptr(L2), _ptr(bias), _ptr(rows_arr), n_rows, _ptr(Y))
+    if fmt == W8A8:
+        rc = lib().oracle_linear_rows_w8(M, N, K, r, _ptr(cx), _ptr(sx), _ptr(XL1), _ptr(cw), _ptr(sw),
+                                         _ptr(L2), _ptr(bias), _ptr(rows_arr), n_rows, _ptr(Y))
+    else:
+        rc = lib().oracle_linear_rows(fmt, M, N, K, r, _ptr(cx), _ptr(sx), _ptr(XL1), _ptr(cw),
+                                      _ptr(sw), _ptr(L2), _ptr(bias), _ptr(rows_arr), n_rows, _ptr(Y))
     assert rc == 0
     return Y
 
 
 def dequant(fmt, codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
-    """s * deq(q) for packed codes (rows x K/2) -> fp32 rows x K."""
+    """s * deq(q) for packed codes (rows x K/2) -> fp32 rows x K; W8A8: int8 codes
+    rows x K times the row's fp32 scale."""
     fmt = _FMT[fmt]
+    if fmt == W8A8:
+        return (np.asarray(codes, dtype=np.float32) * np.asarray(scales, dtype=np.float32)[:, None])
     rows, K = codes.shape[0], codes.shape[1] * 2
     out = np.zeros((rows, K), dtype=np.float32)
     rc = lib().oracle_dequant(fmt, rows, K, _ptr(np.ascontiguousarray(codes)),

@@ -44,6 +44,9 @@
 #define ORACLE_NVFP4 0
 #define ORACLE_INT4 1
 #define ORACLE_FP4G32 2
+/* W8A8 (the paper's 8-bit setting) has its own functions below: int8 codes one
+ * per byte, one fp32 scale per token row (activations) or per output channel
+ * (weights), taken over the whole of K. */
 
 /* Group size along K and bytes per scale of each format. */
 static int fmt_group(int fmt) { return fmt == ORACLE_NVFP4 ? 16 : (fmt == ORACLE_FP4G32 ? 32 : 64); }
@@ -407,4 +410,89 @@ void oracle_e2m1_round_array(const float *x, long n, uint8_t *out) {
 
 void oracle_fp16_round_array(const float *x, long n, uint16_t *out) {
     for (long i = 0; i < n; ++i) out[i] = oracle_fp16_round_sat(x[i]);
+}
+
+/* ------------------------------------------------------------------------- */
+/* W8A8 (Sec. 5.1 "Implementation details", 8-bit setting): per-token dynamic */
+/* activation quantization and per-channel weight quantization, q_max = 127   */
+/* (Sec. 3: 2^(b-1) - 1 for signed b-bit integers).                           */
+/*   s = amax / 127 (IEEE fp32, kept in fp32: a dynamic scale has no storage  */
+/*   format of its own); q = clamp(rint_even(v * RN(1/s)), -127, 127); s = 0  */
+/*   gives zero codes.                                                         */
+/* ------------------------------------------------------------------------- */
+static void quant_int8(const float *v, long n, long stride, int8_t *codes, float *scale) {
+    float amax = 0.0f;
+    for (long i = 0; i < n; ++i) amax = fmaxf(amax, fabsf(v[i * stride]));
+    float s = amax / 127.0f;
+    *scale = s;
+    if (s == 0.0f) {
+        for (long i = 0; i < n; ++i) codes[i] = 0;
+        return;
+    }
+    float inv = 1.0f / s;
+    for (long i = 0; i < n; ++i) {
+        float q = round_half_even(v[i * stride] * inv);
+        if (q > 127.0f) q = 127.0f;
+        if (q < -127.0f) q = -127.0f;
+        codes[i] = (int8_t)q;
+    }
+}
+
+/* Activations: codes M x K int8, scales M fp32, XL1 M x r fp32 (as above). */
+int oracle_act_quant_w8(int M, int K, int r, const uint16_t *X, const float *inv_lambda,
+                        const uint16_t *L1s, int8_t *codes, float *scales, float *XL1) {
+#pragma omp parallel
+    {
+        float *xh = (float *)__builtin_alloca(sizeof(float) * (size_t)K);
+        float *xf = (float *)__builtin_alloca(sizeof(float) * (size_t)K);
+#pragma omp for schedule(static)
+        for (int m = 0; m < M; ++m) {
+            const uint16_t *xr = X + (long)m * K;
+            for (int k = 0; k < K; ++k) {
+                xf[k] = oracle_bf16_decode(xr[k]);
+                xh[k] = inv_lambda ? xf[k] * inv_lambda[k] : xf[k];
+            }
+            quant_int8(xh, K, 1, codes + (long)m * K, scales + m);
+            for (int j = 0; j < r; ++j) {
+                float acc = 0.0f;
+                for (int k = 0; k < K; ++k)
+                    acc += xf[k] * oracle_bf16_decode(L1s[(long)k * r + j]);
+                XL1[(long)m * r + j] = acc;
+            }
+        }
+    }
+    return 0;
+}
+
+/* Weights: R K x N fp32 -> codes N x K int8 (per output channel), scales N fp32. */
+int oracle_weight_quant_w8(int K, int N, const float *R, int8_t *codes, float *scales) {
+#pragma omp parallel for schedule(static)
+    for (int n = 0; n < N; ++n) quant_int8(R + n, K, N, codes + (long)n * K, scales + n);
+    return 0;
+}
+
+/* y[m,n] = bf16( float(sum_k qx qw) * (s_x[m] s_w[n]) + sum_j XL1[m,j] L2[j,n] + bias[n] ):
+ * the integer dot product is exact (|sum| < 127^2 K < 2^31 for K < 2^17) and
+ * rounded once to fp32. */
+int oracle_linear_rows_w8(int M, int N, int K, int r, const int8_t *codes_x, const float *scales_x,
+                          const float *XL1, const int8_t *codes_w, const float *scales_w,
+                          const uint16_t *L2, const uint16_t *bias, const int *rows, int n_rows,
+                          uint16_t *Y) {
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int i = 0; i < n_rows; ++i) {
+        int m = rows ? rows[i] : i;
+        if (m < 0 || m >= M) continue;
+        const int8_t *cx = codes_x + (long)m * K;
+        for (int n = 0; n < N; ++n) {
+            const int8_t *cw = codes_w + (long)n * K;
+            long long dot = 0;
+            for (int k = 0; k < K; ++k) dot += (long long)cx[k] * (long long)cw[k];
+            float acc = (float)dot * (scales_x[m] * scales_w[n]);
+            for (int j = 0; j < r; ++j)
+                acc += XL1[(long)m * r + j] * oracle_bf16_decode(L2[(long)j * N + n]);
+            if (bias) acc += oracle_bf16_decode(bias[n]);
+            Y[(long)i * N + n] = oracle_bf16_round((double)acc);
+        }
+    }
+    return 0;
 }
