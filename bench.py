@@ -157,11 +157,22 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+# Per format: tensor-core instruction family (int8 formats run kind::i8, whose
+# peak is half the FP4 one), activation code bytes per value, GEMM kernel.
+INT8_KIND = ("int4", "w8a8")
+GEMM_KERNEL = {"nvfp4": "gemm_nvfp4_kernel", "fp4g32": "gemm_nvfp4_kernel",
+               "int4": "gemm_int4_kernel", "w8a8": "gemm_w8a8_kernel"}
+DTYPE = {"nvfp4": "e2m1xe2m1+bf16 (fp32 acc)", "fp4g32": "e2m1xe2m1+bf16 (fp32 acc)",
+         "int4": "s8xs8+bf16 (fp32 acc)", "w8a8": "s8xs8 (s32 acc)+bf16 (fp32 acc)"}
+
+
 def layer_inputs(args):
+    import dataclasses
     spec = WL.layer_spec(args.config, args.layer)
     if getattr(args, "fmt", None):
-        import dataclasses
         spec = dataclasses.replace(spec, fmt=args.fmt)
+    if getattr(args, "rank", None) is not None:
+        spec = dataclasses.replace(spec, rank=args.rank)
     M = args.M or WL.CONFIGS[args.config].Ms[-1 if args.config == "c5_block" else 0]
     return spec, M
 
@@ -257,7 +268,7 @@ def tensor_ceiling(S, fmt, stream):
     """The tensor cores' own ceiling for the GEMM's instruction (no global
     traffic): a ~5 ms burst and a ~1 s sustained run, in TFLOP/s."""
     sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
-    flop_step = sms * 4 * 2 * 128 * 256 * (64 if fmt != "int4" else 32)
+    flop_step = sms * 4 * 2 * 128 * 256 * (32 if fmt in INT8_KIND else 64)
 
     def run(steps):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -275,7 +286,7 @@ def tensor_ceiling(S, fmt, stream):
     steps_long = max(2000, int(2000 * 1.0 / t))
     sustained = flop_step * steps_long / run(steps_long) / 1e12
     return {"burst": round(burst, 1), "sustained": round(sustained, 1), "unit": "TFLOP/s",
-            "what": "tcgen05 " + ("kind::mxf4nvf4 128x256x64" if fmt != "int4" else "kind::i8 128x256x32")
+            "what": "tcgen05 " + ("kind::i8 128x256x32" if fmt in INT8_KIND else "kind::mxf4nvf4 128x256x64")
                     + " back to back from shared memory on every SM, no global loads"}
 
 
@@ -304,7 +315,10 @@ def run_ours(args):
     Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
-    launches_per_step = 2 + (1 if (spec.fmt != "int4" and K % 256) else 0)
+    # activation kernel + GEMM; FP4 formats zero the scale padding when K % 256,
+    # W8A8 first computes the per-token scales
+    launches_per_step = 2 + (1 if (spec.fmt in ("nvfp4", "fp4g32") and K % 256) else 0) \
+        + (1 if spec.fmt == "w8a8" else 0)
 
     sampler = ClockSampler(local)
     t_q, t_g, clocks = time_layer(S, w, X, ws, Y, M, flush, stream, args.steps, args.warmup, world, sampler)
@@ -337,22 +351,22 @@ def run_ours(args):
     flops = 2.0 * M * K * N
     r = w.rank
     pk = peaks()
-    fp_peak = pk["bf16"] * (4.0 if spec.fmt != "int4" else 2.0)
+    fp_peak = pk["bf16"] * (2.0 if spec.fmt in INT8_KIND else 4.0)
     gemm_flops = flops + 2.0 * M * r * N
     achieved = gemm_flops / tg_mean / 1e12
     # activation kernel: algorithmic bytes (X read, codes + scales + XL1 written)
-    code_bytes = M * K / 2 if spec.fmt != "int4" else M * K
-    scale_bytes = {"nvfp4": M * K / 16, "fp4g32": M * K / 16, "int4": M * K / 64 * 2}[spec.fmt]
+    code_bytes = M * K if spec.fmt in INT8_KIND else M * K / 2
+    scale_bytes = {"nvfp4": M * K / 16, "fp4g32": M * K / 16, "int4": M * K / 64 * 2, "w8a8": M * 4}[spec.fmt]
     q_bytes = 2.0 * M * K + code_bytes + scale_bytes + 2.0 * M * w.rank_padded
     q_gbs = q_bytes / tq_mean / 1e9
     value = job_throughput(world, flops, args.steps, total)
-    gemm_kernel = "gemm_nvfp4_kernel" if spec.fmt != "int4" else "gemm_int4_kernel"
+    gemm_kernel = GEMM_KERNEL[spec.fmt]
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(total / args.steps * 1e3, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "e2m1xe2m1+bf16 (fp32 acc)" if spec.fmt != "int4" else "s8xs8+bf16 (fp32 acc)",
+        "dtype": DTYPE[spec.fmt],
         "data": "synthetic (seeded FLUX-shaped activations and weights; no checkpoints)",
         "config": {"workload": f"{args.config}/{spec.name}: M={M} K={K} N={N} rank={r} {spec.fmt}",
                    "M": M, "K": K, "N": N, "rank": r, "format": spec.fmt,
@@ -364,7 +378,7 @@ def run_ours(args):
                      "achieved": round(achieved, 1), "peak": round(fp_peak, 1), "unit": "TFLOP/s",
                      "frac": round(achieved / fp_peak, 4),
                      "traffic": ncu_traffic(gemm_kernel, f"{args.config}/{spec.name}", M),
-                     "peak_note": f"{pk['source']}: bf16 {pk['bf16']} TF/s x {'4 (FP4)' if spec.fmt != 'int4' else '2 (INT8)'}"},
+                     "peak_note": f"{pk['source']}: bf16 {pk['bf16']} TF/s x {'2 (INT8)' if spec.fmt in INT8_KIND else '4 (FP4)'}"},
         "roofline_quant": {"bound": "hbm", "kernel": "quant_act_kernel", "achieved": round(q_gbs, 1),
                            "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": round(q_gbs / pk["hbm_gbs"], 4),
                            "algorithmic_bytes": int(q_bytes),
@@ -490,8 +504,10 @@ def main():
     ap.add_argument("--config", default="c2_qkv", choices=sorted(WL.CONFIGS))
     ap.add_argument("--layer", default=None)
     ap.add_argument("--M", type=int, default=None)
-    ap.add_argument("--fmt", choices=["nvfp4", "int4", "fp4g32"], default=None,
-                    help="override the workload's 4-bit format")
+    ap.add_argument("--fmt", choices=["nvfp4", "int4", "fp4g32", "w8a8"], default=None,
+                    help="override the workload's format")
+    ap.add_argument("--rank", type=int, default=None,
+                    help="override the workload's low-rank branch rank (the paper pairs W8A8 with 16)")
     ap.add_argument("--cpu-rows", type=int, default=64)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--rank-sweep", type=lambda v: [int(x) for x in v.split(",")], default=None,

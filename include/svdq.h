@@ -16,6 +16,11 @@
  *   SVDQ_FP4G32: E2M1 codes with one E4M3 scale per 32 values along K (the
  *               paper's FP4 setting of Sec. 5.1: groups of 32, an FP8 scale).
  *               It runs on the NVFP4 kernels with each scale stored twice.
+ *   SVDQ_W8A8 : the 8-bit setting of Sec. 5.1: int8 codes in [-127, 127],
+ *               one fp32 scale per token for the activations (computed on the
+ *               fly over all of K) and one per output channel for the
+ *               weights; the integer dot product is exact and scaled once.
+ *               The paper pairs it with rank 16.
  *
  * Conventions for every call:
  *   - "device" pointers are CUDA global-memory pointers on the current device;
@@ -59,7 +64,7 @@ typedef enum {
   SVDQ_ERR_LIBRARY = 6            /* cuSOLVER / cuBLAS failed during preparation */
 } svdq_status;
 
-typedef enum { SVDQ_NVFP4 = 0, SVDQ_INT4 = 1, SVDQ_FP4G32 = 2 } svdq_format;
+typedef enum { SVDQ_NVFP4 = 0, SVDQ_INT4 = 1, SVDQ_FP4G32 = 2, SVDQ_W8A8 = 3 } svdq_format;
 
 /* Opaque prepared layer: 4-bit residual codes and scales, the bf16 low-rank
  * factors, 1/lambda and the bias, all in device memory owned by the handle. */
@@ -173,13 +178,16 @@ SVDQ_API int svdq_forward_noalloc(const svdq_weights* w, const void* X, int M, v
 /* Debug export of a filled workspace in plain layouts (host outputs, any may
  * be NULL; synchronizes the device):
  *   codes  M x K/2 bytes, element 2i in the low nibble (INT4: two's complement);
- *   scales M x K/16 E4M3 bytes (NVFP4) or M x K/64 fp16 (INT4);
+ *          W8A8: M x K int8;
+ *   scales M x K/16 E4M3 bytes (NVFP4), M x K/32 E4M3 bytes (FP4 g32),
+ *          M x K/64 fp16 (INT4) or M fp32 (W8A8);
  *   xl1    M x rank fp32 (X_hat L1 at fp32 precision; stored as a bf16 pair). */
 SVDQ_API int svdq_export_act(const svdq_weights* w, const void* workspace, int M,
                              uint8_t* codes, void* scales, void* xl1);
 
 /* Debug export of a handle in plain layouts (host outputs, any may be NULL):
- *   codes N x K/2 (per output column, along K), scales N x K/16 or N x K/64,
+ *   codes N x K/2 (per output column, along K; W8A8: N x K int8), scales
+ *   N x K/16, N x K/32, N x K/64 (as for svdq_export_act) or N fp32 (W8A8),
  *   L1 K x rank bf16, L2 rank x N bf16, inv_lambda K floats, lambda K floats. */
 SVDQ_API int svdq_export_weights(const svdq_weights* w, uint8_t* codes, void* scales, void* L1,
                                  void* L2, float* inv_lambda, float* lambda);

@@ -11,6 +11,8 @@ the full SVD, which would take minutes at these sizes).  Checked:
   * Y: sampled rows (first and last 32 rows and 32 seeded random rows, all N
     columns), within |dy| <= 2^-7 |y| + 1e-3 rms(y).
 """
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -23,12 +25,14 @@ from gpu_common import (bits, close_f32, load_from_oracle, require_gpu, svdq, to
 pytestmark = pytest.mark.gpu
 
 CASES = [
-    ("c1_small", None, 256),
-    ("c2_qkv", None, 4608),
-    ("c3_mlp", "fc1", 4608),
-    ("c3_mlp", "fc2", 4608),
-    ("c4_int4_lora", None, 4608),
-] + [("c5_block", layer, M) for layer in ("qkv", "out", "fc1", "fc2") for M in (1024, 4096, 16384)]
+    ("c1_small", None, 256, None),
+    ("c2_qkv", None, 4608, None),
+    ("c3_mlp", "fc1", 4608, None),
+    ("c3_mlp", "fc2", 4608, None),
+    ("c4_int4_lora", None, 4608, None),
+    ("c2_qkv", None, 4608, ("w8a8", 16)),    # the paper's 8-bit setting: W8A8 with rank 16
+    ("c3_mlp", "fc2", 4608, ("w8a8", 16)),
+] + [("c5_block", layer, M, None) for layer in ("qkv", "out", "fc1", "fc2") for M in (1024, 4096, 16384)]
 
 _parts = {}
 
@@ -41,11 +45,12 @@ def S():
 
 def _prepared(spec):
     """Oracle parts of one layer, computed once per layer for every M."""
-    key = (spec.name, spec.K, spec.N, spec.seed, spec.fmt)
+    key = (spec.name, spec.K, spec.N, spec.seed, spec.fmt, spec.rank)
     if key not in _parts:
         W, bias, A, B = WL.make_weights(spec)
         # calibration: the layer's largest token batch of the workload
-        M_cal = max(m for c in WL.CONFIGS.values() for l in c.layers if l is spec for m in c.Ms)
+        M_cal = max(m for c in WL.CONFIGS.values() for l in c.layers
+                    if dataclasses.replace(l, fmt=spec.fmt, rank=spec.rank) == spec for m in c.Ms)
         Xc = WL.bf16_bits(WL.make_activations(spec, M_cal))
         prep = O.prepare(WL.bf16_bits(W), O.calib_absmax(Xc), spec.rank,
                          WL.bf16_bits(A) if A is not None else None,
@@ -63,9 +68,17 @@ def _sample_rows(M, seed):
     return np.unique(rows).astype(np.int32)
 
 
-@pytest.mark.parametrize("config,layer,M", CASES)
-def test_fullsize_parity(S, config, layer, M):
+def _case_id(case):
+    config, layer, M, override = case
+    return "-".join([config] + ([layer] if layer else []) + [str(M)] +
+                    ([f"{override[0]}_r{override[1]}"] if override else []))
+
+
+@pytest.mark.parametrize("config,layer,M,override", CASES, ids=[_case_id(c) for c in CASES])
+def test_fullsize_parity(S, config, layer, M, override):
     spec = WL.layer_spec(config, layer)
+    if override is not None:
+        spec = dataclasses.replace(spec, fmt=override[0], rank=override[1])
     prep, wq, bias_bits = _prepared(spec)
     w = load_from_oracle(S, spec.fmt, prep, bias_bits)
     try:

@@ -67,6 +67,59 @@ def test_weight_quantizer_edge_values(S):
         assert np.array_equal(got["codes"], codes), (fmt, np.argwhere(got["codes"] != codes)[:8])
 
 
+def test_weight_quantizer_edge_values_w8a8(S):
+    """W8A8 per-channel int8: exact ties at scale 1 and 1/2 (round half to
+    even), an all-zero channel, tiny and large channels."""
+    K = 256
+    rng = np.random.default_rng(12)
+    cols = []
+    c = np.zeros(K, dtype=np.float32)
+    c[:8] = [127, 2.5, -0.5, 3.5, 1.5, -126.5, 0.5, -2.5]          # s = 1
+    cols.append(c)
+    c = np.zeros(K, dtype=np.float32)
+    c[:6] = [63.5, 0.25, 0.75, -0.25, -63.25, 1.25]                 # s = 1/2
+    cols.append(c)
+    cols.append(np.zeros(K, dtype=np.float32))
+    cols.append((rng.standard_normal(K) * 1e-3).astype(np.float32))
+    cols.append((rng.standard_normal(K) * 3000).astype(np.float32))
+    while len(cols) < 32:
+        cols.append((rng.standard_normal(K) * 10.0 ** rng.uniform(-4, 3)).astype(np.float32))
+    R = np.stack(cols, axis=1).astype(np.float32)     # K x 32
+    w = S.svdq_load_weights(to_dev_f32(R), fmt="w8a8")
+    got = S.svdq_export_weights(w)
+    codes, scales = O.weight_quant("w8a8", R)
+    assert np.array_equal(got["scales"], scales)
+    assert np.array_equal(got["codes"], codes), np.argwhere(got["codes"] != codes)[:8]
+    assert list(got["codes"][0, :8]) == [127, 2, 0, 4, 2, -126, 0, -2]
+    assert list(got["codes"][1, :6]) == [127, 0, 2, 0, -126, 2]
+    assert got["scales"][2] == 0 and not got["codes"][2].any()
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4", "fp4g32", "w8a8"])
+def test_act_quantizer_edge_rows(S, fmt):
+    """Activation rows with exact ties, an all-zero row, huge and tiny rows,
+    through svdq_quantize_act with lambda = 1; codes and scales bit-exact."""
+    K, N, M = 256, 64, 40
+    rng = np.random.default_rng(13)
+    X = (rng.standard_normal((M, K)) * 10.0 ** rng.uniform(-2, 2, size=(M, 1))).astype(np.float32)
+    X[0] = 0
+    X[0, :8] = [127, 2.5, -0.5, 3.5, 1.5, -126.5, 0.5, -2.5]
+    X[1] = 0
+    X[2] *= 1e4
+    X[3] *= 1e-30
+    X[4, :16] = [6, 3, -1.5, 0.25, 5, 2.5, 0.75, 1.25, 1.75, 3.5, -5, -0.25, 0.5, 0, 0, 0]
+    Xb = WL.bf16_bits(torch.from_numpy(X).to(torch.bfloat16))
+    R = (rng.standard_normal((K, N)) * 0.02).astype(np.float32)
+    ones = np.ones(K, dtype=np.float32)
+    w = S.svdq_load_weights(to_dev_f32(R), fmt=fmt, inv_lambda=to_dev_f32(ones), lam=to_dev_f32(ones))
+    ws, Y = _run_layer(S, w, Xb)
+    codes, scales, _ = S.svdq_export_act(w, ws, M)
+    want = O.act_quant(fmt, Xb, ones, None)
+    assert np.array_equal(scales, want[1]), np.argwhere(scales != want[1])[:8]
+    assert np.array_equal(codes, want[0]), np.argwhere(codes != want[0])[:8]
+    w.close()
+
+
 SHAPES = [
     # M, K, N, rank, fmt, bias
     (1, 256, 256, 32, "nvfp4", False),
@@ -81,6 +134,10 @@ SHAPES = [
     (64, 256, 272, 0, "int4", False),
     (77, 512, 384, 32, "fp4g32", True),      # one E4M3 scale per 32 values, stored per 16
     (300, 320, 272, 48, "fp4g32", False),
+    (77, 512, 384, 16, "w8a8", True),        # int8, per-token / per-channel scales
+    (300, 320, 272, 16, "w8a8", False),      # K % 128 != 0: the last K step is half padding
+    (129, 512, 256, 0, "w8a8", True),        # plain W8A8
+    (200, 1024, 512, 64, "w8a8", False),
 ]
 
 
@@ -137,7 +194,7 @@ def test_prepare_weights_invariants(S):
     assert e_lib <= 1.1 * e_ora + 1e-3, (e_lib, e_ora)
 
 
-@pytest.mark.parametrize("fmt", ["nvfp4", "int4", "fp4g32"])
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4", "fp4g32", "w8a8"])
 def test_lora_fold_parity(S, fmt):
     M, K, N, r, rl = 160, 512, 384, 32, 16
     data = WL.make_small(M, K, N, rank=r, fmt=fmt, lora_rank=rl, seed=9)
@@ -178,7 +235,7 @@ def test_empty_batch_is_a_noop(S):
     assert Y.shape == (0, 256)
 
 
-@pytest.mark.parametrize("fmt", ["nvfp4", "int4", "fp4g32"])
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4", "fp4g32", "w8a8"])
 def test_prepare_refinement(S, fmt):
     """Iterative refinement of the branch in svdq_prepare_weights: the kept
     error is what the exported parts give, it drops below the SVD start, and

@@ -19,9 +19,20 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libsvdq.so")
 
-NVFP4, INT4, FP4G32 = 0, 1, 2
-_FMT = {"nvfp4": NVFP4, "int4": INT4, "fp4g32": FP4G32, NVFP4: NVFP4, INT4: INT4, FP4G32: FP4G32}
-GROUP = {NVFP4: 16, INT4: 64, FP4G32: 32}
+NVFP4, INT4, FP4G32, W8A8 = 0, 1, 2, 3
+_FMT = {"nvfp4": NVFP4, "int4": INT4, "fp4g32": FP4G32, "w8a8": W8A8,
+        NVFP4: NVFP4, INT4: INT4, FP4G32: FP4G32, W8A8: W8A8}
+GROUP = {NVFP4: 16, INT4: 64, FP4G32: 32}   # W8A8: one scale per row over all of K
+
+
+def _code_scale_arrays(fmt: int, rows: int, K: int):
+    """Host arrays for exported codes and scales of `rows` rows: 4-bit formats
+    give packed nibble pairs (rows x K/2) and per-group scales; W8A8 gives int8
+    codes (rows x K) and one fp32 scale per row."""
+    if fmt == W8A8:
+        return np.zeros((rows, K), dtype=np.int8), np.zeros(rows, dtype=np.float32)
+    return (np.zeros((rows, K // 2), dtype=np.uint8),
+            np.zeros((rows, K // GROUP[fmt]), dtype=np.uint16 if fmt == INT4 else np.uint8))
 
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "device allocation failed",
           4: "CUDA error", 5: "device wait timed out", 6: "cuSOLVER/cuBLAS error"}
@@ -276,10 +287,9 @@ def svdq_forward_noalloc(w: Weights, X: torch.Tensor, Y: Optional[torch.Tensor] 
 
 
 def svdq_export_act(w: Weights, workspace: torch.Tensor, M: int):
-    """(codes M x K/2 uint8, scales M x K/g, xl1 M x rank float32) on the host."""
-    g = GROUP[w.fmt]
-    codes = np.zeros((M, w.K // 2), dtype=np.uint8)
-    scales = np.zeros((M, w.K // g), dtype=np.uint16 if w.fmt == INT4 else np.uint8)
+    """(codes, scales, xl1 M x rank float32) on the host: codes M x K/2 uint8 and
+    scales M x K/g for the 4-bit formats, int8 M x K and fp32 M for W8A8."""
+    codes, scales = _code_scale_arrays(w.fmt, M, w.K)
     xl1 = np.zeros((M, w.rank), dtype=np.float32)
     _check(lib().svdq_export_act(w.handle, _ptr(workspace), int(M), codes.ctypes.data_as(ctypes.c_void_p),
                                  scales.ctypes.data_as(ctypes.c_void_p),
@@ -289,9 +299,7 @@ def svdq_export_act(w: Weights, workspace: torch.Tensor, M: int):
 
 
 def svdq_export_weights(w: Weights) -> dict:
-    g = GROUP[w.fmt]
-    codes = np.zeros((w.N, w.K // 2), dtype=np.uint8)
-    scales = np.zeros((w.N, w.K // g), dtype=np.uint16 if w.fmt == INT4 else np.uint8)
+    codes, scales = _code_scale_arrays(w.fmt, w.N, w.K)
     L1 = np.zeros((w.K, w.rank), dtype=np.uint16)
     L2 = np.zeros((w.rank, w.N), dtype=np.uint16)
     inv = np.zeros(w.K, dtype=np.float32)
@@ -316,7 +324,7 @@ def svdq_weights_refine_error(w: "Weights"):
 
 def svdq_tensor_peak(fmt: str, steps: int, stream=None):
     """Launch the tensor-core ceiling kernel (see include/svdq.h); time it with
-    CUDA events.  FLOP = SMs * steps * 4 * 2 * 128 * 256 * (64 NVFP4 / FP4 g32 | 32 INT4)."""
+    CUDA events.  FLOP = SMs * steps * 4 * 2 * 128 * 256 * (64 NVFP4 / FP4 g32 | 32 INT4, W8A8)."""
     _check(lib().svdq_tensor_peak(_FMT[fmt], int(steps), _stream(stream)), "svdq_tensor_peak")
 
 

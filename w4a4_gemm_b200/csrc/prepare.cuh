@@ -322,6 +322,10 @@ __device__ __forceinline__ double deq_weight(int fmt, const uint8_t* __restrict_
     const int8_t q = reinterpret_cast<const int8_t*>(codes)[static_cast<size_t>(n) * K + k];
     return static_cast<double>(q) * static_cast<double>(sf32[static_cast<size_t>(k / 64) * N_pad + n]);
   }
+  if (fmt == 3) {   // W8A8: one fp32 scale per output channel
+    const int8_t q = reinterpret_cast<const int8_t*>(codes)[static_cast<size_t>(n) * K + k];
+    return static_cast<double>(__fmul_rn(static_cast<float>(q), reinterpret_cast<const float*>(sf)[n]));
+  }
   const uint8_t b = codes[static_cast<size_t>(n) * (K / 2) + k / 2];
   const uint32_t c = (k & 1) ? (b >> 4) : (b & 15u);
   const int g = k / 16;
@@ -369,6 +373,24 @@ __global__ void refine_error_kernel(const double* __restrict__ What,
     for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) t += part[w];
     atomicAdd(sum, t);
   }
+}
+
+// W8A8 weights (SVDQuant paper, Sec. 5.1, 8-bit setting): per output channel n,
+// s = max_k |R[k,n]| / 127 (IEEE fp32), codes clamp(rint_even(R * RN(1/s)), -127, 127)
+// stored N x K int8; s = 0 gives zero codes.  One thread per column.
+__global__ void quant_weight_w8_kernel(const float* __restrict__ R, int K, int N,
+                                       int8_t* __restrict__ codes, float* __restrict__ sw) {
+  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  if (n >= N) return;
+  float amax = 0.0f;
+  for (int k = 0; k < K; ++k) amax = fmaxf(amax, fabsf(R[static_cast<size_t>(k) * N + n]));
+  const float s = __fdiv_rn(amax, 127.0f);
+  const float inv = s == 0.0f ? 0.0f : __frcp_rn(s);
+  for (int k = 0; k < K; ++k) {
+    const int q = max(-127, min(127, __float2int_rn(__fmul_rn(R[static_cast<size_t>(k) * N + n], inv))));
+    codes[static_cast<size_t>(n) * K + k] = static_cast<int8_t>(q);
+  }
+  sw[n] = s;
 }
 
 }  // namespace svdq

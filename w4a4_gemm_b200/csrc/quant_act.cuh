@@ -40,8 +40,8 @@ constexpr int kQuantWarps = 4 * kQuantGroups;   // quantizer warps (one per lane
 constexpr int kQuantThreads = 32 * (2 + kQuantWarps);
 constexpr uint32_t kQuantSmemBudget = 220u * 1024u;    // shared memory for stages + code staging
 
-// Bytes of codes one row of a 64-wide sub-tile produces: 64 E2M1 (NVFP4, FP4 g32) or 64 int8 (INT4).
-__host__ __device__ constexpr uint32_t quant_code_row_bytes(int fmt) { return fmt == 1 ? 64u : 32u; }
+// Bytes of codes one row of a 64-wide sub-tile produces: 64 E2M1 (NVFP4, FP4 g32) or 64 int8 (INT4, W8A8).
+__host__ __device__ constexpr uint32_t quant_code_row_bytes(int fmt) { return (fmt == 1 || fmt == 3) ? 64u : 32u; }
 
 struct QuantParams {
   int M, K;
@@ -86,7 +86,8 @@ __host__ __device__ inline QuantSmem quant_smem_layout(int fmt, int r_pad, int S
   return L;
 }
 
-template <int FMT>  // 0 = NVFP4 (groups of 16), 1 = INT4 (groups of 64), 2 = FP4 g32 (groups of 32)
+template <int FMT>  // 0 = NVFP4 (groups of 16), 1 = INT4 (groups of 64), 2 = FP4 g32 (groups of 32),
+                    // 3 = W8A8 (int8, the per-token scale computed beforehand by w8_row_scale_kernel)
 __global__ void __launch_bounds__(kQuantThreads, 1)
     quant_act_kernel(const __grid_constant__ CUtensorMap tm_x,
                      const __grid_constant__ CUtensorMap tm_l1t,
@@ -124,7 +125,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (FMT != 1 && warp >= 2 && warp < 6) fill_e4m3_rcp_table(rcp_tab, threadIdx.x - 64, 128);
+  if ((FMT == 0 || FMT == 2) && warp >= 2 && warp < 6) fill_e4m3_rcp_table(rcp_tab, threadIdx.x - 64, 128);
   if (warp == 1 && has_lr) {
     tmem_alloc(tmem_holder, tmem_cols);
     tmem_relinquish();
@@ -256,6 +257,21 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
         const uint32_t s0 = quant32_fp4(v, out, rcp_tab);
         const uint32_t s1 = quant32_fp4(v + 32, out + 4, rcp_tab);
         sfw = s0 * 0x0101u | (s1 * 0x0101u) << 16;
+      } else if constexpr (FMT == 3) {
+        // int8 codes of this row with its per-token scale
+        const float sd = reinterpret_cast<const float*>(p.sf)[row_ok ? m : 0];
+        const float inv = (sd == 0.0f || !row_ok) ? 0.0f : __frcp_rn(sd);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          uint32_t w = 0;
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            const int q = max(-127, min(127, __float2int_rn(__fmul_rn(v[4 * e + b], inv))));
+            w |= (static_cast<uint32_t>(q) & 0xFFu) << (8 * b);
+          }
+          out[e] = w;
+        }
+        sfw = 0;
       } else {
         float amax = 0.0f;
 #pragma unroll
@@ -280,7 +296,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
       named_bar_sync(bar_free, 128);
       {
         const uint32_t row_addr = smem_u32(buf) + R * RB;
-        const uint32_t sw = FMT != 1 ? ((R >> 2) & 1u) : ((R >> 1) & 3u);
+        const uint32_t sw = RB == 32 ? ((R >> 2) & 1u) : ((R >> 1) & 3u);
 #pragma unroll
         for (uint32_t c = 0; c < RB / 16; ++c)
           asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row_addr + ((c ^ sw) << 4)),
@@ -296,8 +312,8 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
         }
         bulk_commit_group();
       }
-      if (ok && col_ok) {
-        if constexpr (FMT != 1) {
+      if (ok && col_ok && FMT != 3) {   // W8A8 scales are written before this kernel
+        if constexpr (FMT == 0 || FMT == 2) {
           // scale atom: 128 rows x 4 scales, byte (m % 32) * 16 + (m % 128 / 32) * 4 + k4
           uint8_t* atom = p.sf + (static_cast<size_t>(m / 128) * p.sf_kcols + kcol) * 512;
           *reinterpret_cast<uint32_t*>(atom + (m & 31) * 16 + ((m & 127) >> 5) * 4) = row_ok ? sfw : 0u;
@@ -378,6 +394,28 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, tmem_cols);
   }
+}
+
+// W8A8 per-token scale (SVDQuant paper, Sec. 5.1, 8-bit setting):
+// s_x[m] = max_k |fp32(x[m,k]) * (1/lambda_k)| / 127, IEEE fp32, one warp per row.
+__global__ void w8_row_scale_kernel(const __nv_bfloat16* __restrict__ X, const float* __restrict__ inv_lambda,
+                                    int M, int K, float* __restrict__ sx) {
+  const int m = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (m >= M) return;
+  const uint4* xr = reinterpret_cast<const uint4*>(X + static_cast<size_t>(m) * K);
+  const float4* il = reinterpret_cast<const float4*>(inv_lambda);
+  float amax = 0.0f;
+  for (int c = lane; c < K / 8; c += 32) {
+    const uint4 raw = __ldg(xr + c);
+    const float4 l0 = __ldg(il + 2 * c), l1 = __ldg(il + 2 * c + 1);
+    amax = fmax3(amax, fabsf(__fmul_rn(bf16_lo(raw.x), l0.x)), fabsf(__fmul_rn(bf16_hi(raw.x), l0.y)));
+    amax = fmax3(amax, fabsf(__fmul_rn(bf16_lo(raw.y), l0.z)), fabsf(__fmul_rn(bf16_hi(raw.y), l0.w)));
+    amax = fmax3(amax, fabsf(__fmul_rn(bf16_lo(raw.z), l1.x)), fabsf(__fmul_rn(bf16_hi(raw.z), l1.y)));
+    amax = fmax3(amax, fabsf(__fmul_rn(bf16_lo(raw.w), l1.z)), fabsf(__fmul_rn(bf16_hi(raw.w), l1.w)));
+  }
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if (lane == 0) sx[m] = __fdiv_rn(amax, 127.0f);
 }
 
 }  // namespace svdq

@@ -20,6 +20,7 @@
 #include "../../include/svdq.h"
 #include "gemm_int4.cuh"
 #include "gemm_nvfp4.cuh"
+#include "gemm_w8a8.cuh"
 #include "peak.cuh"
 #include "prepare.cuh"
 #include "quant_act.cuh"
@@ -159,6 +160,9 @@ int device_setup(int dev) {
   SVDQ_CUDA(cudaFuncSetAttribute(quant_act_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, qmax));
   SVDQ_CUDA(cudaFuncSetAttribute(quant_act_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, qmax));
   SVDQ_CUDA(cudaFuncSetAttribute(quant_act_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, qmax));
+  SVDQ_CUDA(cudaFuncSetAttribute(quant_act_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, qmax));
+  SVDQ_CUDA(cudaFuncSetAttribute(gemm_w8a8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kW8SmemBytes));
   SVDQ_CUDA(cudaFuncSetAttribute(gemm_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kGemmSmemBytes));
   SVDQ_CUDA(cudaFuncSetAttribute(gemm_int4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -197,8 +201,9 @@ ActLayout act_layout(const svdq_weights* w, int M) {
   L.M_pad = round_up(std::max(M, 1), 128);
   L.codes_bytes = is_fp4(w->fmt) ? static_cast<size_t>(M) * w->K / 2
                                        : static_cast<size_t>(M) * w->K;
-  L.sf_bytes = is_fp4(w->fmt) ? static_cast<size_t>(L.M_pad / 128) * w->sf_kcols * 512
-                                    : static_cast<size_t>(w->K / 64) * L.M_pad * 2;
+  L.sf_bytes = is_fp4(w->fmt)            ? static_cast<size_t>(L.M_pad / 128) * w->sf_kcols * 512
+               : w->fmt == SVDQ_W8A8 ? static_cast<size_t>(L.M_pad) * 4          // fp32 per token
+                                     : static_cast<size_t>(w->K / 64) * L.M_pad * 2;
   L.xl1_bytes = static_cast<size_t>(M) * 2 * w->r_pad * 2;   // bf16 hi | lo
   L.codes_off = 0;
   L.sf_off = align256(L.codes_bytes);
@@ -213,15 +218,17 @@ int encode_weight_maps(svdq_weights* w) {
   int rc;
   if (is_fp4(w->fmt))
     rc = make_map(&w->tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->wcodes, w->K / 2, w->N, 128, kGemmBN);
+  else if (w->fmt == SVDQ_W8A8)
+    rc = make_map(&w->tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->wcodes, w->K, w->N, kW8BKB, kW8BN);
   else
     rc = make_map(&w->tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->wcodes, w->K, w->N, 64, kI4BN);
   if (rc) return rc;
   if (w->r_pad > 0) {
     rc = make_map(&w->tm_l1t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w->l1st, w->K, w->r_pad, 64, w->r_pad);
     if (rc) return rc;
-    const int lc = is_fp4(w->fmt) ? lr_chunk_cols(2 * w->r_pad) : i4_lr_chunk_cols(2 * w->r_pad);
+    const int lc = w->fmt != SVDQ_INT4 ? lr_chunk_cols(2 * w->r_pad) : i4_lr_chunk_cols(2 * w->r_pad);
     rc = make_map(&w->tm_l2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w->l2t2, 2 * w->r_pad, w->N, lc,
-                  is_fp4(w->fmt) ? kGemmBN : kI4BN);
+                  w->fmt != SVDQ_INT4 ? kGemmBN : kI4BN);
     if (rc) return rc;
   } else {
     w->tm_l1t = w->tm_b;
@@ -246,7 +253,8 @@ void free_weights(svdq_weights* w) {
 }
 
 int check_shape(int fmt, int K, int N, int rank) {
-  if (fmt != SVDQ_NVFP4 && fmt != SVDQ_INT4 && fmt != SVDQ_FP4G32) return SVDQ_ERR_INVALID_ARG;
+  if (fmt != SVDQ_NVFP4 && fmt != SVDQ_INT4 && fmt != SVDQ_FP4G32 && fmt != SVDQ_W8A8)
+    return SVDQ_ERR_INVALID_ARG;
   if (K <= 0 || N <= 0 || K % 64 != 0 || N % 16 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
   if (rank < 0 || rank > 256 || rank > std::min(K, N)) return SVDQ_ERR_UNSUPPORTED_SHAPE;
   return SVDQ_OK;
@@ -260,8 +268,9 @@ int alloc_weights(svdq_weights* w, cudaStream_t st) {
   w->r_pad = rank_padded(w->rank);
   const size_t codes = is_fp4(w->fmt) ? static_cast<size_t>(w->N) * w->K / 2
                                             : static_cast<size_t>(w->N) * w->K;
-  const size_t sfb = is_fp4(w->fmt) ? static_cast<size_t>(w->N_pad / 128) * w->sf_kcols * 512
-                                          : static_cast<size_t>(w->K / 64) * w->N_pad * 2;
+  const size_t sfb = is_fp4(w->fmt)            ? static_cast<size_t>(w->N_pad / 128) * w->sf_kcols * 512
+                     : w->fmt == SVDQ_W8A8 ? static_cast<size_t>(w->N_pad) * 4   // fp32 per channel
+                                           : static_cast<size_t>(w->K / 64) * w->N_pad * 2;
   // 1/lambda is read in 512-value blocks by the activation kernel: zero-pad it
   const size_t il_bytes = static_cast<size_t>(round_up(w->K, 512)) * sizeof(float);
   if (cudaMalloc(&w->inv_lambda, il_bytes) != cudaSuccess ||
@@ -295,6 +304,10 @@ int quantize_residual(svdq_weights* w, const float* R, cudaStream_t st) {
   } else if (w->fmt == SVDQ_FP4G32) {
     const dim3 grid((w->N + 127) / 128, w->K / 32);
     quant_weight_fp4g32_kernel<<<grid, blk, 0, st>>>(R, w->K, w->N, w->sf_kcols, w->wcodes, w->wsf);
+  } else if (w->fmt == SVDQ_W8A8) {
+    quant_weight_w8_kernel<<<(w->N + 127) / 128, blk, 0, st>>>(R, w->K, w->N,
+                                                                reinterpret_cast<int8_t*>(w->wcodes),
+                                                                reinterpret_cast<float*>(w->wsf));
   } else {
     const dim3 grid((w->N + 127) / 128, w->K / 64);
     quant_weight_int4_kernel<<<grid, blk, 0, st>>>(R, w->K, w->N, w->N_pad,
@@ -463,9 +476,10 @@ int weight_error(svdq_weights* w, const double* What, double* err_dev, double* o
 int refine_branch(svdq_weights* w, const double* What, float* R, int iters, cudaStream_t st) {
   const size_t KN = static_cast<size_t>(w->K) * w->N;
   const size_t l1b = static_cast<size_t>(w->r_pad) * w->K * 2, l2b = static_cast<size_t>(w->N) * w->r_pad * 2;
-  const size_t cb = w->fmt == SVDQ_INT4 ? KN : KN / 2;
-  const size_t sfb = w->fmt == SVDQ_INT4 ? static_cast<size_t>(w->K / 64) * w->N_pad * 2
-                                         : static_cast<size_t>(w->N_pad / 128) * w->sf_kcols * 512;
+  const size_t cb = is_fp4(w->fmt) ? KN / 2 : KN;
+  const size_t sfb = is_fp4(w->fmt)            ? static_cast<size_t>(w->N_pad / 128) * w->sf_kcols * 512
+                     : w->fmt == SVDQ_W8A8 ? static_cast<size_t>(w->N_pad) * 4
+                                           : static_cast<size_t>(w->K / 64) * w->N_pad * 2;
   const size_t sf32b = w->fmt == SVDQ_INT4 ? static_cast<size_t>(w->K / 64) * w->N_pad * 4 : 0;
   DeviceBuf E, err, b_l1, b_l2, b_codes, b_sf, b_sf32;
   if (!E.alloc(KN * 8) || !err.alloc(sizeof(double)) || !b_l1.alloc(l1b) || !b_l2.alloc(l2b) ||
@@ -527,7 +541,8 @@ SVDQ_API const char* svdq_status_string(int s) {
 }
 
 SVDQ_API int svdq_tensor_peak(int fmt, long long steps, void* stream) {
-  if ((fmt != SVDQ_NVFP4 && fmt != SVDQ_INT4 && fmt != SVDQ_FP4G32) || steps < 1) return SVDQ_ERR_INVALID_ARG;
+  if ((fmt != SVDQ_NVFP4 && fmt != SVDQ_INT4 && fmt != SVDQ_FP4G32 && fmt != SVDQ_W8A8) || steps < 1)
+    return SVDQ_ERR_INVALID_ARG;
   int dev;
   int rc = current_device(&dev);
   if (rc) return rc;
@@ -763,7 +778,7 @@ SVDQ_API int svdq_quantize_act(const svdq_weights* w, const void* X, int M, void
   if ((rc = make_map(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, w->K, M, kQuantBK, BM)))
     return rc;
   // codes: NVFP4 M x K/2 packed E2M1, INT4 M x K int8; one box = one sub-tile's BM rows
-  const uint32_t rb = quant_code_row_bytes(is_fp4(w->fmt) ? 0 : 1);
+  const uint32_t rb = quant_code_row_bytes(w->fmt);
   if ((rc = make_map(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base + L.codes_off,
                      is_fp4(w->fmt) ? w->K / 2 : w->K, M, rb, BM)))
     return rc;
@@ -784,14 +799,19 @@ SVDQ_API int svdq_quantize_act(const svdq_weights* w, const void* X, int M, void
     const size_t off = static_cast<size_t>(w->K / 64) * 512;
     SVDQ_CUDA(cudaMemset2DAsync(p.sf + off, pitch, 0, pitch - off, L.M_pad / 128, st));
   }
-  const QuantSmem Q = quant_smem_layout(is_fp4(w->fmt) ? 0 : 1, w->r_pad, S);
+  const QuantSmem Q = quant_smem_layout(w->fmt, w->r_pad, S);
   const dim3 grid((M + BM - 1) / BM);
   const CUtensorMap& tm_l1t = w->r_pad > 0 ? w->tm_l1t : tm_x;
   if (w->fmt == SVDQ_NVFP4)
     quant_act_kernel<0><<<grid, kQuantThreads, Q.total, st>>>(tm_x, tm_l1t, tm_codes, p);
   else if (w->fmt == SVDQ_FP4G32)
     quant_act_kernel<2><<<grid, kQuantThreads, Q.total, st>>>(tm_x, tm_l1t, tm_codes, p);
-  else
+  else if (w->fmt == SVDQ_W8A8) {
+    // the per-token scales first: they need all of K before any code
+    w8_row_scale_kernel<<<(M + 7) / 8, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(X), w->inv_lambda,
+                                                     M, w->K, reinterpret_cast<float*>(p.sf));
+    quant_act_kernel<3><<<grid, kQuantThreads, Q.total, st>>>(tm_x, tm_l1t, tm_codes, p);
+  } else
     quant_act_kernel<1><<<grid, kQuantThreads, Q.total, st>>>(tm_x, tm_l1t, tm_codes, p);
   SVDQ_CHECK_LAUNCH();
   return SVDQ_OK;
@@ -811,17 +831,19 @@ SVDQ_API int svdq_linear(const svdq_weights* w, const void* ws, int M, void* Y, 
   const uint8_t* base = static_cast<const uint8_t*>(ws);
   CUtensorMap tm_a, tm_xl1;
   const int m_tiles = L.M_pad / 128;
-  const int n_tiles = is_fp4(w->fmt) ? (w->N + kGemmBN - 1) / kGemmBN : (w->N + kI4BN - 1) / kI4BN;
+  const int n_tiles = w->fmt != SVDQ_INT4 ? (w->N + kGemmBN - 1) / kGemmBN : (w->N + kI4BN - 1) / kI4BN;
   const int tiles = m_tiles * n_tiles;
   const int grid = std::min(tiles, g_dev[dev].sms);
   if (is_fp4(w->fmt))
     rc = make_map(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base + L.codes_off, w->K / 2, M, 128, kGemmBM);
+  else if (w->fmt == SVDQ_W8A8)
+    rc = make_map(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base + L.codes_off, w->K, M, kW8BKB, kW8BM);
   else
     rc = make_map(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base + L.codes_off, w->K, M, 64, kI4BM);
   if (rc) return rc;
   if (w->r_pad > 0) {
     if ((rc = make_map(&tm_xl1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base + L.xl1_off, 2 * w->r_pad, M,
-                       is_fp4(w->fmt) ? lr_chunk_cols(2 * w->r_pad) : i4_lr_chunk_cols(2 * w->r_pad),
+                       w->fmt != SVDQ_INT4 ? lr_chunk_cols(2 * w->r_pad) : i4_lr_chunk_cols(2 * w->r_pad),
                        128)))
       return rc;
   } else {
@@ -846,6 +868,23 @@ SVDQ_API int svdq_linear(const svdq_weights* w, const void* ws, int M, void* Y, 
     p.budget = wait_budget();
     gemm_nvfp4_kernel<<<grid, kGemmThreads, kGemmSmemBytes, st>>>(tm_a, w->tm_b, tm_xl1, w->tm_l2t,
                                                                   tm_y, p);
+  } else if (w->fmt == SVDQ_W8A8) {
+    CUtensorMap tm_y;
+    if ((rc = make_map(&tm_y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Y, w->N, M, 16, 32))) return rc;
+    GemmW8Params p;
+    p.M = M;
+    p.N = w->N;
+    p.K = w->K;
+    p.kt_total = (w->K + kW8BKB - 1) / kW8BKB;
+    p.m_tiles = m_tiles;
+    p.n_tiles = n_tiles;
+    p.num_tiles = tiles;
+    p.r_tail = 2 * w->r_pad;
+    p.sx = reinterpret_cast<const float*>(base + L.sf_off);
+    p.sw = reinterpret_cast<const float*>(w->wsf);
+    p.bias = w->bias;
+    p.budget = wait_budget();
+    gemm_w8a8_kernel<<<grid, kW8Threads, kW8SmemBytes, st>>>(tm_a, w->tm_b, tm_xl1, w->tm_l2t, tm_y, p);
   } else {
     GemmI4Params p;
     p.M = M;
@@ -929,7 +968,8 @@ SVDQ_API int svdq_export_act(const svdq_weights* w, const void* ws, int M, uint8
   const uint8_t* base = static_cast<const uint8_t*>(ws);
   const int K = w->K;
   if (codes) {
-    if (is_fp4(w->fmt)) {
+    if (is_fp4(w->fmt) || w->fmt == SVDQ_W8A8) {
+      // packed E2M1 pairs, or W8A8's int8 codes as they are
       SVDQ_CUDA(cudaMemcpy(codes, base + L.codes_off, L.codes_bytes, cudaMemcpyDeviceToHost));
     } else {
       std::vector<int8_t> tmp(L.codes_bytes);
@@ -952,6 +992,8 @@ SVDQ_API int svdq_export_act(const svdq_weights* w, const void* ws, int M, uint8
           const size_t atom = (static_cast<size_t>(m / 128) * w->sf_kcols + b / 4) * 512;
           out[static_cast<size_t>(m) * G + g] = tmp[atom + (m % 32) * 16 + ((m % 128) / 32) * 4 + b % 4];
         }
+    } else if (w->fmt == SVDQ_W8A8) {
+      std::memcpy(scales, tmp.data(), static_cast<size_t>(M) * 4);   // fp32 per token
     } else {
       uint16_t* out = static_cast<uint16_t*>(scales);
       const uint16_t* in = reinterpret_cast<const uint16_t*>(tmp.data());
@@ -988,6 +1030,8 @@ SVDQ_API int svdq_export_weights(const svdq_weights* w, uint8_t* codes, void* sc
   if (codes) {
     if (is_fp4(w->fmt)) {
       SVDQ_CUDA(cudaMemcpy(codes, w->wcodes, static_cast<size_t>(N) * K / 2, cudaMemcpyDeviceToHost));
+    } else if (w->fmt == SVDQ_W8A8) {
+      SVDQ_CUDA(cudaMemcpy(codes, w->wcodes, static_cast<size_t>(N) * K, cudaMemcpyDeviceToHost));
     } else {
       std::vector<int8_t> tmp(static_cast<size_t>(N) * K);
       SVDQ_CUDA(cudaMemcpy(tmp.data(), w->wcodes, tmp.size(), cudaMemcpyDeviceToHost));
@@ -1009,6 +1053,8 @@ SVDQ_API int svdq_export_weights(const svdq_weights* w, uint8_t* codes, void* sc
           const size_t atom = (static_cast<size_t>(n / 128) * w->sf_kcols + b / 4) * 512;
           out[static_cast<size_t>(n) * G + g] = tmp[atom + (n % 32) * 16 + ((n % 128) / 32) * 4 + b % 4];
         }
+    } else if (w->fmt == SVDQ_W8A8) {
+      SVDQ_CUDA(cudaMemcpy(scales, w->wsf, static_cast<size_t>(N) * 4, cudaMemcpyDeviceToHost));
     } else {
       const int G = K / 64;
       std::vector<uint16_t> tmp(static_cast<size_t>(G) * w->N_pad);
