@@ -201,6 +201,19 @@ SVDQ_API int svdq_get_error(void);
  * second; the environment variable SVDQ_WAIT_BUDGET_CYCLES also sets it). */
 SVDQ_API int svdq_set_wait_budget(long long cycles);
 
+/* Launch shape of the activation kernel for every later svdq_quantize_act
+ * (process-wide; a tuning and testing aid).  S = stacked 64-wide K sub-tiles
+ * per pipeline stage (rows per CTA cluster = 128 / S), C = CTAs per cluster,
+ * each on its own K range, whose partial X_hat L1 sums meet in distributed
+ * shared memory.  S, C in {1, 2, 4, 8}; 0, 0 restores the automatic choice
+ * (a cost model over the SM count and the resident clusters of each size).
+ * A forced shape the layer cannot use (S above 256 / rank_padded, C above
+ * 128 / S or above the number of stages, no resident cluster of C CTAs)
+ * falls back to the automatic choice for that call.  The results do not
+ * depend on the shape beyond the summation order of X_hat L1 (fp32).
+ * SVDQ_ERR_INVALID_ARG for other values. */
+SVDQ_API int svdq_set_quant_split(int S, int C);
+
 SVDQ_API const char* svdq_status_string(int status);
 
 /* Measurement helper, not a step of the layer: every SM of the current device

@@ -161,6 +161,36 @@ def test_layer_parity_small(S, M, K, N, rank, fmt, bias):
     assert ok, ("Y", info)
 
 
+@pytest.mark.parametrize("M,K,N,rank,fmt", [
+    (300, 320, 272, 48, "nvfp4"),    # 5 sub-tiles: clusters of 4 leave one CTA without a K range
+    (200, 512, 256, 32, "int4"),
+    (130, 1024, 256, 16, "fp4g32"),
+    (77, 512, 384, 16, "w8a8"),
+])
+def test_forced_launch_shapes(S, M, K, N, rank, fmt):
+    """Every launch shape of the activation kernel (stacked sub-tiles x CTAs per
+    cluster) gives the oracle's codes and scales bit for bit and X_hat L1, Y
+    within tolerance; shapes a layer cannot use fall back to the automatic one."""
+    data = WL.make_small(M, K, N, rank=rank, fmt=fmt, seed=M + K + 1)
+    ref = oracle_layer(fmt, data, rank)
+    w = load_from_oracle(S, fmt, ref["prep"])
+    try:
+        for st in (1, 2, 4, 8):
+            for cl in (1, 2, 4, 8):
+                S.svdq_set_quant_split(st, cl)
+                ws, Y = _run_layer(S, w, WL.bf16_bits(data["X"]))
+                codes, scales, xl1 = S.svdq_export_act(w, ws, M)
+                assert np.array_equal(scales, ref["act"][1]), (st, cl, "scales")
+                assert np.array_equal(codes, ref["act"][0]), (st, cl, "codes")
+                ok, info = close_f32(xl1, ref["act"][2])
+                assert ok, (st, cl, "XL1", info)
+                ok, info = y_within_tol(bits(Y), ref["Y"])
+                assert ok, (st, cl, "Y", info)
+    finally:
+        S.svdq_set_quant_split(0, 0)
+        w.close()
+
+
 def test_prepare_weights_invariants(S):
     """The library's own preparation (cuSOLVER on the fp64 Gram matrix):
     1/lambda bit-exact, the branch spans the oracle's optimal rank-r subspace,

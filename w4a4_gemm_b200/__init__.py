@@ -40,7 +40,8 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "device all
 EXPORTED = ("svdq_calib_absmax", "svdq_prepare_weights", "svdq_load_weights", "svdq_append_lora",
             "svdq_weights_info", "svdq_weights_refine_error", "svdq_act_workspace_bytes", "svdq_quantize_act", "svdq_linear",
             "svdq_forward", "svdq_forward_noalloc", "svdq_export_act", "svdq_export_weights", "svdq_get_error",
-            "svdq_set_wait_budget", "svdq_status_string", "svdq_tensor_peak", "svdq_weights_destroy")
+            "svdq_set_wait_budget", "svdq_set_quant_split", "svdq_status_string", "svdq_tensor_peak",
+            "svdq_weights_destroy")
 
 
 class SvdqError(RuntimeError):
@@ -91,6 +92,7 @@ def lib() -> ctypes.CDLL:
     L.svdq_export_weights.argtypes = [P, P, P, P, P, P, P]
     L.svdq_get_error.argtypes = []
     L.svdq_set_wait_budget.argtypes = [LL]
+    L.svdq_set_quant_split.argtypes = [I, I]
     L.svdq_status_string.argtypes = [I]
     L.svdq_status_string.restype = ctypes.c_char_p
     L.svdq_tensor_peak.argtypes = [I, LL, P]
@@ -330,3 +332,8 @@ def svdq_tensor_peak(fmt: str, steps: int, stream=None):
 
 def svdq_set_wait_budget(cycles: int):
     _check(lib().svdq_set_wait_budget(int(cycles)), "svdq_set_wait_budget")
+
+
+def svdq_set_quant_split(S: int = 0, C: int = 0):
+    """Force the activation kernel's launch shape (see include/svdq.h); 0, 0 = automatic."""
+    _check(lib().svdq_set_quant_split(int(S), int(C)), "svdq_set_quant_split")

@@ -142,6 +142,7 @@ __global__ void __launch_bounds__(kI4Threads, 1)
   const int lr_cols = i4_lr_chunk_cols(p.r_tail);
   const int steps_per_tile = p.groups + n_lr;
 
+  griddep_launch_dependents();
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
@@ -174,6 +175,7 @@ __global__ void __launch_bounds__(kI4Threads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  griddep_wait();   // the activation codes, scales and XL1 come from the previous kernel
 
   if (warp == 0) {
     if (elect_one()) {

@@ -148,6 +148,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int lr_cols = lr_chunk_cols(p.r_tail);
   const int steps_per_tile = p.kt_total + n_lr;
 
+  griddep_launch_dependents();
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
@@ -167,6 +168,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  griddep_wait();   // the activation codes, scales and XL1 come from the previous kernel
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer

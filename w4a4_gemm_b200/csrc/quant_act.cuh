@@ -7,15 +7,23 @@
 // the tensor core reads the TMA-loaded X tile as it is, in parallel with the
 // quantizer warps.
 //
-// One CTA owns BM = 128 / S token rows over the whole of K, so no partial sum
-// ever leaves the CTA.  Each pipeline stage holds S consecutive 64-wide K
-// sub-tiles of those rows stacked on top of each other as the 128-row A
-// operand of one tcgen05 MMA, and the S matching 64 x r_pad slices of the
-// folded factor L1s side by side as its N = S * r_pad wide B operand:
+// A cluster of C CTAs owns BM = 128 / S token rows; its CTA of rank t takes
+// the t-th of C consecutive K ranges.  Each pipeline stage holds S consecutive
+// 64-wide K sub-tiles of those rows stacked on top of each other as the
+// 128-row A operand of one tcgen05 MMA, and the S matching 64 x r_pad slices
+// of the folded factor L1s side by side as its N = S * r_pad wide B operand:
 //   D[j*BM + i, j'*r_pad + c] += sum_k x[i, sub-tile j, k] * L1s[sub-tile j', k, c]
-// Only the diagonal blocks j == j' are wanted; summing them over j gives
-// X L1s = X_hat L1 for row i.  The host picks the smallest S (1, 2, 4 or 8, at most
-// 256 / r_pad) that gives about one CTA per SM.
+// Only the diagonal blocks j == j' are wanted; summing them over j and over
+// the cluster's K ranges gives X L1s = X_hat L1 for row i.  The partial sums
+// meet in distributed shared memory: each CTA parks its blocks in its own
+// shared memory and sums, for its share of the rows, every CTA's blocks in a
+// fixed order (the result does not depend on timing).  Codes and scales are
+// local to a 64-wide group and need no exchange.
+//
+// Every stage carries L1s as well as X: r_pad / BM bytes of factor per byte of
+// X.  Stacking (S > 1) fills the MMA at small M but raises that ratio; the K
+// split (C > 1) keeps BM large and still gives every SM a CTA.  The host picks
+// (S, C) from the SM count and the resident clusters of each size.
 //   warp 0      : TMA producer (S X boxes BM x 64, S L1s^T boxes r_pad x 64, 1/lambda)
 //   warp 1      : TMEM owner; one lane issues the kind::f16 MMAs
 //   warps 2..13 : quantizers in three groups of four; group k takes every
@@ -34,9 +42,11 @@ namespace svdq {
 
 constexpr int kQuantTileRows = 128;   // rows of the MMA A operand
 constexpr int kQuantBK = 64;          // K width of one sub-tile
-constexpr int kQuantMaxStages = 8;
+constexpr int kQuantMaxStages = 12;
+constexpr int kQuantMaxSplit = 8;     // CTAs per cluster splitting K
 constexpr int kQuantGroups = 3;       // quantizer groups working on consecutive stages
-constexpr int kQuantWarps = 4 * kQuantGroups;   // quantizer warps (one per lane quarter per group)
+constexpr int kQuantGroupWarps = 4;   // warps per group: one lane per row of a 128-row stage
+constexpr int kQuantWarps = kQuantGroupWarps * kQuantGroups;
 constexpr int kQuantThreads = 32 * (2 + kQuantWarps);
 constexpr uint32_t kQuantSmemBudget = 220u * 1024u;    // shared memory for stages + code staging
 
@@ -46,7 +56,9 @@ __host__ __device__ constexpr uint32_t quant_code_row_bytes(int fmt) { return (f
 struct QuantParams {
   int M, K;
   int r_pad;        // 0 = no low-rank branch; else 16, 32, 64, 128, 192 or 256
-  int S;            // stacked K sub-tiles per stage (BM = 128 / S rows per CTA)
+  int S;            // stacked K sub-tiles per stage (BM = 128 / S rows per cluster)
+  int C;            // CTAs per cluster, each on its own K range (1, 2, 4 or 8; C <= BM)
+  int per;          // stages per cluster rank: rank t takes stages [t per, min((t+1) per, total))
   int M_pad;        // M rounded up to 128 (scale atoms)
   int sf_kcols;     // NVFP4: K_pad / 64 scale atoms per 128-row block
   const float* inv_lambda;  // K rounded up to 512 (zero padded)
@@ -109,17 +121,21 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
   const bool has_lr = p.r_pad > 0;
   const int S = p.S;
   const int BM = kQuantTileRows / S;
-  const int m0 = blockIdx.x * BM;
+  const int rank = static_cast<int>(blockIdx.x) % p.C;  // rank in the 1-D cluster of C CTAs
+  const int m0 = (static_cast<int>(blockIdx.x) / p.C) * BM;
   const int kstep = S * kQuantBK;                       // K columns per stage
-  const int nkt = (p.K + kstep - 1) / kstep;
+  const int nkt = (p.K + kstep - 1) / kstep;            // stages over all of K
+  const int i0 = min(rank * p.per, nkt);                // this CTA's stages: i0 .. i0 + n_local - 1
+  const int n_local = min(nkt - i0, p.per);
   const int n_mma = S * p.r_pad;                        // MMA N
   const uint32_t tmem_cols = n_mma <= 32 ? 32u : (n_mma <= 64 ? 64u : (n_mma <= 128 ? 128u : 256u));
 
+  griddep_launch_dependents();
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 1);
       // released by the quantizer warps and, with a low-rank branch, the MMAs
-      mbar_init(&empty[s], 4 + (has_lr ? 1 : 0));
+      mbar_init(&empty[s], kQuantGroupWarps + (has_lr ? 1 : 0));
     }
     mbar_init(acc_full, 1);
     *abort_flag = 0;
@@ -134,6 +150,8 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = has_lr ? *tmem_holder : 0u;
+  // X and the previous contents of the workspace belong to earlier kernels
+  griddep_wait();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -142,9 +160,10 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
       if (has_lr) prefetch_tmap(&tm_l1t);
       const uint32_t tx = S * (BM * kQuantBK * 2 + (has_lr ? p.r_pad * 128 : 0) + kQuantBK * 4);
       int issued = 0;
-      for (int i = 0; i < nkt; ++i) {
-        const int s = i % NS;
-        const uint32_t ph = (i / NS) & 1;
+      for (int li = 0; li < n_local; ++li) {
+        const int i = i0 + li;
+        const int s = li % NS;
+        const uint32_t ph = (li / NS) & 1;
         if (!mbar_wait(&empty[s], ph ^ 1, p.budget, abort_flag)) {
           raise_error(kErrWaitQuant);
           *abort_flag = 1;
@@ -158,7 +177,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
           if (has_lr) tma_load_2d(st + L.l1_off + j * p.r_pad * 128, &tm_l1t, &full[s], k, 0);
         }
         bulk_load(st + L.il_off, p.inv_lambda + i * kstep, S * kQuantBK * 4, &full[s]);
-        issued = i + 1;
+        issued = li + 1;
       }
       // never leave while a copy into this CTA's shared memory is still in flight
       if (*abort_flag) {
@@ -170,9 +189,9 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (has_lr && elect_one()) {
       const uint32_t idesc = idesc_bf16_f32(kQuantTileRows, n_mma);
-      for (int i = 0; i < nkt; ++i) {
-        const int s = i % NS;
-        const uint32_t ph = (i / NS) & 1;
+      for (int li = 0; li < n_local; ++li) {
+        const int s = li % NS;
+        const uint32_t ph = (li / NS) & 1;
         if (!mbar_wait(&full[s], ph, p.budget, abort_flag)) {
           raise_error(kErrWaitQuant);
           *abort_flag = 1;
@@ -184,7 +203,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
 #pragma unroll
         for (int k = 0; k < kQuantBK / 16; ++k) {
           mma_bf16(tmem_base, make_kmajor_desc(a0 + 32 * k, 128), make_kmajor_desc(b0 + 32 * k, 128),
-                   idesc, (i > 0 || k > 0) ? 1u : 0u);
+                   idesc, (li > 0 || k > 0) ? 1u : 0u);
         }
         tc_commit(&empty[s]);
       }
@@ -210,9 +229,10 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
     const int m = m0 + static_cast<int>(R) % BM;
     const bool row_ok = m < p.M;
     int use = 0;
-    for (int i = grp; i < nkt; i += kQuantGroups, ++use) {
-      const int s = i % NS;
-      const uint32_t ph = (i / NS) & 1;
+    for (int li = grp; li < n_local; li += kQuantGroups, ++use) {
+      const int i = i0 + li;
+      const int s = li % NS;
+      const uint32_t ph = (li / NS) & 1;
       const bool ok = warp_wait(&full[s], ph, p.budget, abort_flag);
       if (!ok) {
         if (lane == 0) raise_error(kErrWaitQuant);
@@ -328,10 +348,16 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
   __syncwarp();
 
   // ---------------------------------------------------------------- XL1 out
-  // Diagonal block j of the accumulator = the K sub-tiles j (mod S); warps
-  // 2..5 park them in shared memory (the stage buffers are free by now) and
-  // the CTA sums them over j in fixed order and rounds to bf16.
+  // Diagonal block j of the accumulator = the K sub-tiles j (mod S) of this
+  // CTA's K range; warps 2..5 park them in shared memory over the first stage
+  // buffers.  Those are free only once every quantizer group has read its last
+  // stage (the accumulator is complete as soon as the last stage has landed,
+  // and another group may still be reading a late stage in buffer 0): hence
+  // the CTA barrier first.  Then each CTA of the cluster takes BM / C of the
+  // rows and sums, for them, the parked blocks of every CTA (rank 0 first)
+  // over j in fixed order, and rounds to bf16.
   float* red = reinterpret_cast<float*>(smem);   // [128][r_pad] fp32
+  __syncthreads();
   if (has_lr && warp >= 2 && warp < 6) {
     const uint32_t q = warp & 3u;
     const uint32_t R = q * 32 + lane;
@@ -347,8 +373,13 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
     for (int jj = j_first; jj <= j_last; ++jj) {
       for (int c = 0; c < p.r_pad; c += 16) {
         uint32_t r[16];
-        tmem_ld16(tmem_base + ((q * 32u) << 16) + jj * p.r_pad + c, r);
-        tmem_wait_ld();
+        if (n_local > 0) {
+          tmem_ld16(tmem_base + ((q * 32u) << 16) + jj * p.r_pad + c, r);
+          tmem_wait_ld();
+        } else {   // an empty K range contributes zero (its accumulator was never written)
+#pragma unroll
+          for (int e = 0; e < 16; ++e) r[e] = 0u;
+        }
         if (jj == j) {
 #pragma unroll
           for (int e = 0; e < 16; e += 4)
@@ -360,18 +391,23 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
     }
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();   // every CTA of the cluster has parked its blocks (C = 1: the CTA)
   if (has_lr) {
-    // BM rows x r_pad columns, 8 columns per thread over all threads
-    const int units = BM * (p.r_pad / 8);
+    // this CTA's BM / C rows x r_pad columns, 8 columns per thread over all threads
+    const int rows = BM / p.C;
+    const int units = rows * (p.r_pad / 8);
     for (int u = threadIdx.x; u < units; u += kQuantThreads) {
-      const int i = u / (p.r_pad / 8);
+      const int i = rank * rows + u / (p.r_pad / 8);
       const int c = (u % (p.r_pad / 8)) * 8;
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      for (int jj = 0; jj < S; ++jj) {
-        const float* src = red + (jj * BM + i) * p.r_pad + c;
+      for (int t = 0; t < p.C; ++t) {
+        for (int jj = 0; jj < S; ++jj) {
+          const uint32_t src = map_shared_rank(smem_u32(red + (jj * BM + i) * p.r_pad + c), t);
+          const float4 a = ld_shared_cluster_f32x4(src), b = ld_shared_cluster_f32x4(src + 16);
+          const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = __fadd_rn(acc[e], src[e]);
+          for (int e = 0; e < 8; ++e) acc[e] = __fadd_rn(acc[e], v[e]);
+        }
       }
       if (m0 + i < p.M) {
         // hi = bf16(acc), lo = bf16(acc - hi): hi + lo carries acc to ~2^-17
@@ -387,6 +423,8 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
       }
     }
   }
+  // no CTA leaves while a peer may still read its shared memory
+  if (p.C > 1) cluster_sync();
   if (warp == 1 && has_lr) {
     // every MMA this CTA issued has retired before its TMEM is released
     mbar_wait(acc_full, 0, p.budget, nullptr);
@@ -402,6 +440,8 @@ __global__ void w8_row_scale_kernel(const __nv_bfloat16* __restrict__ X, const f
                                     int M, int K, float* __restrict__ sx) {
   const int m = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
+  griddep_launch_dependents();
+  griddep_wait();
   if (m >= M) return;
   const uint4* xr = reinterpret_cast<const uint4*>(X + static_cast<size_t>(m) * K);
   const float4* il = reinterpret_cast<const float4*>(inv_lambda);

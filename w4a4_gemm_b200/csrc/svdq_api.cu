@@ -14,6 +14,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <utility>
 #include <mutex>
 #include <vector>
 
@@ -92,6 +93,34 @@ int rank_padded(int r) {
 
 #define SVDQ_CHECK_LAUNCH() SVDQ_CUDA(cudaGetLastError())
 
+// Launch a hot-path kernel with programmatic stream serialization: it may be
+// scheduled while the previous kernel on the stream drains, does its own setup,
+// and waits for that kernel (griddep_wait) before it touches memory that other
+// kernels read or write.  Every kernel launched this way calls griddep_wait.
+// cluster_x > 0 also groups the CTAs into 1-D clusters of that size.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       unsigned cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.numAttrs = 1;
+  if (cluster_x > 0) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = cluster_x;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
+  }
+  cfg.attrs = attr;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // ------------------------------------------------------------ tensor maps ---
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -142,6 +171,7 @@ int make_map(CUtensorMap* m, CUtensorMapDataType dt, size_t elem, const void* ba
 // ------------------------------------------------------------ device info ---
 struct DeviceInfo {
   int sms = 0;
+  int qclusters[kQuantMaxSplit + 1] = {};   // resident activation-kernel clusters of size C
   bool attrs_set = false;
 };
 DeviceInfo g_dev[64];
@@ -171,6 +201,24 @@ int device_setup(int dev) {
                                  kPeakSmemBytes));
   SVDQ_CUDA(cudaFuncSetAttribute(tensor_peak_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kPeakSmemBytes));
+  // how many clusters of each size the activation kernel can keep resident
+  // (GPCs do not divide evenly into clusters of 4 or 8)
+  for (int C = 1; C <= kQuantMaxSplit; C *= 2) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(C * d.sms);
+    cfg.blockDim = dim3(kQuantThreads);
+    cfg.dynamicSmemBytes = qmax;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    SVDQ_CUDA(cudaOccupancyMaxActiveClusters(&n, quant_act_kernel<1>, &cfg));
+    d.qclusters[C] = n;
+  }
   d.attrs_set = true;
   return SVDQ_OK;
 }
@@ -181,13 +229,49 @@ int current_device(int* dev) {
 }
 
 // ------------------------------------------------------------ workspace ---
-// Stacked K sub-tiles of the activation kernel (rows per CTA = 128 / S): the
-// smallest S that gives about one CTA per SM, as far as the rank allows.
-int quant_stack_for(int M, int r_pad, int sms) {
+// Shape of the activation kernel's launch: S stacked K sub-tiles per stage
+// (BM = 128 / S rows per cluster) and C CTAs per cluster splitting K.  A CTA
+// consumes one 128 x 64 stage in about the same time whatever S is (its four
+// quantizer warps per stage set the pace), so the model is
+//   time = waves * (fixed + [C > 1] * exchange + stages per CTA * stage)
+// with the cycle counts measured on B200 (setup, first load and XL1 epilogue;
+// the cluster exchange of partial sums; one stage).  Ties go to the smaller C,
+// then the smaller S.
+struct QuantSplit {
+  int S, C;
+};
+constexpr double kQuantFixedCycles = 10000.0;
+constexpr double kQuantExchangeCycles = 2000.0;
+constexpr double kQuantStageCycles = 1100.0;
+QuantSplit g_forced_split{0, 0};   // svdq_set_quant_split; {0, 0} = automatic
+
+QuantSplit quant_split_for(int M, int K, int r_pad, const DeviceInfo& d) {
   const int smax = r_pad > 0 ? quant_stack_max(r_pad) : 8;
-  int S = 1;
-  while (S < smax && (M + 128 / S - 1) / (128 / S) < (9 * sms) / 10) S *= 2;
-  return S;
+  const QuantSplit f = g_forced_split;
+  if (f.S > 0 && f.S <= smax && f.C <= kQuantTileRows / f.S &&
+      f.C <= (K + f.S * kQuantBK - 1) / (f.S * kQuantBK) && d.qclusters[f.C] > 0)
+    return f;
+  QuantSplit best{1, 1};
+  double best_t = 1e300;
+  for (int C = 1; C <= kQuantMaxSplit; C *= 2) {
+    const int slots = d.qclusters[C] * C;   // resident CTAs in clusters of C
+    if (slots <= 0) continue;
+    for (int S = 1; S <= smax; S *= 2) {
+      const int BM = kQuantTileRows / S;
+      const int stages = (K + S * kQuantBK - 1) / (S * kQuantBK);
+      if (C > BM || C > stages) continue;
+      const long long ctas = static_cast<long long>((M + BM - 1) / BM) * C;
+      const long long waves = (ctas + slots - 1) / slots;
+      const int per = (stages + C - 1) / C;
+      const double t = static_cast<double>(waves) *
+                       (kQuantFixedCycles + (C > 1 ? kQuantExchangeCycles : 0.0) + per * kQuantStageCycles);
+      if (t < best_t * 0.98) {
+        best_t = t;
+        best = {S, C};
+      }
+    }
+  }
+  return best;
 }
 
 struct ActLayout {
@@ -555,6 +639,17 @@ SVDQ_API int svdq_tensor_peak(int fmt, long long steps, void* stream) {
   return SVDQ_OK;
 }
 
+SVDQ_API int svdq_set_quant_split(int S, int C) {
+  auto pow2_le8 = [](int v) { return v == 1 || v == 2 || v == 4 || v == 8; };
+  if (S == 0 && C == 0) {
+    g_forced_split = {0, 0};
+    return SVDQ_OK;
+  }
+  if (!pow2_le8(S) || !pow2_le8(C)) return SVDQ_ERR_INVALID_ARG;
+  g_forced_split = {S, C};
+  return SVDQ_OK;
+}
+
 SVDQ_API int svdq_set_wait_budget(long long cycles) {
   if (cycles <= 0) return SVDQ_ERR_INVALID_ARG;
   g_budget = cycles;
@@ -772,7 +867,8 @@ SVDQ_API int svdq_quantize_act(const svdq_weights* w, const void* X, int M, void
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const ActLayout L = act_layout(w, M);
   uint8_t* base = static_cast<uint8_t*>(ws);
-  const int S = quant_stack_for(M, w->r_pad, g_dev[dev].sms);
+  const QuantSplit sp = quant_split_for(M, w->K, w->r_pad, g_dev[dev]);
+  const int S = sp.S;
   const int BM = kQuantTileRows / S;
   CUtensorMap tm_x, tm_codes;
   if ((rc = make_map(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, w->K, M, kQuantBK, BM)))
@@ -787,6 +883,8 @@ SVDQ_API int svdq_quantize_act(const svdq_weights* w, const void* X, int M, void
   p.K = w->K;
   p.r_pad = w->r_pad;
   p.S = S;
+  p.C = sp.C;
+  p.per = ((w->K + S * kQuantBK - 1) / (S * kQuantBK) + sp.C - 1) / sp.C;
   p.M_pad = L.M_pad;
   p.sf_kcols = w->sf_kcols;
   p.inv_lambda = w->inv_lambda;
@@ -800,20 +898,24 @@ SVDQ_API int svdq_quantize_act(const svdq_weights* w, const void* X, int M, void
     SVDQ_CUDA(cudaMemset2DAsync(p.sf + off, pitch, 0, pitch - off, L.M_pad / 128, st));
   }
   const QuantSmem Q = quant_smem_layout(w->fmt, w->r_pad, S);
-  const dim3 grid((M + BM - 1) / BM);
+  // clusters of C consecutive CTAs share a row block, one K range each
+  const dim3 grid(((M + BM - 1) / BM) * sp.C);
+  const unsigned C = static_cast<unsigned>(sp.C);
   const CUtensorMap& tm_l1t = w->r_pad > 0 ? w->tm_l1t : tm_x;
-  if (w->fmt == SVDQ_NVFP4)
-    quant_act_kernel<0><<<grid, kQuantThreads, Q.total, st>>>(tm_x, tm_l1t, tm_codes, p);
-  else if (w->fmt == SVDQ_FP4G32)
-    quant_act_kernel<2><<<grid, kQuantThreads, Q.total, st>>>(tm_x, tm_l1t, tm_codes, p);
-  else if (w->fmt == SVDQ_W8A8) {
+  const dim3 blk(kQuantThreads);
+  if (w->fmt == SVDQ_NVFP4) {
+    SVDQ_CUDA(launch_pdl(quant_act_kernel<0>, grid, blk, Q.total, st, C, tm_x, tm_l1t, tm_codes, p));
+  } else if (w->fmt == SVDQ_FP4G32) {
+    SVDQ_CUDA(launch_pdl(quant_act_kernel<2>, grid, blk, Q.total, st, C, tm_x, tm_l1t, tm_codes, p));
+  } else if (w->fmt == SVDQ_W8A8) {
     // the per-token scales first: they need all of K before any code
-    w8_row_scale_kernel<<<(M + 7) / 8, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(X), w->inv_lambda,
-                                                     M, w->K, reinterpret_cast<float*>(p.sf));
-    quant_act_kernel<3><<<grid, kQuantThreads, Q.total, st>>>(tm_x, tm_l1t, tm_codes, p);
-  } else
-    quant_act_kernel<1><<<grid, kQuantThreads, Q.total, st>>>(tm_x, tm_l1t, tm_codes, p);
-  SVDQ_CHECK_LAUNCH();
+    SVDQ_CUDA(launch_pdl(w8_row_scale_kernel, dim3((M + 7) / 8), dim3(256), 0, st, 0u,
+                         static_cast<const __nv_bfloat16*>(X), static_cast<const float*>(w->inv_lambda), M,
+                         w->K, reinterpret_cast<float*>(p.sf)));
+    SVDQ_CUDA(launch_pdl(quant_act_kernel<3>, grid, blk, Q.total, st, C, tm_x, tm_l1t, tm_codes, p));
+  } else {
+    SVDQ_CUDA(launch_pdl(quant_act_kernel<1>, grid, blk, Q.total, st, C, tm_x, tm_l1t, tm_codes, p));
+  }
   return SVDQ_OK;
 }
 
@@ -866,8 +968,8 @@ SVDQ_API int svdq_linear(const svdq_weights* w, const void* ws, int M, void* Y, 
     p.sf_kcols = w->sf_kcols;
     p.bias = w->bias;
     p.budget = wait_budget();
-    gemm_nvfp4_kernel<<<grid, kGemmThreads, kGemmSmemBytes, st>>>(tm_a, w->tm_b, tm_xl1, w->tm_l2t,
-                                                                  tm_y, p);
+    SVDQ_CUDA(launch_pdl(gemm_nvfp4_kernel, dim3(grid), dim3(kGemmThreads), kGemmSmemBytes, st, 0u, tm_a,
+                         w->tm_b, tm_xl1, w->tm_l2t, tm_y, p));
   } else if (w->fmt == SVDQ_W8A8) {
     CUtensorMap tm_y;
     if ((rc = make_map(&tm_y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Y, w->N, M, 16, 32))) return rc;
@@ -884,7 +986,8 @@ SVDQ_API int svdq_linear(const svdq_weights* w, const void* ws, int M, void* Y, 
     p.sw = reinterpret_cast<const float*>(w->wsf);
     p.bias = w->bias;
     p.budget = wait_budget();
-    gemm_w8a8_kernel<<<grid, kW8Threads, kW8SmemBytes, st>>>(tm_a, w->tm_b, tm_xl1, w->tm_l2t, tm_y, p);
+    SVDQ_CUDA(launch_pdl(gemm_w8a8_kernel, dim3(grid), dim3(kW8Threads), kW8SmemBytes, st, 0u, tm_a, w->tm_b,
+                         tm_xl1, w->tm_l2t, tm_y, p));
   } else {
     GemmI4Params p;
     p.M = M;
@@ -902,7 +1005,8 @@ SVDQ_API int svdq_linear(const svdq_weights* w, const void* ws, int M, void* Y, 
     p.bias = w->bias;
     p.Y = static_cast<__nv_bfloat16*>(Y);
     p.budget = wait_budget();
-    gemm_int4_kernel<<<grid, kI4Threads, kI4SmemBytes, st>>>(tm_a, w->tm_b, tm_xl1, w->tm_l2t, p);
+    SVDQ_CUDA(launch_pdl(gemm_int4_kernel, dim3(grid), dim3(kI4Threads), kI4SmemBytes, st, 0u, tm_a, w->tm_b,
+                         tm_xl1, w->tm_l2t, p));
   }
   SVDQ_CHECK_LAUNCH();
   return SVDQ_OK;

@@ -289,6 +289,19 @@ __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// ------------------------------------------- programmatic dependent launch ---
+// A kernel launched with programmatic stream serialization may start while the
+// previous kernel on its stream is still running.  griddep_wait() blocks until
+// that kernel has completed and its memory is visible; every access to memory
+// another kernel produces or consumes must come after it.  Setup that touches
+// only this CTA's own resources (barriers, TMEM, descriptor prefetch) may come
+// before.  griddep_launch_dependents() lets the next kernel in the stream be
+// scheduled as this grid's CTAs retire, so its setup overlaps this one's tail.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------- TMA store ---
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int x, int y) {
   asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
@@ -319,6 +332,9 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
   return r;
 }
 
+// Cluster-wide barrier: every thread of every CTA in the cluster arrives; the
+// release/acquire pair makes each CTA's earlier shared-memory writes visible to
+// the other CTAs' later distributed-shared-memory reads.
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
                    : "memory");
