@@ -66,14 +66,16 @@ def peaks():
 # reports null.  Y of the QKV layer (85 MB) is still mostly dirty in the
 # 126 MB L2 when the GEMM ends, so its write traffic is below Y's size.
 NCU_TRAFFIC = {
-    ("gemm_nvfp4_kernel", "c2_qkv/qkv", 4608): (60281344, "454e3f84fc5c6294"),
-    ("quant_act_kernel", "c2_qkv/qkv", 4608): (28556544, "bf98e5d72b08526b"),
-    ("gemm_int4_kernel", "c4_int4_lora/proj", 4608): (26704640, "330358d37af68794"),
+    ("gemm_nvfp4_kernel", "c2_qkv/qkv", 4608, "nvfp4"): (60545280, "ad5e0c5a2b61f3f0"),
+    ("quant_act_kernel", "c2_qkv/qkv", 4608, "nvfp4"): (28568320, "5fb8f3c157533352"),
+    ("gemm_int4_kernel", "c4_int4_lora/proj", 4608, "int4"): (26791680, "ebe4fe5fb792944f"),
+    ("gemm_w8a8_kernel", "c2_qkv/qkv", 4608, "w8a8"): (86310144, "f42f28fb8882d75e"),
 }
 KERNEL_SOURCES = {
     "gemm_nvfp4_kernel": ("gemm_nvfp4.cuh", "svdq_ptx.cuh", "svdq_formats.cuh"),
     "quant_act_kernel": ("quant_act.cuh", "svdq_ptx.cuh", "svdq_formats.cuh"),
     "gemm_int4_kernel": ("gemm_int4.cuh", "gemm_nvfp4.cuh", "svdq_ptx.cuh", "svdq_formats.cuh"),
+    "gemm_w8a8_kernel": ("gemm_w8a8.cuh", "gemm_nvfp4.cuh", "svdq_ptx.cuh", "svdq_formats.cuh"),
 }
 
 
@@ -86,10 +88,10 @@ def kernel_fingerprint(kernel):
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel, workload, M):
+def ncu_traffic(kernel, workload, M, fmt):
     """Measured DRAM bytes per launch, or None if not captured for this
-    workload or the kernel changed since."""
-    entry = NCU_TRAFFIC.get((kernel, workload, M))
+    workload and format or the kernel changed since."""
+    entry = NCU_TRAFFIC.get((kernel, workload, M, fmt))
     if entry is None or kernel_fingerprint(kernel) != entry[1]:
         return None
     return entry[0]
@@ -389,12 +391,12 @@ def run_ours(args):
         "roofline": {"bound": "tensor", "kernel": gemm_kernel,
                      "achieved": round(achieved, 1), "peak": round(fp_peak, 1), "unit": "TFLOP/s",
                      "frac": round(achieved / fp_peak, 4),
-                     "traffic": ncu_traffic(gemm_kernel, f"{args.config}/{spec.name}", M),
+                     "traffic": ncu_traffic(gemm_kernel, f"{args.config}/{spec.name}", M, spec.fmt),
                      "peak_note": f"{pk['source']}: bf16 {pk['bf16']} TF/s x {'2 (INT8)' if spec.fmt in INT8_KIND else '4 (FP4)'}"},
         "roofline_quant": {"bound": "hbm", "kernel": "quant_act_kernel", "achieved": round(q_gbs, 1),
                            "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": round(q_gbs / pk["hbm_gbs"], 4),
                            "algorithmic_bytes": int(q_bytes),
-                           "traffic": ncu_traffic("quant_act_kernel", f"{args.config}/{spec.name}", M)},
+                           "traffic": ncu_traffic("quant_act_kernel", f"{args.config}/{spec.name}", M, spec.fmt)},
         "e2e": {"value": round(flops / t_e2e / 1e12, 3), "unit": UNIT,
                 "h2d_bytes_per_step": int(X.numel() * 2), "d2h_bytes_per_step": int(Y.numel() * 2)},
         "gpu_launches": launches_per_step * args.steps,

@@ -435,7 +435,9 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
 }
 
 // W8A8 per-token scale (SVDQuant paper, Sec. 5.1, 8-bit setting):
-// s_x[m] = max_k |fp32(x[m,k]) * (1/lambda_k)| / 127, IEEE fp32, one warp per row.
+// s_x[m] = max_k |fp32(x[m,k]) * (1/lambda_k)| / 127, IEEE fp32, one warp per
+// row.  Each lane keeps four 16-byte loads of the row in flight; the guards
+// keep every load inside the row.
 __global__ void w8_row_scale_kernel(const __nv_bfloat16* __restrict__ X, const float* __restrict__ inv_lambda,
                                     int M, int K, float* __restrict__ sx) {
   const int m = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -445,17 +447,32 @@ __global__ void w8_row_scale_kernel(const __nv_bfloat16* __restrict__ X, const f
   if (m >= M) return;
   const uint4* xr = reinterpret_cast<const uint4*>(X + static_cast<size_t>(m) * K);
   const float4* il = reinterpret_cast<const float4*>(inv_lambda);
-  float amax = 0.0f;
-  for (int c = lane; c < K / 8; c += 32) {
-    const uint4 raw = __ldg(xr + c);
-    const float4 l0 = __ldg(il + 2 * c), l1 = __ldg(il + 2 * c + 1);
-    amax = fmax3(amax, fabsf(__fmul_rn(bf16_lo(raw.x), l0.x)), fabsf(__fmul_rn(bf16_hi(raw.x), l0.y)));
-    amax = fmax3(amax, fabsf(__fmul_rn(bf16_lo(raw.y), l0.z)), fabsf(__fmul_rn(bf16_hi(raw.y), l0.w)));
-    amax = fmax3(amax, fabsf(__fmul_rn(bf16_lo(raw.z), l1.x)), fabsf(__fmul_rn(bf16_hi(raw.z), l1.y)));
-    amax = fmax3(amax, fabsf(__fmul_rn(bf16_lo(raw.w), l1.z)), fabsf(__fmul_rn(bf16_hi(raw.w), l1.w)));
+  const int n8 = K / 8;   // 16-byte chunks of the row
+  float amax[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  for (int c0 = lane; c0 < n8; c0 += 4 * 32) {
+    uint4 raw[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int c = c0 + 32 * u;
+      raw[u] = c < n8 ? __ldg(xr + c) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int c = c0 + 32 * u;
+      if (c < n8) {
+        const float4 l0 = __ldg(il + 2 * c), l1 = __ldg(il + 2 * c + 1);
+        float a = amax[u];
+        a = fmax3(a, fabsf(__fmul_rn(bf16_lo(raw[u].x), l0.x)), fabsf(__fmul_rn(bf16_hi(raw[u].x), l0.y)));
+        a = fmax3(a, fabsf(__fmul_rn(bf16_lo(raw[u].y), l0.z)), fabsf(__fmul_rn(bf16_hi(raw[u].y), l0.w)));
+        a = fmax3(a, fabsf(__fmul_rn(bf16_lo(raw[u].z), l1.x)), fabsf(__fmul_rn(bf16_hi(raw[u].z), l1.y)));
+        a = fmax3(a, fabsf(__fmul_rn(bf16_lo(raw[u].w), l1.z)), fabsf(__fmul_rn(bf16_hi(raw[u].w), l1.w)));
+        amax[u] = a;
+      }
+    }
   }
-  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  if (lane == 0) sx[m] = __fdiv_rn(amax, 127.0f);
+  float a = fmaxf(fmaxf(amax[0], amax[1]), fmaxf(amax[2], amax[3]));
+  for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+  if (lane == 0) sx[m] = __fdiv_rn(a, 127.0f);
 }
 
 }  // namespace svdq
