@@ -124,8 +124,7 @@ __global__ void __launch_bounds__(kI4Threads, 1)
                      const __grid_constant__ CUtensorMap tm_xl1,
                      const __grid_constant__ CUtensorMap tm_l2t, const GemmI4Params p) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* smem = align_smem_1024(smem_raw);
   constexpr int S = kI4Stages;
   constexpr int NB = kI4Bufs;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kI4StageBytes * S);

@@ -58,8 +58,7 @@ __global__ void __launch_bounds__(kW8Threads, 1)
                      const __grid_constant__ CUtensorMap tm_y, const GemmW8Params p) {
   constexpr int STAGES = kW8Stages;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* smem = align_smem_1024(smem_raw);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kW8BarOff);
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;

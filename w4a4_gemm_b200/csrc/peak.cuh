@@ -25,8 +25,7 @@ template <int FMT>
 __global__ void __launch_bounds__(kPeakThreads, 1)
     tensor_peak_kernel(long long n_steps, long long budget) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* smem = align_smem_1024(smem_raw);
   uint64_t* done = reinterpret_cast<uint64_t*>(smem + kPeakSfOff + 12 * 512);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(done + 1);
   const uint32_t warp = warp_id();

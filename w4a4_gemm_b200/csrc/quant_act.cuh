@@ -106,8 +106,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
                      const __grid_constant__ CUtensorMap tm_codes, const QuantParams p) {
   extern __shared__ uint8_t smem_raw[];
   const QuantSmem L = quant_smem_layout(FMT, p.r_pad, p.S);
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* smem = align_smem_1024(smem_raw);
   const int NS = static_cast<int>(L.stages);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bar_off);
   uint64_t* empty = full + kQuantMaxStages;

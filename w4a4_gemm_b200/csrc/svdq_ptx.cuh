@@ -289,6 +289,16 @@ __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// ------------------------------------------------ dynamic shared memory ---
+// Dynamic shared memory rounded up to a 1024-byte boundary (the 128-byte TMA
+// swizzle repeats every 1024 bytes).  Offsetting the __shared__ array itself,
+// instead of rounding the pointer as an integer, keeps it visibly in the
+// shared window, so plain loads and stores through it compile to
+// shared-memory instructions rather than generic ones.
+__device__ __forceinline__ uint8_t* align_smem_1024(uint8_t* smem_raw) {
+  return smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+}
+
 // ------------------------------------------- programmatic dependent launch ---
 // A kernel launched with programmatic stream serialization may start while the
 // previous kernel on its stream is still running.  griddep_wait() blocks until
