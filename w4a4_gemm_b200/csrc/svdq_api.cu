@@ -230,19 +230,23 @@ int current_device(int* dev) {
 
 // ------------------------------------------------------------ workspace ---
 // Shape of the activation kernel's launch: S stacked K sub-tiles per stage
-// (BM = 128 / S rows per cluster) and C CTAs per cluster splitting K.  A CTA
-// consumes one 128 x 64 stage in about the same time whatever S is (its four
-// quantizer warps per stage set the pace), so the model is
-//   time = waves * (fixed + [C > 1] * exchange + stages per CTA * stage)
-// with the cycle counts measured on B200 (setup, first load and XL1 epilogue;
-// the cluster exchange of partial sums; one stage).  Ties go to the smaller C,
-// then the smaller S.
+// (BM = 128 / S rows per cluster) and C CTAs per cluster splitting K.  Cost
+// model, in cycles, fitted to forced launches of every shape on B200:
+//   time = waves * (fixed + [C > 1] (exchange + C * per_peer)
+//                   + stages per CTA * (stage + l1 * r_pad / BM))
+// fixed: setup, the first stage's round trip and the XL1 epilogue; exchange and
+// per_peer: the cluster barriers and the distributed-shared-memory reads of the
+// peers' partial sums; stage and l1: one 128 x 64 stage, whose L1s share
+// (r_pad / BM bytes per byte of X) travels and is read with it.  Ties go to
+// the smaller C, then the smaller S.
 struct QuantSplit {
   int S, C;
 };
 constexpr double kQuantFixedCycles = 10000.0;
 constexpr double kQuantExchangeCycles = 2000.0;
-constexpr double kQuantStageCycles = 1100.0;
+constexpr double kQuantPerPeerCycles = 1000.0;
+constexpr double kQuantStageCycles = 800.0;
+constexpr double kQuantL1Cycles = 300.0;
 QuantSplit g_forced_split{0, 0};   // svdq_set_quant_split; {0, 0} = automatic
 
 QuantSplit quant_split_for(int M, int K, int r_pad, const DeviceInfo& d) {
@@ -264,7 +268,8 @@ QuantSplit quant_split_for(int M, int K, int r_pad, const DeviceInfo& d) {
       const long long waves = (ctas + slots - 1) / slots;
       const int per = (stages + C - 1) / C;
       const double t = static_cast<double>(waves) *
-                       (kQuantFixedCycles + (C > 1 ? kQuantExchangeCycles : 0.0) + per * kQuantStageCycles);
+                       (kQuantFixedCycles + (C > 1 ? kQuantExchangeCycles + C * kQuantPerPeerCycles : 0.0) +
+                        per * (kQuantStageCycles + kQuantL1Cycles * r_pad / BM));
       if (t < best_t * 0.98) {
         best_t = t;
         best = {S, C};
