@@ -355,7 +355,10 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
   // the CTA barrier first.  Then each CTA of the cluster takes BM / C of the
   // rows and sums, for them, the parked blocks of every CTA (rank 0 first)
   // over j in fixed order, and rounds to bf16.
-  float* red = reinterpret_cast<float*>(smem);   // [128][r_pad] fp32
+  // [128][r_pad + 4] fp32: the 16-byte pad puts consecutive rows on different
+  // banks, so the lanes' row-wise float4 stores do not conflict
+  float* red = reinterpret_cast<float*>(smem);
+  const int rs = p.r_pad + 4;
   __syncthreads();
   if (has_lr && warp >= 2 && warp < 6) {
     const uint32_t q = warp & 3u;
@@ -382,7 +385,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
         if (jj == j) {
 #pragma unroll
           for (int e = 0; e < 16; e += 4)
-            *reinterpret_cast<float4*>(red + R * p.r_pad + c + e) =
+            *reinterpret_cast<float4*>(red + R * rs + c + e) =
                 make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]),
                             __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
         }
@@ -401,7 +404,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       for (int t = 0; t < p.C; ++t) {
         for (int jj = 0; jj < S; ++jj) {
-          const uint32_t src = map_shared_rank(smem_u32(red + (jj * BM + i) * p.r_pad + c), t);
+          const uint32_t src = map_shared_rank(smem_u32(red + (jj * BM + i) * rs + c), t);
           const float4 a = ld_shared_cluster_f32x4(src), b = ld_shared_cluster_f32x4(src + 16);
           const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
