@@ -26,10 +26,11 @@
 // (S, C) from the SM count and the resident clusters of each size.
 //   warp 0      : TMA producer (S X boxes BM x 64, S L1s^T boxes r_pad x 64, 1/lambda)
 //   warp 1      : TMEM owner; one lane issues the kind::f16 MMAs
-//   warps 2..13 : quantizers in three groups of four; group k takes every
-//                 third stage, and its warp w serves A-tile rows 32 (w % 4) .. + 31,
-//                 one lane per row over the whole 64-wide sub-tile.  They smooth
-//                 X, quantize it, release the stage and store codes and scales.
+//   warps 2..17 : quantizers in up to four groups of four (as many groups as
+//                 there are pipeline stages); group k takes every G-th stage,
+//                 and its warp w serves A-tile rows 32 (w % 4) .. + 31, one lane
+//                 per row over the whole 64-wide sub-tile.  They smooth X,
+//                 quantize it, release the stage and store codes and scales.
 //                 At the end warps 2..5 read the diagonal blocks and the CTA
 //                 sums them into XL1, kept at fp32 precision as a bf16 pair
 //                 hi + lo for the GEMM's tail MMA.
@@ -44,7 +45,7 @@ constexpr int kQuantTileRows = 128;   // rows of the MMA A operand
 constexpr int kQuantBK = 64;          // K width of one sub-tile
 constexpr int kQuantMaxStages = 12;
 constexpr int kQuantMaxSplit = 8;     // CTAs per cluster splitting K
-constexpr int kQuantGroups = 3;       // quantizer groups working on consecutive stages
+constexpr int kQuantGroups = 4;       // quantizer groups working on consecutive stages (at most)
 constexpr int kQuantGroupWarps = 4;   // warps per group: one lane per row of a 128-row stage
 constexpr int kQuantWarps = kQuantGroupWarps * kQuantGroups;
 constexpr int kQuantThreads = 32 * (2 + kQuantWarps);
@@ -59,6 +60,7 @@ struct QuantParams {
   int S;            // stacked K sub-tiles per stage (BM = 128 / S rows per cluster)
   int C;            // CTAs per cluster, each on its own K range (1, 2, 4 or 8; C <= BM)
   int per;          // stages per cluster rank: rank t takes stages [t per, min((t+1) per, total))
+  int groups;       // active quantizer groups G, 1 <= G <= min(kQuantGroups, pipeline stages)
   int M_pad;        // M rounded up to 128 (scale atoms)
   int sf_kcols;     // NVFP4: K_pad / 64 scale atoms per 128-row block
   const float* inv_lambda;  // K rounded up to 512 (zero padded)
@@ -210,7 +212,10 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ quantizers
-    // Group k = (warp - 2) / 4 takes the stages k, k + G, k + 2G, ... (G groups);
+    // Group k = (warp - 2) / 4 takes the stages k, k + G, k + 2G, ... (G active
+    // groups).  G never exceeds the number of stage buffers: a group then never
+    // waits on a stage whose buffer has not yet finished its previous fill, which
+    // the one-bit phase parity of the barrier could not tell apart.
     // its warp of lane quarter q quantizes rows 32 q .. 32 q + 31 of the
     // stacked tile, one lane per row over the whole 64-wide sub-tile: four
     // independent NVFP4 groups of 16 (or one INT4 group of 64) per lane.  The
@@ -228,7 +233,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
     const int m = m0 + static_cast<int>(R) % BM;
     const bool row_ok = m < p.M;
     int use = 0;
-    for (int li = grp; li < n_local; li += kQuantGroups, ++use) {
+    for (int li = grp < p.groups ? grp : n_local; li < n_local; li += p.groups, ++use) {
       const int i = i0 + li;
       const int s = li % NS;
       const uint32_t ph = (li / NS) & 1;

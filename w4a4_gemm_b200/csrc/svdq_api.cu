@@ -896,13 +896,15 @@ SVDQ_API int svdq_quantize_act(const svdq_weights* w, const void* X, int M, void
   p.sf = base + L.sf_off;
   p.xl1 = reinterpret_cast<__nv_bfloat16*>(base + L.xl1_off);
   p.budget = wait_budget();
+  const QuantSmem Q = quant_smem_layout(w->fmt, w->r_pad, S);
+  p.groups = std::min(kQuantGroups, static_cast<int>(Q.stages));
+  if (p.groups < 1) return SVDQ_ERR_UNSUPPORTED_SHAPE;
   if (is_fp4(w->fmt) && w->sf_kcols * 64 != w->K) {
     // zero the scale atoms of the K padding (read by the GEMM's last K step)
     const size_t pitch = static_cast<size_t>(w->sf_kcols) * 512;
     const size_t off = static_cast<size_t>(w->K / 64) * 512;
     SVDQ_CUDA(cudaMemset2DAsync(p.sf + off, pitch, 0, pitch - off, L.M_pad / 128, st));
   }
-  const QuantSmem Q = quant_smem_layout(w->fmt, w->r_pad, S);
   // clusters of C consecutive CTAs share a row block, one K range each
   const dim3 grid(((M + BM - 1) / BM) * sp.C);
   const unsigned C = static_cast<unsigned>(sp.C);

@@ -336,12 +336,6 @@ __device__ __forceinline__ void bulk_wait_group_all() {
 }
 
 // ---------------------------------------------------------------- cluster ---
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-
 // Cluster-wide barrier: every thread of every CTA in the cluster arrives; the
 // release/acquire pair makes each CTA's earlier shared-memory writes visible to
 // the other CTAs' later distributed-shared-memory reads.
@@ -355,12 +349,6 @@ __device__ __forceinline__ uint32_t map_shared_rank(uint32_t saddr, uint32_t ran
   uint32_t r;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
   return r;
-}
-
-__device__ __forceinline__ float ld_shared_cluster_f32(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-  return v;
 }
 
 __device__ __forceinline__ float4 ld_shared_cluster_f32x4(uint32_t addr) {
