@@ -66,10 +66,11 @@ def peaks():
 # reports null.  Y of the QKV layer (85 MB) is still mostly dirty in the
 # 126 MB L2 when the GEMM ends, so its write traffic is below Y's size.
 NCU_TRAFFIC = {
-    ("gemm_nvfp4_kernel", "c2_qkv/qkv", 4608, "nvfp4"): (60545280, "ad5e0c5a2b61f3f0"),
-    ("quant_act_kernel", "c2_qkv/qkv", 4608, "nvfp4"): (28568320, "5fb8f3c157533352"),
-    ("gemm_int4_kernel", "c4_int4_lora/proj", 4608, "int4"): (26791680, "ebe4fe5fb792944f"),
-    ("gemm_w8a8_kernel", "c2_qkv/qkv", 4608, "w8a8"): (86310144, "f42f28fb8882d75e"),
+    ("gemm_nvfp4_kernel", "c2_qkv/qkv", 4608, "nvfp4"): (60871936, "53a792da76c08882"),
+    ("quant_act_kernel", "c2_qkv/qkv", 4608, "nvfp4"): (28560640, "f61da2976a94a454"),
+    ("quant_act_kernel", "c5_block/fc2", 16384, "nvfp4"): (498567680, "f61da2976a94a454"),
+    ("gemm_int4_kernel", "c4_int4_lora/proj", 4608, "int4"): (26797312, "cea79a7c0c6f4575"),
+    ("gemm_w8a8_kernel", "c2_qkv/qkv", 4608, "w8a8"): (86851072, "0c1cad6d3aa86dc5"),
 }
 KERNEL_SOURCES = {
     "gemm_nvfp4_kernel": ("gemm_nvfp4.cuh", "svdq_ptx.cuh", "svdq_formats.cuh"),
