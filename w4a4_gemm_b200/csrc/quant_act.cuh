@@ -60,7 +60,6 @@ struct QuantParams {
   int S;            // stacked K sub-tiles per stage (BM = 128 / S rows per cluster)
   int C;            // CTAs per cluster, each on its own K range (1, 2, 4 or 8; C <= BM)
   int per;          // stages per cluster rank: rank t takes stages [t per, min((t+1) per, total))
-  int groups;       // active quantizer groups G, 1 <= G <= min(kQuantGroups, pipeline stages)
   int M_pad;        // M rounded up to 128 (scale atoms)
   int sf_kcols;     // NVFP4: K_pad / 64 scale atoms per 128-row block
   const float* inv_lambda;  // K rounded up to 512 (zero padded)
@@ -78,11 +77,21 @@ __host__ __device__ inline int quant_stack_max(int r_pad) {
 }
 
 struct QuantSmem {
-  uint32_t x_off, l1_off, il_off, stage_bytes, stages, stg_off, stg_bytes, bar_off, total;
+  uint32_t x_off, l1_off, il_off, stage_bytes, stages, groups, stg_off, stg_bytes, bar_off, total;
 };
 
 // Per stage: the stacked X tile, S slices of L1s^T and 1/lambda.  After the
 // stages: two code staging buffers (128 rows of codes) per quantizer group.
+// G groups take the stages in turn, and the buffer count is a multiple of G,
+// so stage buffer b always serves group b mod G; G is 4 or 3, whichever keeps
+// more of the buffers that fit (4 on a tie: the quantizers set the pace), or
+// the buffer count itself when fewer than three fit.  A group
+// waits on its next stage by the one-bit phase parity of the buffer's full
+// barrier; that parity is unambiguous only if the buffer's previous fill has
+// landed, which holds when that previous fill was this group's own stage.
+// (With buffers shared between groups, a group could wait while another
+// group's stage was still in flight to the same buffer -- TMA fills complete
+// out of order under load -- and match the phase before it.)
 __host__ __device__ inline QuantSmem quant_smem_layout(int fmt, int r_pad, int S) {
   QuantSmem L;
   L.x_off = 0;
@@ -94,6 +103,13 @@ __host__ __device__ inline QuantSmem quant_smem_layout(int fmt, int r_pad, int S
   const uint32_t stg_total = 2u * kQuantGroups * L.stg_bytes;
   L.stages = (kQuantSmemBudget - stg_total) / L.stage_bytes;
   if (L.stages > static_cast<uint32_t>(kQuantMaxStages)) L.stages = kQuantMaxStages;
+  if (L.stages < 3u) {
+    L.groups = L.stages;
+  } else {
+    static_assert(kQuantGroups == 4, "the group rule below picks 4 or 3 groups");
+    L.groups = (L.stages - L.stages % 4u) >= (L.stages - L.stages % 3u) ? 4u : 3u;
+  }
+  if (L.groups > 0) L.stages -= L.stages % L.groups;
   L.stg_off = L.stage_bytes * L.stages;
   L.bar_off = L.stg_off + stg_total;
   L.total = L.bar_off + 256 + 512 + 1024;                  // barriers, 1/scale table, alignment
@@ -213,9 +229,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
   } else {
     // ------------------------------------------------------------ quantizers
     // Group k = (warp - 2) / 4 takes the stages k, k + G, k + 2G, ... (G active
-    // groups).  G never exceeds the number of stage buffers: a group then never
-    // waits on a stage whose buffer has not yet finished its previous fill, which
-    // the one-bit phase parity of the barrier could not tell apart.
+    // groups; stage buffer b always serves group b mod G, see quant_smem_layout);
     // its warp of lane quarter q quantizes rows 32 q .. 32 q + 31 of the
     // stacked tile, one lane per row over the whole 64-wide sub-tile: four
     // independent NVFP4 groups of 16 (or one INT4 group of 64) per lane.  The
@@ -233,7 +247,8 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
     const int m = m0 + static_cast<int>(R) % BM;
     const bool row_ok = m < p.M;
     int use = 0;
-    for (int li = grp < p.groups ? grp : n_local; li < n_local; li += p.groups, ++use) {
+    const int G = static_cast<int>(L.groups);
+    for (int li = grp < G ? grp : n_local; li < n_local; li += G, ++use) {
       const int i = i0 + li;
       const int s = li % NS;
       const uint32_t ph = (li / NS) & 1;

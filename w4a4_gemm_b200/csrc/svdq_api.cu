@@ -897,8 +897,7 @@ SVDQ_API int svdq_quantize_act(const svdq_weights* w, const void* X, int M, void
   p.xl1 = reinterpret_cast<__nv_bfloat16*>(base + L.xl1_off);
   p.budget = wait_budget();
   const QuantSmem Q = quant_smem_layout(w->fmt, w->r_pad, S);
-  p.groups = std::min(kQuantGroups, static_cast<int>(Q.stages));
-  if (p.groups < 1) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  if (Q.groups < 1 || Q.stages % Q.groups != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
   if (is_fp4(w->fmt) && w->sf_kcols * 64 != w->K) {
     // zero the scale atoms of the K padding (read by the GEMM's last K step)
     const size_t pitch = static_cast<size_t>(w->sf_kcols) * 512;
