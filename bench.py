@@ -67,8 +67,8 @@ def peaks():
 # 126 MB L2 when the GEMM ends, so its write traffic is below Y's size.
 NCU_TRAFFIC = {
     ("gemm_nvfp4_kernel", "c2_qkv/qkv", 4608, "nvfp4"): (60871936, "53a792da76c08882"),
-    ("quant_act_kernel", "c2_qkv/qkv", 4608, "nvfp4"): (28560640, "f61da2976a94a454"),
-    ("quant_act_kernel", "c5_block/fc2", 16384, "nvfp4"): (498567680, "f61da2976a94a454"),
+    ("quant_act_kernel", "c2_qkv/qkv", 4608, "nvfp4"): (28561152, "325548569b93b04d"),
+    ("quant_act_kernel", "c5_block/fc2", 16384, "nvfp4"): (498218752, "325548569b93b04d"),
     ("gemm_int4_kernel", "c4_int4_lora/proj", 4608, "int4"): (26797312, "cea79a7c0c6f4575"),
     ("gemm_w8a8_kernel", "c2_qkv/qkv", 4608, "w8a8"): (86851072, "0c1cad6d3aa86dc5"),
 }
