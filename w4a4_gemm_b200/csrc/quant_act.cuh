@@ -246,6 +246,11 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
     const int j = static_cast<int>(R) / BM;    // K sub-tile
     const int m = m0 + static_cast<int>(R) % BM;
     const bool row_ok = m < p.M;
+    float w8_inv = 0.0f;   // W8A8: 1 / this row's token scale, fixed for every stage
+    if constexpr (FMT == 3) {
+      const float sd = reinterpret_cast<const float*>(p.sf)[row_ok ? m : 0];
+      w8_inv = (sd == 0.0f || !row_ok) ? 0.0f : __frcp_rn(sd);
+    }
     int use = 0;
     const int G = static_cast<int>(L.groups);
     for (int li = grp < G ? grp : n_local; li < n_local; li += G, ++use) {
@@ -298,8 +303,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
         sfw = s0 * 0x0101u | (s1 * 0x0101u) << 16;
       } else if constexpr (FMT == 3) {
         // int8 codes of this row with its per-token scale
-        const float sd = reinterpret_cast<const float*>(p.sf)[row_ok ? m : 0];
-        const float inv = (sd == 0.0f || !row_ok) ? 0.0f : __frcp_rn(sd);
+        const float inv = w8_inv;
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           uint32_t w = 0;
