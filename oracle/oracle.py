@@ -87,7 +87,7 @@ def lib() -> ctypes.CDLL:
         _lib.oracle_fold_l1.argtypes = [I, I, P, P, P]
         _lib.oracle_fold_l1.restype = None
         _lib.oracle_weight_quant.argtypes = [I, I, I, P, P, P]
-        _lib.oracle_linear_rows.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, P, I, P]
+        _lib.oracle_linear_rows.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, P, I, I, P]
         _lib.oracle_dequant.argtypes = [I, I, I, P, P, P]
     return _lib
 
@@ -310,11 +310,34 @@ def prepare(W_bits: np.ndarray, x_absmax: Optional[np.ndarray], rank: int,
 # quantization and the layer (C oracle)
 # --------------------------------------------------------------------------
 
-def weight_quant(fmt, R: np.ndarray):
+def prescale_exponent(fmt, R: np.ndarray) -> int:
+    """The optional power-of-two prescale of the weight residual (FP4 formats):
+    the largest integer e with 2^e * s_max <= 448, the top of the E4M3 range,
+    where s_max = fp32(max|R| / 6) is the largest group scale before rounding;
+    0 when R is zero or the format's scales are not E4M3.  The E4M3 scale
+    bottoms out at subnormals near 2^-9; multiplying R by 2^e (exact) lifts
+    small residuals' scales back into the normal range.  The paper has no
+    global scale for its FP4 groups; this is an opt-in reading."""
+    fmt = _FMT[fmt]
+    if fmt not in (NVFP4, FP4G32):
+        return 0
+    amax = np.float32(np.max(np.abs(np.asarray(R, dtype=np.float32)))) if np.size(R) else np.float32(0)
+    s_max = np.float32(amax) / np.float32(6.0)
+    if s_max == 0:
+        return 0
+    f, q = np.frexp(np.float64(s_max))   # s_max = f 2^q, 0.5 <= f < 1; 448 = 0.875 * 2^9
+    e = (9 - int(q)) if f <= 0.875 else (8 - int(q))
+    return max(-64, min(64, e))
+
+
+def weight_quant(fmt, R: np.ndarray, exp: int = 0):
     """Quantize R (K x N fp32) along K per output column -> codes (N x K/2), scales (N x K/g);
-    W8A8: codes N x K int8, scales N fp32 (one per output channel)."""
+    W8A8: codes N x K int8, scales N fp32 (one per output channel).  exp != 0
+    quantizes R * 2^exp (the prescale, exact in fp32)."""
     fmt = _FMT[fmt]
     R = np.ascontiguousarray(R, dtype=np.float32)
+    if exp:
+        R = np.ldexp(R, np.int32(exp)).astype(np.float32)
     K, N = R.shape
     if fmt == W8A8:
         codes = np.zeros((N, K), dtype=np.int8)
@@ -369,8 +392,10 @@ def act_quant(fmt, X_bits: np.ndarray, inv_lambda: Optional[np.ndarray], L1_bits
 
 
 def linear(fmt, act, wq, L2_bits: Optional[np.ndarray], bias_bits: Optional[np.ndarray],
-           N: int, rows: Optional[np.ndarray] = None) -> np.ndarray:
-    """Y rows (bf16 bits): 4-bit GEMM over groups + XL1 L2 + bias, fp32 accumulation."""
+           N: int, rows: Optional[np.ndarray] = None, w_exp: int = 0) -> np.ndarray:
+    """Y rows (bf16 bits): 4-bit GEMM over groups + XL1 L2 + bias, fp32 accumulation.
+    w_exp: the weights were quantized with the prescale 2^w_exp; the group sum is
+    scaled back by 2^-w_exp before the branch and the bias are added."""
     fmt = _FMT[fmt]
     cx, sx, XL1 = act
     cw, sw = wq
@@ -389,7 +414,8 @@ def linear(fmt, act, wq, L2_bits: Optional[np.ndarray], bias_bits: Optional[np.n
                                          _ptr(L2), _ptr(bias), _ptr(rows_arr), n_rows, _ptr(Y))
     else:
         rc = lib().oracle_linear_rows(fmt, M, N, K, r, _ptr(cx), _ptr(sx), _ptr(XL1), _ptr(cw),
-                                      _ptr(sw), _ptr(L2), _ptr(bias), _ptr(rows_arr), n_rows, _ptr(Y))
+                                      _ptr(sw), _ptr(L2), _ptr(bias), _ptr(rows_arr), n_rows, int(w_exp),
+                                      _ptr(Y))
     assert rc == 0
     return Y
 
@@ -409,13 +435,14 @@ def dequant(fmt, codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
 
 
 def layer(fmt, X_bits, W_bits, rank: int, bias_bits=None, lora_A_bits=None, lora_B_bits=None,
-          x_absmax=None, smooth: bool = True, rows=None) -> dict:
+          x_absmax=None, smooth: bool = True, rows=None, pow2_prescale: bool = False) -> dict:
     """The whole layer: prepare (fp64), quantize W and X, GEMM; returns every intermediate."""
     if smooth and x_absmax is None:
         x_absmax = calib_absmax(X_bits)
     prep = prepare(W_bits, x_absmax if smooth else None, rank, lora_A_bits, lora_B_bits)
-    wq = weight_quant(fmt, prep["R"])
+    w_exp = prescale_exponent(fmt, prep["R"]) if pow2_prescale else 0
+    wq = weight_quant(fmt, prep["R"], w_exp)
     r = prep["rank"]
     act = act_quant(fmt, X_bits, prep["inv_lambda"], prep["L1"] if r else None)
-    Y = linear(fmt, act, wq, prep["L2"] if r else None, bias_bits, W_bits.shape[1], rows)
-    return {"prep": prep, "wq": wq, "act": act, "Y": Y}
+    Y = linear(fmt, act, wq, prep["L2"] if r else None, bias_bits, W_bits.shape[1], rows, w_exp)
+    return {"prep": prep, "wq": wq, "act": act, "Y": Y, "w_exp": w_exp}

@@ -342,10 +342,13 @@ int oracle_weight_quant(int fmt, int K, int N, const float *R, uint8_t *codes, v
 /* for the rows listed in `rows` (all rows if rows == NULL, n_rows = M) and   */
 /* all N columns; Y is n_rows x N bf16.  L2: r x N bf16; bias may be NULL.   */
 /* ------------------------------------------------------------------------- */
+/* w_exp: the weight codes and scales are those of R * 2^w_exp (the optional
+ * power-of-two prescale of the weight residual); the group sum is multiplied
+ * by 2^-w_exp (exact) before the branch and the bias are added. */
 int oracle_linear_rows(int fmt, int M, int N, int K, int r, const uint8_t *codes_x,
                        const void *scales_x, const float *XL1, const uint8_t *codes_w,
                        const void *scales_w, const uint16_t *L2, const uint16_t *bias,
-                       const int *rows, int n_rows, uint16_t *Y) {
+                       const int *rows, int n_rows, int w_exp, uint16_t *Y) {
     int g = fmt_group(fmt);
     if (K % g) return 1;
     int G = K / g;
@@ -371,6 +374,7 @@ int oracle_linear_rows(int fmt, int M, int N, int K, int r, const uint8_t *codes
                     part += deq_code(fmt, get_nibble(cx, k)) * deq_code(fmt, get_nibble(cw, k));
                 acc += (sx * sw) * part;
             }
+            acc = ldexpf(acc, -w_exp);
             for (int j = 0; j < r; ++j)
                 acc += XL1[(long)m * r + j] * oracle_bf16_decode(L2[(long)j * N + n]);
             if (bias) acc += oracle_bf16_decode(bias[n]);
