@@ -71,6 +71,18 @@ typedef enum { SVDQ_NVFP4 = 0, SVDQ_INT4 = 1, SVDQ_FP4G32 = 2, SVDQ_W8A8 = 3 } s
 typedef struct svdq_weights svdq_weights;
 
 /* Inputs of svdq_prepare_weights (all device pointers). */
+/* Preparation flags.
+ * SVDQ_WEIGHT_POW2_PRESCALE (FP4 formats; ignored by INT4 and W8A8): quantize
+ *   the residual as R * 2^e, e the largest integer with 2^e * max|R| / 6 <= 448,
+ *   so that small residuals keep normal E4M3 group scales (the E4M3 range ends
+ *   in subnormals near 2^-9, and a weight whose group maxima sit near 10^-3
+ *   would lose its scales there); the GEMM multiplies its group sum by 2^-e
+ *   (exact) before the low-rank branch and the bias are added.  The paper has
+ *   no global scale for its 4-bit groups; off by default.  The exponent is
+ *   reported by svdq_weights_scale_exponent; the exported codes and scales are
+ *   those of R * 2^e. */
+#define SVDQ_WEIGHT_POW2_PRESCALE 1u
+
 typedef struct {
   int fmt;                 /* svdq_format */
   int K, N;                /* W is K x N: input channels x output channels */
@@ -82,6 +94,7 @@ typedef struct {
   const void* lora_B;      /* bf16 lora_rank x N, or NULL */
   int lora_rank;           /* 0 = no LoRA */
   int refine_iters;        /* iterative updates of the low-rank branch (Sec. 4.2), 0 = none */
+  unsigned flags;          /* SVDQ_WEIGHT_POW2_PRESCALE or 0 */
 } svdq_prepare_desc;
 
 /* Inputs of svdq_load_weights: an already decomposed layer (device pointers). */
@@ -93,6 +106,7 @@ typedef struct {
   const void* L2;          /* bf16 rank x N (ignored if rank == 0) */
   const float* R;          /* fp32 K x N residual, quantized here */
   const void* bias;        /* bf16 N, or NULL */
+  unsigned flags;          /* SVDQ_WEIGHT_POW2_PRESCALE or 0 */
 } svdq_parts_desc;
 
 /* Calibration statistic for the smoothing factor (Sec. 4.2):
@@ -130,6 +144,9 @@ SVDQ_API int svdq_append_lora(svdq_weights* w, const void* lora_A, const void* l
 /* Weight error ||W_hat - L1 L2 - deq(Q(R))||_F of the SVD start and of the
  * kept iterate of svdq_prepare_weights' refinement (both -1 without it). */
 SVDQ_API int svdq_weights_refine_error(const svdq_weights* w, double* initial, double* kept);
+
+/* The weight prescale exponent e of a handle (0 without SVDQ_WEIGHT_POW2_PRESCALE). */
+SVDQ_API int svdq_weights_scale_exponent(const svdq_weights* w, int* exponent);
 
 /* Shape of a handle; any output pointer may be NULL. */
 SVDQ_API int svdq_weights_info(const svdq_weights* w, int* fmt, int* K, int* N, int* rank,

@@ -50,6 +50,10 @@ def test_host_side_argument_rejection(L):
         assert L.svdq_prepare_weights(ctypes.byref(d), None, ctypes.byref(h)) == want, (K, N, rank, fmt)
     d = S._PrepareDesc(0, 256, 256, 16, fake.value, None, None, fake.value, None, 8)
     assert L.svdq_prepare_weights(ctypes.byref(d), None, ctypes.byref(h)) == 1   # LoRA B missing
+    d = S._PrepareDesc(0, 256, 256, 16, fake.value, None, None, None, None, 0, 0, 6)
+    assert L.svdq_prepare_weights(ctypes.byref(d), None, ctypes.byref(h)) == 1   # unknown flag bits
+    e = ctypes.c_int()
+    assert L.svdq_weights_scale_exponent(None, ctypes.byref(e)) == 1
     n = ctypes.c_size_t()
     assert L.svdq_act_workspace_bytes(None, 16, ctypes.byref(n)) == 1
     assert L.svdq_quantize_act(None, fake, 16, fake, None) == 1

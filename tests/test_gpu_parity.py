@@ -191,6 +191,72 @@ def test_forced_launch_shapes(S, M, K, N, rank, fmt):
         w.close()
 
 
+@pytest.mark.parametrize("fmt", ["nvfp4", "fp4g32"])
+def test_pow2_prescale_parity(S, fmt):
+    """Small weights with the power-of-two prescale: the library's exponent, weight
+    codes and scales are the oracle's for R * 2^e, and Y (also after a LoRA is
+    appended, which rebuilds the scaled tail operand) is within tolerance of the
+    oracle's layer that scales the group sum back by 2^-e."""
+    M, K, N, r, rl = 150, 512, 384, 32, 16
+    d = WL.make_small(M, K, N, rank=r, fmt=fmt, bias=True, lora_rank=rl, seed=31)
+    Xb = WL.bf16_bits(d["X"])
+    Wb = WL.bf16_bits((d["W"].float() * 0.01).to(torch.bfloat16))
+    bb = WL.bf16_bits(d["bias"])
+    prep = O.prepare(Wb, O.calib_absmax(Xb), r)
+    e = O.prescale_exponent(fmt, prep["R"])
+    assert e > 0
+    wq = O.weight_quant(fmt, prep["R"], e)
+    w = S.svdq_load_weights(to_dev_f32(prep["R"]), fmt=fmt, L1=to_dev_bits(prep["L1"]),
+                            L2=to_dev_bits(prep["L2"]), inv_lambda=to_dev_f32(prep["inv_lambda"]),
+                            lam=to_dev_f32(prep["lam"]), bias=to_dev_bits(bb), pow2_prescale=True)
+    try:
+        assert S.svdq_weights_scale_exponent(w) == e
+        ex = S.svdq_export_weights(w)
+        assert np.array_equal(ex["scales"], wq[1]) and np.array_equal(ex["codes"], wq[0])
+        assert np.array_equal(ex["L2"], prep["L2"])          # the exported factor is unscaled
+        act = O.act_quant(fmt, Xb, prep["inv_lambda"], prep["L1"])
+        y_ref = O.linear(fmt, act, wq, prep["L2"], bb, N, w_exp=e)
+        ws, Y = _run_layer(S, w, Xb)
+        ok, info = y_within_tol(bits(Y), y_ref)
+        assert ok, ("Y", info)
+        # LoRA folded into the branch of the prescaled handle
+        S.svdq_append_lora(w, d["lora_A"].cuda(), d["lora_B"].cuda())
+        ref = O.prepare(Wb, O.calib_absmax(Xb), r, WL.bf16_bits(d["lora_A"]), WL.bf16_bits(d["lora_B"]))
+        act = O.act_quant(fmt, Xb, ref["inv_lambda"], ref["L1"])
+        y_ref = O.linear(fmt, act, wq, ref["L2"], bb, N, w_exp=e)
+        ws, Y = _run_layer(S, w, Xb)
+        ok, info = y_within_tol(bits(Y), y_ref)
+        assert ok, ("Y after LoRA", info)
+    finally:
+        w.close()
+
+
+def test_pow2_prescale_in_preparation(S):
+    """svdq_prepare_weights with the prescale: the codes are the oracle quantizer's
+    of R * 2^e for the library's own residual, and on a weight whose scales would
+    sit in the E4M3 subnormal range the layer is much closer to X W."""
+    M, K, N = 128, 512, 256
+    d = WL.make_small(M, K, N, rank=0, seed=32, x_outliers=0)
+    Wt = (d["W"].float() * 0.02).to(torch.bfloat16)
+    Xb, Wb = WL.bf16_bits(d["X"]), WL.bf16_bits(Wt)
+    exact = O.bf16_decode(Xb).astype(np.float64) @ O.bf16_decode(Wb).astype(np.float64)
+    err = {}
+    for pre in (False, True):
+        w = S.svdq_prepare_weights(Wt.cuda(), 0, "nvfp4", pow2_prescale=pre)
+        try:
+            e = S.svdq_weights_scale_exponent(w)
+            R = O.bf16_decode(Wb).astype(np.float32)        # rank 0, lambda = 1: R = W
+            assert e == (O.prescale_exponent("nvfp4", R) if pre else 0)
+            ex = S.svdq_export_weights(w)
+            codes, scales = O.weight_quant("nvfp4", R, e)
+            assert np.array_equal(ex["scales"], scales) and np.array_equal(ex["codes"], codes)
+            ws, Y = _run_layer(S, w, Xb)
+            err[pre] = np.linalg.norm(O.bf16_decode(bits(Y)) - exact) / np.linalg.norm(exact)
+        finally:
+            w.close()
+    assert err[True] < 0.25 and err[False] > 0.9, err
+
+
 def test_prepare_weights_invariants(S):
     """The library's own preparation (cuSOLVER on the fp64 Gram matrix):
     1/lambda bit-exact, the branch spans the oracle's optimal rank-r subspace,

@@ -38,7 +38,7 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "device all
           4: "CUDA error", 5: "device wait timed out", 6: "cuSOLVER/cuBLAS error"}
 
 EXPORTED = ("svdq_calib_absmax", "svdq_prepare_weights", "svdq_load_weights", "svdq_append_lora",
-            "svdq_weights_info", "svdq_weights_refine_error", "svdq_act_workspace_bytes", "svdq_quantize_act", "svdq_linear",
+            "svdq_weights_info", "svdq_weights_refine_error", "svdq_weights_scale_exponent", "svdq_act_workspace_bytes", "svdq_quantize_act", "svdq_linear",
             "svdq_forward", "svdq_forward_noalloc", "svdq_export_act", "svdq_export_weights", "svdq_get_error",
             "svdq_set_wait_budget", "svdq_set_quant_split", "svdq_status_string", "svdq_tensor_peak",
             "svdq_weights_destroy")
@@ -55,14 +55,17 @@ class _PrepareDesc(ctypes.Structure):
                 ("rank", ctypes.c_int), ("W", ctypes.c_void_p), ("x_absmax", ctypes.c_void_p),
                 ("bias", ctypes.c_void_p), ("lora_A", ctypes.c_void_p),
                 ("lora_B", ctypes.c_void_p), ("lora_rank", ctypes.c_int),
-                ("refine_iters", ctypes.c_int)]
+                ("refine_iters", ctypes.c_int), ("flags", ctypes.c_uint)]
 
 
 class _PartsDesc(ctypes.Structure):
     _fields_ = [("fmt", ctypes.c_int), ("K", ctypes.c_int), ("N", ctypes.c_int),
                 ("rank", ctypes.c_int), ("inv_lambda", ctypes.c_void_p),
                 ("lambda_", ctypes.c_void_p), ("L1", ctypes.c_void_p), ("L2", ctypes.c_void_p),
-                ("R", ctypes.c_void_p), ("bias", ctypes.c_void_p)]
+                ("R", ctypes.c_void_p), ("bias", ctypes.c_void_p), ("flags", ctypes.c_uint)]
+
+
+WEIGHT_POW2_PRESCALE = 1   # svdq_prepare_desc / svdq_parts_desc flag (see include/svdq.h)
 
 
 _lib = None
@@ -83,6 +86,7 @@ def lib() -> ctypes.CDLL:
     L.svdq_append_lora.argtypes = [P, P, P, I, P]
     L.svdq_weights_info.argtypes = [P] + [ctypes.POINTER(I)] * 5
     L.svdq_weights_refine_error.argtypes = [P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)]
+    L.svdq_weights_scale_exponent.argtypes = [P, ctypes.POINTER(ctypes.c_int)]
     L.svdq_act_workspace_bytes.argtypes = [P, I, ctypes.POINTER(ctypes.c_size_t)]
     L.svdq_quantize_act.argtypes = [P, P, I, P, P]
     L.svdq_linear.argtypes = [P, P, I, P, P]
@@ -176,7 +180,7 @@ def svdq_calib_absmax(X: torch.Tensor, out: Optional[torch.Tensor] = None, accum
 def svdq_prepare_weights(W: torch.Tensor, rank: int, fmt="nvfp4", x_absmax: Optional[torch.Tensor] = None,
                          bias: Optional[torch.Tensor] = None, lora_A: Optional[torch.Tensor] = None,
                          lora_B: Optional[torch.Tensor] = None, refine_iters: int = 0,
-                         stream=None) -> Weights:
+                         pow2_prescale: bool = False, stream=None) -> Weights:
     _dev(W, torch.bfloat16, "W")
     K, N = W.shape
     if x_absmax is not None:
@@ -192,7 +196,8 @@ def svdq_prepare_weights(W: torch.Tensor, rank: int, fmt="nvfp4", x_absmax: Opti
                      x_absmax.data_ptr() if x_absmax is not None else None,
                      bias.data_ptr() if bias is not None else None,
                      lora_A.data_ptr() if lora_A is not None else None,
-                     lora_B.data_ptr() if lora_B is not None else None, rl, int(refine_iters))
+                     lora_B.data_ptr() if lora_B is not None else None, rl, int(refine_iters),
+                     WEIGHT_POW2_PRESCALE if pow2_prescale else 0)
     h = ctypes.c_void_p()
     _check(lib().svdq_prepare_weights(ctypes.byref(d), _stream(stream), ctypes.byref(h)),
            "svdq_prepare_weights")
@@ -202,7 +207,7 @@ def svdq_prepare_weights(W: torch.Tensor, rank: int, fmt="nvfp4", x_absmax: Opti
 def svdq_load_weights(R: torch.Tensor, fmt="nvfp4", L1: Optional[torch.Tensor] = None,
                       L2: Optional[torch.Tensor] = None, inv_lambda: Optional[torch.Tensor] = None,
                       lam: Optional[torch.Tensor] = None, bias: Optional[torch.Tensor] = None,
-                      stream=None) -> Weights:
+                      pow2_prescale: bool = False, stream=None) -> Weights:
     _dev(R, torch.float32, "R")
     K, N = R.shape
     r = 0 if L1 is None else L1.shape[1]
@@ -217,7 +222,8 @@ def svdq_load_weights(R: torch.Tensor, fmt="nvfp4", L1: Optional[torch.Tensor] =
     d = _PartsDesc(_FMT[fmt], K, N, r, inv_lambda.data_ptr() if inv_lambda is not None else None,
                    lam.data_ptr() if lam is not None else None,
                    L1.data_ptr() if r else None, L2.data_ptr() if r else None, R.data_ptr(),
-                   bias.data_ptr() if bias is not None else None)
+                   bias.data_ptr() if bias is not None else None,
+                   WEIGHT_POW2_PRESCALE if pow2_prescale else 0)
     h = ctypes.c_void_p()
     _check(lib().svdq_load_weights(ctypes.byref(d), _stream(stream), ctypes.byref(h)), "svdq_load_weights")
     return Weights(h)
@@ -314,6 +320,13 @@ def svdq_export_weights(w: Weights) -> dict:
 
 def svdq_get_error() -> int:
     return int(lib().svdq_get_error())
+
+
+def svdq_weights_scale_exponent(w: "Weights") -> int:
+    """e of the weight prescale: the stored codes and scales are those of R * 2^e."""
+    e = ctypes.c_int()
+    _check(lib().svdq_weights_scale_exponent(w.handle, ctypes.byref(e)), "svdq_weights_scale_exponent")
+    return e.value
 
 
 def svdq_weights_refine_error(w: "Weights"):

@@ -66,6 +66,7 @@ struct GemmParams {
   const uint8_t* sfb;  // weight scale atoms     [N_pad/128][sf_kcols][512]
   int sf_kcols;        // K_pad / 64, K_pad = K rounded up to 256
   const __nv_bfloat16* bias;  // N or nullptr
+  float out_scale;     // 2^-e of the weight prescale: y = acc * out_scale + b (exact scaling)
   long long budget;
 };
 
@@ -81,13 +82,14 @@ __device__ __forceinline__ uint64_t sf_desc(uint32_t saddr) {
 }
 
 // Epilogue: 16 fp32 accumulators of this lane's row (columns n0 .. n0 + 15)
-// + bias -> bf16 -> the warp's buffer (32 rows of 32 bytes in the TMA 32-byte
+// times out_scale (a power of two: exact) + bias -> bf16 -> the warp's buffer (32 rows of 32 bytes in the TMA 32-byte
 // swizzle: the 16-byte half c of row r sits at half c ^ ((r >> 2) & 1)) ->
 // one TMA store of the 32 x 16 box at (n0, row0).  The store clips rows past M
 // and columns past N; the bias is read only below N (N % 16 == 0).
 __device__ __forceinline__ void epi_store_16(const uint32_t* r, uint8_t* buf, const CUtensorMap* tm_y,
                                              int n0, int row0, int N,
-                                             const __nv_bfloat16* __restrict__ bias, uint32_t lane) {
+                                             const __nv_bfloat16* __restrict__ bias, float out_scale,
+                                             uint32_t lane) {
   float bb[16];
 #pragma unroll
   for (int j = 0; j < 16; ++j) bb[j] = 0.f;
@@ -106,7 +108,8 @@ __device__ __forceinline__ void epi_store_16(const uint32_t* r, uint8_t* buf, co
   uint32_t w[8];
 #pragma unroll
   for (int t = 0; t < 8; ++t)
-    w[t] = pack_bf16x2(__uint_as_float(r[2 * t]) + bb[2 * t], __uint_as_float(r[2 * t + 1]) + bb[2 * t + 1]);
+    w[t] = pack_bf16x2(__fmaf_rn(__uint_as_float(r[2 * t]), out_scale, bb[2 * t]),
+                       __fmaf_rn(__uint_as_float(r[2 * t + 1]), out_scale, bb[2 * t + 1]));
   if (lane == 0) bulk_wait_group_read<0>();   // the previous store has read the buffer
   __syncwarp();
   const uint32_t row_addr = smem_u32(buf) + lane * 32u;
@@ -312,7 +315,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
         for (int c = 0; c < 8; ++c)
           if (nb + 16 * c < p.N)
-            epi_store_16(&v[c / 2][16 * (c % 2)], ebuf, &tm_y, nb + 16 * c, row0, p.N, p.bias, lane);
+            epi_store_16(&v[c / 2][16 * (c % 2)], ebuf, &tm_y, nb + 16 * c, row0, p.N, p.bias, p.out_scale,
+                         lane);
       }
     }
     if (lane == 0) bulk_wait_group_all();

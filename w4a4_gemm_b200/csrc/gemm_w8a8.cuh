@@ -230,8 +230,8 @@ __global__ void __launch_bounds__(kW8Threads, 1)
           }
         }
         if (row0 < p.M) {
-          if (n0 < p.N) epi_store_16(y, ebuf, &tm_y, n0, row0, p.N, p.bias, lane);
-          if (n0 + 16 < p.N) epi_store_16(y + 16, ebuf, &tm_y, n0 + 16, row0, p.N, p.bias, lane);
+          if (n0 < p.N) epi_store_16(y, ebuf, &tm_y, n0, row0, p.N, p.bias, 1.0f, lane);
+          if (n0 + 16 < p.N) epi_store_16(y + 16, ebuf, &tm_y, n0 + 16, row0, p.N, p.bias, 1.0f, lane);
         }
       }
     }

@@ -211,12 +211,15 @@ __global__ void fold_l1_kernel(const __nv_bfloat16* __restrict__ l1t, const floa
 
 // The up-projection operand of the GEMM's tail: [L2^T | L2^T] (N x 2 r_pad), so
 // that one MMA over K = 2 r_pad adds (hi + lo) L2 for X_hat L1 = hi + lo.
-__global__ void dup_l2_kernel(const __nv_bfloat16* __restrict__ l2t, int N, int r_pad,
+// l2t2 = scale * [L2^T | L2^T]; scale is a power of two (the weight prescale,
+// 1 without it), so the bf16 products are exact.
+__global__ void dup_l2_kernel(const __nv_bfloat16* __restrict__ l2t, int N, int r_pad, float scale,
                               __nv_bfloat16* __restrict__ l2t2) {
   const int n = blockIdx.x * blockDim.x + threadIdx.x;
   if (n >= N) return;
   for (int j = 0; j < r_pad; ++j) {
-    const __nv_bfloat16 v = l2t[static_cast<size_t>(n) * r_pad + j];
+    const __nv_bfloat16 v =
+        __float2bfloat16_rn(__fmul_rn(__bfloat162float(l2t[static_cast<size_t>(n) * r_pad + j]), scale));
     l2t2[static_cast<size_t>(n) * 2 * r_pad + j] = v;
     l2t2[static_cast<size_t>(n) * 2 * r_pad + r_pad + j] = v;
   }
@@ -242,8 +245,10 @@ __global__ void residual_kernel(const double* __restrict__ What,
 // NVFP4: one thread per (n, group of 16): codes N x K/2, scales in 512-byte atoms
 //        (128 columns x 4 groups; byte (n % 32) * 16 + (n % 128 / 32) * 4 + g % 4).
 // INT4 : one thread per (n, group of 64): int8 codes N x K, fp16 scales [K/64][N_pad].
+// pre: the power-of-two weight prescale (1 without it); R * pre is exact.
 __global__ void quant_weight_nvfp4_kernel(const float* __restrict__ R, int K, int N, int sf_kcols,
-                                          uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
+                                          float pre, uint8_t* __restrict__ codes,
+                                          uint8_t* __restrict__ sf) {
   __shared__ float rcp_tab[128];
   fill_e4m3_rcp_table(rcp_tab, threadIdx.x, blockDim.x);
   __syncthreads();
@@ -252,7 +257,7 @@ __global__ void quant_weight_nvfp4_kernel(const float* __restrict__ R, int K, in
   if (n >= N) return;
   float v[16];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = R[static_cast<size_t>(16 * g + i) * N + n];
+  for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(R[static_cast<size_t>(16 * g + i) * N + n], pre);
   uint32_t cw[2];
   const uint32_t s8 = quant16_nvfp4(v, cw, rcp_tab);
   uint32_t* dst = reinterpret_cast<uint32_t*>(codes + static_cast<size_t>(n) * (K / 2) + 8 * g);
@@ -285,7 +290,8 @@ __global__ void quant_weight_int4_kernel(const float* __restrict__ R, int K, int
 // FP4 g32: one E4M3 scale per 32 values of K, stored in both 16-value slots of
 // the scale atom so the NVFP4 GEMM (block16) applies it to both halves.
 __global__ void quant_weight_fp4g32_kernel(const float* __restrict__ R, int K, int N, int sf_kcols,
-                                           uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
+                                           float pre, uint8_t* __restrict__ codes,
+                                           uint8_t* __restrict__ sf) {
   __shared__ float rcp_tab[128];
   fill_e4m3_rcp_table(rcp_tab, threadIdx.x, blockDim.x);
   __syncthreads();
@@ -294,7 +300,7 @@ __global__ void quant_weight_fp4g32_kernel(const float* __restrict__ R, int K, i
   if (n >= N) return;
   float v[32];
 #pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = R[static_cast<size_t>(32 * g + i) * N + n];
+  for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(R[static_cast<size_t>(32 * g + i) * N + n], pre);
   uint32_t cw[4];
   const uint32_t s8 = quant32_fp4(v, cw, rcp_tab);
   uint4* dst = reinterpret_cast<uint4*>(codes + static_cast<size_t>(n) * (K / 2) + 16 * g);
@@ -314,10 +320,11 @@ __global__ void quant_weight_fp4g32_kernel(const float* __restrict__ R, int K, i
 // deq(Q(R))[k, n] from the handle's codes and scales (fmt: 0 NVFP4, 1 INT4,
 // 2 FP4 g32 -- whose scale sits in both 16-value slots, so the block-of-16
 // lookup serves it too).
+// post: 2^-e of the weight prescale (FP4 formats; 1 without it).
 __device__ __forceinline__ double deq_weight(int fmt, const uint8_t* __restrict__ codes,
                                              const uint8_t* __restrict__ sf,
                                              const float* __restrict__ sf32, int K, int N_pad,
-                                             int sf_kcols, int k, int n) {
+                                             int sf_kcols, double post, int k, int n) {
   if (fmt == 1) {
     const int8_t q = reinterpret_cast<const int8_t*>(codes)[static_cast<size_t>(n) * K + k];
     return static_cast<double>(q) * static_cast<double>(sf32[static_cast<size_t>(k / 64) * N_pad + n]);
@@ -331,19 +338,19 @@ __device__ __forceinline__ double deq_weight(int fmt, const uint8_t* __restrict_
   const int g = k / 16;
   const uint8_t s8 = sf[(static_cast<size_t>(n / 128) * sf_kcols + g / 4) * 512 + (n & 31) * 16 +
                         ((n & 127) >> 5) * 4 + (g & 3)];
-  return static_cast<double>(e2m1_value(c)) * static_cast<double>(e4m3_value(s8));
+  return static_cast<double>(e2m1_value(c)) * static_cast<double>(e4m3_value(s8)) * post;
 }
 
 // E = W_hat - deq(Q(R)), fp64 K x N.
 __global__ void refine_target_kernel(const double* __restrict__ What, int fmt,
                                      const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sf,
                                      const float* __restrict__ sf32, int K, int N, int N_pad,
-                                     int sf_kcols, double* __restrict__ E) {
+                                     int sf_kcols, double post, double* __restrict__ E) {
   const int n = blockIdx.x * blockDim.x + threadIdx.x;
   const int k = blockIdx.y;
   if (n >= N) return;
   const size_t i = static_cast<size_t>(k) * N + n;
-  E[i] = What[i] - deq_weight(fmt, codes, sf, sf32, K, N_pad, sf_kcols, k, n);
+  E[i] = What[i] - deq_weight(fmt, codes, sf, sf32, K, N_pad, sf_kcols, post, k, n);
 }
 
 // *sum += sum over the block's elements of (W_hat - L1 L2 - deq(Q(R)))^2, fp64.
@@ -352,7 +359,7 @@ __global__ void refine_error_kernel(const double* __restrict__ What,
                                     const __nv_bfloat16* __restrict__ l2t, int r, int r_pad, int fmt,
                                     const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sf,
                                     const float* __restrict__ sf32, int K, int N, int N_pad,
-                                    int sf_kcols, double* __restrict__ sum) {
+                                    int sf_kcols, double post, double* __restrict__ sum) {
   __shared__ double part[8];
   const int n = blockIdx.x * blockDim.x + threadIdx.x;
   const int k = blockIdx.y;
@@ -362,7 +369,7 @@ __global__ void refine_error_kernel(const double* __restrict__ What,
     for (int j = 0; j < r; ++j)
       acc -= static_cast<double>(__bfloat162float(l1t[static_cast<size_t>(j) * K + k])) *
              static_cast<double>(__bfloat162float(l2t[static_cast<size_t>(n) * r_pad + j]));
-    acc -= deq_weight(fmt, codes, sf, sf32, K, N_pad, sf_kcols, k, n);
+    acc -= deq_weight(fmt, codes, sf, sf32, K, N_pad, sf_kcols, post, k, n);
     d2 = acc * acc;
   }
   for (int o = 16; o > 0; o >>= 1) d2 += __shfl_xor_sync(0xffffffffu, d2, o);
@@ -391,6 +398,17 @@ __global__ void quant_weight_w8_kernel(const float* __restrict__ R, int K, int N
     codes[static_cast<size_t>(n) * K + k] = static_cast<int8_t>(q);
   }
   sw[n] = s;
+}
+
+// *out = max(*out, max |R|) as the bits of a non-negative float (which order
+// like the unsigned integers); *out starts at 0.  Grid-stride over n values.
+__global__ void absmax_f32_kernel(const float* __restrict__ R, size_t n, unsigned int* __restrict__ out) {
+  float m = 0.0f;
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x)
+    m = fmaxf(m, fabsf(R[i]));
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) atomicMax(out, __float_as_uint(m));
 }
 
 }  // namespace svdq

@@ -11,6 +11,7 @@
 #include <cusolverDn.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -52,6 +53,8 @@ struct svdq_weights {
   __nv_bfloat16* bias = nullptr;
   CUtensorMap tm_b, tm_l1t, tm_l2t;
   double refine_err0 = -1.0, refine_err = -1.0;   // weight error: SVD start, kept iterate
+  unsigned flags = 0;  // SVDQ_WEIGHT_POW2_PRESCALE
+  int w_exp = 0;       // the codes and scales are those of R * 2^w_exp (FP4 formats)
 };
 
 namespace {
@@ -385,14 +388,59 @@ int alloc_weights(svdq_weights* w, cudaStream_t st) {
   return SVDQ_OK;
 }
 
+struct DeviceBuf {
+  void* p = nullptr;
+  ~DeviceBuf() { if (p) cudaFree(p); }
+  bool alloc(size_t n) { return cudaMalloc(&p, n) == cudaSuccess; }
+  template <class T> T* as() const { return static_cast<T*>(p); }
+};
+
+// The optional power-of-two prescale of the weight residual: the largest e
+// with 2^e * s_max <= 448 (the top of the E4M3 range), s_max = fp32(max|R| / 6)
+// the largest group scale before rounding; 0 for a zero residual.  Computed
+// from the bits: s_max = f 2^q with 0.5 <= f < 1 and 448 = 0.875 * 2^9.
+int prescale_exponent(float amax) {
+  const float s_max = amax / 6.0f;
+  if (!(s_max > 0.0f)) return 0;
+  int q = 0;
+  const float f = std::frexp(s_max, &q);
+  const int e = f <= 0.875f ? 9 - q : 8 - q;
+  return std::max(-64, std::min(64, e));
+}
+
+// Derived operand of the tail MMA: l2t2 = 2^w_exp [L2^T | L2^T].
+int build_l2t2(svdq_weights* w, cudaStream_t st) {
+  if (w->rank == 0 || w->l2t2 == nullptr) return SVDQ_OK;
+  dup_l2_kernel<<<(w->N + 255) / 256, 256, 0, st>>>(w->l2t, w->N, w->r_pad, std::ldexp(1.0f, w->w_exp),
+                                                    w->l2t2);
+  SVDQ_CHECK_LAUNCH();
+  return SVDQ_OK;
+}
+
 int quantize_residual(svdq_weights* w, const float* R, cudaStream_t st) {
   const dim3 blk(128);
+  const int e_old = w->w_exp;
+  w->w_exp = 0;
+  if ((w->flags & SVDQ_WEIGHT_POW2_PRESCALE) && is_fp4(w->fmt)) {
+    DeviceBuf amax;
+    if (!amax.alloc(sizeof(unsigned))) return SVDQ_ERR_ALLOC;
+    SVDQ_CUDA(cudaMemsetAsync(amax.p, 0, sizeof(unsigned), st));
+    absmax_f32_kernel<<<4 * 148, 256, 0, st>>>(R, static_cast<size_t>(w->K) * w->N, amax.as<unsigned>());
+    SVDQ_CHECK_LAUNCH();
+    unsigned bits = 0;
+    SVDQ_CUDA(cudaMemcpyAsync(&bits, amax.p, sizeof bits, cudaMemcpyDeviceToHost, st));
+    SVDQ_CUDA(cudaStreamSynchronize(st));
+    float a;
+    std::memcpy(&a, &bits, sizeof a);
+    w->w_exp = prescale_exponent(a);
+  }
+  const float pre = std::ldexp(1.0f, w->w_exp);
   if (w->fmt == SVDQ_NVFP4) {
     const dim3 grid((w->N + 127) / 128, w->K / 16);
-    quant_weight_nvfp4_kernel<<<grid, blk, 0, st>>>(R, w->K, w->N, w->sf_kcols, w->wcodes, w->wsf);
+    quant_weight_nvfp4_kernel<<<grid, blk, 0, st>>>(R, w->K, w->N, w->sf_kcols, pre, w->wcodes, w->wsf);
   } else if (w->fmt == SVDQ_FP4G32) {
     const dim3 grid((w->N + 127) / 128, w->K / 32);
-    quant_weight_fp4g32_kernel<<<grid, blk, 0, st>>>(R, w->K, w->N, w->sf_kcols, w->wcodes, w->wsf);
+    quant_weight_fp4g32_kernel<<<grid, blk, 0, st>>>(R, w->K, w->N, w->sf_kcols, pre, w->wcodes, w->wsf);
   } else if (w->fmt == SVDQ_W8A8) {
     quant_weight_w8_kernel<<<(w->N + 127) / 128, blk, 0, st>>>(R, w->K, w->N,
                                                                 reinterpret_cast<int8_t*>(w->wcodes),
@@ -404,6 +452,7 @@ int quantize_residual(svdq_weights* w, const float* R, cudaStream_t st) {
                                                    reinterpret_cast<uint16_t*>(w->wsf), w->wsf32);
   }
   SVDQ_CHECK_LAUNCH();
+  if (w->w_exp != e_old) return build_l2t2(w, st);   // the tail carries the same 2^e
   return SVDQ_OK;
 }
 
@@ -415,7 +464,7 @@ int refold_l1(svdq_weights* w, cudaStream_t st) {
   w->l2t2 = nullptr;
   if (cudaMalloc(&w->l2t2, static_cast<size_t>(w->N) * 2 * w->r_pad * 2) != cudaSuccess)
     return SVDQ_ERR_ALLOC;
-  dup_l2_kernel<<<(w->N + 255) / 256, 256, 0, st>>>(w->l2t, w->N, w->r_pad, w->l2t2);
+  if (int rc = build_l2t2(w, st)) return rc;
   fold_l1_kernel<<<dim3((w->K + 255) / 256, w->rank), 256, 0, st>>>(w->l1t, w->inv_lambda, w->K,
                                                                      w->rank, w->l1st);
   SVDQ_CHECK_LAUNCH();
@@ -428,13 +477,6 @@ int copy_bias(svdq_weights* w, const void* bias, cudaStream_t st) {
   SVDQ_CUDA(cudaMemcpyAsync(w->bias, bias, static_cast<size_t>(w->N) * 2, cudaMemcpyDeviceToDevice, st));
   return SVDQ_OK;
 }
-
-struct DeviceBuf {
-  void* p = nullptr;
-  ~DeviceBuf() { if (p) cudaFree(p); }
-  bool alloc(size_t n) { return cudaMalloc(&p, n) == cudaSuccess; }
-  template <class T> T* as() const { return static_cast<T*>(p); }
-};
 
 int do_append_lora(svdq_weights* w, const void* A, const void* B, int rl, cudaStream_t st) {
   if (rl <= 0) return SVDQ_OK;
@@ -550,7 +592,7 @@ int weight_error(svdq_weights* w, const double* What, double* err_dev, double* o
   SVDQ_CUDA(cudaMemsetAsync(err_dev, 0, sizeof(double), st));
   refine_error_kernel<<<dim3((w->N + 255) / 256, w->K), 256, 0, st>>>(
       What, w->l1t, w->l2t, w->rank, w->r_pad, w->fmt, w->wcodes, w->wsf, w->wsf32, w->K, w->N,
-      w->N_pad, w->sf_kcols, err_dev);
+      w->N_pad, w->sf_kcols, std::ldexp(1.0, -w->w_exp), err_dev);
   SVDQ_CHECK_LAUNCH();
   double h = 0.0;
   SVDQ_CUDA(cudaMemcpyAsync(&h, err_dev, sizeof(double), cudaMemcpyDeviceToHost, st));
@@ -592,7 +634,8 @@ int refine_branch(svdq_weights* w, const double* What, float* R, int iters, cuda
   if ((rc = save(true))) return rc;
   for (int t = 0; t < iters; ++t) {
     refine_target_kernel<<<dim3((w->N + 255) / 256, w->K), 256, 0, st>>>(
-        What, w->fmt, w->wcodes, w->wsf, w->wsf32, w->K, w->N, w->N_pad, w->sf_kcols, E.as<double>());
+        What, w->fmt, w->wcodes, w->wsf, w->wsf32, w->K, w->N, w->N_pad, w->sf_kcols,
+        std::ldexp(1.0, -w->w_exp), E.as<double>());
     SVDQ_CHECK_LAUNCH();
     if ((rc = lowrank_factors(w, E.as<double>(), st))) return rc;
     residual_kernel<<<dim3((w->N + 255) / 256, w->K), 256, 0, st>>>(What, w->l1t, w->l2t, w->K, w->N,
@@ -693,6 +736,7 @@ SVDQ_API int svdq_prepare_weights(const svdq_prepare_desc* d, void* stream, svdq
   if (d->rank + d->lora_rank > 256 || d->rank + d->lora_rank > std::min(d->K, d->N))
     return SVDQ_ERR_UNSUPPORTED_SHAPE;
   if (d->refine_iters < 0 || d->refine_iters > 64) return SVDQ_ERR_INVALID_ARG;
+  if (d->flags & ~SVDQ_WEIGHT_POW2_PRESCALE) return SVDQ_ERR_INVALID_ARG;
   int dev;
   if ((rc = current_device(&dev))) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -702,6 +746,7 @@ SVDQ_API int svdq_prepare_weights(const svdq_prepare_desc* d, void* stream, svdq
   w->K = d->K;
   w->N = d->N;
   w->rank = d->rank;
+  w->flags = d->flags;
   const int K = d->K, N = d->N;
   do {
     if ((rc = alloc_weights(w, st))) break;
@@ -757,6 +802,7 @@ SVDQ_API int svdq_load_weights(const svdq_parts_desc* d, void* stream, svdq_weig
   int rc = check_shape(d->fmt, d->K, d->N, d->rank);
   if (rc) return rc;
   if (d->rank > 0 && (d->L1 == nullptr || d->L2 == nullptr)) return SVDQ_ERR_INVALID_ARG;
+  if (d->flags & ~SVDQ_WEIGHT_POW2_PRESCALE) return SVDQ_ERR_INVALID_ARG;
   int dev;
   if ((rc = current_device(&dev))) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -766,6 +812,7 @@ SVDQ_API int svdq_load_weights(const svdq_parts_desc* d, void* stream, svdq_weig
   w->K = d->K;
   w->N = d->N;
   w->rank = d->rank;
+  w->flags = d->flags;
   const int K = d->K, N = d->N;
   do {
     if ((rc = alloc_weights(w, st))) break;
@@ -834,6 +881,12 @@ SVDQ_API int svdq_append_lora(svdq_weights* w, const void* A, const void* B, int
   if (rc) return rc;
   if (dev != w->device) return SVDQ_ERR_INVALID_ARG;
   return do_append_lora(w, A, B, rl, static_cast<cudaStream_t>(stream));
+}
+
+SVDQ_API int svdq_weights_scale_exponent(const svdq_weights* w, int* exponent) {
+  if (w == nullptr || exponent == nullptr) return SVDQ_ERR_INVALID_ARG;
+  *exponent = w->w_exp;
+  return SVDQ_OK;
 }
 
 SVDQ_API int svdq_weights_refine_error(const svdq_weights* w, double* initial, double* kept) {
@@ -973,6 +1026,7 @@ SVDQ_API int svdq_linear(const svdq_weights* w, const void* ws, int M, void* Y, 
     p.sfb = w->wsf;
     p.sf_kcols = w->sf_kcols;
     p.bias = w->bias;
+    p.out_scale = std::ldexp(1.0f, -w->w_exp);
     p.budget = wait_budget();
     SVDQ_CUDA(launch_pdl(gemm_nvfp4_kernel, dim3(grid), dim3(kGemmThreads), kGemmSmemBytes, st, 0u, tm_a,
                          w->tm_b, tm_xl1, w->tm_l2t, tm_y, p));
