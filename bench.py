@@ -65,6 +65,12 @@ def peaks():
 # fingerprint of the kernel's sources: a kernel changed since the capture
 # reports null.  Y of the QKV layer (85 MB) is still mostly dirty in the
 # 126 MB L2 when the GEMM ends, so its write traffic is below Y's size.
+# Vendor figures for one B200, for the fractions reported beside the measured
+# denominators: dense FP4 and INT8 tensor peaks (NVIDIA's doubled figures are
+# with 2:4 sparsity) and the HBM3e bandwidth.
+DATASHEET_FP4_TFLOPS = 9000.0
+DATASHEET_INT8_TOPS = 4500.0
+NOMINAL_HBM_GBS = 8000.0
 NCU_TRAFFIC = {
     ("gemm_nvfp4_kernel", "c2_qkv/qkv", 4608, "nvfp4"): (60871936, "53a792da76c08882"),
     ("quant_act_kernel", "c2_qkv/qkv", 4608, "nvfp4"): (28561152, "325548569b93b04d"),
@@ -432,9 +438,13 @@ def run_ours(args):
                      "achieved": round(achieved, 1), "peak": round(fp_peak, 1), "unit": "TFLOP/s",
                      "frac": round(achieved / fp_peak, 4),
                      "traffic": ncu_traffic(gemm_kernel, f"{args.config}/{spec.name}", M, spec.fmt),
-                     "peak_note": f"{pk['source']}: bf16 {pk['bf16']} TF/s x {'2 (INT8)' if spec.fmt in INT8_KIND else '4 (FP4)'}"},
+                     "peak_note": f"{pk['source']}: bf16 {pk['bf16']} TF/s x {'2 (INT8)' if spec.fmt in INT8_KIND else '4 (FP4)'}",
+                     "datasheet_peak": DATASHEET_INT8_TOPS if spec.fmt in INT8_KIND else DATASHEET_FP4_TFLOPS,
+                     "frac_of_datasheet": round(achieved / (DATASHEET_INT8_TOPS if spec.fmt in INT8_KIND
+                                                            else DATASHEET_FP4_TFLOPS), 4)},
         "roofline_quant": {"bound": "hbm", "kernel": "quant_act_kernel", "achieved": round(q_gbs, 1),
                            "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": round(q_gbs / pk["hbm_gbs"], 4),
+                           "nominal_peak": NOMINAL_HBM_GBS, "frac_of_nominal": round(q_gbs / NOMINAL_HBM_GBS, 4),
                            "algorithmic_bytes": int(q_bytes),
                            "traffic": ncu_traffic("quant_act_kernel", f"{args.config}/{spec.name}", M, spec.fmt)},
         "e2e": {"value": round(flops / t_e2e / 1e12, 3), "unit": UNIT,
