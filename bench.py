@@ -72,11 +72,11 @@ DATASHEET_FP4_TFLOPS = 9000.0
 DATASHEET_INT8_TOPS = 4500.0
 NOMINAL_HBM_GBS = 8000.0
 NCU_TRAFFIC = {
-    ("gemm_nvfp4_kernel", "c2_qkv/qkv", 4608, "nvfp4"): (60871936, "53a792da76c08882"),
-    ("quant_act_kernel", "c2_qkv/qkv", 4608, "nvfp4"): (28561152, "325548569b93b04d"),
-    ("quant_act_kernel", "c5_block/fc2", 16384, "nvfp4"): (498218752, "325548569b93b04d"),
-    ("gemm_int4_kernel", "c4_int4_lora/proj", 4608, "int4"): (26797312, "cea79a7c0c6f4575"),
-    ("gemm_w8a8_kernel", "c2_qkv/qkv", 4608, "w8a8"): (86851072, "0c1cad6d3aa86dc5"),
+    ("gemm_nvfp4_kernel", "c2_qkv/qkv", 4608, "nvfp4"): (60754688, "c75505201d43dc8a"),
+    ("quant_act_kernel", "c2_qkv/qkv", 4608, "nvfp4"): (28561408, "7535e0940e8751a3"),
+    ("quant_act_kernel", "c5_block/fc2", 16384, "nvfp4"): (498098944, "7535e0940e8751a3"),
+    ("gemm_int4_kernel", "c4_int4_lora/proj", 4608, "int4"): (26840576, "b63229ae4c1e56af"),
+    ("gemm_w8a8_kernel", "c2_qkv/qkv", 4608, "w8a8"): (86607872, "fce99d9aabbce8f4"),
 }
 KERNEL_SOURCES = {
     "gemm_nvfp4_kernel": ("gemm_nvfp4.cuh", "svdq_ptx.cuh", "svdq_formats.cuh"),
