@@ -520,6 +520,106 @@ def _oracle_step(O, spec, prep, wq, sample, bias):
     O.linear(spec.fmt, act, wq, prep["L2"] if prep["rank"] else None, bias, spec.N)
 
 
+def run_block(args):
+    """--layer all: the workload's layers back to back as one step (one DiT
+    block's four linears at M tokens, each on its own seeded input), under one
+    event pair with the L2 flushed before every step.  The activation kernel of
+    each layer is launched while the previous GEMM drains (programmatic
+    dependent launch).  Reports the block and each layer's share."""
+    import w4a4_gemm_b200 as S
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    S.lib()
+    cfg = WL.CONFIGS[args.config]
+    M = args.M or cfg.Ms[-1]
+    layers = []
+    for spec in cfg.layers:
+        W, bias, A, B = WL.make_weights(spec)
+        X = WL.make_activations(spec, M).to(dev)
+        w = S.svdq_prepare_weights(W.to(dev), spec.rank, spec.fmt, x_absmax=S.svdq_calib_absmax(X),
+                                   bias=bias.to(dev) if bias is not None else None)
+        layers.append((spec, w, X, S.alloc_workspace(w, M, dev),
+                       torch.empty(M, spec.N, dtype=torch.bfloat16, device=dev)))
+        del W
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def block(evs=None, split=False):
+        for i, (spec, w, X, ws, Y) in enumerate(layers):
+            if evs is not None and (split or i == 0):
+                evs[i].record(stream)
+            S.svdq_quantize_act(w, X, ws)
+            S.svdq_linear(w, ws, M, Y)
+        if evs is not None:
+            evs[-1].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        block()
+    torch.cuda.synchronize()
+    if S.svdq_get_error():
+        raise RuntimeError("device wait timed out during warm-up")
+    n = len(layers)
+
+    def run(split):
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n + 1)] for _ in range(args.steps)]
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        for e in evs:
+            flush.zero_()
+            block(e, split)
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        return evs
+
+    # the block under one event pair (the layers' kernels overlap at their
+    # boundaries), then a second pass with an event before every layer
+    sampler = ClockSampler(local)
+    sampler.start()
+    whole = run(False)
+    clocks = sampler.stop()
+    split = run(True)
+    if S.svdq_get_error():
+        raise RuntimeError("device wait timed out during timing")
+    t_block = np.array([e[0].elapsed_time(e[n]) for e in whole]) * 1e-3
+    t_layer = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(n)] for e in split]).mean(axis=0) * 1e-3
+    flops = sum(2.0 * M * spec.K * spec.N for spec, *_ in layers)
+    total = float(t_block.sum())
+    (total,) = max_over_ranks([total], world, dev)
+    pk = peaks()
+    line = {
+        "metric": METRIC, "value": round(job_throughput(world, flops, args.steps, total), 2), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(total / args.steps * 1e3, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": DTYPE[layers[0][0].fmt],
+        "data": "synthetic (seeded FLUX-shaped activations and weights; no checkpoints)",
+        "config": {"workload": f"{args.config}: one block ({', '.join(s.name for s, *_ in layers)}) at M={M}",
+                   "M": M, "layers": [{"name": s.name, "K": s.K, "N": s.N, "rank": s.rank} for s, *_ in layers],
+                   "l2": "flushed between steps (512 MiB write)", "parallelism": f"dp{world} (token batches)"},
+        "us_per_block": round(total / args.steps * 1e6, 2),
+        "us_per_layer_in_block": {s.name: round(float(t) * 1e6, 2) for (s, *_), t in zip(layers, t_layer)},
+        "us_split_how": "us_per_block: the block under one event pair; us_per_layer_in_block: a second pass "
+                        "with an event before every layer",
+        "pct_fp4_peak_block": round(100.0 * flops / (total / args.steps) / 1e12 / (pk["bf16"] * 4.0), 2),
+        "gpu_launches": 2 * n * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    for _, w, *_ in layers:
+        w.close()
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
 def cpu_baseline(spec, M, rows):
     O, prep, wq, sample, bias = _oracle_setup(spec, M, rows)
     t0 = time.perf_counter()
@@ -568,7 +668,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="c2_qkv", choices=sorted(WL.CONFIGS))
-    ap.add_argument("--layer", default=None)
+    ap.add_argument("--layer", default=None,
+                    help="a layer of the config, or 'all': the config's layers back to back as one step")
     ap.add_argument("--M", type=int, default=None)
     ap.add_argument("--fmt", choices=["nvfp4", "int4", "fp4g32", "w8a8"], default=None,
                     help="override the workload's format")
@@ -585,6 +686,8 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.layer == "all":
+        run_block(args)
     else:
         run_ours(args)
 
