@@ -72,11 +72,12 @@ DATASHEET_FP4_TFLOPS = 9000.0
 DATASHEET_INT8_TOPS = 4500.0
 NOMINAL_HBM_GBS = 8000.0
 NCU_TRAFFIC = {
-    ("gemm_nvfp4_kernel", "c2_qkv/qkv", 4608, "nvfp4"): (60754688, "c75505201d43dc8a"),
+    ("gemm_nvfp4_kernel", "c2_qkv/qkv", 4608, "nvfp4"): (64887552, "4ca905a3b65027bb"),
+    ("gemm_nvfp4_kernel", "c5_block/fc2", 16384, "nvfp4"): (228391424, "4ca905a3b65027bb"),
     ("quant_act_kernel", "c2_qkv/qkv", 4608, "nvfp4"): (28561408, "7535e0940e8751a3"),
     ("quant_act_kernel", "c5_block/fc2", 16384, "nvfp4"): (498098944, "7535e0940e8751a3"),
-    ("gemm_int4_kernel", "c4_int4_lora/proj", 4608, "int4"): (26840576, "b63229ae4c1e56af"),
-    ("gemm_w8a8_kernel", "c2_qkv/qkv", 4608, "w8a8"): (86607872, "fce99d9aabbce8f4"),
+    ("gemm_int4_kernel", "c4_int4_lora/proj", 4608, "int4"): (26637056, "b98bf8b57d772110"),
+    ("gemm_w8a8_kernel", "c2_qkv/qkv", 4608, "w8a8"): (100051968, "5ea041ecba00a81f"),
 }
 KERNEL_SOURCES = {
     "gemm_nvfp4_kernel": ("gemm_nvfp4.cuh", "svdq_ptx.cuh", "svdq_formats.cuh"),
@@ -283,6 +284,49 @@ def unfused_foil(S, w, w0, X, ws, Y, M, flush, stream, steps, warmup):
     return float(np.mean([a.elapsed_time(b) for a, b in ts])) * 1e-3
 
 
+def vendor_gemm(M, K, N, flush, stream, steps, warmup):
+    """Seconds per launch of cuBLAS's NVFP4 block-scaled GEMM (torch scaled_mm:
+    E2M1 operands, an E4M3 scale per 16 values in the 128 x 4 swizzled layout,
+    bf16 out) on random codes of the layer's M, K and N: a comparison point for
+    gemm_nvfp4_kernel at rank 0 (no low-rank tail, no bias).  Not part of the
+    product; None with the reason when this torch or shape cannot run it."""
+    if M % 128 or (K // 16) % 4:
+        return None, "needs M % 128 == 0 and K % 64 == 0"
+    try:
+        import torch.nn.functional as F
+        from torch.nn.functional import ScalingType, SwizzleType
+        dev = torch.device("cuda", torch.cuda.current_device())
+        g = torch.Generator(device=dev)
+        g.manual_seed(7)
+        a = torch.randint(0, 256, (M, K // 2), dtype=torch.uint8, device=dev, generator=g).view(torch.float4_e2m1fn_x2)
+        b = torch.randint(0, 256, (N, K // 2), dtype=torch.uint8, device=dev, generator=g).view(torch.float4_e2m1fn_x2)
+        sa = (torch.rand(M, K // 16, device=dev, generator=g) * 1.5 + 0.25).to(torch.float8_e4m3fn)
+        sb = (torch.rand(N, K // 16, device=dev, generator=g) * 1.5 + 0.25).to(torch.float8_e4m3fn)
+        sw = SwizzleType.SWIZZLE_32_4_4
+
+        def step():
+            F.scaled_mm(a, b.t(), sa, ScalingType.BlockWise1x16, sb, ScalingType.BlockWise1x16,
+                        swizzle_a=sw, swizzle_b=sw, output_dtype=torch.bfloat16)
+
+        step()
+        torch.cuda.synchronize()
+    except Exception as e:   # an older torch or cuBLAS without NVFP4
+        return None, str(e).splitlines()[0][:160]
+    for _ in range(warmup):
+        flush.zero_()
+        step()
+    ts = []
+    for _ in range(steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        step()
+        e1.record(stream)
+        ts.append((e0, e1))
+    torch.cuda.synchronize()
+    return float(np.mean([x.elapsed_time(y) for x, y in ts])) * 1e-3, None
+
+
 def e2e_pipelined(S, w, X, Y, ws, steps):
     """Seconds per step of the layer served end to end through svdq_forward:
     every step copies its X from pinned host memory to the device and its Y
@@ -473,6 +517,17 @@ def run_ours(args):
                 "us_layer": round(t_unf * 1e6, 2), "layer": round(t_unf / l0 - 1.0, 4),
                 "what": "rank-0 layer, then smoothing, X_hat L1 and (X_hat L1) L2 as separate cuBLAS bf16 "
                         "GEMMs and an addition into Y (the unfused design the fused kernels replace)"}
+        if spec.fmt == "nvfp4":
+            t_v, why = vendor_gemm(M, spec.K, spec.N, flush, stream, args.steps, args.warmup)
+            if t_v is None:
+                line["vendor_gemm"] = {"unavailable": why}
+            else:
+                line["vendor_gemm"] = {
+                    "us": round(t_v * 1e6, 2), "tflops": round(2.0 * M * spec.K * spec.N / t_v / 1e12, 1),
+                    "ours_rank0_us": round(float(g0.mean()) * 1e6, 2),
+                    "ours_over_vendor_time": round(float(g0.mean()) / t_v, 4),
+                    "what": "cuBLAS NVFP4 block-scaled GEMM (torch scaled_mm, BlockWise1x16, swizzled E4M3 "
+                            "scales) on random codes of the same M, K, N, against gemm_nvfp4_kernel at rank 0"}
         if args.rank_sweep:
             sweep = []
             for rr in args.rank_sweep:

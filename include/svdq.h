@@ -231,6 +231,16 @@ SVDQ_API int svdq_set_wait_budget(long long cycles);
  * SVDQ_ERR_INVALID_ARG for other values. */
 SVDQ_API int svdq_set_quant_split(int S, int C);
 
+/* Tile order of the GEMM for every later svdq_linear (process-wide; a tuning
+ * and testing aid).  The persistent GEMM walks its 128-row x 256-column output
+ * tiles in groups of `group_m` row blocks: all of a group's tiles, row block
+ * fastest, before the next group.  Small groups keep fewer activation row
+ * blocks and more weight column blocks in flight at once.  group_m above the
+ * number of row blocks is clamped to it (one group: the whole of M for each
+ * weight column block); 0 restores the automatic choice.  The result does not
+ * depend on the order.  SVDQ_ERR_INVALID_ARG for group_m < 0. */
+SVDQ_API int svdq_set_gemm_raster(int group_m);
+
 SVDQ_API const char* svdq_status_string(int status);
 
 /* Measurement helper, not a step of the layer: every SM of the current device

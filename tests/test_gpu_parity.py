@@ -191,6 +191,29 @@ def test_forced_launch_shapes(S, M, K, N, rank, fmt):
         w.close()
 
 
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4", "w8a8"])
+def test_forced_gemm_raster(S, fmt):
+    """The GEMM's tile order changes which CTA computes a tile and when, not what
+    it computes: every order gives the same Y bit for bit, within tolerance of
+    the oracle (5 row blocks, 4 column blocks with a ragged last one)."""
+    M, K, N, rank = 600, 512, 784, 16
+    data = WL.make_small(M, K, N, rank=rank, fmt=fmt, seed=91)
+    ref = oracle_layer(fmt, data, rank)
+    w = load_from_oracle(S, fmt, ref["prep"])
+    try:
+        S.svdq_set_gemm_raster(0)
+        _, Y0 = _run_layer(S, w, WL.bf16_bits(data["X"]))
+        ok, info = y_within_tol(bits(Y0), ref["Y"])
+        assert ok, ("auto", info)
+        for g in (1, 2, 3, 5, 64):
+            S.svdq_set_gemm_raster(g)
+            _, Y = _run_layer(S, w, WL.bf16_bits(data["X"]))
+            assert np.array_equal(bits(Y), bits(Y0)), g
+    finally:
+        S.svdq_set_gemm_raster(0)
+        w.close()
+
+
 @pytest.mark.parametrize("fmt", ["nvfp4", "fp4g32"])
 def test_pow2_prescale_parity(S, fmt):
     """Small weights with the power-of-two prescale: the library's exponent, weight

@@ -40,7 +40,7 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "device all
 EXPORTED = ("svdq_calib_absmax", "svdq_prepare_weights", "svdq_load_weights", "svdq_append_lora",
             "svdq_weights_info", "svdq_weights_refine_error", "svdq_weights_scale_exponent", "svdq_act_workspace_bytes", "svdq_quantize_act", "svdq_linear",
             "svdq_forward", "svdq_forward_noalloc", "svdq_export_act", "svdq_export_weights", "svdq_get_error",
-            "svdq_set_wait_budget", "svdq_set_quant_split", "svdq_status_string", "svdq_tensor_peak",
+            "svdq_set_wait_budget", "svdq_set_quant_split", "svdq_set_gemm_raster", "svdq_status_string", "svdq_tensor_peak",
             "svdq_weights_destroy")
 
 
@@ -97,6 +97,7 @@ def lib() -> ctypes.CDLL:
     L.svdq_get_error.argtypes = []
     L.svdq_set_wait_budget.argtypes = [LL]
     L.svdq_set_quant_split.argtypes = [I, I]
+    L.svdq_set_gemm_raster.argtypes = [I]
     L.svdq_status_string.argtypes = [I]
     L.svdq_status_string.restype = ctypes.c_char_p
     L.svdq_tensor_peak.argtypes = [I, LL, P]
@@ -350,3 +351,8 @@ def svdq_set_wait_budget(cycles: int):
 def svdq_set_quant_split(S: int = 0, C: int = 0):
     """Force the activation kernel's launch shape (see include/svdq.h); 0, 0 = automatic."""
     _check(lib().svdq_set_quant_split(int(S), int(C)), "svdq_set_quant_split")
+
+
+def svdq_set_gemm_raster(group_m: int = 0):
+    """Force the GEMM's tile order (row blocks per group, see include/svdq.h); 0 = automatic."""
+    _check(lib().svdq_set_gemm_raster(int(group_m)), "svdq_set_gemm_raster")

@@ -58,6 +58,7 @@ struct GemmI4Params {
   int M, N, K;
   int groups;          // K / 64
   int m_tiles, n_tiles, num_tiles;
+  int group_m;         // tile order (gemm_tile_coords)
   int r_tail;          // tail K: 2 r_pad (X_hat L1 as hi | lo against L2^T | L2^T), 0 = none
   const uint16_t* sx;  // fp16 [K/64][M_pad]
   const float* sw;     // fp32 [K/64][N_pad] (exact copies of the fp16 weight scales)
@@ -189,7 +190,8 @@ __global__ void __launch_bounds__(kI4Threads, 1)
       int it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
-        const int m_blk = tile % p.m_tiles, n_blk = tile / p.m_tiles;
+        int m_blk, n_blk;
+        gemm_tile_coords(p.m_tiles, p.n_tiles, p.group_m, tile, m_blk, n_blk);
         const int m0 = m_blk * kI4BM, n0 = n_blk * kI4BN;
         for (int step = 0; step < steps_per_tile; ++step, ++it) {
           const int s = it % S;
@@ -272,7 +274,8 @@ __global__ void __launch_bounds__(kI4Threads, 1)
     int it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
-      const int m_blk = tile % p.m_tiles, n_blk = tile / p.m_tiles;
+      int m_blk, n_blk;
+      gemm_tile_coords(p.m_tiles, p.n_tiles, p.group_m, tile, m_blk, n_blk);
       const int m = m_blk * kI4BM + static_cast<int>(row);
       unsigned long long acc[32];   // 64 fp32 accumulators, pairs of adjacent columns
 #pragma unroll

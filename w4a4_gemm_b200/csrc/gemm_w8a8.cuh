@@ -44,6 +44,7 @@ struct GemmW8Params {
   int M, N, K;
   int kt_total;        // ceil(K / 128)
   int m_tiles, n_tiles, num_tiles;
+  int group_m;         // tile order (gemm_tile_coords)
   int r_tail;          // 2 r_pad, 0 = no low-rank branch
   const float* sx;     // M_pad per-token scales
   const float* sw;     // N_pad per-channel scales
@@ -109,7 +110,7 @@ __global__ void __launch_bounds__(kW8Threads, 1)
       bool ok = true;
       for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
         int m_blk, n_blk;
-        gemm_tile_coords(p.m_tiles, tile, m_blk, n_blk);
+        gemm_tile_coords(p.m_tiles, p.n_tiles, p.group_m, tile, m_blk, n_blk);
         const int m0 = m_blk * kW8BM, n0 = n_blk * kW8BN;
         for (int step = 0; step < steps_per_tile; ++step, ++it) {
           const int s = it % STAGES;
@@ -193,7 +194,7 @@ __global__ void __launch_bounds__(kW8Threads, 1)
     int t_local = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++t_local) {
       int m_blk, n_blk;
-      gemm_tile_coords(p.m_tiles, tile, m_blk, n_blk);
+      gemm_tile_coords(p.m_tiles, p.n_tiles, p.group_m, tile, m_blk, n_blk);
       if (!warp_wait(acc_full, t_local & 1, p.budget, abort_flag)) {
         if (lane == 0) raise_error(kErrWaitGemm);
         *abort_flag = 1;

@@ -251,6 +251,7 @@ constexpr double kQuantPerPeerCycles = 1000.0;
 constexpr double kQuantStageCycles = 800.0;
 constexpr double kQuantL1Cycles = 300.0;
 QuantSplit g_forced_split{0, 0};   // svdq_set_quant_split; {0, 0} = automatic
+int g_forced_group_m = 0;          // svdq_set_gemm_raster; 0 = automatic
 
 QuantSplit quant_split_for(int M, int K, int r_pad, const DeviceInfo& d) {
   const int smax = r_pad > 0 ? quant_stack_max(r_pad) : 8;
@@ -687,6 +688,12 @@ SVDQ_API int svdq_tensor_peak(int fmt, long long steps, void* stream) {
   return SVDQ_OK;
 }
 
+SVDQ_API int svdq_set_gemm_raster(int group_m) {
+  if (group_m < 0) return SVDQ_ERR_INVALID_ARG;
+  g_forced_group_m = group_m;
+  return SVDQ_OK;
+}
+
 SVDQ_API int svdq_set_quant_split(int S, int C) {
   auto pow2_le8 = [](int v) { return v == 1 || v == 2 || v == 4 || v == 8; };
   if (S == 0 && C == 0) {
@@ -978,6 +985,14 @@ SVDQ_API int svdq_quantize_act(const svdq_weights* w, const void* X, int M, void
   return SVDQ_OK;
 }
 
+// Row blocks per group of the GEMMs' tile order (gemm_tile_coords).
+int gemm_group_m(int m_tiles, int n_tiles, int grid) {
+  if (g_forced_group_m > 0) return std::min(g_forced_group_m, m_tiles);
+  (void)n_tiles;
+  (void)grid;
+  return std::min(kGemmGroupM, m_tiles);
+}
+
 SVDQ_API int svdq_linear(const svdq_weights* w, const void* ws, int M, void* Y, void* stream) {
   if (w == nullptr || M < 0) return SVDQ_ERR_INVALID_ARG;
   if (M == 0) return SVDQ_OK;
@@ -995,6 +1010,7 @@ SVDQ_API int svdq_linear(const svdq_weights* w, const void* ws, int M, void* Y, 
   const int n_tiles = w->fmt != SVDQ_INT4 ? (w->N + kGemmBN - 1) / kGemmBN : (w->N + kI4BN - 1) / kI4BN;
   const int tiles = m_tiles * n_tiles;
   const int grid = std::min(tiles, g_dev[dev].sms);
+  const int group_m = gemm_group_m(m_tiles, n_tiles, grid);
   if (is_fp4(w->fmt))
     rc = make_map(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base + L.codes_off, w->K / 2, M, 128, kGemmBM);
   else if (w->fmt == SVDQ_W8A8)
@@ -1021,6 +1037,7 @@ SVDQ_API int svdq_linear(const svdq_weights* w, const void* ws, int M, void* Y, 
     p.m_tiles = m_tiles;
     p.n_tiles = n_tiles;
     p.num_tiles = tiles;
+    p.group_m = group_m;
     p.r_tail = 2 * w->r_pad;
     p.sfa = base + L.sf_off;
     p.sfb = w->wsf;
@@ -1041,6 +1058,7 @@ SVDQ_API int svdq_linear(const svdq_weights* w, const void* ws, int M, void* Y, 
     p.m_tiles = m_tiles;
     p.n_tiles = n_tiles;
     p.num_tiles = tiles;
+    p.group_m = group_m;
     p.r_tail = 2 * w->r_pad;
     p.sx = reinterpret_cast<const float*>(base + L.sf_off);
     p.sw = reinterpret_cast<const float*>(w->wsf);
@@ -1057,6 +1075,7 @@ SVDQ_API int svdq_linear(const svdq_weights* w, const void* ws, int M, void* Y, 
     p.m_tiles = m_tiles;
     p.n_tiles = n_tiles;
     p.num_tiles = tiles;
+    p.group_m = group_m;
     p.r_tail = 2 * w->r_pad;
     p.sx = reinterpret_cast<const uint16_t*>(base + L.sf_off);
     p.sw = w->wsf32;
