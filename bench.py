@@ -72,15 +72,16 @@ DATASHEET_FP4_TFLOPS = 9000.0
 DATASHEET_INT8_TOPS = 4500.0
 NOMINAL_HBM_GBS = 8000.0
 NCU_TRAFFIC = {
-    ("gemm_nvfp4_kernel", "c2_qkv/qkv", 4608, "nvfp4"): (64887552, "4ca905a3b65027bb"),
-    ("gemm_nvfp4_kernel", "c5_block/fc2", 16384, "nvfp4"): (228391424, "4ca905a3b65027bb"),
-    ("quant_act_kernel", "c2_qkv/qkv", 4608, "nvfp4"): (28561408, "7535e0940e8751a3"),
-    ("quant_act_kernel", "c5_block/fc2", 16384, "nvfp4"): (498098944, "7535e0940e8751a3"),
-    ("gemm_int4_kernel", "c4_int4_lora/proj", 4608, "int4"): (26637056, "b98bf8b57d772110"),
-    ("gemm_w8a8_kernel", "c2_qkv/qkv", 4608, "w8a8"): (100051968, "5ea041ecba00a81f"),
+    ("gemm_nvfp4_pair_kernel", "c2_qkv/qkv", 4608, "nvfp4"): (63419392, "f895356c38d662a7"),
+    ("gemm_nvfp4_pair_kernel", "c5_block/fc2", 16384, "nvfp4"): (222889216, "f895356c38d662a7"),
+    ("quant_act_kernel", "c2_qkv/qkv", 4608, "nvfp4"): (28561408, "97712fa48aaac990"),
+    ("quant_act_kernel", "c5_block/fc2", 16384, "nvfp4"): (498574592, "97712fa48aaac990"),
+    ("gemm_int4_kernel", "c4_int4_lora/proj", 4608, "int4"): (26690816, "4e6665236c6ea587"),
+    ("gemm_w8a8_kernel", "c2_qkv/qkv", 4608, "w8a8"): (100859392, "2d56831f05842901"),
 }
 KERNEL_SOURCES = {
     "gemm_nvfp4_kernel": ("gemm_nvfp4.cuh", "svdq_ptx.cuh", "svdq_formats.cuh"),
+    "gemm_nvfp4_pair_kernel": ("gemm_nvfp4_pair.cuh", "gemm_nvfp4.cuh", "svdq_ptx.cuh", "svdq_formats.cuh"),
     "quant_act_kernel": ("quant_act.cuh", "svdq_ptx.cuh", "svdq_formats.cuh"),
     "gemm_int4_kernel": ("gemm_int4.cuh", "gemm_nvfp4.cuh", "svdq_ptx.cuh", "svdq_formats.cuh"),
     "gemm_w8a8_kernel": ("gemm_w8a8.cuh", "gemm_nvfp4.cuh", "svdq_ptx.cuh", "svdq_formats.cuh"),
@@ -170,7 +171,7 @@ class ClockSampler:
 # Per format: tensor-core instruction family (int8 formats run kind::i8, whose
 # peak is half the FP4 one), activation code bytes per value, GEMM kernel.
 INT8_KIND = ("int4", "w8a8")
-GEMM_KERNEL = {"nvfp4": "gemm_nvfp4_kernel", "fp4g32": "gemm_nvfp4_kernel",
+GEMM_KERNEL = {"nvfp4": "gemm_nvfp4_pair_kernel", "fp4g32": "gemm_nvfp4_pair_kernel",
                "int4": "gemm_int4_kernel", "w8a8": "gemm_w8a8_kernel"}
 DTYPE = {"nvfp4": "e2m1xe2m1+bf16 (fp32 acc)", "fp4g32": "e2m1xe2m1+bf16 (fp32 acc)",
          "int4": "s8xs8+bf16 (fp32 acc)", "w8a8": "s8xs8 (s32 acc)+bf16 (fp32 acc)"}
@@ -288,7 +289,7 @@ def vendor_gemm(M, K, N, flush, stream, steps, warmup):
     """Seconds per launch of cuBLAS's NVFP4 block-scaled GEMM (torch scaled_mm:
     E2M1 operands, an E4M3 scale per 16 values in the 128 x 4 swizzled layout,
     bf16 out) on random codes of the layer's M, K and N: a comparison point for
-    gemm_nvfp4_kernel at rank 0 (no low-rank tail, no bias).  Not part of the
+    the FP4 GEMM at rank 0 (no low-rank tail, no bias).  Not part of the
     product; None with the reason when this torch or shape cannot run it."""
     if M % 128 or (K // 16) % 4:
         return None, "needs M % 128 == 0 and K % 64 == 0"
@@ -527,7 +528,7 @@ def run_ours(args):
                     "ours_rank0_us": round(float(g0.mean()) * 1e6, 2),
                     "ours_over_vendor_time": round(float(g0.mean()) / t_v, 4),
                     "what": "cuBLAS NVFP4 block-scaled GEMM (torch scaled_mm, BlockWise1x16, swizzled E4M3 "
-                            "scales) on random codes of the same M, K, N, against gemm_nvfp4_kernel at rank 0"}
+                            "scales) on random codes of the same M, K, N, against our FP4 GEMM at rank 0"}
         if args.rank_sweep:
             sweep = []
             for rr in args.rank_sweep:

@@ -241,6 +241,17 @@ SVDQ_API int svdq_set_quant_split(int S, int C);
  * depend on the order.  SVDQ_ERR_INVALID_ARG for group_m < 0. */
 SVDQ_API int svdq_set_gemm_raster(int group_m);
 
+/* GEMM kernel of the FP4 formats for every later svdq_linear (process-wide; a
+ * tuning and testing aid): 1 = one CTA per 128 x 256 output tile, 2 = a pair of
+ * CTAs (a cluster of two) per 256 x 256 tile, each CTA staging its own 128 rows
+ * of the activations and half of the weight columns for tcgen05 MMAs that span
+ * both; 0 restores the automatic choice.  Both give the same Y bit for bit (the
+ * same products summed in the same order).  The INT4 and W8A8 formats have one
+ * kernel each and ignore it.  With kind 2 the raster group of
+ * svdq_set_gemm_raster counts 128-row blocks and is rounded up to pairs.
+ * SVDQ_ERR_INVALID_ARG for other values. */
+SVDQ_API int svdq_set_gemm_kernel(int kind);
+
 SVDQ_API const char* svdq_status_string(int status);
 
 /* Measurement helper, not a step of the layer: every SM of the current device

@@ -191,6 +191,34 @@ def test_forced_launch_shapes(S, M, K, N, rank, fmt):
         w.close()
 
 
+@pytest.mark.parametrize("M,K,N,rank,fmt", [
+    (600, 512, 784, 16, "nvfp4"),    # odd number of 128-row blocks: the last pair's second CTA has no rows
+    (130, 1024, 256, 32, "fp4g32"),
+    (256, 256, 512, 0, "nvfp4"),     # no low-rank tail
+    (1000, 768, 272, 48, "nvfp4"),   # ragged last column block, 3 tail chunks
+    (384, 320, 1024, 32, "nvfp4"),   # K below two K steps
+])
+def test_forced_gemm_kernel(S, M, K, N, rank, fmt):
+    """The FP4 GEMM on single CTAs (128 x 256 tiles) and on CTA pairs (256 x 256,
+    cta_group::2 MMAs) sums the same products in the same order: Y bit for bit
+    the same, within tolerance of the oracle."""
+    data = WL.make_small(M, K, N, rank=rank, fmt=fmt, seed=M + K)
+    ref = oracle_layer(fmt, data, rank)
+    w = load_from_oracle(S, fmt, ref["prep"])
+    try:
+        Ys = {}
+        for kind in (1, 2):
+            S.svdq_set_gemm_kernel(kind)
+            _, Y = _run_layer(S, w, WL.bf16_bits(data["X"]))
+            ok, info = y_within_tol(bits(Y), ref["Y"])
+            assert ok, (kind, info)
+            Ys[kind] = bits(Y)
+        assert np.array_equal(Ys[1], Ys[2])
+    finally:
+        S.svdq_set_gemm_kernel(0)
+        w.close()
+
+
 @pytest.mark.parametrize("fmt", ["nvfp4", "int4", "w8a8"])
 def test_forced_gemm_raster(S, fmt):
     """The GEMM's tile order changes which CTA computes a tile and when, not what

@@ -40,7 +40,7 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "device all
 EXPORTED = ("svdq_calib_absmax", "svdq_prepare_weights", "svdq_load_weights", "svdq_append_lora",
             "svdq_weights_info", "svdq_weights_refine_error", "svdq_weights_scale_exponent", "svdq_act_workspace_bytes", "svdq_quantize_act", "svdq_linear",
             "svdq_forward", "svdq_forward_noalloc", "svdq_export_act", "svdq_export_weights", "svdq_get_error",
-            "svdq_set_wait_budget", "svdq_set_quant_split", "svdq_set_gemm_raster", "svdq_status_string", "svdq_tensor_peak",
+            "svdq_set_wait_budget", "svdq_set_quant_split", "svdq_set_gemm_raster", "svdq_set_gemm_kernel", "svdq_status_string", "svdq_tensor_peak",
             "svdq_weights_destroy")
 
 
@@ -98,6 +98,7 @@ def lib() -> ctypes.CDLL:
     L.svdq_set_wait_budget.argtypes = [LL]
     L.svdq_set_quant_split.argtypes = [I, I]
     L.svdq_set_gemm_raster.argtypes = [I]
+    L.svdq_set_gemm_kernel.argtypes = [I]
     L.svdq_status_string.argtypes = [I]
     L.svdq_status_string.restype = ctypes.c_char_p
     L.svdq_tensor_peak.argtypes = [I, LL, P]
@@ -351,6 +352,11 @@ def svdq_set_wait_budget(cycles: int):
 def svdq_set_quant_split(S: int = 0, C: int = 0):
     """Force the activation kernel's launch shape (see include/svdq.h); 0, 0 = automatic."""
     _check(lib().svdq_set_quant_split(int(S), int(C)), "svdq_set_quant_split")
+
+
+def svdq_set_gemm_kernel(kind: int = 0):
+    """Force the FP4 GEMM kernel: 1 = one CTA per tile, 2 = CTA pairs; 0 = automatic (see include/svdq.h)."""
+    _check(lib().svdq_set_gemm_kernel(int(kind)), "svdq_set_gemm_kernel")
 
 
 def svdq_set_gemm_raster(group_m: int = 0):

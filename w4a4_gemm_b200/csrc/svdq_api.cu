@@ -22,6 +22,7 @@
 #include "../../include/svdq.h"
 #include "gemm_int4.cuh"
 #include "gemm_nvfp4.cuh"
+#include "gemm_nvfp4_pair.cuh"
 #include "gemm_w8a8.cuh"
 #include "peak.cuh"
 #include "prepare.cuh"
@@ -52,6 +53,7 @@ struct svdq_weights {
   __nv_bfloat16* l2t2 = nullptr; // N x 2 r_pad: [L2^T | L2^T], the tail MMA's B operand
   __nv_bfloat16* bias = nullptr;
   CUtensorMap tm_b, tm_l1t, tm_l2t;
+  CUtensorMap tm_b_half, tm_l2t_half, tm_sfb;   // FP4 CTA-pair GEMM: 128-row boxes, scale atoms
   double refine_err0 = -1.0, refine_err = -1.0;   // weight error: SVD start, kept iterate
   unsigned flags = 0;  // SVDQ_WEIGHT_POW2_PRESCALE
   int w_exp = 0;       // the codes and scales are those of R * 2^w_exp (FP4 formats)
@@ -171,9 +173,30 @@ int make_map(CUtensorMap* m, CUtensorMapDataType dt, size_t elem, const void* ba
   return SVDQ_OK;
 }
 
+// Map over an array of 512-byte scale atoms as [atoms][128 x 32-bit words]; a
+// box is 4 consecutive atoms (one 256-wide K step of 128 rows), no swizzle.
+int make_atom_map(CUtensorMap* m, const void* base, uint64_t atoms) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return SVDQ_ERR_CUDA;
+  const cuuint64_t dims[2] = {128, atoms};
+  const cuuint64_t strides[1] = {512};
+  const cuuint32_t box[2] = {128, 4};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    std::fprintf(stderr, "svdq: cuTensorMapEncodeTiled failed (%d) for %llu scale atoms\n", static_cast<int>(r),
+                 static_cast<unsigned long long>(atoms));
+    return SVDQ_ERR_CUDA;
+  }
+  return SVDQ_OK;
+}
+
 // ------------------------------------------------------------ device info ---
 struct DeviceInfo {
   int sms = 0;
+  int pair_clusters = 0;                    // resident clusters of the CTA-pair GEMM
   int qclusters[kQuantMaxSplit + 1] = {};   // resident activation-kernel clusters of size C
   bool attrs_set = false;
 };
@@ -198,6 +221,8 @@ int device_setup(int dev) {
                                  kW8SmemBytes));
   SVDQ_CUDA(cudaFuncSetAttribute(gemm_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kGemmSmemBytes));
+  SVDQ_CUDA(cudaFuncSetAttribute(gemm_nvfp4_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kPairSmemBytes));
   SVDQ_CUDA(cudaFuncSetAttribute(gemm_int4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kI4SmemBytes));
   SVDQ_CUDA(cudaFuncSetAttribute(tensor_peak_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -221,6 +246,22 @@ int device_setup(int dev) {
     int n = 0;
     SVDQ_CUDA(cudaOccupancyMaxActiveClusters(&n, quant_act_kernel<1>, &cfg));
     d.qclusters[C] = n;
+  }
+  {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(d.sms & ~1);
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = kPairSmemBytes;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    SVDQ_CUDA(cudaOccupancyMaxActiveClusters(&n, gemm_nvfp4_pair_kernel, &cfg));
+    d.pair_clusters = n;
   }
   d.attrs_set = true;
   return SVDQ_OK;
@@ -252,6 +293,7 @@ constexpr double kQuantStageCycles = 800.0;
 constexpr double kQuantL1Cycles = 300.0;
 QuantSplit g_forced_split{0, 0};   // svdq_set_quant_split; {0, 0} = automatic
 int g_forced_group_m = 0;          // svdq_set_gemm_raster; 0 = automatic
+int g_forced_gemm_kind = 0;        // svdq_set_gemm_kernel; 0 = automatic, 1 = one CTA, 2 = CTA pairs
 
 QuantSplit quant_split_for(int M, int K, int r_pad, const DeviceInfo& d) {
   const int smax = r_pad > 0 ? quant_stack_max(r_pad) : 8;
@@ -309,9 +351,11 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 int encode_weight_maps(svdq_weights* w) {
   int rc;
-  if (is_fp4(w->fmt))
+  if (is_fp4(w->fmt)) {
     rc = make_map(&w->tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->wcodes, w->K / 2, w->N, 128, kGemmBN);
-  else if (w->fmt == SVDQ_W8A8)
+    if (!rc) rc = make_map(&w->tm_b_half, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->wcodes, w->K / 2, w->N, 128, 128);
+    if (!rc) rc = make_atom_map(&w->tm_sfb, w->wsf, static_cast<uint64_t>(w->N_pad / 128) * w->sf_kcols);
+  } else if (w->fmt == SVDQ_W8A8)
     rc = make_map(&w->tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->wcodes, w->K, w->N, kW8BKB, kW8BN);
   else
     rc = make_map(&w->tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->wcodes, w->K, w->N, 64, kI4BN);
@@ -323,9 +367,13 @@ int encode_weight_maps(svdq_weights* w) {
     rc = make_map(&w->tm_l2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w->l2t2, 2 * w->r_pad, w->N, lc,
                   w->fmt != SVDQ_INT4 ? kGemmBN : kI4BN);
     if (rc) return rc;
+    if (is_fp4(w->fmt) &&
+        (rc = make_map(&w->tm_l2t_half, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w->l2t2, 2 * w->r_pad, w->N, lc, 128)))
+      return rc;
   } else {
     w->tm_l1t = w->tm_b;
     w->tm_l2t = w->tm_b;
+    w->tm_l2t_half = w->tm_b;
   }
   return SVDQ_OK;
 }
@@ -688,6 +736,12 @@ SVDQ_API int svdq_tensor_peak(int fmt, long long steps, void* stream) {
   return SVDQ_OK;
 }
 
+SVDQ_API int svdq_set_gemm_kernel(int kind) {
+  if (kind < 0 || kind > 2) return SVDQ_ERR_INVALID_ARG;
+  g_forced_gemm_kind = kind;
+  return SVDQ_OK;
+}
+
 SVDQ_API int svdq_set_gemm_raster(int group_m) {
   if (group_m < 0) return SVDQ_ERR_INVALID_ARG;
   g_forced_group_m = group_m;
@@ -993,6 +1047,13 @@ int gemm_group_m(int m_tiles, int n_tiles, int grid) {
   return std::min(kGemmGroupM, m_tiles);
 }
 
+// FP4 GEMM on CTA pairs (256 x 256 tiles) or on single CTAs (128 x 256).
+bool use_pair_gemm(const svdq_weights* w, const DeviceInfo& d) {
+  if (!is_fp4(w->fmt) || d.pair_clusters <= 0) return false;
+  if (g_forced_gemm_kind != 0) return g_forced_gemm_kind == 2;
+  return true;   // as fast or faster at every layer shape of the FLUX block
+}
+
 SVDQ_API int svdq_linear(const svdq_weights* w, const void* ws, int M, void* Y, void* stream) {
   if (w == nullptr || M < 0) return SVDQ_ERR_INVALID_ARG;
   if (M == 0) return SVDQ_OK;
@@ -1026,7 +1087,32 @@ SVDQ_API int svdq_linear(const svdq_weights* w, const void* ws, int M, void* Y, 
   } else {
     tm_xl1 = tm_a;
   }
-  if (is_fp4(w->fmt)) {
+  if (is_fp4(w->fmt) && use_pair_gemm(w, g_dev[dev])) {
+    CUtensorMap tm_y, tm_sfa;
+    if ((rc = make_map(&tm_y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Y, w->N, M, 16, 32))) return rc;
+    if ((rc = make_atom_map(&tm_sfa, base + L.sf_off, static_cast<uint64_t>(L.M_pad / 128) * w->sf_kcols)))
+      return rc;
+    GemmParams p;
+    p.M = M;
+    p.N = w->N;
+    p.K = w->K;
+    p.kt_total = (w->K + 255) / 256;
+    p.m_tiles = (M + kPairBM - 1) / kPairBM;
+    p.n_tiles = (w->N + kPairBN - 1) / kPairBN;
+    p.num_tiles = p.m_tiles * p.n_tiles;
+    p.group_m = g_forced_group_m > 0 ? std::min((g_forced_group_m + 1) / 2, p.m_tiles)
+                                     : std::min(kPairGroupM, p.m_tiles);
+    p.r_tail = 2 * w->r_pad;
+    p.sfa = nullptr;
+    p.sfb = nullptr;
+    p.sf_kcols = w->sf_kcols;
+    p.bias = w->bias;
+    p.out_scale = std::ldexp(1.0f, -w->w_exp);
+    p.budget = wait_budget();
+    const int pairs = std::min(p.num_tiles, g_dev[dev].pair_clusters);
+    SVDQ_CUDA(launch_pdl(gemm_nvfp4_pair_kernel, dim3(2 * pairs), dim3(kGemmThreads), kPairSmemBytes, st, 2u,
+                         tm_a, w->tm_b_half, tm_sfa, w->tm_sfb, tm_xl1, w->tm_l2t_half, tm_y, p));
+  } else if (is_fp4(w->fmt)) {
     CUtensorMap tm_y;
     if ((rc = make_map(&tm_y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Y, w->N, M, 16, 32))) return rc;
     GemmParams p;
