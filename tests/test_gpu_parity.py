@@ -197,23 +197,26 @@ def test_forced_launch_shapes(S, M, K, N, rank, fmt):
     (256, 256, 512, 0, "nvfp4"),     # no low-rank tail
     (1000, 768, 272, 48, "nvfp4"),   # ragged last column block, 3 tail chunks
     (384, 320, 1024, 32, "nvfp4"),   # K below two K steps
+    (520, 512, 208, 32, "nvfp4"),    # one 192-column tile and a 16-column one
 ])
 def test_forced_gemm_kernel(S, M, K, N, rank, fmt):
-    """The FP4 GEMM on single CTAs (128 x 256 tiles) and on CTA pairs (256 x 256,
-    cta_group::2 MMAs) sums the same products in the same order: Y bit for bit
-    the same, within tolerance of the oracle."""
+    """The FP4 GEMM on single CTAs (128 x 256 tiles), on CTA pairs with 256 x 256
+    tiles and on CTA pairs with 256 x 192 tiles and two accumulators (cta_group::2
+    MMAs) sums the same products in the same order: Y bit for bit the same,
+    within tolerance of the oracle."""
     data = WL.make_small(M, K, N, rank=rank, fmt=fmt, seed=M + K)
     ref = oracle_layer(fmt, data, rank)
     w = load_from_oracle(S, fmt, ref["prep"])
     try:
         Ys = {}
-        for kind in (1, 2):
+        for kind in (1, 2, 3):
             S.svdq_set_gemm_kernel(kind)
             _, Y = _run_layer(S, w, WL.bf16_bits(data["X"]))
             ok, info = y_within_tol(bits(Y), ref["Y"])
             assert ok, (kind, info)
             Ys[kind] = bits(Y)
         assert np.array_equal(Ys[1], Ys[2])
+        assert np.array_equal(Ys[1], Ys[3])
     finally:
         S.svdq_set_gemm_kernel(0)
         w.close()

@@ -1,21 +1,29 @@
-// gemm_nvfp4_pair.cuh -- the fused 4-bit GEMM on CTA pairs (256 x 256 tiles).
+// gemm_nvfp4_pair.cuh -- the fused 4-bit GEMM on CTA pairs (256 x BN tiles,
+// BN = 256 or 192).
 //
 // Computes what gemm_nvfp4_kernel computes (SVDQuant Sec. 4.2, Eq. 5 and the
 // fused low-rank branch of Sec. 4.3, Fig. 6b):
 //   Y = Q(X_hat) Q(R) + (X_hat L1) L2 + b
 // with every output tile shared by the two CTAs of a cluster.  The pair's
-// 256 x 256 tile is one tcgen05.mma.cta_group::2 of M = 256, N = 256 per 64
-// values of K: each CTA stages its own 128 activation rows and one half (128
+// 256 x BN tile is one tcgen05.mma.cta_group::2 of M = 256, N = BN per 64
+// values of K: each CTA stages its own 128 activation rows and one half (BN / 2
 // weight columns) of B, and the MMA, issued by rank 0, reads both CTAs'
-// operands and accumulates each CTA's 128 x 256 block in that CTA's TMEM.
+// operands and accumulates each CTA's 128 x BN block in that CTA's TMEM.
 // Against one CTA per 128 x 256 tile, an SM then pulls 32 KB of codes per
-// 256-wide K step instead of 48 KB for the same tensor-core work, and the
-// smaller stages fit five to a CTA instead of four.
+// 256-wide K step instead of 48 KB for the same tensor-core work (BN = 256),
+// and the smaller stages fit five to a CTA instead of four.
+//
+// BN = 256 leaves room in TMEM for one accumulator: the MMAs of a tile wait
+// until the epilogue has copied the previous tile's accumulator to registers.
+// BN = 192 fits two accumulators (TMEM columns 0 and 256) beside the scale
+// factors, so the MMAs run on into the next tile while the epilogue drains the
+// last one; it moves more operand bytes per MMA and pays where the K loop of a
+// tile is short.
 //
 // Per CTA of the pair:
 //   warp 0    : TMA producer for this CTA's stage buffers: A codes (128 x 128 B),
-//               its half of B (128 x 128 B), the A scale atoms of its rows and
-//               the B scale atoms of all 256 columns (every CTA's TMEM needs
+//               its half of B (BN / 2 x 128 B), the A scale atoms of its rows and
+//               the B scale atoms of all BN columns (every CTA's TMEM needs
 //               them), then the low-rank operands (its XL1 rows, its half of
 //               [L2^T | L2^T]).  All of them count on rank 0's stage barrier;
 //               rank 0 alone arms it with both CTAs' bytes.
@@ -24,7 +32,7 @@
 //               issues the pair MMAs; each commit signals the matching barrier
 //               in both CTAs.
 //   warps 2-9 : epilogue of this CTA's 128 rows, as in gemm_nvfp4_kernel; the
-//               hand-back of the accumulator counts on rank 0's barrier, which
+//               hand-back of an accumulator counts on rank 0's barrier, which
 //               waits for all sixteen epilogue warps of the pair.
 #pragma once
 
@@ -33,21 +41,43 @@
 namespace svdq {
 
 constexpr int kPairBM = 256;                   // rows per pair tile (128 per CTA)
-constexpr int kPairBN = 256;                   // weight columns per pair tile (128 per CTA)
-constexpr int kPairStages = 5;
 constexpr int kPairGroupM = 4;                 // pair row blocks per tile-order group
-constexpr uint32_t kPairAOff = 0;                                 // 128 x 128 B
-constexpr uint32_t kPairBOff = 128 * kGemmBKB;                    // 16384: 128 x 128 B
-constexpr uint32_t kPairSfaOff = kPairBOff + 128 * kGemmBKB;      // 32768: 4 atoms
-constexpr uint32_t kPairSfbOff = kPairSfaOff + 4 * 512;           // 34816: 2 x 4 atoms
-constexpr uint32_t kPairStageBytes = kPairSfbOff + 8 * 512;       // 38912 (38 x 1024)
-constexpr uint32_t kPairEpiOff = kPairStageBytes * kPairStages;
-constexpr uint32_t kPairBarOff = kPairEpiOff + kGemmEpiWarps * kGemmEpiBufBytes;
-constexpr uint32_t kPairSmemBytes = kPairBarOff + 256 + 1024;
 constexpr uint16_t kPairMask = 3;              // both CTAs of the pair
 
-// p.m_tiles counts pair row blocks (256 rows); p.sfa / p.sfb are unused (the
-// scale atoms come through tm_sfa / tm_sfb: [atoms][128 x 32-bit words]).
+// Shape of the pair kernel for a tile width BN (weight columns per pair tile,
+// BN / 2 per CTA).  BN = 256 keeps one accumulator in TMEM (256 columns of the
+// 512, the scale factors in 48 more); BN = 192 fits two (columns 0 and 256),
+// so the MMAs of the next tile need not wait for the epilogue to empty the
+// last one.
+template <int BN>
+struct PairShape {
+  static_assert(BN == 256 || BN == 192, "pair tiles are 256 or 192 columns wide");
+  static constexpr int kBH = BN / 2;                                      // weight columns per CTA
+  static constexpr int kAcc = BN == 256 ? 1 : 2;                          // accumulators in TMEM
+  static constexpr int kStages = BN == 256 ? 5 : 6;
+  static constexpr uint32_t kAOff = 0;                                    // 128 x 128 B
+  static constexpr uint32_t kBOff = 128 * kGemmBKB;                       // kBH x 128 B
+  static constexpr uint32_t kSfaOff = kBOff + kBH * kGemmBKB;             // 4 atoms
+  static constexpr uint32_t kSfbOff = kSfaOff + 4 * 512;                  // 2 x 4 atoms
+  static constexpr uint32_t kStageBytes = kSfbOff + 8 * 512;              // 38912 / 34816
+  static constexpr uint32_t kEpiOff = kStageBytes * kStages;
+  static constexpr uint32_t kBarOff = kEpiOff + kGemmEpiWarps * kGemmEpiBufBytes;
+  static constexpr uint32_t kSmemBytes = kBarOff + 256 + 1024;
+  static constexpr uint32_t kAccStride = 256;                             // TMEM columns between accumulators
+  static constexpr uint32_t kSfaCol = kAccStride * (kAcc - 1) + BN;       // 256 / 448
+  static constexpr uint32_t kSfbCol = kSfaCol + 16;                       // 272 / 464
+  static_assert(kStageBytes % 1024 == 0, "stage buffers keep the 1024-byte swizzle alignment");
+  static_assert(kSfbCol + 32 <= kGemmTmemCols, "accumulators and scale factors fit in TMEM");
+};
+constexpr uint32_t kPairSmemBytes = PairShape<256>::kSmemBytes;
+constexpr uint32_t kPair192SmemBytes = PairShape<192>::kSmemBytes;
+
+// p.m_tiles counts pair row blocks (256 rows), p.n_tiles weight column blocks
+// of BN; p.sfa / p.sfb are unused (the scale atoms come through tm_sfa / tm_sfb:
+// [atoms][128 x 32-bit words]; for tm_sfb, atom slot 2 nb + a of a K step holds
+// the scales of weight columns nb BN + 128 a .. + 127).  tm_b and tm_l2t have
+// boxes of BN / 2 rows.
+template <int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_nvfp4_pair_kernel(const __grid_constant__ CUtensorMap tm_a,
                            const __grid_constant__ CUtensorMap tm_b,
@@ -56,14 +86,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                            const __grid_constant__ CUtensorMap tm_xl1,
                            const __grid_constant__ CUtensorMap tm_l2t,
                            const __grid_constant__ CUtensorMap tm_y, const GemmParams p) {
-  constexpr int STAGES = kPairStages;
+  using Sh = PairShape<BN>;
+  constexpr int STAGES = Sh::kStages;
+  constexpr int ACC = Sh::kAcc;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_smem_1024(smem_raw);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kPairBarOff);   // rank 0's are used
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Sh::kBarOff);   // rank 0's are used
   uint64_t* empty = full + STAGES;
-  uint64_t* acc_full = empty + STAGES;
-  uint64_t* acc_empty = acc_full + 1;                                  // rank 0's is used
-  uint64_t* mma_done = acc_empty + 1;
+  uint64_t* acc_full = empty + STAGES;                                 // [ACC]
+  uint64_t* acc_empty = acc_full + ACC;                                // [ACC], rank 0's are used
+  uint64_t* mma_done = acc_empty + ACC;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
@@ -82,8 +114,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 2 * kGemmEpiWarps);
+    for (int b = 0; b < ACC; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 2 * kGemmEpiWarps);
+    }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -111,8 +145,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         prefetch_tmap(&tm_l2t);
       }
       const uint32_t full0 = map_shared_rank(smem_u32(&full[0]), 0);   // rank 0's stage barriers
-      const uint32_t main_tx = 2 * kPairStageBytes;
-      const uint32_t lr_tx = 2 * 2 * 128 * static_cast<uint32_t>(lr_cols) * 2;
+      const uint32_t main_tx = 2 * Sh::kStageBytes;
+      const uint32_t lr_tx = 2 * (128 + Sh::kBH) * static_cast<uint32_t>(lr_cols) * 2;
       int it = 0;
       bool ok = true;
       for (int tile = pair; tile < p.num_tiles && ok; tile += n_pairs) {
@@ -120,7 +154,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         gemm_tile_coords(p.m_tiles, p.n_tiles, p.group_m, tile, mp, nb);
         const int m_blk = 2 * mp + static_cast<int>(rank);    // this CTA's 128-row block
         const int m0 = m_blk * 128;
-        const int nh0 = nb * kPairBN + 128 * static_cast<int>(rank);
+        const int nh0 = nb * BN + Sh::kBH * static_cast<int>(rank);
         for (int step = 0; step < steps_per_tile; ++step, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
@@ -130,21 +164,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             ok = false;
             break;
           }
-          uint8_t* st = smem + s * kPairStageBytes;
+          uint8_t* st = smem + s * Sh::kStageBytes;
           const uint32_t fb = full0 + static_cast<uint32_t>(s) * 8u;
           if (step < p.kt_total) {
             const int kt = step;
             if (rank == 0) mbar_arrive_expect_tx(&full[s], main_tx);
-            tma_load_2d_pair(st + kPairAOff, &tm_a, fb, kt * kGemmBKB, m0);
-            tma_load_2d_pair(st + kPairBOff, &tm_b, fb, kt * kGemmBKB, nh0);
-            tma_load_2d_pair(st + kPairSfaOff, &tm_sfa, fb, 0, m_blk * p.sf_kcols + 4 * kt);
-            tma_load_2d_pair(st + kPairSfbOff, &tm_sfb, fb, 0, (2 * nb) * p.sf_kcols + 4 * kt);
-            tma_load_2d_pair(st + kPairSfbOff + 2048, &tm_sfb, fb, 0, (2 * nb + 1) * p.sf_kcols + 4 * kt);
+            tma_load_2d_pair(st + Sh::kAOff, &tm_a, fb, kt * kGemmBKB, m0);
+            tma_load_2d_pair(st + Sh::kBOff, &tm_b, fb, kt * kGemmBKB, nh0);
+            tma_load_2d_pair(st + Sh::kSfaOff, &tm_sfa, fb, 0, m_blk * p.sf_kcols + 4 * kt);
+            tma_load_2d_pair(st + Sh::kSfbOff, &tm_sfb, fb, 0, (2 * nb) * p.sf_kcols + 4 * kt);
+            tma_load_2d_pair(st + Sh::kSfbOff + 2048, &tm_sfb, fb, 0, (2 * nb + 1) * p.sf_kcols + 4 * kt);
           } else {
             const int c = step - p.kt_total;
             if (rank == 0) mbar_arrive_expect_tx(&full[s], lr_tx);
-            tma_load_2d_pair(st + kPairAOff, &tm_xl1, fb, c * 64, m0);
-            tma_load_2d_pair(st + kPairBOff, &tm_l2t, fb, c * 64, nh0);
+            tma_load_2d_pair(st + Sh::kAOff, &tm_xl1, fb, c * 64, m0);
+            tma_load_2d_pair(st + Sh::kBOff, &tm_l2t, fb, c * 64, nh0);
           }
         }
       }
@@ -156,14 +190,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer (rank 0)
     if (rank == 0 && elect_one()) {
-      const uint32_t idesc_main = idesc_e2m1_ue4m3(kPairBM, kPairBN);
-      const uint32_t idesc_lr = idesc_bf16_f32(kPairBM, kPairBN);
+      const uint32_t idesc_main = idesc_e2m1_ue4m3(kPairBM, BN);
+      const uint32_t idesc_lr = idesc_bf16_f32(kPairBM, BN);
       const uint32_t lr_row_bytes = static_cast<uint32_t>(lr_cols) * 2;
-      const uint32_t d_tmem = tmem_base;
+      const uint32_t sfa_col = tmem_base + Sh::kSfaCol;
+      const uint32_t sfb_col = tmem_base + Sh::kSfbCol;
       int it = 0, t_local = 0;
       bool ok = true;
       for (int tile = pair; tile < p.num_tiles && ok; tile += n_pairs, ++t_local) {
-        if (!mbar_wait(acc_empty, (t_local & 1) ^ 1, p.budget, abort_flag)) {
+        // accumulator b of this tile; its previous tile's epilogue must have emptied it
+        const int b = t_local % ACC;
+        const uint32_t d_tmem = tmem_base + Sh::kAccStride * static_cast<uint32_t>(b);
+        if (!mbar_wait(&acc_empty[b], ((t_local / ACC) & 1) ^ 1, p.budget, abort_flag)) {
           raise_error(kErrWaitGemm);
           *abort_flag = 1;
           break;
@@ -180,23 +218,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             break;
           }
           tc_fence_after();
-          uint8_t* st = smem + s * kPairStageBytes;
-          const uint32_t a0 = smem_u32(st + kPairAOff);
-          const uint32_t b0 = smem_u32(st + kPairBOff);
+          uint8_t* st = smem + s * Sh::kStageBytes;
+          const uint32_t a0 = smem_u32(st + Sh::kAOff);
+          const uint32_t b0 = smem_u32(st + Sh::kBOff);
           if (!tail) {
-            const uint32_t sfa_s = smem_u32(st + kPairSfaOff);
-            const uint32_t sfb_s = smem_u32(st + kPairSfbOff);
+            const uint32_t sfa_s = smem_u32(st + Sh::kSfaOff);
+            const uint32_t sfb_s = smem_u32(st + Sh::kSfbOff);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              tmem_cp_32x128b_x4_pair(tmem_base + kGemmSfaCol + 4 * j, sf_desc(sfa_s + 512 * j));
-              tmem_cp_32x128b_x4_pair(tmem_base + kGemmSfbCol + 8 * j, sf_desc(sfb_s + 512 * j));
-              tmem_cp_32x128b_x4_pair(tmem_base + kGemmSfbCol + 8 * j + 4, sf_desc(sfb_s + 2048 + 512 * j));
+              tmem_cp_32x128b_x4_pair(sfa_col + 4 * j, sf_desc(sfa_s + 512 * j));
+              tmem_cp_32x128b_x4_pair(sfb_col + 8 * j, sf_desc(sfb_s + 512 * j));
+              tmem_cp_32x128b_x4_pair(sfb_col + 8 * j + 4, sf_desc(sfb_s + 2048 + 512 * j));
             }
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               mma_nvf4_pair(d_tmem, make_kmajor_desc(a0 + 32 * j, 128), make_kmajor_desc(b0 + 32 * j, 128),
-                            idesc_main, tmem_base + kGemmSfaCol + 4 * j, tmem_base + kGemmSfbCol + 8 * j,
-                            (step > 0 || j > 0) ? 1u : 0u);
+                            idesc_main, sfa_col + 4 * j, sfb_col + 8 * j, (step > 0 || j > 0) ? 1u : 0u);
             }
           } else {
             for (int j = 0; j < lr_cols / 16; ++j) {
@@ -207,7 +244,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tc_commit_pair(&empty[s], kPairMask);
         }
         if (!ok) break;
-        tc_commit_pair(acc_full, kPairMask);
+        tc_commit_pair(&acc_full[b], kPairMask);
       }
       tc_commit_pair(mma_done, kPairMask);   // retires once every MMA and copy issued above has completed
     }
@@ -215,31 +252,33 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ---------------------------------------------------------------- epilogue
     const uint32_t q = warp & 3u;
     const uint32_t h = (warp - 2) >> 2;
-    uint8_t* ebuf = smem + kPairEpiOff + (warp - 2) * kGemmEpiBufBytes;
-    const uint32_t acc_empty0 = map_shared_rank(smem_u32(acc_empty), 0);
+    constexpr int CH = Sh::kBH / 32;   // 32-column chunks of this warp's half of the tile
+    uint8_t* ebuf = smem + Sh::kEpiOff + (warp - 2) * kGemmEpiBufBytes;
     int t_local = 0;
     for (int tile = pair; tile < p.num_tiles; tile += n_pairs, ++t_local) {
       int mp, nb;
       gemm_tile_coords(p.m_tiles, p.n_tiles, p.group_m, tile, mp, nb);
-      if (!warp_wait(acc_full, t_local & 1, p.budget, abort_flag)) {
+      const int b = t_local % ACC;
+      if (!warp_wait(&acc_full[b], (t_local / ACC) & 1, p.budget, abort_flag)) {
         if (lane == 0) raise_error(kErrWaitGemm);
         *abort_flag = 1;
         break;
       }
       tc_fence_after();
-      uint32_t v[4][32];
-      const uint32_t taddr = tmem_base + ((q * 32u) << 16) + 128u * h;
+      uint32_t v[CH][32];
+      const uint32_t taddr = tmem_base + ((q * 32u) << 16) + Sh::kAccStride * static_cast<uint32_t>(b) +
+                             static_cast<uint32_t>(Sh::kBH) * h;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(taddr + 32 * c, v[c]);
+      for (int c = 0; c < CH; ++c) tmem_ld32(taddr + 32 * c, v[c]);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(acc_empty0);
+      if (lane == 0) mbar_arrive_cluster(map_shared_rank(smem_u32(&acc_empty[b]), 0));
       const int row0 = mp * kPairBM + 128 * static_cast<int>(rank) + static_cast<int>(q) * 32;
-      const int ncol = nb * kPairBN + 128 * static_cast<int>(h);
+      const int ncol = nb * BN + Sh::kBH * static_cast<int>(h);
       if (row0 < p.M) {
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
+        for (int c = 0; c < 2 * CH; ++c)
           if (ncol + 16 * c < p.N)
             epi_store_16(&v[c / 2][16 * (c % 2)], ebuf, &tm_y, ncol + 16 * c, row0, p.N, p.bias,
                          p.out_scale, lane);

@@ -267,6 +267,29 @@ __global__ void quant_weight_nvfp4_kernel(const float* __restrict__ R, int K, in
   atom[(n & 31) * 16 + ((n & 127) >> 5) * 4 + (g & 3)] = static_cast<uint8_t>(s8);
 }
 
+// The weight scale atoms regrouped for the 192-column pair GEMM tiles: atom slot
+// 2 nb + a (a = 0, 1) of K step kc holds the scales of weight columns
+// nb * 192 + 128 a .. + 127 in the atom layout above (columns past the tile or
+// past N hold 0), so that a tile's scales start at an atom boundary.  One
+// thread per byte of the output, [2 * n_tiles][sf_kcols][512].
+__global__ void pair192_scale_atoms_kernel(const uint8_t* __restrict__ sf, int N, int sf_kcols, int n_tiles,
+                                           uint8_t* __restrict__ out) {
+  const size_t total = static_cast<size_t>(2 * n_tiles) * sf_kcols * 512;
+  const size_t o = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (o >= total) return;
+  const int i = static_cast<int>(o % 512);
+  const int kc = static_cast<int>((o / 512) % sf_kcols);
+  const int ts = static_cast<int>(o / (512 * static_cast<size_t>(sf_kcols)));
+  const int n = i / 16 + 32 * ((i % 16) / 4);   // column within the atom
+  const int g = i % 4;
+  const int nt = 128 * (ts % 2) + n;            // column within the 192-wide tile
+  const int c = (ts / 2) * 192 + nt;
+  uint8_t v = 0;
+  if (nt < 192 && c < N)
+    v = sf[(static_cast<size_t>(c / 128) * sf_kcols + kc) * 512 + (c % 32) * 16 + ((c % 128) / 32) * 4 + g];
+  out[o] = v;
+}
+
 __global__ void quant_weight_int4_kernel(const float* __restrict__ R, int K, int N, int N_pad,
                                          int8_t* __restrict__ codes, uint16_t* __restrict__ sf,
                                          float* __restrict__ sf32) {

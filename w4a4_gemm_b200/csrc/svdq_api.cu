@@ -46,6 +46,8 @@ struct svdq_weights {
   float* lambda = nullptr;
   uint8_t* wcodes = nullptr;  // NVFP4: N x K/2 packed; INT4: N x K int8
   uint8_t* wsf = nullptr;     // NVFP4: atoms [N_pad/128][sf_kcols][512]; INT4: fp16 [K/64][N_pad]
+  uint8_t* wsf192 = nullptr;  // FP4: the same atoms regrouped per 192-column tile [2 n192][sf_kcols][512]
+  int n192 = 0;               // FP4: 192-column tiles of N
   float* wsf32 = nullptr;     // INT4: the same scales as fp32, read by the GEMM
   __nv_bfloat16* l1t = nullptr;  // r_pad x K
   __nv_bfloat16* l1st = nullptr; // r_pad x K: bf16(diag(1/lambda) L1)^T, read by the activation kernel
@@ -54,6 +56,7 @@ struct svdq_weights {
   __nv_bfloat16* bias = nullptr;
   CUtensorMap tm_b, tm_l1t, tm_l2t;
   CUtensorMap tm_b_half, tm_l2t_half, tm_sfb;   // FP4 CTA-pair GEMM: 128-row boxes, scale atoms
+  CUtensorMap tm_b_96, tm_l2t_96, tm_sfb192;    // FP4 CTA-pair GEMM with 192-column tiles
   double refine_err0 = -1.0, refine_err = -1.0;   // weight error: SVD start, kept iterate
   unsigned flags = 0;  // SVDQ_WEIGHT_POW2_PRESCALE
   int w_exp = 0;       // the codes and scales are those of R * 2^w_exp (FP4 formats)
@@ -196,7 +199,8 @@ int make_atom_map(CUtensorMap* m, const void* base, uint64_t atoms) {
 // ------------------------------------------------------------ device info ---
 struct DeviceInfo {
   int sms = 0;
-  int pair_clusters = 0;                    // resident clusters of the CTA-pair GEMM
+  int pair_clusters = 0;                    // resident clusters of the CTA-pair GEMM (256-column tiles)
+  int pair192_clusters = 0;                 // the same with 192-column tiles
   int qclusters[kQuantMaxSplit + 1] = {};   // resident activation-kernel clusters of size C
   bool attrs_set = false;
 };
@@ -221,8 +225,10 @@ int device_setup(int dev) {
                                  kW8SmemBytes));
   SVDQ_CUDA(cudaFuncSetAttribute(gemm_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kGemmSmemBytes));
-  SVDQ_CUDA(cudaFuncSetAttribute(gemm_nvfp4_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  SVDQ_CUDA(cudaFuncSetAttribute(gemm_nvfp4_pair_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kPairSmemBytes));
+  SVDQ_CUDA(cudaFuncSetAttribute(gemm_nvfp4_pair_kernel<192>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kPair192SmemBytes));
   SVDQ_CUDA(cudaFuncSetAttribute(gemm_int4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kI4SmemBytes));
   SVDQ_CUDA(cudaFuncSetAttribute(tensor_peak_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -247,11 +253,11 @@ int device_setup(int dev) {
     SVDQ_CUDA(cudaOccupancyMaxActiveClusters(&n, quant_act_kernel<1>, &cfg));
     d.qclusters[C] = n;
   }
-  {
+  for (int bn : {256, 192}) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(d.sms & ~1);
     cfg.blockDim = dim3(kGemmThreads);
-    cfg.dynamicSmemBytes = kPairSmemBytes;
+    cfg.dynamicSmemBytes = bn == 256 ? kPairSmemBytes : kPair192SmemBytes;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
@@ -260,8 +266,13 @@ int device_setup(int dev) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    SVDQ_CUDA(cudaOccupancyMaxActiveClusters(&n, gemm_nvfp4_pair_kernel, &cfg));
-    d.pair_clusters = n;
+    if (bn == 256) {
+      SVDQ_CUDA(cudaOccupancyMaxActiveClusters(&n, gemm_nvfp4_pair_kernel<256>, &cfg));
+      d.pair_clusters = n;
+    } else {
+      SVDQ_CUDA(cudaOccupancyMaxActiveClusters(&n, gemm_nvfp4_pair_kernel<192>, &cfg));
+      d.pair192_clusters = n;
+    }
   }
   d.attrs_set = true;
   return SVDQ_OK;
@@ -293,7 +304,8 @@ constexpr double kQuantStageCycles = 800.0;
 constexpr double kQuantL1Cycles = 300.0;
 QuantSplit g_forced_split{0, 0};   // svdq_set_quant_split; {0, 0} = automatic
 int g_forced_group_m = 0;          // svdq_set_gemm_raster; 0 = automatic
-int g_forced_gemm_kind = 0;        // svdq_set_gemm_kernel; 0 = automatic, 1 = one CTA, 2 = CTA pairs
+int g_forced_gemm_kind = 0;        // svdq_set_gemm_kernel; 0 = automatic, 1 = one CTA, 2 = CTA pairs,
+                                   // 3 = CTA pairs on 192-column tiles
 
 QuantSplit quant_split_for(int M, int K, int r_pad, const DeviceInfo& d) {
   const int smax = r_pad > 0 ? quant_stack_max(r_pad) : 8;
@@ -355,6 +367,8 @@ int encode_weight_maps(svdq_weights* w) {
     rc = make_map(&w->tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->wcodes, w->K / 2, w->N, 128, kGemmBN);
     if (!rc) rc = make_map(&w->tm_b_half, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->wcodes, w->K / 2, w->N, 128, 128);
     if (!rc) rc = make_atom_map(&w->tm_sfb, w->wsf, static_cast<uint64_t>(w->N_pad / 128) * w->sf_kcols);
+    if (!rc) rc = make_map(&w->tm_b_96, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->wcodes, w->K / 2, w->N, 128, 96);
+    if (!rc) rc = make_atom_map(&w->tm_sfb192, w->wsf192, static_cast<uint64_t>(2 * w->n192) * w->sf_kcols);
   } else if (w->fmt == SVDQ_W8A8)
     rc = make_map(&w->tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->wcodes, w->K, w->N, kW8BKB, kW8BN);
   else
@@ -370,10 +384,14 @@ int encode_weight_maps(svdq_weights* w) {
     if (is_fp4(w->fmt) &&
         (rc = make_map(&w->tm_l2t_half, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w->l2t2, 2 * w->r_pad, w->N, lc, 128)))
       return rc;
+    if (is_fp4(w->fmt) &&
+        (rc = make_map(&w->tm_l2t_96, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w->l2t2, 2 * w->r_pad, w->N, lc, 96)))
+      return rc;
   } else {
     w->tm_l1t = w->tm_b;
     w->tm_l2t = w->tm_b;
     w->tm_l2t_half = w->tm_b;
+    w->tm_l2t_96 = w->tm_b;
   }
   return SVDQ_OK;
 }
@@ -384,6 +402,7 @@ void free_weights(svdq_weights* w) {
   cudaFree(w->lambda);
   cudaFree(w->wcodes);
   cudaFree(w->wsf);
+  cudaFree(w->wsf192);
   cudaFree(w->wsf32);
   cudaFree(w->l1t);
   cudaFree(w->l1st);
@@ -420,6 +439,12 @@ int alloc_weights(svdq_weights* w, cudaStream_t st) {
     return SVDQ_ERR_ALLOC;
   SVDQ_CUDA(cudaMemsetAsync(w->inv_lambda, 0, il_bytes, st));
   SVDQ_CUDA(cudaMemsetAsync(w->wsf, 0, sfb, st));
+  if (is_fp4(w->fmt)) {
+    w->n192 = (w->N + 191) / 192;
+    const size_t sf192 = static_cast<size_t>(2 * w->n192) * w->sf_kcols * 512;
+    if (cudaMalloc(&w->wsf192, sf192) != cudaSuccess) return SVDQ_ERR_ALLOC;
+    SVDQ_CUDA(cudaMemsetAsync(w->wsf192, 0, sf192, st));
+  }
   if (w->fmt == SVDQ_INT4) {
     const size_t sf32 = static_cast<size_t>(w->K / 64) * w->N_pad * sizeof(float);
     if (cudaMalloc(&w->wsf32, sf32) != cudaSuccess) return SVDQ_ERR_ALLOC;
@@ -501,6 +526,12 @@ int quantize_residual(svdq_weights* w, const float* R, cudaStream_t st) {
                                                    reinterpret_cast<uint16_t*>(w->wsf), w->wsf32);
   }
   SVDQ_CHECK_LAUNCH();
+  if (is_fp4(w->fmt)) {
+    const size_t sf192 = static_cast<size_t>(2 * w->n192) * w->sf_kcols * 512;
+    pair192_scale_atoms_kernel<<<static_cast<unsigned>((sf192 + 255) / 256), 256, 0, st>>>(
+        w->wsf, w->N, w->sf_kcols, w->n192, w->wsf192);
+    SVDQ_CHECK_LAUNCH();
+  }
   if (w->w_exp != e_old) return build_l2t2(w, st);   // the tail carries the same 2^e
   return SVDQ_OK;
 }
@@ -737,7 +768,7 @@ SVDQ_API int svdq_tensor_peak(int fmt, long long steps, void* stream) {
 }
 
 SVDQ_API int svdq_set_gemm_kernel(int kind) {
-  if (kind < 0 || kind > 2) return SVDQ_ERR_INVALID_ARG;
+  if (kind < 0 || kind > 3) return SVDQ_ERR_INVALID_ARG;
   g_forced_gemm_kind = kind;
   return SVDQ_OK;
 }
@@ -1047,11 +1078,18 @@ int gemm_group_m(int m_tiles, int n_tiles, int grid) {
   return std::min(kGemmGroupM, m_tiles);
 }
 
-// FP4 GEMM on CTA pairs (256 x 256 tiles) or on single CTAs (128 x 256).
-bool use_pair_gemm(const svdq_weights* w, const DeviceInfo& d) {
-  if (!is_fp4(w->fmt) || d.pair_clusters <= 0) return false;
-  if (g_forced_gemm_kind != 0) return g_forced_gemm_kind == 2;
-  return true;   // as fast or faster at every layer shape of the FLUX block
+// FP4 GEMM kernel: 1 = single CTAs (128 x 256 tiles), 2 = CTA pairs on
+// 256 x 256 tiles, 3 = CTA pairs on 256 x 192 tiles with two accumulators.
+// With one accumulator the MMAs of a tile wait until the epilogue has copied
+// the previous tile out of TMEM; two accumulators hide that hand-off, which
+// weighs most when the tiles are short in K.  On B200 the 192-column tiles are
+// 3-5 % faster at K = 3072 (FLUX QKV, out and fc1 layers) and 6 % slower at
+// K = 12288 (fc2), where a tile's K loop is four times longer.
+int fp4_gemm_kind(const svdq_weights* w, const DeviceInfo& d) {
+  int kind = g_forced_gemm_kind != 0 ? g_forced_gemm_kind : (w->K <= 4096 ? 3 : 2);
+  if (kind == 3 && d.pair192_clusters <= 0) kind = 2;
+  if (kind == 2 && d.pair_clusters <= 0) kind = 1;
+  return kind;
 }
 
 SVDQ_API int svdq_linear(const svdq_weights* w, const void* ws, int M, void* Y, void* stream) {
@@ -1087,7 +1125,9 @@ SVDQ_API int svdq_linear(const svdq_weights* w, const void* ws, int M, void* Y, 
   } else {
     tm_xl1 = tm_a;
   }
-  if (is_fp4(w->fmt) && use_pair_gemm(w, g_dev[dev])) {
+  const int fp4_kind = is_fp4(w->fmt) ? fp4_gemm_kind(w, g_dev[dev]) : 0;
+  if (fp4_kind == 2 || fp4_kind == 3) {
+    const int bn = fp4_kind == 2 ? 256 : 192;
     CUtensorMap tm_y, tm_sfa;
     if ((rc = make_map(&tm_y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Y, w->N, M, 16, 32))) return rc;
     if ((rc = make_atom_map(&tm_sfa, base + L.sf_off, static_cast<uint64_t>(L.M_pad / 128) * w->sf_kcols)))
@@ -1098,7 +1138,7 @@ SVDQ_API int svdq_linear(const svdq_weights* w, const void* ws, int M, void* Y, 
     p.K = w->K;
     p.kt_total = (w->K + 255) / 256;
     p.m_tiles = (M + kPairBM - 1) / kPairBM;
-    p.n_tiles = (w->N + kPairBN - 1) / kPairBN;
+    p.n_tiles = (w->N + bn - 1) / bn;
     p.num_tiles = p.m_tiles * p.n_tiles;
     p.group_m = g_forced_group_m > 0 ? std::min((g_forced_group_m + 1) / 2, p.m_tiles)
                                      : std::min(kPairGroupM, p.m_tiles);
@@ -1109,9 +1149,15 @@ SVDQ_API int svdq_linear(const svdq_weights* w, const void* ws, int M, void* Y, 
     p.bias = w->bias;
     p.out_scale = std::ldexp(1.0f, -w->w_exp);
     p.budget = wait_budget();
-    const int pairs = std::min(p.num_tiles, g_dev[dev].pair_clusters);
-    SVDQ_CUDA(launch_pdl(gemm_nvfp4_pair_kernel, dim3(2 * pairs), dim3(kGemmThreads), kPairSmemBytes, st, 2u,
-                         tm_a, w->tm_b_half, tm_sfa, w->tm_sfb, tm_xl1, w->tm_l2t_half, tm_y, p));
+    if (bn == 256) {
+      const int pairs = std::min(p.num_tiles, g_dev[dev].pair_clusters);
+      SVDQ_CUDA(launch_pdl(gemm_nvfp4_pair_kernel<256>, dim3(2 * pairs), dim3(kGemmThreads), kPairSmemBytes, st,
+                           2u, tm_a, w->tm_b_half, tm_sfa, w->tm_sfb, tm_xl1, w->tm_l2t_half, tm_y, p));
+    } else {
+      const int pairs = std::min(p.num_tiles, g_dev[dev].pair192_clusters);
+      SVDQ_CUDA(launch_pdl(gemm_nvfp4_pair_kernel<192>, dim3(2 * pairs), dim3(kGemmThreads), kPair192SmemBytes,
+                           st, 2u, tm_a, w->tm_b_96, tm_sfa, w->tm_sfb192, tm_xl1, w->tm_l2t_96, tm_y, p));
+    }
   } else if (is_fp4(w->fmt)) {
     CUtensorMap tm_y;
     if ((rc = make_map(&tm_y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Y, w->N, M, 16, 32))) return rc;
