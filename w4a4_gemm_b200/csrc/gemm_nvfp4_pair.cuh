@@ -31,7 +31,8 @@
 //               CTAs' scales into their TMEM (tcgen05.cp.cta_group::2) and
 //               issues the pair MMAs; each commit signals the matching barrier
 //               in both CTAs.
-//   warps 2-9 : epilogue of this CTA's 128 rows, as in gemm_nvfp4_kernel; the
+//   warps 2-9 : epilogue of this CTA's 128 rows, as in gemm_nvfp4_kernel but
+//               with 32-column TMA boxes (a 2 KB buffer per warp); the
 //               hand-back of an accumulator counts on rank 0's barrier, which
 //               waits for all sixteen epilogue warps of the pair.
 #pragma once
@@ -61,7 +62,8 @@ struct PairShape {
   static constexpr uint32_t kSfbOff = kSfaOff + 4 * 512;                  // 2 x 4 atoms
   static constexpr uint32_t kStageBytes = kSfbOff + 8 * 512;              // 38912 / 34816
   static constexpr uint32_t kEpiOff = kStageBytes * kStages;
-  static constexpr uint32_t kBarOff = kEpiOff + kGemmEpiWarps * kGemmEpiBufBytes;
+  static constexpr uint32_t kEpiBufBytes = 32 * 64;                      // 32 rows x 32 bf16 per warp
+  static constexpr uint32_t kBarOff = kEpiOff + kGemmEpiWarps * kEpiBufBytes;
   static constexpr uint32_t kSmemBytes = kBarOff + 256 + 1024;
   static constexpr uint32_t kAccStride = 256;                             // TMEM columns between accumulators
   static constexpr uint32_t kSfaCol = kAccStride * (kAcc - 1) + BN;       // 256 / 448
@@ -253,7 +255,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t q = warp & 3u;
     const uint32_t h = (warp - 2) >> 2;
     constexpr int CH = Sh::kBH / 32;   // 32-column chunks of this warp's half of the tile
-    uint8_t* ebuf = smem + Sh::kEpiOff + (warp - 2) * kGemmEpiBufBytes;
+    uint8_t* ebuf = smem + Sh::kEpiOff + (warp - 2) * Sh::kEpiBufBytes;
     int t_local = 0;
     for (int tile = pair; tile < p.num_tiles; tile += n_pairs, ++t_local) {
       int mp, nb;
@@ -278,10 +280,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int ncol = nb * BN + Sh::kBH * static_cast<int>(h);
       if (row0 < p.M) {
 #pragma unroll
-        for (int c = 0; c < 2 * CH; ++c)
-          if (ncol + 16 * c < p.N)
-            epi_store_16(&v[c / 2][16 * (c % 2)], ebuf, &tm_y, ncol + 16 * c, row0, p.N, p.bias,
-                         p.out_scale, lane);
+        for (int c = 0; c < CH; ++c)
+          if (ncol + 32 * c < p.N)
+            epi_store_32(v[c], ebuf, &tm_y, ncol + 32 * c, row0, p.N, p.bias, p.out_scale, lane);
       }
     }
     if (lane == 0) bulk_wait_group_all();

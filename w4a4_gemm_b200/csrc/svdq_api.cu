@@ -1129,7 +1129,7 @@ SVDQ_API int svdq_linear(const svdq_weights* w, const void* ws, int M, void* Y, 
   if (fp4_kind == 2 || fp4_kind == 3) {
     const int bn = fp4_kind == 2 ? 256 : 192;
     CUtensorMap tm_y, tm_sfa;
-    if ((rc = make_map(&tm_y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Y, w->N, M, 16, 32))) return rc;
+    if ((rc = make_map(&tm_y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Y, w->N, M, 32, 32))) return rc;
     if ((rc = make_atom_map(&tm_sfa, base + L.sf_off, static_cast<uint64_t>(L.M_pad / 128) * w->sf_kcols)))
       return rc;
     GemmParams p;
