@@ -72,7 +72,7 @@ DATASHEET_FP4_TFLOPS = 9000.0
 DATASHEET_INT8_TOPS = 4500.0
 NOMINAL_HBM_GBS = 8000.0
 NCU_TRAFFIC = {
-    ("gemm_nvfp4_pair_kernel", "c2_qkv/qkv", 4608, "nvfp4"): (63905536, "11d238ee1892f8dd"),
+    ("gemm_nvfp4_pair_kernel", "c2_qkv/qkv", 4608, "nvfp4"): (63905536, "ab2d6aed3c92a25a"),
     ("gemm_nvfp4_pair_kernel", "c5_block/fc2", 16384, "nvfp4"): (222889216, "f895356c38d662a7"),
     ("quant_act_kernel", "c2_qkv/qkv", 4608, "nvfp4"): (28561408, "97712fa48aaac990"),
     ("quant_act_kernel", "c5_block/fc2", 16384, "nvfp4"): (498574592, "97712fa48aaac990"),

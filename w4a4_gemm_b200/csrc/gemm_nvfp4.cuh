@@ -145,51 +145,6 @@ __device__ __forceinline__ void epi_store_16(const uint32_t* r, uint8_t* buf, co
   }
 }
 
-// The same for 32 columns (n0 .. n0 + 31): a 2 KB buffer of 32 rows of 64 bytes
-// in the TMA 64-byte swizzle (16-byte chunk c of row r at c ^ ((r >> 1) & 3)),
-// one TMA store of the 32 x 32 box.  Used by the CTA-pair kernels: half the
-// stores of 16-column boxes for the same bytes.
-__device__ __forceinline__ void epi_store_32(const uint32_t* r, uint8_t* buf, const CUtensorMap* tm_y,
-                                             int n0, int row0, int N,
-                                             const __nv_bfloat16* __restrict__ bias, float out_scale,
-                                             uint32_t lane) {
-  uint32_t w[16];
-#pragma unroll
-  for (int h = 0; h < 4; ++h) {
-    float bb[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) bb[j] = 0.f;
-    if (bias != nullptr && n0 + 8 * h < N) {
-      const uint4 b = __ldg(reinterpret_cast<const uint4*>(bias + n0 + 8 * h));
-      const uint32_t b4[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        bb[2 * t] = bf16_lo(b4[t]);
-        bb[2 * t + 1] = bf16_hi(b4[t]);
-      }
-    }
-#pragma unroll
-    for (int t = 0; t < 4; ++t)
-      w[4 * h + t] = pack_bf16x2(__fmaf_rn(__uint_as_float(r[8 * h + 2 * t]), out_scale, bb[2 * t]),
-                                 __fmaf_rn(__uint_as_float(r[8 * h + 2 * t + 1]), out_scale, bb[2 * t + 1]));
-  }
-  if (lane == 0) bulk_wait_group_read<0>();   // the previous store has read the buffer
-  __syncwarp();
-  const uint32_t row_addr = smem_u32(buf) + lane * 64u;
-  const uint32_t sw = (lane >> 1) & 3u;
-#pragma unroll
-  for (uint32_t c = 0; c < 4; ++c)
-    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row_addr + ((c ^ sw) << 4)),
-                 "r"(w[4 * c]), "r"(w[4 * c + 1]), "r"(w[4 * c + 2]), "r"(w[4 * c + 3])
-                 : "memory");
-  fence_proxy_async_smem();
-  __syncwarp();
-  if (lane == 0) {
-    tma_store_2d(tm_y, buf, n0, row0);
-    bulk_commit_group();
-  }
-}
-
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a,
                       const __grid_constant__ CUtensorMap tm_b,
