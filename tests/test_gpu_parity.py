@@ -412,3 +412,38 @@ def test_prepare_refinement(S, fmt):
     codes, scales = O.weight_quant(fmt, R)
     assert np.array_equal(scales, e["scales"]) and np.array_equal(codes, e["codes"])
     w.close()
+
+
+@pytest.mark.parametrize("fmt,pre", [("nvfp4", False), ("nvfp4", True), ("fp4g32", False), ("int4", False)])
+def test_refined_weights_through_the_gemm(S, fmt, pre):
+    """After a refinement that may keep an earlier iterate, every GEMM kernel reads
+    the kept codes and scales (and the layouts derived from them): Y from each
+    kernel is the oracle's layer of the exported parts, bit for bit the same
+    across the FP4 kernels.  With the prescale, the kept iterate's exponent."""
+    M, K, N, r = 300, 512, 400, 16
+    data = WL.make_small(M, K, N, w_outlier_rows=6, seed=13)
+    Xb = WL.bf16_bits(data["X"])
+    W = data["W"]
+    if pre:
+        W = (W.float() * 0.02).to(torch.bfloat16)   # residual scales in the E4M3 subnormal range
+    w = S.svdq_prepare_weights(W.cuda(), r, fmt, x_absmax=S.svdq_calib_absmax(data["X"].cuda()),
+                               refine_iters=4, pow2_prescale=pre)
+    try:
+        e = S.svdq_export_weights(w)
+        exp = S.svdq_weights_scale_exponent(w)
+        act = O.act_quant(fmt, Xb, e["inv_lambda"], e["L1"])
+        Y_ora = O.linear(fmt, act, (e["codes"], e["scales"]), e["L2"], None, N, w_exp=exp)
+        kinds = (1, 2, 3) if fmt != "int4" else (0,)
+        Ys = []
+        for kind in kinds:
+            S.svdq_set_gemm_kernel(kind)
+            _, Y = _run_layer(S, w, Xb)
+            ok, info = y_within_tol(bits(Y), Y_ora)
+            assert ok, (kind, info)
+            Ys.append(bits(Y))
+        for y in Ys[1:]:
+            assert np.array_equal(y, Ys[0])
+    finally:
+        S.svdq_set_gemm_kernel(0)
+        w.close()
+

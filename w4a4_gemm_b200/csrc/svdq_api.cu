@@ -491,6 +491,19 @@ int build_l2t2(svdq_weights* w, cudaStream_t st) {
   return SVDQ_OK;
 }
 
+// Scale layouts derived from the weight scales in w->wsf, redone whenever
+// those change (quantization, or a refinement restoring an earlier iterate):
+// FP4 formats: the atoms regrouped per 192-column tile of the pair GEMM.
+int derive_scale_layouts(svdq_weights* w, cudaStream_t st) {
+  if (is_fp4(w->fmt)) {
+    const size_t sf192 = static_cast<size_t>(2 * w->n192) * w->sf_kcols * 512;
+    pair192_scale_atoms_kernel<<<static_cast<unsigned>((sf192 + 255) / 256), 256, 0, st>>>(
+        w->wsf, w->N, w->sf_kcols, w->n192, w->wsf192);
+    SVDQ_CHECK_LAUNCH();
+  }
+  return SVDQ_OK;
+}
+
 int quantize_residual(svdq_weights* w, const float* R, cudaStream_t st) {
   const dim3 blk(128);
   const int e_old = w->w_exp;
@@ -526,12 +539,7 @@ int quantize_residual(svdq_weights* w, const float* R, cudaStream_t st) {
                                                    reinterpret_cast<uint16_t*>(w->wsf), w->wsf32);
   }
   SVDQ_CHECK_LAUNCH();
-  if (is_fp4(w->fmt)) {
-    const size_t sf192 = static_cast<size_t>(2 * w->n192) * w->sf_kcols * 512;
-    pair192_scale_atoms_kernel<<<static_cast<unsigned>((sf192 + 255) / 256), 256, 0, st>>>(
-        w->wsf, w->N, w->sf_kcols, w->n192, w->wsf192);
-    SVDQ_CHECK_LAUNCH();
-  }
+  if (int rc = derive_scale_layouts(w, st)) return rc;
   if (w->w_exp != e_old) return build_l2t2(w, st);   // the tail carries the same 2^e
   return SVDQ_OK;
 }
@@ -712,6 +720,7 @@ int refine_branch(svdq_weights* w, const double* What, float* R, int iters, cuda
   if ((rc = weight_error(w, What, err.as<double>(), &best, st))) return rc;
   w->refine_err0 = best;
   if ((rc = save(true))) return rc;
+  int best_exp = w->w_exp;   // the prescale exponent the kept codes and scales were made with
   for (int t = 0; t < iters; ++t) {
     refine_target_kernel<<<dim3((w->N + 255) / 256, w->K), 256, 0, st>>>(
         What, w->fmt, w->wcodes, w->wsf, w->wsf32, w->K, w->N, w->N_pad, w->sf_kcols,
@@ -725,10 +734,13 @@ int refine_branch(svdq_weights* w, const double* What, float* R, int iters, cuda
     if ((rc = weight_error(w, What, err.as<double>(), &e, st))) return rc;
     if (e < best) {
       best = e;
+      best_exp = w->w_exp;
       if ((rc = save(true))) return rc;
     }
   }
   if ((rc = save(false))) return rc;
+  w->w_exp = best_exp;   // the caller rebuilds [L2^T | L2^T] (refold_l1) with it
+  if ((rc = derive_scale_layouts(w, st))) return rc;
   w->refine_err = best;
   SVDQ_CUDA(cudaStreamSynchronize(st));
   return SVDQ_OK;
