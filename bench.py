@@ -73,7 +73,7 @@ DATASHEET_INT8_TOPS = 4500.0
 NOMINAL_HBM_GBS = 8000.0
 NCU_TRAFFIC = {
     ("gemm_nvfp4_pair_kernel", "c2_qkv/qkv", 4608, "nvfp4"): (63905536, "ab2d6aed3c92a25a"),
-    ("gemm_nvfp4_pair_kernel", "c5_block/fc2", 16384, "nvfp4"): (222889216, "f895356c38d662a7"),
+    ("gemm_nvfp4_pair_kernel", "c5_block/fc2", 16384, "nvfp4"): (221753856, "ab2d6aed3c92a25a"),
     ("quant_act_kernel", "c2_qkv/qkv", 4608, "nvfp4"): (28561408, "97712fa48aaac990"),
     ("quant_act_kernel", "c5_block/fc2", 16384, "nvfp4"): (498574592, "97712fa48aaac990"),
     ("gemm_int4_kernel", "c4_int4_lora/proj", 4608, "int4"): (26690816, "4e6665236c6ea587"),
