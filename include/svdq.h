@@ -232,8 +232,9 @@ SVDQ_API int svdq_set_wait_budget(long long cycles);
 SVDQ_API int svdq_set_quant_split(int S, int C);
 
 /* Tile order of the GEMM for every later svdq_linear (process-wide; a tuning
- * and testing aid).  The persistent GEMM walks its 128-row x 256-column output
- * tiles in groups of `group_m` row blocks: all of a group's tiles, row block
+ * and testing aid).  The persistent GEMM walks its output tiles (128 rows
+ * per row block; 256 or 192 weight columns per column block) in groups of
+ * `group_m` row blocks: all of a group's tiles, row block
  * fastest, before the next group.  Small groups keep fewer activation row
  * blocks and more weight column blocks in flight at once.  group_m above the
  * number of row blocks is clamped to it (one group: the whole of M for each
