@@ -11,6 +11,7 @@
 #include <cusolverDn.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdio>
 #include <cstdlib>
@@ -64,19 +65,25 @@ struct svdq_weights {
 
 namespace {
 
-long long g_budget = -1;
+// Process-wide state is read by the hot calls from any host thread: every
+// lazily set or tunable value is atomic, and one-time set-up is published with
+// a release store after it is complete.
+std::atomic<long long> g_budget{-1};
 std::mutex g_mutex;
 
 long long wait_budget() {
-  if (g_budget < 0) {
+  long long b = g_budget.load(std::memory_order_acquire);
+  if (b < 0) {
     std::lock_guard<std::mutex> lk(g_mutex);
-    if (g_budget < 0) {
+    b = g_budget.load(std::memory_order_relaxed);
+    if (b < 0) {
       const char* env = std::getenv("SVDQ_WAIT_BUDGET_CYCLES");
       long long v = env ? std::atoll(env) : 0;
-      g_budget = v > 0 ? v : (1LL << 31);
+      b = v > 0 ? v : (1LL << 31);
+      g_budget.store(b, std::memory_order_release);
     }
   }
-  return g_budget;
+  return b;
 }
 
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -202,16 +209,16 @@ struct DeviceInfo {
   int pair_clusters = 0;                    // resident clusters of the CTA-pair GEMM (256-column tiles)
   int pair192_clusters = 0;                 // the same with 192-column tiles
   int qclusters[kQuantMaxSplit + 1] = {};   // resident activation-kernel clusters of size C
-  bool attrs_set = false;
+  std::atomic<bool> attrs_set{false};   // set (release) once every field above is filled
 };
 DeviceInfo g_dev[64];
 
 int device_setup(int dev) {
   if (dev < 0 || dev >= 64) return SVDQ_ERR_CUDA;
   DeviceInfo& d = g_dev[dev];
-  if (d.attrs_set) return SVDQ_OK;
+  if (d.attrs_set.load(std::memory_order_acquire)) return SVDQ_OK;
   std::lock_guard<std::mutex> lk(g_mutex);
-  if (d.attrs_set) return SVDQ_OK;
+  if (d.attrs_set.load(std::memory_order_relaxed)) return SVDQ_OK;
   SVDQ_CUDA(cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev));
   uint32_t qmax = 0;
   for (int rp : {0, 16, 32, 64, 128, 192, 256})
@@ -274,7 +281,7 @@ int device_setup(int dev) {
       d.pair192_clusters = n;
     }
   }
-  d.attrs_set = true;
+  d.attrs_set.store(true, std::memory_order_release);
   return SVDQ_OK;
 }
 
@@ -302,14 +309,15 @@ constexpr double kQuantExchangeCycles = 2000.0;
 constexpr double kQuantPerPeerCycles = 1000.0;
 constexpr double kQuantStageCycles = 800.0;
 constexpr double kQuantL1Cycles = 300.0;
-QuantSplit g_forced_split{0, 0};   // svdq_set_quant_split; {0, 0} = automatic
-int g_forced_group_m = 0;          // svdq_set_gemm_raster; 0 = automatic
-int g_forced_gemm_kind = 0;        // svdq_set_gemm_kernel; 0 = automatic, 1 = one CTA, 2 = CTA pairs,
-                                   // 3 = CTA pairs on 192-column tiles
+std::atomic<int> g_forced_split{0};      // svdq_set_quant_split: 16 S + C; 0 = automatic
+std::atomic<int> g_forced_group_m{0};    // svdq_set_gemm_raster; 0 = automatic
+std::atomic<int> g_forced_gemm_kind{0};  // svdq_set_gemm_kernel; 0 = automatic, 1 = one CTA, 2 = CTA pairs,
+                                         // 3 = CTA pairs on 192-column tiles
 
 QuantSplit quant_split_for(int M, int K, int r_pad, const DeviceInfo& d) {
   const int smax = r_pad > 0 ? quant_stack_max(r_pad) : 8;
-  const QuantSplit f = g_forced_split;
+  const int fs = g_forced_split.load(std::memory_order_relaxed);
+  const QuantSplit f{fs / 16, fs % 16};
   if (f.S > 0 && f.S <= smax && f.C <= kQuantTileRows / f.S &&
       f.C <= (K + f.S * kQuantBK - 1) / (f.S * kQuantBK) && d.qclusters[f.C] > 0)
     return f;
@@ -781,30 +789,30 @@ SVDQ_API int svdq_tensor_peak(int fmt, long long steps, void* stream) {
 
 SVDQ_API int svdq_set_gemm_kernel(int kind) {
   if (kind < 0 || kind > 3) return SVDQ_ERR_INVALID_ARG;
-  g_forced_gemm_kind = kind;
+  g_forced_gemm_kind.store(kind, std::memory_order_relaxed);
   return SVDQ_OK;
 }
 
 SVDQ_API int svdq_set_gemm_raster(int group_m) {
   if (group_m < 0) return SVDQ_ERR_INVALID_ARG;
-  g_forced_group_m = group_m;
+  g_forced_group_m.store(group_m, std::memory_order_relaxed);
   return SVDQ_OK;
 }
 
 SVDQ_API int svdq_set_quant_split(int S, int C) {
   auto pow2_le8 = [](int v) { return v == 1 || v == 2 || v == 4 || v == 8; };
   if (S == 0 && C == 0) {
-    g_forced_split = {0, 0};
+    g_forced_split.store(0, std::memory_order_relaxed);
     return SVDQ_OK;
   }
   if (!pow2_le8(S) || !pow2_le8(C)) return SVDQ_ERR_INVALID_ARG;
-  g_forced_split = {S, C};
+  g_forced_split.store(16 * S + C, std::memory_order_relaxed);
   return SVDQ_OK;
 }
 
 SVDQ_API int svdq_set_wait_budget(long long cycles) {
   if (cycles <= 0) return SVDQ_ERR_INVALID_ARG;
-  g_budget = cycles;
+  g_budget.store(cycles, std::memory_order_release);
   return SVDQ_OK;
 }
 
@@ -1084,7 +1092,8 @@ SVDQ_API int svdq_quantize_act(const svdq_weights* w, const void* X, int M, void
 
 // Row blocks per group of the GEMMs' tile order (gemm_tile_coords).
 int gemm_group_m(int m_tiles, int n_tiles, int grid) {
-  if (g_forced_group_m > 0) return std::min(g_forced_group_m, m_tiles);
+  const int g = g_forced_group_m.load(std::memory_order_relaxed);
+  if (g > 0) return std::min(g, m_tiles);
   (void)n_tiles;
   (void)grid;
   return std::min(kGemmGroupM, m_tiles);
@@ -1098,7 +1107,8 @@ int gemm_group_m(int m_tiles, int n_tiles, int grid) {
 // 3-5 % faster at K = 3072 (FLUX QKV, out and fc1 layers) and 6 % slower at
 // K = 12288 (fc2), where a tile's K loop is four times longer.
 int fp4_gemm_kind(const svdq_weights* w, const DeviceInfo& d) {
-  int kind = g_forced_gemm_kind != 0 ? g_forced_gemm_kind : (w->K <= 4096 ? 3 : 2);
+  const int forced = g_forced_gemm_kind.load(std::memory_order_relaxed);
+  int kind = forced != 0 ? forced : (w->K <= 4096 ? 3 : 2);
   if (kind == 3 && d.pair192_clusters <= 0) kind = 2;
   if (kind == 2 && d.pair_clusters <= 0) kind = 1;
   return kind;
@@ -1152,8 +1162,8 @@ SVDQ_API int svdq_linear(const svdq_weights* w, const void* ws, int M, void* Y, 
     p.m_tiles = (M + kPairBM - 1) / kPairBM;
     p.n_tiles = (w->N + bn - 1) / bn;
     p.num_tiles = p.m_tiles * p.n_tiles;
-    p.group_m = g_forced_group_m > 0 ? std::min((g_forced_group_m + 1) / 2, p.m_tiles)
-                                     : std::min(kPairGroupM, p.m_tiles);
+    const int forced_g = g_forced_group_m.load(std::memory_order_relaxed);
+    p.group_m = forced_g > 0 ? std::min((forced_g + 1) / 2, p.m_tiles) : std::min(kPairGroupM, p.m_tiles);
     p.r_tail = 2 * w->r_pad;
     p.sfa = nullptr;
     p.sfb = nullptr;
@@ -1250,7 +1260,7 @@ SVDQ_API int svdq_forward(const svdq_weights* w, const void* X, int M, void* Y, 
 static __device__ __align__(256) uint8_t g_noalloc_workspace[SVDQ_NOALLOC_WORKSPACE_BYTES];
 
 SVDQ_API int svdq_forward_noalloc(const svdq_weights* w, const void* X, int M, void* Y, void* stream) {
-  static void* ws_ptr[64] = {};
+  static std::atomic<void*> ws_ptr[64] = {};
   if (w == nullptr || M < 0) return SVDQ_ERR_INVALID_ARG;
   if (M == 0) return SVDQ_OK;
   const size_t need = act_layout(w, M).total;
@@ -1265,25 +1275,26 @@ SVDQ_API int svdq_forward_noalloc(const svdq_weights* w, const void* X, int M, v
   int rc = current_device(&dev);
   if (rc) return rc;
   if (dev != w->device) return SVDQ_ERR_INVALID_ARG;
-  if (ws_ptr[dev] == nullptr) {
+  void* ws = ws_ptr[dev].load(std::memory_order_acquire);
+  if (ws == nullptr) {
     // first call on this device: look up the array's device address once
     // (host code cannot use the symbol itself as a device pointer)
     std::lock_guard<std::mutex> lk(g_mutex);
-    if (ws_ptr[dev] == nullptr) {
-      void* p = nullptr;
-      const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_workspace);
+    ws = ws_ptr[dev].load(std::memory_order_relaxed);
+    if (ws == nullptr) {
+      const cudaError_t e = cudaGetSymbolAddress(&ws, g_noalloc_workspace);
       if (e != cudaSuccess) {
         std::fprintf(stderr, "svdq_forward_noalloc: cudaGetSymbolAddress failed: %s\n",
                      cudaGetErrorString(e));
         return SVDQ_ERR_CUDA;
       }
-      ws_ptr[dev] = p;
+      ws_ptr[dev].store(ws, std::memory_order_release);
     }
   }
   // The activation kernel rewrites every workspace byte the GEMM reads for this
   // M (codes, scales including the K padding, XL1), so the array's previous
   // contents never leak into the result.
-  return svdq_forward(w, X, M, Y, ws_ptr[dev], stream);
+  return svdq_forward(w, X, M, Y, ws, stream);
 }
 
 SVDQ_API int svdq_export_act(const svdq_weights* w, const void* ws, int M, uint8_t* codes,
