@@ -84,8 +84,6 @@ def lib() -> ctypes.CDLL:
             getattr(_lib, name).argtypes = [P, L, P]
             getattr(_lib, name).restype = None
         _lib.oracle_act_quant.argtypes = [I, I, I, I, P, P, P, P, P, P]
-        _lib.oracle_fold_l1.argtypes = [I, I, P, P, P]
-        _lib.oracle_fold_l1.restype = None
         _lib.oracle_weight_quant.argtypes = [I, I, I, P, P, P]
         _lib.oracle_linear_rows.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, P, I, I, P]
         _lib.oracle_dequant.argtypes = [I, I, I, P, P, P]
@@ -352,20 +350,11 @@ def weight_quant(fmt, R: np.ndarray, exp: int = 0):
     return codes, scales
 
 
-def fold_l1(L1_bits: np.ndarray, inv_lambda: Optional[np.ndarray]) -> np.ndarray:
-    """The down-projection factor with the smoothing folded in:
-    L1s = bf16(diag(inv_lambda) L1), so that X_hat L1 = X L1s (Sec. 4.2)."""
-    L1 = np.ascontiguousarray(L1_bits, dtype=np.uint16)
-    K, r = L1.shape
-    out = np.zeros((K, r), dtype=np.uint16)
-    inv = None if inv_lambda is None else np.ascontiguousarray(inv_lambda, dtype=np.float32)
-    lib().oracle_fold_l1(K, r, _ptr(inv), _ptr(L1), _ptr(out))
-    return out
-
-
 def act_quant(fmt, X_bits: np.ndarray, inv_lambda: Optional[np.ndarray], L1_bits: Optional[np.ndarray]):
     """Smooth and quantize X (M x K bf16) -> codes, scales, and the down-projection
-    XL1 = X fold_l1(L1, inv_lambda) (M x r fp32, fp32 accumulation in increasing k)."""
+    XL1 = X_hat L1 (M x r fp32): x_hat = fp32(x) * inv_lambda, the value the
+    quantizer sees, times the bf16 factor L1, fp32 products and sums in
+    increasing k (Sec. 4.2: X_hat = X diag(lambda)^-1; the branch X_hat L1)."""
     fmt = _FMT[fmt]
     X_bits = np.ascontiguousarray(X_bits, dtype=np.uint16)
     M, K = X_bits.shape
@@ -376,16 +365,16 @@ def act_quant(fmt, X_bits: np.ndarray, inv_lambda: Optional[np.ndarray], L1_bits
         codes = np.zeros((M, K), dtype=np.int8)
         scales = np.zeros(M, dtype=np.float32)
         XL1 = np.zeros((M, r), dtype=np.float32)
-        L1s = None if L1_bits is None else fold_l1(L1_bits, inv)
-        assert lib().oracle_act_quant_w8(M, K, r, _ptr(X_bits), _ptr(inv), _ptr(L1s), _ptr(codes),
+        L1 = None if L1_bits is None else np.ascontiguousarray(L1_bits, dtype=np.uint16)
+        assert lib().oracle_act_quant_w8(M, K, r, _ptr(X_bits), _ptr(inv), _ptr(L1), _ptr(codes),
                                          _ptr(scales), _ptr(XL1)) == 0
         return codes, scales, XL1
     g = GROUP[fmt]
     codes = np.zeros((M, K // 2), dtype=np.uint8)
     scales = np.zeros((M, K // g), dtype=np.uint16 if fmt == INT4 else np.uint8)
     XL1 = np.zeros((M, r), dtype=np.float32)
-    L1s = None if L1_bits is None else fold_l1(L1_bits, inv)
-    rc = lib().oracle_act_quant(fmt, M, K, r, _ptr(X_bits), _ptr(inv), _ptr(L1s),
+    L1 = None if L1_bits is None else np.ascontiguousarray(L1_bits, dtype=np.uint16)
+    rc = lib().oracle_act_quant(fmt, M, K, r, _ptr(X_bits), _ptr(inv), _ptr(L1),
                                 _ptr(codes), _ptr(scales), _ptr(XL1))
     assert rc == 0
     return codes, scales, XL1

@@ -29,10 +29,10 @@
  *   - codes round to nearest, ties to the even code; a zero scale gives zero
  *     codes; the sign bit of an E2M1 code is the sign of X * RN(1/s);
  *   - INT4 codes are clamped to [-7, 7] (symmetric, q_max = 7);
- *   - the down-projection folds the smoothing into its factor,
- *     X_hat L1 = X (diag(lambda)^-1 L1), with the folded factor rounded to
- *     bf16 once; X itself is already 16-bit; the branch's intermediate X_hat L1
- *     stays at fp32 accumulator precision (only the factors are 16-bit);
+ *   - the down-projection is X_hat L1 itself: x_hat = fp32(x) * inv_lambda
+ *     (the value the quantizer sees) times the bf16 factor L1, accumulated in
+ *     fp32 in increasing k; the branch's intermediate X_hat L1 stays at fp32
+ *     accumulator precision (only the factors L1, L2 are 16-bit);
  *   - the GEMM accumulates in fp32: exact per-group integer/E2M1 partial sums,
  *     scaled by s_x * s_w, summed over groups in increasing order, then the
  *     low-rank term sum_j XL1[m,j] L2[j,n] in increasing j, then the bias.
@@ -262,18 +262,18 @@ static void quantize_row(int fmt, const float *v, int K, uint8_t *codes_row, voi
 }
 
 /* ------------------------------------------------------------------------- */
-/* Activation side (the fused "quantize + down-projection" of Sec. 4.3).     */
-/*   x_hat[m,k] = fp32(x[m,k]) * inv_lambda[k]                                */
+/* Activation side (the fused "quantize + down-projection" of Sec. 4.3; the  */
+/* smoothing X_hat = X diag(lambda)^-1 and the branch X_hat L1 of Sec. 4.2). */
+/*   x_hat[m,k] = fp32(x[m,k]) * inv_lambda[k]        (one fp32 rounding)     */
 /*   codes/scales = Q(x_hat) per group                                         */
-/*   XL1[m,j]   = sum_k fp32(x[m,k]) * L1s[k,j], fp32, increasing k (kept fp32)*/
-/* where L1s = bf16(diag(inv_lambda) L1) is the down-projection factor with  */
-/* the smoothing folded in (X_hat L1 = X diag(lambda)^-1 L1), computed by     */
-/* oracle_fold_l1.  X: M x K bf16; L1s: K x r bf16 (row-major); codes:         */
-/* M x K/2 bytes (element 2i in the low nibble); scales: M x K/g (uint8 E4M3  */
-/* or uint16 fp16); XL1: M x r fp32.  inv_lambda may be NULL (lambda = 1).     */
+/*   XL1[m,j]   = sum_k x_hat[m,k] * L1[k,j], fp32 products and sums in       */
+/*                increasing k (kept fp32)                                     */
+/* X: M x K bf16; L1: K x r bf16 (row-major); codes: M x K/2 bytes (element  */
+/* 2i in the low nibble); scales: M x K/g (uint8 E4M3 or uint16 fp16); XL1:   */
+/* M x r fp32.  inv_lambda may be NULL (lambda = 1).                           */
 /* ------------------------------------------------------------------------- */
 int oracle_act_quant(int fmt, int M, int K, int r, const uint16_t *X, const float *inv_lambda,
-                     const uint16_t *L1s, uint8_t *codes, void *scales, float *XL1) {
+                     const uint16_t *L1, uint8_t *codes, void *scales, float *XL1) {
     int g = fmt_group(fmt);
     if (K % g) return 1;
     int ssz = fmt_scale_bytes(fmt);
@@ -293,25 +293,12 @@ int oracle_act_quant(int fmt, int M, int K, int r, const uint16_t *X, const floa
             for (int j = 0; j < r; ++j) {
                 float acc = 0.0f;
                 for (int k = 0; k < K; ++k)
-                    acc += xf[k] * oracle_bf16_decode(L1s[(long)k * r + j]);
+                    acc += xh[k] * oracle_bf16_decode(L1[(long)k * r + j]);
                 XL1[(long)m * r + j] = acc;
             }
         }
     }
     return 0;
-}
-
-/* The smoothing folded into the down-projection factor:
- * L1s[k,j] = bf16( inv_lambda[k] * L1[k,j] ), the product exact in double and
- * rounded once (nearest, ties to even).  L1: K x r bf16; inv_lambda may be
- * NULL (then L1s = L1). */
-void oracle_fold_l1(int K, int r, const float *inv_lambda, const uint16_t *L1, uint16_t *L1s) {
-    for (long k = 0; k < K; ++k)
-        for (int j = 0; j < r; ++j) {
-            double v = (double)oracle_bf16_decode(L1[k * r + j]);
-            if (inv_lambda) v *= (double)inv_lambda[k];
-            L1s[k * r + j] = oracle_bf16_round(v);
-        }
 }
 
 /* ------------------------------------------------------------------------- */
@@ -442,9 +429,9 @@ static void quant_int8(const float *v, long n, long stride, int8_t *codes, float
     }
 }
 
-/* Activations: codes M x K int8, scales M fp32, XL1 M x r fp32 (as above). */
+/* Activations: codes M x K int8, scales M fp32, XL1 M x r fp32 (X_hat L1 as above). */
 int oracle_act_quant_w8(int M, int K, int r, const uint16_t *X, const float *inv_lambda,
-                        const uint16_t *L1s, int8_t *codes, float *scales, float *XL1) {
+                        const uint16_t *L1, int8_t *codes, float *scales, float *XL1) {
 #pragma omp parallel
     {
         float *xh = (float *)__builtin_alloca(sizeof(float) * (size_t)K);
@@ -460,7 +447,7 @@ int oracle_act_quant_w8(int M, int K, int r, const uint16_t *X, const float *inv
             for (int j = 0; j < r; ++j) {
                 float acc = 0.0f;
                 for (int k = 0; k < K; ++k)
-                    acc += xf[k] * oracle_bf16_decode(L1s[(long)k * r + j]);
+                    acc += xh[k] * oracle_bf16_decode(L1[(long)k * r + j]);
                 XL1[(long)m * r + j] = acc;
             }
         }

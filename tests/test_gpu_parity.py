@@ -12,7 +12,7 @@ import torch
 
 import oracle as O
 import workloads as WL
-from gpu_common import (bits, close_f32, load_from_oracle, oracle_layer, require_gpu, svdq,
+from gpu_common import (bits, xl1_within_bound, load_from_oracle, oracle_layer, require_gpu, svdq,
                         to_dev_bits, to_dev_f32, y_within_tol)
 
 pytestmark = pytest.mark.gpu
@@ -155,7 +155,7 @@ def test_layer_parity_small(S, M, K, N, rank, fmt, bias):
     assert np.array_equal(scales, ref["act"][1]), "activation scales differ"
     assert np.array_equal(codes, ref["act"][0]), "activation codes differ"
     if rank:
-        ok, info = close_f32(xl1, ref["act"][2])
+        ok, info = xl1_within_bound(xl1, ref["act"][2], WL.bf16_bits(data["X"]), prep["inv_lambda"], prep["L1"])
         assert ok, ("XL1", info)
     ok, info = y_within_tol(bits(Y), ref["Y"])
     assert ok, ("Y", info)
@@ -182,7 +182,8 @@ def test_forced_launch_shapes(S, M, K, N, rank, fmt):
                 codes, scales, xl1 = S.svdq_export_act(w, ws, M)
                 assert np.array_equal(scales, ref["act"][1]), (st, cl, "scales")
                 assert np.array_equal(codes, ref["act"][0]), (st, cl, "codes")
-                ok, info = close_f32(xl1, ref["act"][2])
+                ok, info = xl1_within_bound(xl1, ref["act"][2], WL.bf16_bits(data["X"]),
+                                            ref["prep"]["inv_lambda"], ref["prep"]["L1"])
                 assert ok, (st, cl, "XL1", info)
                 ok, info = y_within_tol(bits(Y), ref["Y"])
                 assert ok, (st, cl, "Y", info)

@@ -218,6 +218,14 @@ def test_hand_worked_tiny_layer(golden):
     assert act[2][0, 0] == 3.0
     Y = O.bf16_decode(O.linear("nvfp4", act, (cw, sw), L2, bias, N))
     assert np.array_equal(Y[0], vec("y_full").astype(np.float32))
+    # smooth: 1/lambda = 0.75 on channel 0 reaches both the quantizer and the branch
+    act = O.act_quant("nvfp4", Xb, vec("inv_l").astype(np.float32), L1)
+    c = hexv("xs_codes")
+    assert np.array_equal(act[0][0] & 0xF, c[0::2]) and np.array_equal(act[0][0] >> 4, c[1::2])
+    assert act[1][0, 0] == hexv("xs_scale")[0]
+    assert act[2][0, 0] == vec("xs_xl1")[0]
+    Y = O.bf16_decode(O.linear("nvfp4", act, (cw, sw), L2, bias, N))
+    assert np.array_equal(Y[0], vec("y_smooth").astype(np.float32))
 
 
 def test_row_subset_matches_full():
