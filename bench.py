@@ -6,13 +6,15 @@ the fused activation kernel (smoothing + quantize + down-projection) and the
 fused 4-bit GEMM (+ up-projection + bias), both through the C ABI.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--config c2_qkv] [--layer qkv] [--M 4608]
+                    [--config c5_block] [--layer fc2] [--M 16384]
 
-Default workload: the FLUX attention QKV projection, M = 4608 tokens
-(4096 image + 512 text), K = 3072 -> N = 9216, rank 32, NVFP4.  The metric is
-the effective throughput 2*M*K*N / (layer time), in TFLOP/s; the line also
-carries us/layer, the per-kernel times, the GEMM's roofline fraction against
-the FP4 tensor peak and the activation kernel's against HBM bandwidth.
+Default workload: the largest FLUX-shaped GEMM of the workloads, the DiT
+block's MLP fc2 layer at M = 16384 tokens, K = 12288 -> N = 3072, rank 32,
+NVFP4 (bias).  The metric is the effective throughput 2*M*K*N / (layer time),
+in TFLOP/s; the line also carries us/layer, the per-kernel times, the GEMM's
+roofline fraction against the FP4 tensor peak and the activation kernel's
+against HBM bandwidth.  Other layers: --config / --layer / --M (e.g.
+--config c2_qkv for the attention QKV projection at M = 4608).
 
 Between timed steps a 512 MiB buffer is rewritten to flush the 126 MB L2.
 Under torchrun every rank runs its own batch of the same layer (token-parallel
@@ -179,7 +181,10 @@ DTYPE = {"nvfp4": "e2m1xe2m1+bf16 (fp32 acc)", "fp4g32": "e2m1xe2m1+bf16 (fp32 a
 
 def layer_inputs(args):
     import dataclasses
-    spec = WL.layer_spec(args.config, args.layer)
+    layer = args.layer
+    if layer is None and args.config == "c5_block":
+        layer = "fc2"      # the block's largest GEMM (K = 12288 -> N = 3072)
+    spec = WL.layer_spec(args.config, layer)
     if getattr(args, "fmt", None):
         spec = dataclasses.replace(spec, fmt=args.fmt)
     if getattr(args, "rank", None) is not None:
@@ -563,9 +568,11 @@ def _oracle_setup(spec, M, rows):
     X = WL.make_activations(spec, M)
     Xb = WL.bf16_bits(X)
     xm = O.calib_absmax(Xb)
+    # the top-r factors from the Gram matrix (the same subspace as a full SVD,
+    # which takes minutes at FLUX sizes); preparation is not timed
     prep = O.prepare(WL.bf16_bits(W), xm, spec.rank,
                      WL.bf16_bits(A) if A is not None else None,
-                     WL.bf16_bits(B) if B is not None else None)
+                     WL.bf16_bits(B) if B is not None else None, svd="gram")
     wq = O.weight_quant(spec.fmt, prep["R"])
     sample = np.ascontiguousarray(Xb[:rows])
     return O, prep, wq, sample, (WL.bf16_bits(bias) if bias is not None else None)
@@ -676,7 +683,16 @@ def run_block(args):
         torch.distributed.destroy_process_group()
 
 
+def cpu_rows(spec, M, rows):
+    """Rows of the oracle's timed sample: as given, else about 4 GFLOP of the
+    layer (2 K N per row), at least 8 and at most M."""
+    if rows is None:
+        rows = max(8, int(4e9 // (2.0 * spec.K * spec.N)))
+    return max(1, min(M, rows))
+
+
 def cpu_baseline(spec, M, rows):
+    rows = cpu_rows(spec, M, rows)
     O, prep, wq, sample, bias = _oracle_setup(spec, M, rows)
     t0 = time.perf_counter()
     _oracle_step(O, spec, prep, wq, sample, bias)
@@ -693,7 +709,7 @@ def run_reference(args):
     if rank != 0:
         return
     spec, M = layer_inputs(args)
-    rows = args.cpu_rows
+    rows = cpu_rows(spec, M, args.cpu_rows)
     O, prep, wq, sample, bias = _oracle_setup(spec, M, rows)
     for _ in range(args.warmup):
         _oracle_step(O, spec, prep, wq, sample, bias)
@@ -723,7 +739,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", default="c2_qkv", choices=sorted(WL.CONFIGS))
+    ap.add_argument("--config", default="c5_block", choices=sorted(WL.CONFIGS))
     ap.add_argument("--layer", default=None,
                     help="a layer of the config, or 'all': the config's layers back to back as one step")
     ap.add_argument("--M", type=int, default=None)
@@ -731,7 +747,8 @@ def main():
                     help="override the workload's format")
     ap.add_argument("--rank", type=int, default=None,
                     help="override the workload's low-rank branch rank (the paper pairs W8A8 with 16)")
-    ap.add_argument("--cpu-rows", type=int, default=64)
+    ap.add_argument("--cpu-rows", type=int, default=None,
+                    help="token rows of the oracle's sample (default: about 4 GFLOP of the layer, >= 8 rows)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--rank-sweep", type=lambda v: [int(x) for x in v.split(",")], default=None,
                     help="also time the layer at these ranks, e.g. 16,32,48,64")

@@ -214,8 +214,13 @@ SVDQ_API int svdq_export_weights(const svdq_weights* w, uint8_t* codes, void* sc
  * Returns the word (>= 0) or -SVDQ_ERR_CUDA.  Synchronizes the device. */
 SVDQ_API int svdq_get_error(void);
 
-/* Clock-cycle budget of every bounded device wait (default 2^31, about one
- * second; the environment variable SVDQ_WAIT_BUDGET_CYCLES also sets it). */
+/* Clock-cycle budget of every bounded device wait of the hot pipelines
+ * (default 2^31, about one second; the environment variable
+ * SVDQ_WAIT_BUDGET_CYCLES also sets it).  A wait that runs out sets the error
+ * word above and stops its CTA's pipeline; the waits with which a CTA then
+ * drains what it already issued (copies landing, MMAs retiring, before shared
+ * memory and TMEM are released) get max(budget, 2^33) cycles, since issued
+ * work always finishes.  cycles <= 0: SVDQ_ERR_INVALID_ARG. */
 SVDQ_API int svdq_set_wait_budget(long long cycles);
 
 /* Launch shape of the activation kernel for every later svdq_quantize_act

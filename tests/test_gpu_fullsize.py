@@ -8,8 +8,9 @@ the full SVD, which would take minutes at these sizes).  Checked:
   * weight codes and scales: every value, bit-exact;
   * activation codes and scales: every row, bit-exact;
   * X_hat L1: every row, within 2^-14 sum_k |x_hat_k| |L1_kj| (gpu_common);
-  * Y: sampled rows (first and last 32 rows and 32 seeded random rows, all N
-    columns), within |dy| <= 2^-7 |y| + 1e-3 rms(y).
+  * Y: every row up to M = 512; above, the first and last row of every
+    128-row block, a seeded row in each of its middle 32-row slices and 32
+    seeded rows anywhere (all N columns), within |dy| <= 2^-7 |y| + 1e-3 rms(y).
 """
 import dataclasses
 
@@ -62,10 +63,22 @@ def _prepared(spec):
 
 
 def _sample_rows(M, seed):
+    """Rows whose Y is checked: all of them up to 512; above, in every 128-row
+    block its first and last row and one seeded row in each of its two middle
+    32-row slices -- so every (row block, epilogue warp quarter) position of
+    every output tile is checked -- plus 32 seeded rows anywhere."""
+    if M <= 512:
+        return np.arange(M, dtype=np.int32)
     rng = np.random.default_rng(seed)
-    k = min(32, M)
-    rows = np.concatenate([np.arange(k), np.arange(M - k, M), rng.integers(0, M, size=32)])
-    return np.unique(rows).astype(np.int32)
+    rows = [rng.integers(0, M, size=32)]
+    for b in range(0, M, 128):
+        last = min(b + 127, M - 1)
+        rows.append(np.array([b, last]))
+        for q in (1, 2):
+            lo = b + 32 * q
+            if lo <= last:
+                rows.append(rng.integers(lo, min(lo + 32, last + 1), size=1))
+    return np.unique(np.concatenate(rows)).astype(np.int32)
 
 
 def _case_id(case):

@@ -7,7 +7,10 @@ the library keeps the activation workspace in a fixed device array.  These
 tests call the entry point through the C ABI and check its output against
 svdq_forward with a caller workspace, on two calls in a row with different
 inputs (the array keeps the previous call's bytes), for both formats, and
-that a batch too large for the array is refused before anything runs.
+that a batch too large for the array is refused before anything runs.  The
+kernels are deterministic and only the workspace address differs, so the
+outputs must be bit-identical; a second layer whose K and M padding differ
+from the first call's checks that no leftover byte of the array reaches Y.
 
 This file runs last (pytest collects it after every other test file).
 """
@@ -48,8 +51,35 @@ def test_forward_noalloc_matches_forward_on_two_calls(fmt, rank):
         assert _noalloc(S, w, X, Y) == 0
         torch.cuda.synchronize()
         assert S.svdq_get_error() == 0
-        ok, info = y_within_tol(bits(Y), bits(ref))
-        assert ok, info
+        assert torch.equal(Y, ref), y_within_tol(bits(Y), bits(ref))[1]
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4"])
+def test_forward_noalloc_after_a_call_with_other_padding(fmt):
+    """A 1000 x 1024 call leaves the array full of bytes; then a layer with
+    K = 320 (scale atoms padded past K) at M = 130 (a ragged last row block)
+    must still equal svdq_forward bit for bit."""
+    require_gpu()
+    S = svdq()
+    big = WL.make_small(1000, 1024, 512, rank=32, fmt=fmt, seed=41)
+    wb = load_from_oracle(S, fmt, O.prepare(WL.bf16_bits(big["W"]), O.calib_absmax(WL.bf16_bits(big["X"])), 32))
+    small = WL.make_small(130, 320, 272, rank=48, fmt=fmt, bias=True, seed=42)
+    ws = load_from_oracle(S, fmt, O.prepare(WL.bf16_bits(small["W"]), O.calib_absmax(WL.bf16_bits(small["X"])), 48),
+                          WL.bf16_bits(small["bias"]))
+    try:
+        Xb = big["X"].cuda()
+        Yb = torch.empty(1000, 512, dtype=torch.bfloat16, device="cuda")
+        assert _noalloc(S, wb, Xb, Yb) == 0
+        Xs = small["X"].cuda()
+        ref = S.svdq_forward(ws, Xs)
+        Ys = torch.full((130, 272), float("nan"), dtype=torch.bfloat16, device="cuda")
+        assert _noalloc(S, ws, Xs, Ys) == 0
+        torch.cuda.synchronize()
+        assert S.svdq_get_error() == 0
+        assert torch.equal(Ys, ref), y_within_tol(bits(Ys), bits(ref))[1]
+    finally:
+        wb.close()
+        ws.close()
 
 
 def test_forward_noalloc_rejects_batches_beyond_the_array():

@@ -238,10 +238,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
       }
-      if (*abort_flag) {
-        for (int i = (it > STAGES ? it - STAGES : 0); i < it; ++i)
-          mbar_wait(&full[i % STAGES], (i / STAGES) & 1, p.budget, nullptr);
-      }
+      // never leave while a copy into this CTA's shared memory is still in flight
+      // (whether or not a wait ran out, and in whichever role)
+      for (int i = (it > STAGES ? it - STAGES : 0); i < it; ++i)
+        mbar_wait(&full[i % STAGES], (i / STAGES) & 1, drain_budget(p.budget), nullptr);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
@@ -345,7 +345,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   if (warp == 1) {
     // every MMA issued by this CTA has retired before its TMEM is released
-    mbar_wait(mma_done, 0, p.budget, nullptr);
+    mbar_wait(mma_done, 0, drain_budget(p.budget), nullptr);
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem_base, kGemmTmemCols);

@@ -146,6 +146,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* mma_done = acc_empty + ACC;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  // rank 0's copy: stages whose loads each CTA issued (read by rank 0's drain)
+  uint32_t* issued = reinterpret_cast<uint32_t*>(tmem_holder + 2);
 
   const uint32_t warp = warp_id();
   const uint32_t lane = lane_id();
@@ -230,10 +232,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
       }
-      if (*abort_flag && rank == 0) {
-        for (int i = (it > STAGES ? it - STAGES : 0); i < it; ++i)
-          mbar_wait(&full[i % STAGES], (i / STAGES) & 1, p.budget, nullptr);
-      }
+      // publish, in rank 0's shared memory, how many stages this CTA filled
+      st_shared_cluster_u32(map_shared_rank(smem_u32(issued + rank), 0), static_cast<uint32_t>(it));
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer (rank 0)
@@ -336,10 +336,32 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   __syncwarp();
   tc_fence_before();
+  cluster_sync();   // both producers have published their counts
+  if (rank == 0 && threadIdx.x == 0) {
+    // Drain: every load either CTA issued counts on rank 0's barriers and
+    // writes into that CTA's shared memory, so none may still be in flight
+    // when the pair leaves.  After a wait ran out the two producers may have
+    // stopped at different stages: a stage only rank 1 filled is armed here
+    // for rank 1's share, and in a stage only rank 0 filled rank 1's share is
+    // completed without a copy.  Stages older than the last STAGES were all
+    // consumed by the MMAs (a producer refills a buffer only after that).
+    const int c0 = static_cast<int>(issued[0]), c1 = static_cast<int>(issued[1]);
+    const int cmax = c0 > c1 ? c0 : c1;
+    const uint32_t lr_share = (128 + Sh::kBH) * static_cast<uint32_t>(lr_cols) * 2;
+    for (int i = (cmax > STAGES ? cmax - STAGES : 0); i < cmax; ++i) {
+      uint64_t* bar = &full[i % STAGES];
+      const uint32_t share = (i % steps_per_tile) < p.kt_total ? Sh::kStageBytes : lr_share;
+      if (i >= c0)
+        mbar_arrive_expect_tx(bar, share);
+      else if (i >= c1)
+        mbar_complete_tx(bar, share);
+      if (!mbar_wait(bar, (i / STAGES) & 1, drain_budget(p.budget), nullptr)) raise_error(kErrWaitGemm);
+    }
+  }
   __syncthreads();
   if (warp == 1) {
     // every MMA of the pair has retired before its TMEM is released
-    mbar_wait(mma_done, 0, p.budget, nullptr);
+    mbar_wait(mma_done, 0, drain_budget(p.budget), nullptr);
     __syncwarp();
     tc_fence_after();
     tmem_dealloc_pair(tmem_base, kGemmTmemCols);

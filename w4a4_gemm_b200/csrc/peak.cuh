@@ -82,7 +82,8 @@ __global__ void __launch_bounds__(kPeakThreads, 1)
   }
   __syncwarp();
   if (warp == 0) {
-    if (!warp_wait(done, 0, budget, nullptr) && lane_id() == 0) raise_error(kErrWaitOther);
+    // the MMAs run for the whole measurement: wait for them before freeing TMEM
+    if (!warp_wait(done, 0, drain_budget(budget), nullptr) && lane_id() == 0) raise_error(kErrWaitOther);
   }
   tc_fence_before();
   __syncthreads();

@@ -196,17 +196,24 @@ __global__ void lora_l1_kernel(const __nv_bfloat16* __restrict__ A, const float*
   l1t[static_cast<size_t>(col0 + j) * K + k] = bf16_from_f64(v);
 }
 
-// The smoothing folded into the down-projection factor:
-// l1st[j][k] = bf16(inv_lambda[k] * l1t[j][k]) (exact product, one rounding),
-// so that X_hat L1 = X (diag(lambda)^-1 L1) reads X as it is.
+// The smoothing folded into the down-projection factor, carried as a pair of
+// bf16 terms so that it keeps 16 bits more than one bf16 rounding would:
+//   p = inv_lambda[k] * l1t[j][k]           (exact in fp64: 24 x 8 bits)
+//   l1st[j][k]         = hi = bf16(p)
+//   l1st[r_pad + j][k] = lo = bf16(p - hi)  (p - hi exact in fp64)
+// |hi + lo - p| <= 2^-8 |p - hi| <= 2^-16 |p|.  The activation kernel computes
+// X hi + X lo = X (diag(lambda)^-1 L1) = X_hat L1 (SVDQuant Sec. 4.2) with the
+// X tile as loaded; every product of two bf16 values is exact in fp32.
 __global__ void fold_l1_kernel(const __nv_bfloat16* __restrict__ l1t, const float* __restrict__ inv,
-                               int K, int r, __nv_bfloat16* __restrict__ l1st) {
+                               int K, int r, int r_pad, __nv_bfloat16* __restrict__ l1st) {
   const int k = blockIdx.x * blockDim.x + threadIdx.x;
   const int j = blockIdx.y;
   if (k >= K || j >= r) return;
   const double v = static_cast<double>(inv[k]) *
                    static_cast<double>(__bfloat162float(l1t[static_cast<size_t>(j) * K + k]));
-  l1st[static_cast<size_t>(j) * K + k] = bf16_from_f64(v);
+  const __nv_bfloat16 hi = bf16_from_f64(v);
+  l1st[static_cast<size_t>(j) * K + k] = hi;
+  l1st[static_cast<size_t>(r_pad + j) * K + k] = bf16_from_f64(v - static_cast<double>(__bfloat162float(hi)));
 }
 
 // The up-projection operand of the GEMM's tail: [L2^T | L2^T] (N x 2 r_pad), so
@@ -291,8 +298,7 @@ __global__ void pair192_scale_atoms_kernel(const uint8_t* __restrict__ sf, int N
 }
 
 __global__ void quant_weight_int4_kernel(const float* __restrict__ R, int K, int N, int N_pad,
-                                         int8_t* __restrict__ codes, uint16_t* __restrict__ sf,
-                                         float* __restrict__ sf32) {
+                                         uint8_t* __restrict__ codes, uint16_t* __restrict__ sf) {
   const int n = blockIdx.x * blockDim.x + threadIdx.x;
   const int g = blockIdx.y;
   if (n >= N) return;
@@ -301,13 +307,38 @@ __global__ void quant_weight_int4_kernel(const float* __restrict__ R, int K, int
   const uint16_t sh = int4_scale_bits(amax);
   const float sd = __half2float(__ushort_as_half(sh));
   const float inv = sd == 0.f ? 0.f : __frcp_rn(sd);
-  for (int i = 0; i < 64; ++i) {
-    const float v = R[static_cast<size_t>(64 * g + i) * N + n];
-    codes[static_cast<size_t>(n) * K + 64 * g + i] =
-        static_cast<int8_t>(sd == 0.f ? 0 : int4_code(v, inv));
+  // 64 codes -> 32 bytes, element 2i in the low nibble (4-bit two's complement)
+  uint32_t wd[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    uint32_t w = 0;
+#pragma unroll
+    for (int b = 0; b < 8; ++b) {
+      const float v = R[static_cast<size_t>(64 * g + 8 * e + b) * N + n];
+      const uint32_t c = sd == 0.f ? 0u : static_cast<uint32_t>(int4_code(v, inv)) & 0xFu;
+      w |= c << (4 * b);
+    }
+    wd[e] = w;
   }
+  uint4* dst = reinterpret_cast<uint4*>(codes + static_cast<size_t>(n) * (K / 2) + 32 * g);
+  dst[0] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+  dst[1] = make_uint4(wd[4], wd[5], wd[6], wd[7]);
   sf[static_cast<size_t>(g) * N_pad + n] = sh;
-  sf32[static_cast<size_t>(g) * N_pad + n] = sd;   // exact: every fp16 value is an fp32 value
+}
+
+// The INT4 GEMM's per-column constants, derived from the fp16 weight scales:
+// for the column pair (2i, 2i + 1) of group g one float4
+//   (s_w[2i] / 16, s_w[2i+1] / 16, -1.5 * 2^19 * s_w[2i], -1.5 * 2^19 * s_w[2i+1]),
+// all exact (an fp16 value times a power of two, or times 3 * 2^18).  With the
+// partial read back as v = 1.5 * 2^23 + 16 P, fma(v, s_w / 16, c) = P s_w.
+__global__ void int4_column_consts_kernel(const uint16_t* __restrict__ sf, int groups, int N_pad,
+                                          float4* __restrict__ swc) {
+  const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;   // (g, column pair)
+  if (i >= static_cast<size_t>(groups) * (N_pad / 2)) return;
+  const size_t g = i / (N_pad / 2), c2 = i % (N_pad / 2);
+  const float s0 = __half2float(__ushort_as_half(sf[g * N_pad + 2 * c2]));
+  const float s1 = __half2float(__ushort_as_half(sf[g * N_pad + 2 * c2 + 1]));
+  swc[i] = make_float4(s0 * 0.0625f, s1 * 0.0625f, s0 * -786432.0f, s1 * -786432.0f);
 }
 
 // FP4 g32: one E4M3 scale per 32 values of K, stored in both 16-value slots of
@@ -345,12 +376,13 @@ __global__ void quant_weight_fp4g32_kernel(const float* __restrict__ R, int K, i
 // lookup serves it too).
 // post: 2^-e of the weight prescale (FP4 formats; 1 without it).
 __device__ __forceinline__ double deq_weight(int fmt, const uint8_t* __restrict__ codes,
-                                             const uint8_t* __restrict__ sf,
-                                             const float* __restrict__ sf32, int K, int N_pad,
+                                             const uint8_t* __restrict__ sf, int K, int N_pad,
                                              int sf_kcols, double post, int k, int n) {
-  if (fmt == 1) {
-    const int8_t q = reinterpret_cast<const int8_t*>(codes)[static_cast<size_t>(n) * K + k];
-    return static_cast<double>(q) * static_cast<double>(sf32[static_cast<size_t>(k / 64) * N_pad + n]);
+  if (fmt == 1) {   // packed 4-bit two's complement, fp16 scale per 64
+    const uint8_t b = codes[static_cast<size_t>(n) * (K / 2) + k / 2];
+    const int c = static_cast<int>((k & 1) ? (b >> 4) : (b & 15u));
+    const uint16_t sh = reinterpret_cast<const uint16_t*>(sf)[static_cast<size_t>(k / 64) * N_pad + n];
+    return static_cast<double>(c >= 8 ? c - 16 : c) * static_cast<double>(__half2float(__ushort_as_half(sh)));
   }
   if (fmt == 3) {   // W8A8: one fp32 scale per output channel
     const int8_t q = reinterpret_cast<const int8_t*>(codes)[static_cast<size_t>(n) * K + k];
@@ -367,13 +399,13 @@ __device__ __forceinline__ double deq_weight(int fmt, const uint8_t* __restrict_
 // E = W_hat - deq(Q(R)), fp64 K x N.
 __global__ void refine_target_kernel(const double* __restrict__ What, int fmt,
                                      const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sf,
-                                     const float* __restrict__ sf32, int K, int N, int N_pad,
+                                     int K, int N, int N_pad,
                                      int sf_kcols, double post, double* __restrict__ E) {
   const int n = blockIdx.x * blockDim.x + threadIdx.x;
   const int k = blockIdx.y;
   if (n >= N) return;
   const size_t i = static_cast<size_t>(k) * N + n;
-  E[i] = What[i] - deq_weight(fmt, codes, sf, sf32, K, N_pad, sf_kcols, post, k, n);
+  E[i] = What[i] - deq_weight(fmt, codes, sf, K, N_pad, sf_kcols, post, k, n);
 }
 
 // *sum += sum over the block's elements of (W_hat - L1 L2 - deq(Q(R)))^2, fp64.
@@ -381,7 +413,7 @@ __global__ void refine_error_kernel(const double* __restrict__ What,
                                     const __nv_bfloat16* __restrict__ l1t,
                                     const __nv_bfloat16* __restrict__ l2t, int r, int r_pad, int fmt,
                                     const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sf,
-                                    const float* __restrict__ sf32, int K, int N, int N_pad,
+                                    int K, int N, int N_pad,
                                     int sf_kcols, double post, double* __restrict__ sum) {
   __shared__ double part[8];
   const int n = blockIdx.x * blockDim.x + threadIdx.x;
@@ -392,7 +424,7 @@ __global__ void refine_error_kernel(const double* __restrict__ What,
     for (int j = 0; j < r; ++j)
       acc -= static_cast<double>(__bfloat162float(l1t[static_cast<size_t>(j) * K + k])) *
              static_cast<double>(__bfloat162float(l2t[static_cast<size_t>(n) * r_pad + j]));
-    acc -= deq_weight(fmt, codes, sf, sf32, K, N_pad, sf_kcols, post, k, n);
+    acc -= deq_weight(fmt, codes, sf, K, N_pad, sf_kcols, post, k, n);
     d2 = acc * acc;
   }
   for (int o = 16; o > 0; o >>= 1) d2 += __shfl_xor_sync(0xffffffffu, d2, o);

@@ -5,13 +5,18 @@
 // its input with the quantizer, so both are computed from one read of X.  The
 // smoothing is folded into the factor, X_hat L1 = X (diag(lambda)^-1 L1), so
 // the tensor core reads the TMA-loaded X tile as it is, in parallel with the
-// quantizer warps.
+// quantizer warps.  One bf16 rounding of the folded factor (2^-8 per term)
+// would move Y by several times the output tolerance where the branch and the
+// 4-bit part cancel, so the factor is carried as a bf16 pair L1s = hi + lo
+// (2^-16 per term) and each stage issues the MMAs twice, X hi then X lo, into
+// the same accumulator (bf16 x bf16 products are exact in fp32).
 //
 // A cluster of C CTAs owns BM = 128 / S token rows; its CTA of rank t takes
 // the t-th of C consecutive K ranges.  Each pipeline stage holds S consecutive
 // 64-wide K sub-tiles of those rows stacked on top of each other as the
 // 128-row A operand of one tcgen05 MMA, and the S matching 64 x r_pad slices
-// of the folded factor L1s side by side as its N = S * r_pad wide B operand:
+// of the folded factor L1s side by side as its N = S * r_pad wide B operand
+// (once for hi, once for lo):
 //   D[j*BM + i, j'*r_pad + c] += sum_k x[i, sub-tile j, k] * L1s[sub-tile j', k, c]
 // Only the diagonal blocks j == j' are wanted; summing them over j and over
 // the cluster's K ranges gives X L1s = X_hat L1 for row i.  The partial sums
@@ -20,11 +25,13 @@
 // fixed order (the result does not depend on timing).  Codes and scales are
 // local to a 64-wide group and need no exchange.
 //
-// Every stage carries L1s as well as X: r_pad / BM bytes of factor per byte of
-// X.  Stacking (S > 1) fills the MMA at small M but raises that ratio; the K
-// split (C > 1) keeps BM large and still gives every SM a CTA.  The host picks
-// (S, C) from the SM count and the resident clusters of each size.
-//   warp 0      : TMA producer (S X boxes BM x 64, S L1s^T boxes r_pad x 64, 1/lambda)
+// Every stage carries L1s as well as X: 2 r_pad / BM bytes of factor (hi and
+// lo) per byte of X.  Stacking (S > 1) fills the MMA at small M but raises
+// that ratio; the K split (C > 1) keeps BM large and still gives every SM a
+// CTA.  The host picks (S, C) from the SM count and the resident clusters of
+// each size.
+//   warp 0      : TMA producer (S X boxes BM x 64, 2 S L1s^T boxes r_pad x 64
+//                 (hi, lo), 1/lambda)
 //   warp 1      : TMEM owner; one lane issues the kind::f16 MMAs
 //   warps 2..17 : quantizers in up to four groups of four (as many groups as
 //                 there are pipeline stages); group k takes every G-th stage,
@@ -80,8 +87,9 @@ struct QuantSmem {
   uint32_t x_off, l1_off, il_off, stage_bytes, stages, groups, stg_off, stg_bytes, bar_off, total;
 };
 
-// Per stage: the stacked X tile, S slices of L1s^T and 1/lambda.  After the
-// stages: two code staging buffers (128 rows of codes) per quantizer group.
+// Per stage: the stacked X tile, S slices of L1s^T hi then S of lo, and
+// 1/lambda.  After the stages: two code staging buffers (128 rows of codes)
+// per quantizer group.
 // G groups take the stages in turn, and the buffer count is a multiple of G,
 // so stage buffer b always serves group b mod G; G is 4 or 3, whichever keeps
 // more of the buffers that fit (4 on a tie: the quantizers set the pace), or
@@ -96,7 +104,7 @@ __host__ __device__ inline QuantSmem quant_smem_layout(int fmt, int r_pad, int S
   QuantSmem L;
   L.x_off = 0;
   L.l1_off = kQuantTileRows * kQuantBK * 2;                // 16384
-  L.il_off = L.l1_off + S * r_pad * 128;                   // S * r_pad rows of 128 bytes
+  L.il_off = L.l1_off + 2 * S * r_pad * 128;               // 2 S r_pad rows of 128 bytes (hi, lo)
   uint32_t sb = L.il_off + S * kQuantBK * 4;
   L.stage_bytes = (sb + 1023u) & ~1023u;
   L.stg_bytes = kQuantTileRows * quant_code_row_bytes(fmt);   // one staging buffer
@@ -175,7 +183,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
     if (elect_one()) {
       prefetch_tmap(&tm_x);
       if (has_lr) prefetch_tmap(&tm_l1t);
-      const uint32_t tx = S * (BM * kQuantBK * 2 + (has_lr ? p.r_pad * 128 : 0) + kQuantBK * 4);
+      const uint32_t tx = S * (BM * kQuantBK * 2 + (has_lr ? 2 * p.r_pad * 128 : 0) + kQuantBK * 4);
       int issued = 0;
       for (int li = 0; li < n_local; ++li) {
         const int i = i0 + li;
@@ -191,16 +199,18 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
         for (int j = 0; j < S; ++j) {
           const int k = (i * S + j) * kQuantBK;   // may lie past K: the box is zero-filled
           tma_load_2d(st + L.x_off + j * BM * 128, &tm_x, &full[s], k, m0);
-          if (has_lr) tma_load_2d(st + L.l1_off + j * p.r_pad * 128, &tm_l1t, &full[s], k, 0);
+          if (has_lr) {   // rows 0 .. r_pad - 1 of the map hold hi, r_pad .. 2 r_pad - 1 lo
+            tma_load_2d(st + L.l1_off + j * p.r_pad * 128, &tm_l1t, &full[s], k, 0);
+            tma_load_2d(st + L.l1_off + (S + j) * p.r_pad * 128, &tm_l1t, &full[s], k, p.r_pad);
+          }
         }
         bulk_load(st + L.il_off, p.inv_lambda + i * kstep, S * kQuantBK * 4, &full[s]);
         issued = li + 1;
       }
       // never leave while a copy into this CTA's shared memory is still in flight
-      if (*abort_flag) {
-        for (int i = (issued > NS ? issued - NS : 0); i < issued; ++i)
-          mbar_wait(&full[i % NS], (i / NS) & 1, p.budget, nullptr);
-      }
+      // (whether or not a wait ran out, and in whichever role)
+      for (int i = (issued > NS ? issued - NS : 0); i < issued; ++i)
+        mbar_wait(&full[i % NS], (i / NS) & 1, drain_budget(p.budget), nullptr);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -216,12 +226,16 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
         }
         tc_fence_after();
         const uint32_t a0 = smem_u32(smem + s * L.stage_bytes + L.x_off);
-        const uint32_t b0 = smem_u32(smem + s * L.stage_bytes + L.l1_off);
+        const uint32_t b0 = smem_u32(smem + s * L.stage_bytes + L.l1_off);   // hi slices
+        const uint32_t b1 = b0 + static_cast<uint32_t>(S * p.r_pad * 128);    // lo slices
 #pragma unroll
         for (int k = 0; k < kQuantBK / 16; ++k) {
           mma_bf16(tmem_base, make_kmajor_desc(a0 + 32 * k, 128), make_kmajor_desc(b0 + 32 * k, 128),
                    idesc, (li > 0 || k > 0) ? 1u : 0u);
         }
+#pragma unroll
+        for (int k = 0; k < kQuantBK / 16; ++k)
+          mma_bf16(tmem_base, make_kmajor_desc(a0 + 32 * k, 128), make_kmajor_desc(b1 + 32 * k, 128), idesc, 1u);
         tc_commit(&empty[s]);
       }
       tc_commit(acc_full);  // also covers an early exit: waits for every issued MMA
@@ -322,12 +336,16 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
         const uint16_t sh = int4_scale_bits(amax);
         const float sd = __half2float(__ushort_as_half(sh));
         const float inv = sd == 0.0f ? 0.0f : __frcp_rn(sd);
+        // int8 codes in the INT4 GEMM's K order: in each run of eight values the
+        // even positions first, then the odd ones (the order in which the GEMM
+        // unpacks the 4-bit weight codes)
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
+          const int base = 8 * (e >> 1) + (e & 1);
           uint32_t w = 0;
 #pragma unroll
           for (int b = 0; b < 4; ++b)
-            w |= (static_cast<uint32_t>(int4_code(v[4 * e + b], inv)) & 0xFFu) << (8 * b);
+            w |= (static_cast<uint32_t>(int4_code(v[base + 2 * b], inv)) & 0xFFu) << (8 * b);
           out[e] = sd == 0.0f ? 0u : w;
         }
         sfw = sh;
@@ -453,7 +471,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
   if (p.C > 1) cluster_sync();
   if (warp == 1 && has_lr) {
     // every MMA this CTA issued has retired before its TMEM is released
-    mbar_wait(acc_full, 0, p.budget, nullptr);
+    mbar_wait(acc_full, 0, drain_budget(p.budget), nullptr);
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem_base, tmem_cols);

@@ -45,13 +45,14 @@ struct svdq_weights {
   int sf_kcols = 0;    // K_pad / 64
   float* inv_lambda = nullptr;
   float* lambda = nullptr;
-  uint8_t* wcodes = nullptr;  // NVFP4: N x K/2 packed; INT4: N x K int8
+  uint8_t* wcodes = nullptr;  // NVFP4, FP4 g32, INT4: N x K/2 packed (element 2i low nibble); W8A8: N x K int8
   uint8_t* wsf = nullptr;     // NVFP4: atoms [N_pad/128][sf_kcols][512]; INT4: fp16 [K/64][N_pad]
   uint8_t* wsf192 = nullptr;  // FP4: the same atoms regrouped per 192-column tile [2 n192][sf_kcols][512]
   int n192 = 0;               // FP4: 192-column tiles of N
-  float* wsf32 = nullptr;     // INT4: the same scales as fp32, read by the GEMM
+  float4* wswc = nullptr;     // INT4: per column pair (s_w / 16, c) constants of the GEMM's drain
   __nv_bfloat16* l1t = nullptr;  // r_pad x K
-  __nv_bfloat16* l1st = nullptr; // r_pad x K: bf16(diag(1/lambda) L1)^T, read by the activation kernel
+  __nv_bfloat16* l1st = nullptr; // 2 r_pad x K: (diag(1/lambda) L1)^T as hi rows then lo rows, read by
+                                 // the activation kernel
   __nv_bfloat16* l2t = nullptr;  // N x r_pad
   __nv_bfloat16* l2t2 = nullptr; // N x 2 r_pad: [L2^T | L2^T], the tail MMA's B operand
   __nv_bfloat16* bias = nullptr;
@@ -164,7 +165,7 @@ CUtensorMapSwizzle swizzle_for(uint32_t row_bytes) {
 
 // 2-D map over a row-major [rows][cols] array of `elem` bytes per element.
 int make_map(CUtensorMap* m, CUtensorMapDataType dt, size_t elem, const void* base, uint64_t cols,
-             uint64_t rows, uint32_t box_cols, uint32_t box_rows) {
+             uint64_t rows, uint32_t box_cols, uint32_t box_rows, int swizzle = -1) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return SVDQ_ERR_CUDA;
   const cuuint64_t dims[2] = {cols, rows};
@@ -172,7 +173,9 @@ int make_map(CUtensorMap* m, CUtensorMapDataType dt, size_t elem, const void* ba
   const cuuint32_t box[2] = {box_cols, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_for(static_cast<uint32_t>(box_cols * elem)),
+                  CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle >= 0 ? static_cast<CUtensorMapSwizzle>(swizzle)
+                               : swizzle_for(static_cast<uint32_t>(box_cols * elem)),
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     std::fprintf(stderr, "svdq: cuTensorMapEncodeTiled failed (%d): cols=%llu rows=%llu box=%u x %u\n",
@@ -211,10 +214,11 @@ struct DeviceInfo {
   int qclusters[kQuantMaxSplit + 1] = {};   // resident activation-kernel clusters of size C
   std::atomic<bool> attrs_set{false};   // set (release) once every field above is filled
 };
-DeviceInfo g_dev[64];
+constexpr int kMaxDevices = 64;   // device ordinals the per-device tables cover
+DeviceInfo g_dev[kMaxDevices];
 
 int device_setup(int dev) {
-  if (dev < 0 || dev >= 64) return SVDQ_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return SVDQ_ERR_CUDA;
   DeviceInfo& d = g_dev[dev];
   if (d.attrs_set.load(std::memory_order_acquire)) return SVDQ_OK;
   std::lock_guard<std::mutex> lk(g_mutex);
@@ -299,7 +303,7 @@ int current_device(int* dev) {
 // fixed: setup, the first stage's round trip and the XL1 epilogue; exchange and
 // per_peer: the cluster barriers and the distributed-shared-memory reads of the
 // peers' partial sums; stage and l1: one 128 x 64 stage, whose L1s share
-// (r_pad / BM bytes per byte of X) travels and is read with it.  Ties go to
+// (hi and lo: 2 r_pad / BM bytes per byte of X) travels and is read with it.  Ties go to
 // the smaller C, then the smaller S.
 struct QuantSplit {
   int S, C;
@@ -314,7 +318,7 @@ std::atomic<int> g_forced_group_m{0};    // svdq_set_gemm_raster; 0 = automatic
 std::atomic<int> g_forced_gemm_kind{0};  // svdq_set_gemm_kernel; 0 = automatic, 1 = one CTA, 2 = CTA pairs,
                                          // 3 = CTA pairs on 192-column tiles
 
-QuantSplit quant_split_for(int M, int K, int r_pad, const DeviceInfo& d) {
+QuantSplit quant_split_for(int fmt, int M, int K, int r_pad, const DeviceInfo& d) {
   const int smax = r_pad > 0 ? quant_stack_max(r_pad) : 8;
   const int fs = g_forced_split.load(std::memory_order_relaxed);
   const QuantSplit f{fs / 16, fs % 16};
@@ -327,6 +331,9 @@ QuantSplit quant_split_for(int M, int K, int r_pad, const DeviceInfo& d) {
     const int slots = d.qclusters[C] * C;   // resident CTAs in clusters of C
     if (slots <= 0) continue;
     for (int S = 1; S <= smax; S *= 2) {
+      // a stack whose stage no longer leaves room for three stage buffers
+      // loses the pipeline the model assumes
+      if (S > 1 && quant_smem_layout(fmt, r_pad, S).stages < 3) continue;
       const int BM = kQuantTileRows / S;
       const int stages = (K + S * kQuantBK - 1) / (S * kQuantBK);
       if (C > BM || C > stages) continue;
@@ -335,7 +342,7 @@ QuantSplit quant_split_for(int M, int K, int r_pad, const DeviceInfo& d) {
       const int per = (stages + C - 1) / C;
       const double t = static_cast<double>(waves) *
                        (kQuantFixedCycles + (C > 1 ? kQuantExchangeCycles + C * kQuantPerPeerCycles : 0.0) +
-                        per * (kQuantStageCycles + kQuantL1Cycles * r_pad / BM));
+                        per * (kQuantStageCycles + kQuantL1Cycles * 2 * r_pad / BM));
       if (t < best_t * 0.98) {
         best_t = t;
         best = {S, C};
@@ -379,11 +386,12 @@ int encode_weight_maps(svdq_weights* w) {
     if (!rc) rc = make_atom_map(&w->tm_sfb192, w->wsf192, static_cast<uint64_t>(2 * w->n192) * w->sf_kcols);
   } else if (w->fmt == SVDQ_W8A8)
     rc = make_map(&w->tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->wcodes, w->K, w->N, kW8BKB, kW8BN);
-  else
-    rc = make_map(&w->tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->wcodes, w->K, w->N, 64, kI4BN);
+  else   // INT4: the packed codes, 32 bytes (64 codes) x 128 columns per box, read by the drain warps
+    rc = make_map(&w->tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->wcodes, w->K / 2, w->N, 32, kI4BN,
+                  CU_TENSOR_MAP_SWIZZLE_NONE);
   if (rc) return rc;
   if (w->r_pad > 0) {
-    rc = make_map(&w->tm_l1t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w->l1st, w->K, w->r_pad, 64, w->r_pad);
+    rc = make_map(&w->tm_l1t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w->l1st, w->K, 2 * w->r_pad, 64, w->r_pad);
     if (rc) return rc;
     const int lc = w->fmt != SVDQ_INT4 ? lr_chunk_cols(2 * w->r_pad) : i4_lr_chunk_cols(2 * w->r_pad);
     rc = make_map(&w->tm_l2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w->l2t2, 2 * w->r_pad, w->N, lc,
@@ -411,7 +419,7 @@ void free_weights(svdq_weights* w) {
   cudaFree(w->wcodes);
   cudaFree(w->wsf);
   cudaFree(w->wsf192);
-  cudaFree(w->wsf32);
+  cudaFree(w->wswc);
   cudaFree(w->l1t);
   cudaFree(w->l1st);
   cudaFree(w->l2t);
@@ -434,7 +442,7 @@ int alloc_weights(svdq_weights* w, cudaStream_t st) {
   w->N_pad = round_up(w->N, 256);
   w->sf_kcols = w->K_pad / 64;
   w->r_pad = rank_padded(w->rank);
-  const size_t codes = is_fp4(w->fmt) ? static_cast<size_t>(w->N) * w->K / 2
+  const size_t codes = w->fmt != SVDQ_W8A8 ? static_cast<size_t>(w->N) * w->K / 2
                                             : static_cast<size_t>(w->N) * w->K;
   const size_t sfb = is_fp4(w->fmt)            ? static_cast<size_t>(w->N_pad / 128) * w->sf_kcols * 512
                      : w->fmt == SVDQ_W8A8 ? static_cast<size_t>(w->N_pad) * 4   // fp32 per channel
@@ -454,17 +462,17 @@ int alloc_weights(svdq_weights* w, cudaStream_t st) {
     SVDQ_CUDA(cudaMemsetAsync(w->wsf192, 0, sf192, st));
   }
   if (w->fmt == SVDQ_INT4) {
-    const size_t sf32 = static_cast<size_t>(w->K / 64) * w->N_pad * sizeof(float);
-    if (cudaMalloc(&w->wsf32, sf32) != cudaSuccess) return SVDQ_ERR_ALLOC;
-    SVDQ_CUDA(cudaMemsetAsync(w->wsf32, 0, sf32, st));
+    const size_t swc = static_cast<size_t>(w->K / 64) * (w->N_pad / 2) * sizeof(float4);
+    if (cudaMalloc(&w->wswc, swc) != cudaSuccess) return SVDQ_ERR_ALLOC;
+    SVDQ_CUDA(cudaMemsetAsync(w->wswc, 0, swc, st));
   }
   if (w->r_pad > 0) {
     if (cudaMalloc(&w->l1t, static_cast<size_t>(w->r_pad) * w->K * 2) != cudaSuccess ||
-        cudaMalloc(&w->l1st, static_cast<size_t>(w->r_pad) * w->K * 2) != cudaSuccess ||
+        cudaMalloc(&w->l1st, static_cast<size_t>(2 * w->r_pad) * w->K * 2) != cudaSuccess ||
         cudaMalloc(&w->l2t, static_cast<size_t>(w->N) * w->r_pad * 2) != cudaSuccess)
       return SVDQ_ERR_ALLOC;
     SVDQ_CUDA(cudaMemsetAsync(w->l1t, 0, static_cast<size_t>(w->r_pad) * w->K * 2, st));
-    SVDQ_CUDA(cudaMemsetAsync(w->l1st, 0, static_cast<size_t>(w->r_pad) * w->K * 2, st));
+    SVDQ_CUDA(cudaMemsetAsync(w->l1st, 0, static_cast<size_t>(2 * w->r_pad) * w->K * 2, st));
     SVDQ_CUDA(cudaMemsetAsync(w->l2t, 0, static_cast<size_t>(w->N) * w->r_pad * 2, st));
   }
   return SVDQ_OK;
@@ -501,8 +509,15 @@ int build_l2t2(svdq_weights* w, cudaStream_t st) {
 
 // Scale layouts derived from the weight scales in w->wsf, redone whenever
 // those change (quantization, or a refinement restoring an earlier iterate):
-// FP4 formats: the atoms regrouped per 192-column tile of the pair GEMM.
+// FP4 formats: the atoms regrouped per 192-column tile of the pair GEMM;
+// INT4: the drain's per-column-pair constants.
 int derive_scale_layouts(svdq_weights* w, cudaStream_t st) {
+  if (w->fmt == SVDQ_INT4) {
+    const size_t n = static_cast<size_t>(w->K / 64) * (w->N_pad / 2);
+    int4_column_consts_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
+        reinterpret_cast<const uint16_t*>(w->wsf), w->K / 64, w->N_pad, w->wswc);
+    SVDQ_CHECK_LAUNCH();
+  }
   if (is_fp4(w->fmt)) {
     const size_t sf192 = static_cast<size_t>(2 * w->n192) * w->sf_kcols * 512;
     pair192_scale_atoms_kernel<<<static_cast<unsigned>((sf192 + 255) / 256), 256, 0, st>>>(
@@ -542,9 +557,8 @@ int quantize_residual(svdq_weights* w, const float* R, cudaStream_t st) {
                                                                 reinterpret_cast<float*>(w->wsf));
   } else {
     const dim3 grid((w->N + 127) / 128, w->K / 64);
-    quant_weight_int4_kernel<<<grid, blk, 0, st>>>(R, w->K, w->N, w->N_pad,
-                                                   reinterpret_cast<int8_t*>(w->wcodes),
-                                                   reinterpret_cast<uint16_t*>(w->wsf), w->wsf32);
+    quant_weight_int4_kernel<<<grid, blk, 0, st>>>(R, w->K, w->N, w->N_pad, w->wcodes,
+                                                   reinterpret_cast<uint16_t*>(w->wsf));
   }
   SVDQ_CHECK_LAUNCH();
   if (int rc = derive_scale_layouts(w, st)) return rc;
@@ -552,8 +566,8 @@ int quantize_residual(svdq_weights* w, const float* R, cudaStream_t st) {
   return SVDQ_OK;
 }
 
-// The derived operands the kernels read: l1st = bf16(diag(1/lambda) L1)^T and
-// l2t2 = [L2^T | L2^T], from the current l1t, l2t and inv_lambda.
+// The derived operands the kernels read: l1st = (diag(1/lambda) L1)^T as a bf16
+// pair hi | lo and l2t2 = [L2^T | L2^T], from the current l1t, l2t and inv_lambda.
 int refold_l1(svdq_weights* w, cudaStream_t st) {
   if (w->rank == 0) return SVDQ_OK;
   cudaFree(w->l2t2);
@@ -562,7 +576,7 @@ int refold_l1(svdq_weights* w, cudaStream_t st) {
     return SVDQ_ERR_ALLOC;
   if (int rc = build_l2t2(w, st)) return rc;
   fold_l1_kernel<<<dim3((w->K + 255) / 256, w->rank), 256, 0, st>>>(w->l1t, w->inv_lambda, w->K,
-                                                                     w->rank, w->l1st);
+                                                                     w->rank, w->r_pad, w->l1st);
   SVDQ_CHECK_LAUNCH();
   return SVDQ_OK;
 }
@@ -582,7 +596,7 @@ int do_append_lora(svdq_weights* w, const void* A, const void* B, int rl, cudaSt
   const int rp_new = rank_padded(r_new);
   __nv_bfloat16 *l1t = nullptr, *l1st = nullptr, *l2t = nullptr;
   if (cudaMalloc(&l1t, static_cast<size_t>(rp_new) * w->K * 2) != cudaSuccess) return SVDQ_ERR_ALLOC;
-  if (cudaMalloc(&l1st, static_cast<size_t>(rp_new) * w->K * 2) != cudaSuccess) {
+  if (cudaMalloc(&l1st, static_cast<size_t>(2 * rp_new) * w->K * 2) != cudaSuccess) {
     cudaFree(l1t);
     return SVDQ_ERR_ALLOC;
   }
@@ -592,7 +606,7 @@ int do_append_lora(svdq_weights* w, const void* A, const void* B, int rl, cudaSt
     return SVDQ_ERR_ALLOC;
   }
   cudaMemsetAsync(l1t, 0, static_cast<size_t>(rp_new) * w->K * 2, st);
-  cudaMemsetAsync(l1st, 0, static_cast<size_t>(rp_new) * w->K * 2, st);
+  cudaMemsetAsync(l1st, 0, static_cast<size_t>(2 * rp_new) * w->K * 2, st);
   cudaMemsetAsync(l2t, 0, static_cast<size_t>(w->N) * rp_new * 2, st);
   if (r_old > 0) {
     const size_t n1 = static_cast<size_t>(r_old) * w->K;
@@ -687,7 +701,7 @@ int lowrank_factors(svdq_weights* w, const double* What, cudaStream_t st) {
 int weight_error(svdq_weights* w, const double* What, double* err_dev, double* out, cudaStream_t st) {
   SVDQ_CUDA(cudaMemsetAsync(err_dev, 0, sizeof(double), st));
   refine_error_kernel<<<dim3((w->N + 255) / 256, w->K), 256, 0, st>>>(
-      What, w->l1t, w->l2t, w->rank, w->r_pad, w->fmt, w->wcodes, w->wsf, w->wsf32, w->K, w->N,
+      What, w->l1t, w->l2t, w->rank, w->r_pad, w->fmt, w->wcodes, w->wsf, w->K, w->N,
       w->N_pad, w->sf_kcols, std::ldexp(1.0, -w->w_exp), err_dev);
   SVDQ_CHECK_LAUNCH();
   double h = 0.0;
@@ -703,14 +717,13 @@ int weight_error(svdq_weights* w, const double* What, double* err_dev, double* o
 int refine_branch(svdq_weights* w, const double* What, float* R, int iters, cudaStream_t st) {
   const size_t KN = static_cast<size_t>(w->K) * w->N;
   const size_t l1b = static_cast<size_t>(w->r_pad) * w->K * 2, l2b = static_cast<size_t>(w->N) * w->r_pad * 2;
-  const size_t cb = is_fp4(w->fmt) ? KN / 2 : KN;
+  const size_t cb = w->fmt != SVDQ_W8A8 ? KN / 2 : KN;
   const size_t sfb = is_fp4(w->fmt)            ? static_cast<size_t>(w->N_pad / 128) * w->sf_kcols * 512
                      : w->fmt == SVDQ_W8A8 ? static_cast<size_t>(w->N_pad) * 4
                                            : static_cast<size_t>(w->K / 64) * w->N_pad * 2;
-  const size_t sf32b = w->fmt == SVDQ_INT4 ? static_cast<size_t>(w->K / 64) * w->N_pad * 4 : 0;
-  DeviceBuf E, err, b_l1, b_l2, b_codes, b_sf, b_sf32;
+  DeviceBuf E, err, b_l1, b_l2, b_codes, b_sf;
   if (!E.alloc(KN * 8) || !err.alloc(sizeof(double)) || !b_l1.alloc(l1b) || !b_l2.alloc(l2b) ||
-      !b_codes.alloc(cb) || !b_sf.alloc(sfb) || (sf32b && !b_sf32.alloc(sf32b)))
+      !b_codes.alloc(cb) || !b_sf.alloc(sfb))
     return SVDQ_ERR_ALLOC;
   auto save = [&](bool to_best) -> int {
     auto cp = [&](void* best, void* cur, size_t n) {
@@ -718,8 +731,7 @@ int refine_branch(svdq_weights* w, const double* What, float* R, int iters, cuda
                      : cudaMemcpyAsync(cur, best, n, cudaMemcpyDeviceToDevice, st);
     };
     if (cp(b_l1.p, w->l1t, l1b) != cudaSuccess || cp(b_l2.p, w->l2t, l2b) != cudaSuccess ||
-        cp(b_codes.p, w->wcodes, cb) != cudaSuccess || cp(b_sf.p, w->wsf, sfb) != cudaSuccess ||
-        (sf32b && cp(b_sf32.p, w->wsf32, sf32b) != cudaSuccess))
+        cp(b_codes.p, w->wcodes, cb) != cudaSuccess || cp(b_sf.p, w->wsf, sfb) != cudaSuccess)
       return SVDQ_ERR_CUDA;
     return SVDQ_OK;
   };
@@ -731,7 +743,7 @@ int refine_branch(svdq_weights* w, const double* What, float* R, int iters, cuda
   int best_exp = w->w_exp;   // the prescale exponent the kept codes and scales were made with
   for (int t = 0; t < iters; ++t) {
     refine_target_kernel<<<dim3((w->N + 255) / 256, w->K), 256, 0, st>>>(
-        What, w->fmt, w->wcodes, w->wsf, w->wsf32, w->K, w->N, w->N_pad, w->sf_kcols,
+        What, w->fmt, w->wcodes, w->wsf, w->K, w->N, w->N_pad, w->sf_kcols,
         std::ldexp(1.0, -w->w_exp), E.as<double>());
     SVDQ_CHECK_LAUNCH();
     if ((rc = lowrank_factors(w, E.as<double>(), st))) return rc;
@@ -1037,7 +1049,7 @@ SVDQ_API int svdq_quantize_act(const svdq_weights* w, const void* X, int M, void
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const ActLayout L = act_layout(w, M);
   uint8_t* base = static_cast<uint8_t*>(ws);
-  const QuantSplit sp = quant_split_for(M, w->K, w->r_pad, g_dev[dev]);
+  const QuantSplit sp = quant_split_for(w->fmt, M, w->K, w->r_pad, g_dev[dev]);
   const int S = sp.S;
   const int BM = kQuantTileRows / S;
   CUtensorMap tm_x, tm_codes;
@@ -1063,6 +1075,8 @@ SVDQ_API int svdq_quantize_act(const svdq_weights* w, const void* X, int M, void
   p.budget = wait_budget();
   const QuantSmem Q = quant_smem_layout(w->fmt, w->r_pad, S);
   if (Q.groups < 1 || Q.stages % Q.groups != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  // the X_hat L1 epilogue parks [128][r_pad + 4] fp32 over the stage and staging buffers
+  if (static_cast<uint32_t>(kQuantTileRows * (w->r_pad + 4) * 4) > Q.bar_off) return SVDQ_ERR_UNSUPPORTED_SHAPE;
   if (is_fp4(w->fmt) && w->sf_kcols * 64 != w->K) {
     // zero the scale atoms of the K padding (read by the GEMM's last K step)
     const size_t pitch = static_cast<size_t>(w->sf_kcols) * 512;
@@ -1232,7 +1246,7 @@ SVDQ_API int svdq_linear(const svdq_weights* w, const void* ws, int M, void* Y, 
     p.group_m = group_m;
     p.r_tail = 2 * w->r_pad;
     p.sx = reinterpret_cast<const uint16_t*>(base + L.sf_off);
-    p.sw = w->wsf32;
+    p.swc = w->wswc;
     p.M_pad = L.M_pad;
     p.N_pad = w->N_pad;
     p.bias = w->bias;
@@ -1260,7 +1274,7 @@ SVDQ_API int svdq_forward(const svdq_weights* w, const void* X, int M, void* Y, 
 static __device__ __align__(256) uint8_t g_noalloc_workspace[SVDQ_NOALLOC_WORKSPACE_BYTES];
 
 SVDQ_API int svdq_forward_noalloc(const svdq_weights* w, const void* X, int M, void* Y, void* stream) {
-  static std::atomic<void*> ws_ptr[64] = {};
+  static std::atomic<void*> ws_ptr[kMaxDevices] = {};
   if (w == nullptr || M < 0) return SVDQ_ERR_INVALID_ARG;
   if (M == 0) return SVDQ_OK;
   const size_t need = act_layout(w, M).total;
@@ -1275,6 +1289,7 @@ SVDQ_API int svdq_forward_noalloc(const svdq_weights* w, const void* X, int M, v
   int rc = current_device(&dev);
   if (rc) return rc;
   if (dev != w->device) return SVDQ_ERR_INVALID_ARG;
+  if (dev < 0 || dev >= kMaxDevices) return SVDQ_ERR_CUDA;   // (current_device checks this as well)
   void* ws = ws_ptr[dev].load(std::memory_order_acquire);
   if (ws == nullptr) {
     // first call on this device: look up the array's device address once
@@ -1310,10 +1325,15 @@ SVDQ_API int svdq_export_act(const svdq_weights* w, const void* ws, int M, uint8
       // packed E2M1 pairs, or W8A8's int8 codes as they are
       SVDQ_CUDA(cudaMemcpy(codes, base + L.codes_off, L.codes_bytes, cudaMemcpyDeviceToHost));
     } else {
+      // INT4: int8 codes in the GEMM's K order (0 2 4 6 1 3 5 7 in each run of
+      // eight) -> packed nibbles in natural order
       std::vector<int8_t> tmp(L.codes_bytes);
       SVDQ_CUDA(cudaMemcpy(tmp.data(), base + L.codes_off, L.codes_bytes, cudaMemcpyDeviceToHost));
-      for (size_t i = 0; i < tmp.size() / 2; ++i)
-        codes[i] = static_cast<uint8_t>((tmp[2 * i] & 0xF) | ((tmp[2 * i + 1] & 0xF) << 4));
+      for (size_t c = 0; c < tmp.size() / 8; ++c) {
+        const int8_t* e = tmp.data() + 8 * c;   // e[0..3] = k 0 2 4 6, e[4..7] = k 1 3 5 7
+        for (int i = 0; i < 4; ++i)
+          codes[4 * c + i] = static_cast<uint8_t>((e[i] & 0xF) | ((e[4 + i] & 0xF) << 4));
+      }
     }
   }
   if (scales) {
@@ -1366,15 +1386,10 @@ SVDQ_API int svdq_export_weights(const svdq_weights* w, uint8_t* codes, void* sc
   SVDQ_CUDA(cudaDeviceSynchronize());
   const int K = w->K, N = w->N;
   if (codes) {
-    if (is_fp4(w->fmt)) {
-      SVDQ_CUDA(cudaMemcpy(codes, w->wcodes, static_cast<size_t>(N) * K / 2, cudaMemcpyDeviceToHost));
-    } else if (w->fmt == SVDQ_W8A8) {
+    if (w->fmt == SVDQ_W8A8) {
       SVDQ_CUDA(cudaMemcpy(codes, w->wcodes, static_cast<size_t>(N) * K, cudaMemcpyDeviceToHost));
-    } else {
-      std::vector<int8_t> tmp(static_cast<size_t>(N) * K);
-      SVDQ_CUDA(cudaMemcpy(tmp.data(), w->wcodes, tmp.size(), cudaMemcpyDeviceToHost));
-      for (size_t i = 0; i < tmp.size() / 2; ++i)
-        codes[i] = static_cast<uint8_t>((tmp[2 * i] & 0xF) | ((tmp[2 * i + 1] & 0xF) << 4));
+    } else {   // packed nibbles as stored (E2M1, or INT4 two's complement)
+      SVDQ_CUDA(cudaMemcpy(codes, w->wcodes, static_cast<size_t>(N) * K / 2, cudaMemcpyDeviceToHost));
     }
   }
   if (scales) {

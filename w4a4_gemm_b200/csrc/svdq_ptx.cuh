@@ -91,6 +91,23 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long l
   }
 }
 
+// Bound of the waits a kernel makes on its way out: for copies it has issued
+// to land and MMAs it has issued to retire before it frees shared memory or
+// TMEM.  Work already issued always finishes, so these waits get the larger of
+// the caller's budget and 2^33 cycles (4.4 s at 1965 MHz): a short budget that
+// ends a stalled pipeline early must not also cut the drain short.
+constexpr long long kDrainBudget = 1LL << 33;
+__host__ __device__ constexpr long long drain_budget(long long budget) {
+  return budget > kDrainBudget ? budget : kDrainBudget;
+}
+
+// Complete `bytes` of an mbarrier phase's expected transaction count without a
+// copy (for fills a peer CTA armed for but never issued).
+__device__ __forceinline__ void mbar_complete_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.complete_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
 // Warp-wide wait: every lane waits, and the warp leaves converged with one
 // verdict (false if any lane gave up), as required before .sync.aligned
 // tcgen05 instructions and cluster barriers.
@@ -433,6 +450,11 @@ __device__ __forceinline__ void tc_commit_pair(uint64_t* bar, uint16_t cta_mask)
       " [%0], %1;" ::"r"(smem_u32(bar)),
       "h"(cta_mask)
       : "memory");
+}
+
+// Store a 32-bit word to shared memory of this cluster (an address from map_shared_rank).
+__device__ __forceinline__ void st_shared_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
 }
 
 __device__ __forceinline__ float4 ld_shared_cluster_f32x4(uint32_t addr) {
