@@ -10,33 +10,35 @@
 // with scale 1.
 //
 // Weight codes stay at 4 bits in HBM (N x K/2 bytes, element 2i in the low
-// nibble, two's complement).  The drain warps also unpack each stage's packed
-// B tile in shared memory, a few stages ahead of the MMA: every nibble goes to
-// the high half of its own byte, so the int8 the tensor core reads is 16 q
-// (the sign comes along for free, three integer operations per eight codes),
-// and within each run of eight values the bytes come out in the K order
-// 0 2 4 6 1 3 5 7.  The activation codes (int8, written by the activation
-// kernel) are stored in that same order, so every product q_x q_w meets its
-// partner and the group's integer sum is 16 P with P = sum q_x q_w.
+// nibble, two's complement).  Two unpack warps turn each stage's packed B tile
+// into the MMA's int8 layout in shared memory as soon as it lands: every
+// nibble goes to the high half of its own byte, so the int8 the tensor core
+// reads is 16 q (the sign comes along for free, three integer operations per
+// eight codes), and within each run of eight values the bytes come out in the
+// K order 0 2 4 6 1 3 5 7.  The activation codes (int8, written by the
+// activation kernel) are stored in that same order, so every product q_x q_w
+// meets its partner and the group's integer sum is 16 P, P = sum q_x q_w.
 //
-// The partial reaches the drain already as fp32: each buffer is pre-filled
-// with the bit pattern of 1.5 * 2^23 and the MMAs accumulate onto it, so the
+// The partial reaches the drain already as fp32: before a group's two int8
+// MMAs the MMA issuer writes 1.5 * 2^23 into the partial buffer with one bf16
+// MMA of two constant tiles (A rows (1, 0, ...), B rows (1.5 * 2^23, 0, ...),
+// accumulate off), and the int8 MMAs accumulate onto that offset's bits, so the
 // bits read back are those of v = 1.5 * 2^23 + 16 P exactly (|16 P| <= 16 * 64
-// * 49 < 2^22).  After reading a buffer the drain refills it.  Per output and
-// group the drain then issues two fused multiply-adds, on packed pairs:
-//   t   = v * (s_w / 16) + c,   c = -1.5 * 2^19 * s_w     (t = P s_w exactly:
-//         P s_w has at most 23 significant bits, and c is exact)
-//   acc = t * s_x + acc
-// with (s_w / 16, c) prepared per weight column beside the fp16 scales.
+// * 49 < 2^22).  The drain only reads TMEM.  Per output pair and group it issues
+// three packed fp32 operations:
+//   d = v - 1.5 * 2^23   (= 16 P, exact)
+//   s = s_x * (s_w / 16) (exact: two fp16 values and a power of two)
+//   acc = d * s + acc    (one rounding)
+// with s_w / 16 prepared per weight column beside the fp16 scales.
 //
-//   warp 0     : TMA producer (A 128 x 64 int8, the packed B 128 x 32 bytes,
-//                the group's activation scales (fp16) and the weight columns'
-//                (s_w / 16, c) pairs; then the XL1 / L2^T chunks of the tail)
-//   warp 1     : TMEM owner, MMA issuer
-//   warps 2-17 : unpack of B (each a 16th of the tile, kI4Ahead stages ahead)
-//                and drain + epilogue: warp w serves TMEM lane quarter w % 4
-//                and output columns [32 ((w - 2) / 4), +32) of the 128 x 128
-//                tile.  Four warps per scheduler hide the TMEM load latency.
+//   warp 0      : TMA producer (A 128 x 64 int8, the packed B 128 x 32 bytes,
+//                 the group's activation scales (fp16) and the weight columns'
+//                 s_w / 16; then the XL1 / L2^T chunks of the tail)
+//   warp 1      : TMEM owner, MMA issuer
+//   warps 2-9   : drain + epilogue: warp w serves TMEM lane quarter w % 4 and
+//                 output columns [64 ((w - 2) / 4), +64) of the 128 x 128 tile,
+//                 read from TMEM with one 64-column load per group
+//   warps 10-11 : unpack of the packed B tiles, stage by stage as they land
 #pragma once
 
 #include "gemm_nvfp4.cuh"
@@ -48,29 +50,28 @@ namespace svdq {
 constexpr int kI4BM = 128;
 constexpr int kI4BN = 128;
 constexpr int kI4BK = 64;                 // one group
-constexpr int kI4EpiWarps = 16;
-constexpr int kI4Threads = 32 * (2 + kI4EpiWarps);
+constexpr int kI4EpiWarps = 8;
+constexpr int kI4UnpackWarps = 2;
+constexpr int kI4Threads = 32 * (2 + kI4EpiWarps + kI4UnpackWarps);
 constexpr int kI4Bufs = 4;                // TMEM partial buffers of kI4BN columns
-constexpr int kI4Ahead = 2;               // stages the unpack runs ahead of the drain
 constexpr uint32_t kI4AOff = 0;                            // 128 x 64 B (int8 codes or a tail chunk)
-constexpr uint32_t kI4BOff = kI4BM * 64;                   // 8192: unpacked B, 128 x 64 B
-constexpr uint32_t kI4BpOff = kI4BOff + kI4BN * 64;        // 16384: packed B, 128 x 32 B
+constexpr uint32_t kI4BOff = kI4BM * 128;                  // 16384
+constexpr uint32_t kI4BpOff = kI4BOff + kI4BN * 128;       // 32768
 constexpr uint32_t kI4SxOff = kI4BpOff + kI4BN * 32;       // 20480: activation scales, 128 fp16
-constexpr uint32_t kI4SwOff = kI4SxOff + kI4BM * 2;        // 20736: 64 (s_w / 16, c) column pairs
-constexpr uint32_t kI4StageBytes = 22528;                  // 22 KB, multiple of 1024
-constexpr int kI4Stages = 9;
+constexpr uint32_t kI4SwOff = kI4SxOff + kI4BM * 2;        // s_w / 16 of the tile's 128 columns
+constexpr uint32_t kI4StageBytes = 38912;
+constexpr int kI4Stages = 5;
+constexpr uint32_t kI4ConstOff = kI4StageBytes * kI4Stages;  // the offset MMA's two constant 128 x 16 bf16 tiles
 constexpr uint32_t kI4BarBytes = 512;                      // 3 S + 2 NB + 1 mbarriers, TMEM address, flag
-constexpr uint32_t kI4SmemBytes = kI4StageBytes * kI4Stages + kI4BarBytes + 1024;
-constexpr uint32_t kI4Magic = 0x4B400000u;                 // bits of 1.5 * 2^23
-static_assert(kI4SwOff + 64 * 16 <= kI4StageBytes, "stage layout");
-static_assert(kI4Stages >= kI4Ahead + 2, "the unpack look-ahead needs free stages");
+constexpr uint32_t kI4SmemBytes = kI4ConstOff + 8192 + kI4BarBytes + 1024;
+static_assert(kI4SwOff + kI4BN * 4 <= kI4StageBytes, "stage layout");
 static_assert((3 * kI4Stages + 2 * kI4Bufs + 1) * 8 + 8 <= kI4BarBytes, "barrier area");
 
 // Low-rank tail chunks of at most 32 bf16 columns (64-byte rows: they fit the
 // A and B regions of a stage).
-__host__ __device__ inline int i4_lr_chunk_cols(int k_tail) { return k_tail < 32 ? k_tail : 32; }
+__host__ __device__ inline int i4_lr_chunk_cols(int k_tail) { return k_tail < 64 ? k_tail : 64; }
 __host__ __device__ inline int i4_lr_num_chunks(int k_tail) {
-  return k_tail == 0 ? 0 : (k_tail + 31) / 32;
+  return k_tail == 0 ? 0 : (k_tail + 63) / 64;
 }
 
 struct GemmI4Params {
@@ -80,24 +81,31 @@ struct GemmI4Params {
   int group_m;         // tile order (gemm_tile_coords)
   int r_tail;          // tail K: 2 r_pad (X_hat L1 as hi | lo against L2^T | L2^T), 0 = none
   const uint16_t* sx;  // fp16 [K/64][M_pad]
-  const float4* swc;   // [K/64][N_pad/2]: (s_w[2i] / 16, s_w[2i+1] / 16, c[2i], c[2i+1])
+  const float* sw16;   // [K/64][N_pad]: s_w / 16 (exact)
   int M_pad, N_pad;
   const __nv_bfloat16* bias;
   __nv_bfloat16* Y;
   long long budget;
 };
 
-__device__ __forceinline__ void tmem_st32_const(uint32_t taddr, uint32_t v) {
+// 64 consecutive 32-bit TMEM columns of this warp's 32 lanes into 64 registers.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
   asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-      "{%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, "
-      "%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1};" ::"r"(taddr),
-      "r"(v)
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, "
+      "%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, "
+      "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+        "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
+        "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
+        "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr)
       : "memory");
-}
-
-__device__ __forceinline__ void tmem_wait_st() {
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 __device__ __forceinline__ unsigned long long f2_pack(float a, float b) {
@@ -137,31 +145,6 @@ __device__ __forceinline__ uint2 i4_unpack8(uint32_t w) {
   return make_uint2((w << 4) & 0xF0F0F0F0u, w & 0xF0F0F0F0u);
 }
 
-// One drain warp's share of unpacking step u: wait for the stage's copies,
-// turn 8 packed bytes (16 codes) of B into the MMA layout (64-byte rows,
-// 64-byte swizzle: 16-byte chunk c of row r at c ^ ((r >> 1) & 3)), and
-// arrive on the stage's `unpacked` barrier.  Tail steps only arrive.
-__device__ __forceinline__ void i4_unpack_step(int u, uint8_t* smem, uint64_t* full, uint64_t* unpacked,
-                                               int steps_per_tile, int groups, uint32_t u_src, uint32_t u_dst,
-                                               long long budget, volatile int* abort_flag, bool& ok,
-                                               uint32_t lane) {
-  const int s = u % kI4Stages;
-  if (ok && !warp_wait(&full[s], (u / kI4Stages) & 1, budget, abort_flag)) {
-    if (lane == 0) raise_error(kErrWaitGemm);
-    *abort_flag = 1;
-    ok = false;
-  }
-  if (ok && (u % steps_per_tile) < groups) {
-    uint8_t* st = smem + s * kI4StageBytes;
-    const uint2 w = *reinterpret_cast<const uint2*>(st + u_src);
-    const uint2 a = i4_unpack8(w.x), b = i4_unpack8(w.y);
-    *reinterpret_cast<uint4*>(st + u_dst) = make_uint4(a.x, a.y, b.x, b.y);
-    fence_proxy_async_smem();
-  }
-  __syncwarp();
-  if (lane == 0) mbar_arrive(&unpacked[s]);
-}
-
 __global__ void __launch_bounds__(kI4Threads, 1)
     gemm_int4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_bp,
                      const __grid_constant__ CUtensorMap tm_xl1,
@@ -170,7 +153,7 @@ __global__ void __launch_bounds__(kI4Threads, 1)
   uint8_t* smem = align_smem_1024(smem_raw);
   constexpr int S = kI4Stages;
   constexpr int NB = kI4Bufs;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kI4StageBytes * S);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kI4ConstOff + 8192);
   uint64_t* unpacked = full + S;    // [S]: B of the stage is in its MMA layout
   uint64_t* empty = unpacked + S;
   uint64_t* pfull = empty + S;      // [NB]
@@ -195,7 +178,7 @@ __global__ void __launch_bounds__(kI4Threads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&unpacked[s], kI4EpiWarps);
+      mbar_init(&unpacked[s], kI4UnpackWarps);
       mbar_init(&empty[s], 1 + kI4EpiWarps);
     }
     for (int b = 0; b < NB; ++b) {
@@ -206,6 +189,19 @@ __global__ void __launch_bounds__(kI4Threads, 1)
     *abort_flag = 0;
     fence_barrier_init();
   }
+  if (threadIdx.x < 256) {
+    // The offset MMA's operands, 128 x 16 bf16 each, K-major, 32-byte swizzle
+    // (16-byte chunk c of row r at c ^ ((r >> 2) & 1)): A rows (1, 0, ..., 0)
+    // and B rows (1.5 * 2^23, 0, ..., 0), so that D = A B^T is 1.5 * 2^23 in
+    // every element, exactly.
+    const uint32_t t = threadIdx.x & 127u;
+    uint8_t* rowp = smem + kI4ConstOff + (threadIdx.x < 128 ? 0u : 4096u) + t * 32;
+    const uint32_t first = threadIdx.x < 128 ? 0x3F80u : 0x4B40u;   // bf16 1.0 / 1.5 * 2^23
+    const uint32_t c0 = (t >> 2) & 1u;                              // physical chunk of k = 0 .. 7
+    *reinterpret_cast<uint4*>(rowp + (c0 << 4)) = make_uint4(first, 0u, 0u, 0u);
+    *reinterpret_cast<uint4*>(rowp + ((c0 ^ 1u) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+    fence_proxy_async_smem();
+  }
   if (warp == 1) {
     tmem_alloc(tmem_holder, 512);
     tmem_relinquish();
@@ -214,16 +210,6 @@ __global__ void __launch_bounds__(kI4Threads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
-  if (warp >= 2) {
-    // every partial buffer starts out holding the conversion offset
-    const uint32_t q = warp & 3u, h = (warp - 2) >> 2;
-    for (int b = 0; b < NB; ++b)
-      tmem_st32_const(tmem_base + ((q * 32u) << 16) + kI4BN * b + 32u * h, kI4Magic);
-    tmem_wait_st();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
   griddep_wait();   // the activation codes, scales and XL1 come from the previous kernel
 
   if (warp == 0) {
@@ -234,7 +220,7 @@ __global__ void __launch_bounds__(kI4Threads, 1)
         prefetch_tmap(&tm_xl1);
         prefetch_tmap(&tm_l2t);
       }
-      const uint32_t main_tx = kI4BM * 64 + kI4BN * 32 + kI4BM * 2 + (kI4BN / 2) * 16;
+      const uint32_t main_tx = kI4BM * 64 + kI4BN * 32 + kI4BM * 2 + kI4BN * 4;
       const uint32_t lr_tx = (kI4BM + kI4BN) * lr_cols * 2;
       int it = 0;
       bool ok = true;
@@ -258,13 +244,12 @@ __global__ void __launch_bounds__(kI4Threads, 1)
             tma_load_2d(st + kI4AOff, &tm_a, &full[s], g * kI4BK, m0);
             tma_load_2d(st + kI4BpOff, &tm_bp, &full[s], g * (kI4BK / 2), n0);
             bulk_load(st + kI4SxOff, p.sx + static_cast<size_t>(g) * p.M_pad + m0, kI4BM * 2, &full[s]);
-            bulk_load(st + kI4SwOff, p.swc + static_cast<size_t>(g) * (p.N_pad / 2) + n0 / 2, (kI4BN / 2) * 16,
-                      &full[s]);
+            bulk_load(st + kI4SwOff, p.sw16 + static_cast<size_t>(g) * p.N_pad + n0, kI4BN * 4, &full[s]);
           } else {
             const int c = step - p.groups;
             mbar_arrive_expect_tx(&full[s], lr_tx);
-            tma_load_2d(st + kI4AOff, &tm_xl1, &full[s], c * 32, m0);
-            tma_load_2d(st + kI4BOff, &tm_l2t, &full[s], c * 32, n0);
+            tma_load_2d(st + kI4AOff, &tm_xl1, &full[s], c * 64, m0);
+            tma_load_2d(st + kI4BOff, &tm_l2t, &full[s], c * 64, n0);
           }
         }
       }
@@ -278,6 +263,7 @@ __global__ void __launch_bounds__(kI4Threads, 1)
       const uint32_t idesc_main = idesc_s8_s32(kI4BM, kI4BN);
       const uint32_t idesc_lr = idesc_bf16_f32(kI4BM, kI4BN);
       const uint32_t lr_row_bytes = static_cast<uint32_t>(lr_cols) * 2;
+      const uint32_t c_a = smem_u32(smem + kI4ConstOff), c_b = c_a + 4096u;
       for (int it = 0; it < total_steps; ++it) {
         const int s = it % S;
         const uint32_t ph = (it / S) & 1;
@@ -296,7 +282,9 @@ __global__ void __launch_bounds__(kI4Threads, 1)
         const uint32_t a0 = smem_u32(st + kI4AOff), b0 = smem_u32(st + kI4BOff);
         const uint32_t d = tmem_base + kI4BN * b;
         if (!tail) {
-          // accumulate onto the buffer's conversion offset
+          // the buffer := 1.5 * 2^23 (one bf16 MMA of the constant tiles), then
+          // the group's int8 products accumulate onto that offset
+          mma_bf16(d, make_kmajor_desc(c_a, 32), make_kmajor_desc(c_b, 32), idesc_lr, 0u);
 #pragma unroll
           for (int j = 0; j < 2; ++j)
             mma_i8(d, make_kmajor_desc(a0 + 32 * j, 64), make_kmajor_desc(b0 + 32 * j, 64), idesc_main, 1u);
@@ -310,33 +298,54 @@ __global__ void __launch_bounds__(kI4Threads, 1)
       }
       tc_commit(mma_done);
     }
-  } else {
-    // ------------------------------------------------ unpack + drain / epilogue
-    const uint32_t d = warp - 2;               // 0 .. 15
-    const uint32_t q = warp & 3u;              // TMEM lane quarter this warp may access
-    const uint32_t h = d >> 2;                 // 32-column slice of the tile
-    const uint32_t row = q * 32 + lane;
-    // unpack share: 8 packed bytes (16 codes) of B row ur, quarter uq
-    const uint32_t ut = d * 32 + lane;         // 0 .. 511
-    const uint32_t ur = ut >> 2, uq = ut & 3u;
-    const uint32_t u_src = kI4BpOff + ur * 32 + uq * 8;
-    const uint32_t u_dst = kI4BOff + ur * 64 + ((uq ^ ((ur >> 1) & 3u)) << 4);   // 64-byte swizzle
+  } else if (warp >= 2 + kI4EpiWarps) {
+    // ------------------------------------------------------------ unpack
+    // Two warps (64 lanes) turn each landed stage's packed B (128 columns x 32
+    // bytes) into the MMA layout: 64-byte rows, 64-byte swizzle (16-byte chunk
+    // c of row r at c ^ ((r >> 1) & 3)).  Lane task t: 16 packed bytes (32
+    // codes) = half h of row r -> unpacked chunks 2 h and 2 h + 1.
+    const uint32_t ul = (warp - 2 - kI4EpiWarps) * 32 + lane;   // 0 .. 63
     bool ok = true;
-
-    for (int u = 0; u < kI4Ahead && u < total_steps; ++u)
-      i4_unpack_step(u, smem, full, unpacked, steps_per_tile, p.groups, u_src, u_dst, p.budget, abort_flag, ok, lane);
+    for (int u = 0; u < total_steps; ++u) {
+      const int s = u % S;
+      if (ok && !warp_wait(&full[s], (u / S) & 1, p.budget, abort_flag)) {
+        if (lane == 0) raise_error(kErrWaitGemm);
+        *abort_flag = 1;
+        ok = false;
+      }
+      if (ok && (u % steps_per_tile) < p.groups) {
+        uint8_t* st = smem + s * kI4StageBytes;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t t = ul + 64u * i;           // 0 .. 255
+          const uint32_t r = t >> 1, hh = t & 1u;
+          const uint4 w = *reinterpret_cast<const uint4*>(st + kI4BpOff + r * 32 + hh * 16);
+          const uint2 a = i4_unpack8(w.x), b = i4_unpack8(w.y), c = i4_unpack8(w.z), d = i4_unpack8(w.w);
+          const uint32_t sw = (r >> 1) & 3u;
+          uint8_t* row = st + kI4BOff + r * 64;
+          *reinterpret_cast<uint4*>(row + (((2 * hh) ^ sw) << 4)) = make_uint4(a.x, a.y, b.x, b.y);
+          *reinterpret_cast<uint4*>(row + (((2 * hh + 1) ^ sw) << 4)) = make_uint4(c.x, c.y, d.x, d.y);
+        }
+        fence_proxy_async_smem();
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&unpacked[s]);
+    }
+  } else {
+    // ------------------------------------------------------------ drain / epilogue
+    const uint32_t q = warp & 3u;              // TMEM lane quarter this warp may access
+    const uint32_t h = (warp - 2) >> 2;        // 64-column half of the tile
+    const uint32_t row = q * 32 + lane;
+    bool ok = true;
     int it = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
       int m_blk, n_blk;
       gemm_tile_coords(p.m_tiles, p.n_tiles, p.group_m, tile, m_blk, n_blk);
       const int m = m_blk * kI4BM + static_cast<int>(row);
-      unsigned long long acc[16];   // 32 fp32 accumulators, pairs of adjacent columns
+      unsigned long long acc[32];   // 64 fp32 accumulators, pairs of adjacent columns
 #pragma unroll
-      for (int j = 0; j < 16; ++j) acc[j] = 0ull;
+      for (int j = 0; j < 32; ++j) acc[j] = 0ull;
       for (int step = 0; step < steps_per_tile; ++step, ++it) {
-        if (it + kI4Ahead < total_steps)
-          i4_unpack_step(it + kI4Ahead, smem, full, unpacked, steps_per_tile, p.groups, u_src, u_dst, p.budget,
-                         abort_flag, ok, lane);
         const int s = it % S;
         const int b = it % NB;
         const uint32_t pph = (it / NB) & 1;
@@ -348,34 +357,32 @@ __global__ void __launch_bounds__(kI4Threads, 1)
         if (ok) {
           tc_fence_after();
           const uint8_t* st = smem + s * kI4StageBytes;
-          const uint32_t taddr = tmem_base + ((q * 32u) << 16) + kI4BN * b + 32u * h;
+          const uint32_t taddr = tmem_base + ((q * 32u) << 16) + kI4BN * b + 64u * h;
           const bool main_step = step < p.groups;
+          const unsigned long long magic2 = f2_pack(12582912.0f, 12582912.0f);
           unsigned long long sx2 = 0ull;
           if (main_step) {
             const float sx = __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(st + kI4SxOff)[row]));
             sx2 = f2_pack(sx, sx);
           }
-          const ulonglong2* swc = reinterpret_cast<const ulonglong2*>(st + kI4SwOff) + 16 * h;
-          // two halves of 16 columns (16 loaded values live at a time)
+          const unsigned long long* sw2 = reinterpret_cast<const unsigned long long*>(st + kI4SwOff) + 32 * h;
+          uint32_t r[64];
+          tmem_ld64(taddr, r);   // one TMEM round trip per group
+          tmem_wait_ld();
+          if (main_step) {
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            uint32_t r[16];
-            tmem_ld16(taddr + 16u * half, r);
-            tmem_wait_ld();
-            if (main_step) {
-#pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                const ulonglong2 wc = swc[8 * half + j];   // (s_w / 16, c) of columns 32 h + 16 half + 2 j, + 1
-                acc[8 * half + j] =
-                    f2_fma(f2_fma(u2_pack(r[2 * j], r[2 * j + 1]), wc.x, wc.y), sx2, acc[8 * half + j]);
-              }
-            } else {
-#pragma unroll
-              for (int j = 0; j < 8; ++j) acc[8 * half + j] = f2_add(acc[8 * half + j], u2_pack(r[2 * j], r[2 * j + 1]));
+            for (int j = 0; j < 32; ++j) {
+              const unsigned long long w2 = sw2[j];   // s_w / 16 of columns 64 h + 2 j, + 1
+              unsigned long long d, sc, rr;
+              asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(u2_pack(r[2 * j], r[2 * j + 1])), "l"(magic2));
+              asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(sc) : "l"(sx2), "l"(w2));
+              asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(rr) : "l"(d), "l"(sc), "l"(acc[j]));
+              acc[j] = rr;
             }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) acc[j] = f2_add(acc[j], u2_pack(r[2 * j], r[2 * j + 1]));
           }
-          tmem_st32_const(taddr, kI4Magic);   // the buffer holds the offset again
-          tmem_wait_st();
         }
         tc_fence_before();
         __syncwarp();
@@ -385,12 +392,12 @@ __global__ void __launch_bounds__(kI4Threads, 1)
         }
       }
       if (!ok) continue;   // keep walking the steps so the barriers stay matched
-      // bias, bf16, store: 32 columns of this row
-      const int n_base = n_blk * kI4BN + 32 * static_cast<int>(h);
+      // bias, bf16, store: 64 columns of this row
+      const int n_base = n_blk * kI4BN + 64 * static_cast<int>(h);
       if (m < p.M) {
         __nv_bfloat16* yrow = p.Y + static_cast<size_t>(m) * p.N;
 #pragma unroll
-        for (int j = 0; j < 32; j += 8) {
+        for (int j = 0; j < 64; j += 8) {
           const int n = n_base + j;
           if (n < p.N) {
             float bb[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};

@@ -326,19 +326,14 @@ __global__ void quant_weight_int4_kernel(const float* __restrict__ R, int K, int
   sf[static_cast<size_t>(g) * N_pad + n] = sh;
 }
 
-// The INT4 GEMM's per-column constants, derived from the fp16 weight scales:
-// for the column pair (2i, 2i + 1) of group g one float4
-//   (s_w[2i] / 16, s_w[2i+1] / 16, -1.5 * 2^19 * s_w[2i], -1.5 * 2^19 * s_w[2i+1]),
-// all exact (an fp16 value times a power of two, or times 3 * 2^18).  With the
-// partial read back as v = 1.5 * 2^23 + 16 P, fma(v, s_w / 16, c) = P s_w.
-__global__ void int4_column_consts_kernel(const uint16_t* __restrict__ sf, int groups, int N_pad,
-                                          float4* __restrict__ swc) {
-  const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;   // (g, column pair)
-  if (i >= static_cast<size_t>(groups) * (N_pad / 2)) return;
-  const size_t g = i / (N_pad / 2), c2 = i % (N_pad / 2);
-  const float s0 = __half2float(__ushort_as_half(sf[g * N_pad + 2 * c2]));
-  const float s1 = __half2float(__ushort_as_half(sf[g * N_pad + 2 * c2 + 1]));
-  swc[i] = make_float4(s0 * 0.0625f, s1 * 0.0625f, s0 * -786432.0f, s1 * -786432.0f);
+// The INT4 GEMM's per-column scale, derived from the fp16 weight scales:
+// s_w / 16 for group g and column n (exact: an fp16 value times 2^-4).  The
+// GEMM reads the partial as 16 P (its weight operand is 16 q) and scales it by
+// s_x * (s_w / 16).
+__global__ void int4_column_scales_kernel(const uint16_t* __restrict__ sf, size_t count, float* __restrict__ sw16) {
+  const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;   // g * N_pad + n
+  if (i >= count) return;
+  sw16[i] = __half2float(__ushort_as_half(sf[i])) * 0.0625f;
 }
 
 // FP4 g32: one E4M3 scale per 32 values of K, stored in both 16-value slots of

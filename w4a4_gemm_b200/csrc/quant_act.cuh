@@ -107,8 +107,8 @@ __host__ __device__ inline QuantSmem quant_smem_layout(int fmt, int r_pad, int S
   L.il_off = L.l1_off + 2 * S * r_pad * 128;               // 2 S r_pad rows of 128 bytes (hi, lo)
   uint32_t sb = L.il_off + S * kQuantBK * 4;
   L.stage_bytes = (sb + 1023u) & ~1023u;
-  L.stg_bytes = kQuantTileRows * quant_code_row_bytes(fmt);   // one staging buffer
-  const uint32_t stg_total = 2u * kQuantGroups * L.stg_bytes;
+  L.stg_bytes = 32u * quant_code_row_bytes(fmt);           // one staging buffer: a warp's 32 rows
+  const uint32_t stg_total = 2u * kQuantWarps * L.stg_bytes;
   L.stages = (kQuantSmemBudget - stg_total) / L.stage_bytes;
   if (L.stages > static_cast<uint32_t>(kQuantMaxStages)) L.stages = kQuantMaxStages;
   if (L.stages < 3u) {
@@ -246,17 +246,19 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
     // groups; stage buffer b always serves group b mod G, see quant_smem_layout);
     // its warp of lane quarter q quantizes rows 32 q .. 32 q + 31 of the
     // stacked tile, one lane per row over the whole 64-wide sub-tile: four
-    // independent NVFP4 groups of 16 (or one INT4 group of 64) per lane.  The
-    // group stages its 128 rows of codes in shared memory and one of its
-    // threads writes them with a TMA store per sub-tile; each lane writes its
-    // row's scales itself (one 4-byte word or one fp16).  A failed wait does
-    // not leave the loop: the group's named barriers stay matched.
+    // independent NVFP4 groups of 16 (or one INT4 group of 64) per lane.  Each
+    // warp stages its own 32 rows of codes in shared memory (two buffers, used
+    // in turn) and its lane 0 writes them with one TMA store per sub-tile the
+    // rows belong to (boxes of min(32, BM) rows), so no barrier ties the warps
+    // of a group together; each lane writes its row's scales itself (one 4-byte
+    // word or one fp16).
     constexpr uint32_t RB = quant_code_row_bytes(FMT);   // code bytes per row
     const uint32_t q = warp & 3u;
     const int grp = static_cast<int>(warp - 2) >> 2;
-    const bool leader = warp == static_cast<uint32_t>(2 + 4 * grp) && lane == 0;
-    const uint32_t bar_free = 1 + 2 * grp, bar_full = 2 + 2 * grp;   // named barriers of the group
     const uint32_t R = q * 32 + lane;          // row of the stacked A tile
+    const int st_boxes = BM < 32 ? 2 : 1;                               // code stores per stage
+    const int st_j0 = static_cast<int>(q * 32) / BM;                    // sub-tile of the first box
+    const int st_m0 = m0 + static_cast<int>(q * 32) % BM;               // its first token row
     const int j = static_cast<int>(R) / BM;    // K sub-tile
     const int m = m0 + static_cast<int>(R) % BM;
     const bool row_ok = m < p.M;
@@ -350,14 +352,14 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
         }
         sfw = sh;
       }
-      // codes -> this group's staging buffer (rows of RB bytes in the TMA swizzle
-      // of that row length: 16-byte chunk c of row R sits at c ^ ((R >> sh) & mask))
-      uint8_t* buf = smem + L.stg_off + (2 * grp + (use & 1)) * L.stg_bytes;
-      if (leader) bulk_wait_group_read<1>();   // its store from two uses ago has read it
-      named_bar_sync(bar_free, 128);
+      // codes -> this warp's staging buffer (rows of RB bytes in the TMA swizzle
+      // of that row length: 16-byte chunk c of row r sits at c ^ ((r >> sh) & mask))
+      uint8_t* buf = smem + L.stg_off + (2 * (warp - 2) + (use & 1)) * L.stg_bytes;
+      if (lane == 0) bulk_wait_group_read<1>();   // its store from two uses ago has read it
+      __syncwarp();
       {
-        const uint32_t row_addr = smem_u32(buf) + R * RB;
-        const uint32_t sw = RB == 32 ? ((R >> 2) & 1u) : ((R >> 1) & 3u);
+        const uint32_t row_addr = smem_u32(buf) + lane * RB;
+        const uint32_t sw = RB == 32 ? ((lane >> 2) & 1u) : ((lane >> 1) & 3u);
 #pragma unroll
         for (uint32_t c = 0; c < RB / 16; ++c)
           asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row_addr + ((c ^ sw) << 4)),
@@ -365,11 +367,13 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
                        : "memory");
       }
       fence_proxy_async_smem();
-      named_bar_sync(bar_full, 128);
-      if (leader && ok) {
-        for (int jj = 0; jj < S; ++jj) {
-          const int kc = i * S + jj;
-          if (kc * kQuantBK < p.K) tma_store_2d(&tm_codes, buf + jj * BM * RB, kc * RB, m0);
+      __syncwarp();
+      if (lane == 0 && ok) {
+        // rows 32 q .. 32 q + 31 of the stacked tile: one box of 32 rows, or
+        // (BM = 16) two boxes in consecutive sub-tiles
+        for (int b = 0; b < st_boxes; ++b) {
+          const int kc = i * S + st_j0 + b;
+          if (kc * kQuantBK < p.K) tma_store_2d(&tm_codes, buf + b * 16 * RB, kc * RB, st_m0);
         }
         bulk_commit_group();
       }
@@ -384,7 +388,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
         }
       }
     }
-    if (leader) bulk_wait_group_all();
+    if (lane == 0) bulk_wait_group_all();
   }
   __syncwarp();
 

@@ -49,7 +49,7 @@ struct svdq_weights {
   uint8_t* wsf = nullptr;     // NVFP4: atoms [N_pad/128][sf_kcols][512]; INT4: fp16 [K/64][N_pad]
   uint8_t* wsf192 = nullptr;  // FP4: the same atoms regrouped per 192-column tile [2 n192][sf_kcols][512]
   int n192 = 0;               // FP4: 192-column tiles of N
-  float4* wswc = nullptr;     // INT4: per column pair (s_w / 16, c) constants of the GEMM's drain
+  float* wsw16 = nullptr;     // INT4: s_w / 16 per group and column [K/64][N_pad], read by the GEMM
   __nv_bfloat16* l1t = nullptr;  // r_pad x K
   __nv_bfloat16* l1st = nullptr; // 2 r_pad x K: (diag(1/lambda) L1)^T as hi rows then lo rows, read by
                                  // the activation kernel
@@ -419,7 +419,7 @@ void free_weights(svdq_weights* w) {
   cudaFree(w->wcodes);
   cudaFree(w->wsf);
   cudaFree(w->wsf192);
-  cudaFree(w->wswc);
+  cudaFree(w->wsw16);
   cudaFree(w->l1t);
   cudaFree(w->l1st);
   cudaFree(w->l2t);
@@ -462,9 +462,9 @@ int alloc_weights(svdq_weights* w, cudaStream_t st) {
     SVDQ_CUDA(cudaMemsetAsync(w->wsf192, 0, sf192, st));
   }
   if (w->fmt == SVDQ_INT4) {
-    const size_t swc = static_cast<size_t>(w->K / 64) * (w->N_pad / 2) * sizeof(float4);
-    if (cudaMalloc(&w->wswc, swc) != cudaSuccess) return SVDQ_ERR_ALLOC;
-    SVDQ_CUDA(cudaMemsetAsync(w->wswc, 0, swc, st));
+    const size_t sw16 = static_cast<size_t>(w->K / 64) * w->N_pad * sizeof(float);
+    if (cudaMalloc(&w->wsw16, sw16) != cudaSuccess) return SVDQ_ERR_ALLOC;
+    SVDQ_CUDA(cudaMemsetAsync(w->wsw16, 0, sw16, st));
   }
   if (w->r_pad > 0) {
     if (cudaMalloc(&w->l1t, static_cast<size_t>(w->r_pad) * w->K * 2) != cudaSuccess ||
@@ -510,12 +510,12 @@ int build_l2t2(svdq_weights* w, cudaStream_t st) {
 // Scale layouts derived from the weight scales in w->wsf, redone whenever
 // those change (quantization, or a refinement restoring an earlier iterate):
 // FP4 formats: the atoms regrouped per 192-column tile of the pair GEMM;
-// INT4: the drain's per-column-pair constants.
+// INT4: the GEMM's s_w / 16 per group and column.
 int derive_scale_layouts(svdq_weights* w, cudaStream_t st) {
   if (w->fmt == SVDQ_INT4) {
-    const size_t n = static_cast<size_t>(w->K / 64) * (w->N_pad / 2);
-    int4_column_consts_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
-        reinterpret_cast<const uint16_t*>(w->wsf), w->K / 64, w->N_pad, w->wswc);
+    const size_t n = static_cast<size_t>(w->K / 64) * w->N_pad;
+    int4_column_scales_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
+        reinterpret_cast<const uint16_t*>(w->wsf), n, w->wsw16);
     SVDQ_CHECK_LAUNCH();
   }
   if (is_fp4(w->fmt)) {
@@ -1055,10 +1055,11 @@ SVDQ_API int svdq_quantize_act(const svdq_weights* w, const void* X, int M, void
   CUtensorMap tm_x, tm_codes;
   if ((rc = make_map(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, w->K, M, kQuantBK, BM)))
     return rc;
-  // codes: NVFP4 M x K/2 packed E2M1, INT4 M x K int8; one box = one sub-tile's BM rows
+  // codes: NVFP4 M x K/2 packed E2M1, INT4 M x K int8; one box = a warp's
+  // rows of one sub-tile, min(32, BM) rows
   const uint32_t rb = quant_code_row_bytes(w->fmt);
   if ((rc = make_map(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base + L.codes_off,
-                     is_fp4(w->fmt) ? w->K / 2 : w->K, M, rb, BM)))
+                     is_fp4(w->fmt) ? w->K / 2 : w->K, M, rb, std::min(BM, 32))))
     return rc;
   QuantParams p;
   p.M = M;
@@ -1246,7 +1247,7 @@ SVDQ_API int svdq_linear(const svdq_weights* w, const void* ws, int M, void* Y, 
     p.group_m = group_m;
     p.r_tail = 2 * w->r_pad;
     p.sx = reinterpret_cast<const uint16_t*>(base + L.sf_off);
-    p.swc = w->wswc;
+    p.sw16 = w->wsw16;
     p.M_pad = L.M_pad;
     p.N_pad = w->N_pad;
     p.bias = w->bias;
