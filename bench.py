@@ -62,11 +62,11 @@ def peaks():
 
 
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
-# one ncu capture of `bench.py --steps 3 --warmup 3 --no-cpu-baseline
-# --no-extras` (the summaries under profiles/), keyed by kernel, workload and a
-# fingerprint of the kernel's sources: a kernel changed since the capture
-# reports null.  Y of the QKV layer (85 MB) is still mostly dirty in the
-# 126 MB L2 when the GEMM ends, so its write traffic is below Y's size.
+# one ncu capture of `bench.py [--config ...] --steps 3 --warmup 3
+# --no-cpu-baseline --no-extras` (the summaries under profiles/), keyed by
+# kernel, workload and a fingerprint of the kernel's sources: a kernel changed
+# since the capture reports null.  Part of Y is still dirty in the 126 MB L2
+# when a GEMM ends, so the write traffic is below Y's size.
 # Vendor figures for one B200, for the fractions reported beside the measured
 # denominators: dense FP4 and INT8 tensor peaks (NVIDIA's doubled figures are
 # with 2:4 sparsity) and the HBM3e bandwidth.
@@ -74,12 +74,9 @@ DATASHEET_FP4_TFLOPS = 9000.0
 DATASHEET_INT8_TOPS = 4500.0
 NOMINAL_HBM_GBS = 8000.0
 NCU_TRAFFIC = {
-    ("gemm_nvfp4_pair_kernel", "c2_qkv/qkv", 4608, "nvfp4"): (63905536, "ab2d6aed3c92a25a"),
-    ("gemm_nvfp4_pair_kernel", "c5_block/fc2", 16384, "nvfp4"): (221753856, "ab2d6aed3c92a25a"),
-    ("quant_act_kernel", "c2_qkv/qkv", 4608, "nvfp4"): (28561408, "97712fa48aaac990"),
-    ("quant_act_kernel", "c5_block/fc2", 16384, "nvfp4"): (498574592, "97712fa48aaac990"),
-    ("gemm_int4_kernel", "c4_int4_lora/proj", 4608, "int4"): (26690816, "4e6665236c6ea587"),
-    ("gemm_w8a8_kernel", "c2_qkv/qkv", 4608, "w8a8"): (100859392, "2d56831f05842901"),
+    ("gemm_nvfp4_pair_kernel", "c5_block/fc2", 16384, "nvfp4"): (221565696, "97027a9e62004fde"),
+    ("quant_act_kernel", "c5_block/fc2", 16384, "nvfp4"): (499809792, "21b4a8dae4db57e2"),
+    ("gemm_int4_kernel", "c4_int4_lora/proj", 4608, "int4"): (21903616, "69b145f7bae51b3c"),
 }
 KERNEL_SOURCES = {
     "gemm_nvfp4_kernel": ("gemm_nvfp4.cuh", "svdq_ptx.cuh", "svdq_formats.cuh"),

@@ -19,16 +19,16 @@
 // activation kernel) are stored in that same order, so every product q_x q_w
 // meets its partner and the group's integer sum is 16 P, P = sum q_x q_w.
 //
-// The partial reaches the drain already as fp32: before a group's two int8
-// MMAs the MMA issuer writes 1.5 * 2^23 into the partial buffer with one bf16
-// MMA of two constant tiles (A rows (1, 0, ...), B rows (1.5 * 2^23, 0, ...),
-// accumulate off), and the int8 MMAs accumulate onto that offset's bits, so the
-// bits read back are those of v = 1.5 * 2^23 + 16 P exactly (|16 P| <= 16 * 64
-// * 49 < 2^22).  The drain only reads TMEM.  Per output pair and group it issues
-// three packed fp32 operations:
-//   d = v - 1.5 * 2^23   (= 16 P, exact)
-//   s = s_x * (s_w / 16) (exact: two fp16 values and a power of two)
-//   acc = d * s + acc    (one rounding)
+// The partial reaches the drain already as an fp32 value: before a group's two
+// int8 MMAs the MMA issuer writes 1.5 * 2^23 into the partial buffer with one
+// bf16 MMA of two constant tiles (A rows (1, 0, ...), B rows (1.5 * 2^23, 0,
+// ...), accumulate off); the int8 MMAs accumulate onto that offset's bits, which
+// are then the bits of the fp32 value 1.5 * 2^23 + 16 P (|16 P| <= 16 * 64 * 49
+// < 2^22); a second bf16 MMA (B rows -1.5 * 2^23, accumulate on) subtracts the
+// offset in fp32, exactly, leaving 16 P.  The drain only reads TMEM, and per
+// output pair and group issues two packed fp32 operations:
+//   s   = s_x * (s_w / 16)   (exact: two fp16 values and a power of two)
+//   acc = 16 P * s + acc     (one rounding)
 // with s_w / 16 prepared per weight column beside the fp16 scales.
 //
 //   warp 0      : TMA producer (A 128 x 64 int8, the packed B 128 x 32 bytes,
@@ -61,9 +61,10 @@ constexpr uint32_t kI4SxOff = kI4BpOff + kI4BN * 32;       // 20480: activation 
 constexpr uint32_t kI4SwOff = kI4SxOff + kI4BM * 2;        // s_w / 16 of the tile's 128 columns
 constexpr uint32_t kI4StageBytes = 38912;
 constexpr int kI4Stages = 5;
-constexpr uint32_t kI4ConstOff = kI4StageBytes * kI4Stages;  // the offset MMA's two constant 128 x 16 bf16 tiles
+constexpr uint32_t kI4ConstOff = kI4StageBytes * kI4Stages;  // the offset MMAs' constant 128 x 16 bf16 tiles:
+                                                             // A = (1, 0, ...), B = (+-1.5 * 2^23, 0, ...)
 constexpr uint32_t kI4BarBytes = 512;                      // 3 S + 2 NB + 1 mbarriers, TMEM address, flag
-constexpr uint32_t kI4SmemBytes = kI4ConstOff + 8192 + kI4BarBytes + 1024;
+constexpr uint32_t kI4SmemBytes = kI4ConstOff + 12288 + kI4BarBytes + 1024;
 static_assert(kI4SwOff + kI4BN * 4 <= kI4StageBytes, "stage layout");
 static_assert((3 * kI4Stages + 2 * kI4Bufs + 1) * 8 + 8 <= kI4BarBytes, "barrier area");
 
@@ -133,6 +134,12 @@ __device__ __forceinline__ unsigned long long f2_fma(unsigned long long a, unsig
   return r;
 }
 
+__device__ __forceinline__ unsigned long long f2_mul(unsigned long long a, unsigned long long b) {
+  unsigned long long r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
 __device__ __forceinline__ unsigned long long f2_add(unsigned long long a, unsigned long long b) {
   unsigned long long r;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
@@ -153,7 +160,7 @@ __global__ void __launch_bounds__(kI4Threads, 1)
   uint8_t* smem = align_smem_1024(smem_raw);
   constexpr int S = kI4Stages;
   constexpr int NB = kI4Bufs;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kI4ConstOff + 8192);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kI4ConstOff + 12288);
   uint64_t* unpacked = full + S;    // [S]: B of the stage is in its MMA layout
   uint64_t* empty = unpacked + S;
   uint64_t* pfull = empty + S;      // [NB]
@@ -189,14 +196,14 @@ __global__ void __launch_bounds__(kI4Threads, 1)
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (threadIdx.x < 256) {
-    // The offset MMA's operands, 128 x 16 bf16 each, K-major, 32-byte swizzle
-    // (16-byte chunk c of row r at c ^ ((r >> 2) & 1)): A rows (1, 0, ..., 0)
-    // and B rows (1.5 * 2^23, 0, ..., 0), so that D = A B^T is 1.5 * 2^23 in
-    // every element, exactly.
-    const uint32_t t = threadIdx.x & 127u;
-    uint8_t* rowp = smem + kI4ConstOff + (threadIdx.x < 128 ? 0u : 4096u) + t * 32;
-    const uint32_t first = threadIdx.x < 128 ? 0x3F80u : 0x4B40u;   // bf16 1.0 / 1.5 * 2^23
+  if (threadIdx.x < 384) {
+    // The offset MMAs' operands, 128 x 16 bf16 each, K-major, 32-byte swizzle
+    // (16-byte chunk c of row r at c ^ ((r >> 2) & 1)): A rows (1, 0, ..., 0),
+    // B rows (1.5 * 2^23, 0, ..., 0) and (-1.5 * 2^23, 0, ..., 0), so that
+    // D = A B^T is +-1.5 * 2^23 in every element, exactly.
+    const uint32_t t = threadIdx.x & 127u, which = threadIdx.x >> 7;
+    uint8_t* rowp = smem + kI4ConstOff + which * 4096u + t * 32;
+    const uint32_t first = which == 0 ? 0x3F80u : (which == 1 ? 0x4B40u : 0xCB40u);   // 1.0, +-1.5 * 2^23
     const uint32_t c0 = (t >> 2) & 1u;                              // physical chunk of k = 0 .. 7
     *reinterpret_cast<uint4*>(rowp + (c0 << 4)) = make_uint4(first, 0u, 0u, 0u);
     *reinterpret_cast<uint4*>(rowp + ((c0 ^ 1u) << 4)) = make_uint4(0u, 0u, 0u, 0u);
@@ -263,7 +270,7 @@ __global__ void __launch_bounds__(kI4Threads, 1)
       const uint32_t idesc_main = idesc_s8_s32(kI4BM, kI4BN);
       const uint32_t idesc_lr = idesc_bf16_f32(kI4BM, kI4BN);
       const uint32_t lr_row_bytes = static_cast<uint32_t>(lr_cols) * 2;
-      const uint32_t c_a = smem_u32(smem + kI4ConstOff), c_b = c_a + 4096u;
+      const uint32_t c_a = smem_u32(smem + kI4ConstOff), c_b = c_a + 4096u, c_bn = c_a + 8192u;
       for (int it = 0; it < total_steps; ++it) {
         const int s = it % S;
         const uint32_t ph = (it / S) & 1;
@@ -282,12 +289,15 @@ __global__ void __launch_bounds__(kI4Threads, 1)
         const uint32_t a0 = smem_u32(st + kI4AOff), b0 = smem_u32(st + kI4BOff);
         const uint32_t d = tmem_base + kI4BN * b;
         if (!tail) {
-          // the buffer := 1.5 * 2^23 (one bf16 MMA of the constant tiles), then
-          // the group's int8 products accumulate onto that offset
+          // the buffer := 1.5 * 2^23 (one bf16 MMA of the constant tiles); the
+          // group's int8 products accumulate onto that offset's bits, which are
+          // then the fp32 value 1.5 * 2^23 + 16 P; one more bf16 MMA adds
+          // -1.5 * 2^23 in fp32 (exact), leaving the fp32 value 16 P
           mma_bf16(d, make_kmajor_desc(c_a, 32), make_kmajor_desc(c_b, 32), idesc_lr, 0u);
 #pragma unroll
           for (int j = 0; j < 2; ++j)
             mma_i8(d, make_kmajor_desc(a0 + 32 * j, 64), make_kmajor_desc(b0 + 32 * j, 64), idesc_main, 1u);
+          mma_bf16(d, make_kmajor_desc(c_a, 32), make_kmajor_desc(c_bn, 32), idesc_lr, 1u);
         } else {
           for (int j = 0; j < lr_cols / 16; ++j)
             mma_bf16(d, make_kmajor_desc(a0 + 32 * j, lr_row_bytes), make_kmajor_desc(b0 + 32 * j, lr_row_bytes),
@@ -359,25 +369,23 @@ __global__ void __launch_bounds__(kI4Threads, 1)
           const uint8_t* st = smem + s * kI4StageBytes;
           const uint32_t taddr = tmem_base + ((q * 32u) << 16) + kI4BN * b + 64u * h;
           const bool main_step = step < p.groups;
-          const unsigned long long magic2 = f2_pack(12582912.0f, 12582912.0f);
           unsigned long long sx2 = 0ull;
           if (main_step) {
             const float sx = __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(st + kI4SxOff)[row]));
             sx2 = f2_pack(sx, sx);
           }
-          const unsigned long long* sw2 = reinterpret_cast<const unsigned long long*>(st + kI4SwOff) + 32 * h;
+          const ulonglong2* sw4 = reinterpret_cast<const ulonglong2*>(st + kI4SwOff) + 16 * h;
           uint32_t r[64];
           tmem_ld64(taddr, r);   // one TMEM round trip per group
           tmem_wait_ld();
           if (main_step) {
+            // acc += 16 P * (s_x * s_w / 16): the scale product and one fused
+            // multiply-add per column pair; s_w / 16 read four columns at a time
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const unsigned long long w2 = sw2[j];   // s_w / 16 of columns 64 h + 2 j, + 1
-              unsigned long long d, sc, rr;
-              asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(u2_pack(r[2 * j], r[2 * j + 1])), "l"(magic2));
-              asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(sc) : "l"(sx2), "l"(w2));
-              asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(rr) : "l"(d), "l"(sc), "l"(acc[j]));
-              acc[j] = rr;
+            for (int j = 0; j < 32; j += 2) {
+              const ulonglong2 w4 = sw4[j / 2];   // s_w / 16 of columns 64 h + 2 j .. + 3
+              acc[j] = f2_fma(u2_pack(r[2 * j], r[2 * j + 1]), f2_mul(sx2, w4.x), acc[j]);
+              acc[j + 1] = f2_fma(u2_pack(r[2 * j + 2], r[2 * j + 3]), f2_mul(sx2, w4.y), acc[j + 1]);
             }
           } else {
 #pragma unroll
