@@ -312,7 +312,7 @@ constexpr double kQuantFixedCycles = 10000.0;
 constexpr double kQuantExchangeCycles = 2000.0;
 constexpr double kQuantPerPeerCycles = 1000.0;
 constexpr double kQuantStageCycles = 800.0;
-constexpr double kQuantL1Cycles = 300.0;
+constexpr double kQuantL1Cycles = 400.0;   // refitted with the hi + lo factor (a forced-shape sweep on B200)
 std::atomic<int> g_forced_split{0};      // svdq_set_quant_split: 16 S + C; 0 = automatic
 std::atomic<int> g_forced_group_m{0};    // svdq_set_gemm_raster; 0 = automatic
 std::atomic<int> g_forced_gemm_kind{0};  // svdq_set_gemm_kernel; 0 = automatic, 1 = one CTA, 2 = CTA pairs,
