@@ -65,8 +65,10 @@ def peaks():
 # one ncu capture of `bench.py [--config ...] --steps 3 --warmup 3
 # --no-cpu-baseline --no-extras` (the summaries under profiles/), keyed by
 # kernel, workload and a fingerprint of the kernel's sources: a kernel changed
-# since the capture reports null.  Part of Y is still dirty in the 126 MB L2
-# when a GEMM ends, so the write traffic is below Y's size.
+# since the capture reports null.  Part of what a kernel writes is still
+# dirty in the 126 MB L2 when it ends (part of Y after a GEMM; at M = 4608 all
+# of the activation kernel's outputs), so write traffic is below the bytes
+# written.
 # Vendor figures for one B200, for the fractions reported beside the measured
 # denominators: dense FP4 and INT8 tensor peaks (NVIDIA's doubled figures are
 # with 2:4 sparsity) and the HBM3e bandwidth.
@@ -76,7 +78,10 @@ NOMINAL_HBM_GBS = 8000.0
 NCU_TRAFFIC = {
     ("gemm_nvfp4_pair_kernel", "c5_block/fc2", 16384, "nvfp4"): (221565696, "97027a9e62004fde"),
     ("quant_act_kernel", "c5_block/fc2", 16384, "nvfp4"): (499809792, "21b4a8dae4db57e2"),
-    ("gemm_int4_kernel", "c4_int4_lora/proj", 4608, "int4"): (21903616, "69b145f7bae51b3c"),
+    ("gemm_int4_kernel", "c4_int4_lora/proj", 4608, "int4"): (21903616, "94d8e85b38a51e4a"),
+    ("gemm_nvfp4_pair_kernel", "c2_qkv/qkv", 4608, "nvfp4"): (64266752, "97027a9e62004fde"),
+    ("quant_act_kernel", "c2_qkv/qkv", 4608, "nvfp4"): (28757760, "21b4a8dae4db57e2"),
+    ("gemm_w8a8_kernel", "c2_qkv/qkv", 4608, "w8a8"): (93856256, "7bfa1387a77d1a37"),
 }
 KERNEL_SOURCES = {
     "gemm_nvfp4_kernel": ("gemm_nvfp4.cuh", "svdq_ptx.cuh", "svdq_formats.cuh"),
