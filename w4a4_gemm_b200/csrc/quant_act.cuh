@@ -88,8 +88,8 @@ struct QuantSmem {
 };
 
 // Per stage: the stacked X tile, S slices of L1s^T hi then S of lo, and
-// 1/lambda.  After the stages: two code staging buffers (128 rows of codes)
-// per quantizer group.
+// 1/lambda.  After the stages: one code staging buffer (32 rows of codes) per
+// quantizer warp.
 // G groups take the stages in turn, and the buffer count is a multiple of G,
 // so stage buffer b always serves group b mod G; G is 4 or 3, whichever keeps
 // more of the buffers that fit (4 on a tie: the quantizers set the pace), or
@@ -108,7 +108,7 @@ __host__ __device__ inline QuantSmem quant_smem_layout(int fmt, int r_pad, int S
   uint32_t sb = L.il_off + S * kQuantBK * 4;
   L.stage_bytes = (sb + 1023u) & ~1023u;
   L.stg_bytes = 32u * quant_code_row_bytes(fmt);           // one staging buffer: a warp's 32 rows
-  const uint32_t stg_total = 2u * kQuantWarps * L.stg_bytes;
+  const uint32_t stg_total = kQuantWarps * L.stg_bytes;
   L.stages = (kQuantSmemBudget - stg_total) / L.stage_bytes;
   if (L.stages > static_cast<uint32_t>(kQuantMaxStages)) L.stages = kQuantMaxStages;
   if (L.stages < 3u) {
@@ -247,8 +247,9 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
     // its warp of lane quarter q quantizes rows 32 q .. 32 q + 31 of the
     // stacked tile, one lane per row over the whole 64-wide sub-tile: four
     // independent NVFP4 groups of 16 (or one INT4 group of 64) per lane.  Each
-    // warp stages its own 32 rows of codes in shared memory (two buffers, used
-    // in turn) and its lane 0 writes them with one TMA store per sub-tile the
+    // warp stages its own 32 rows of codes in shared memory (one buffer, which
+    // its previous store has read long before the next stage) and its lane 0
+    // writes them with one TMA store per sub-tile the
     // rows belong to (boxes of min(32, BM) rows), so no barrier ties the warps
     // of a group together; each lane writes its row's scales itself (one 4-byte
     // word or one fp16).
@@ -267,9 +268,8 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
       const float sd = reinterpret_cast<const float*>(p.sf)[row_ok ? m : 0];
       w8_inv = (sd == 0.0f || !row_ok) ? 0.0f : __frcp_rn(sd);
     }
-    int use = 0;
     const int G = static_cast<int>(L.groups);
-    for (int li = grp < G ? grp : n_local; li < n_local; li += G, ++use) {
+    for (int li = grp < G ? grp : n_local; li < n_local; li += G) {
       const int i = i0 + li;
       const int s = li % NS;
       const uint32_t ph = (li / NS) & 1;
@@ -354,8 +354,8 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
       }
       // codes -> this warp's staging buffer (rows of RB bytes in the TMA swizzle
       // of that row length: 16-byte chunk c of row r sits at c ^ ((r >> sh) & mask))
-      uint8_t* buf = smem + L.stg_off + (2 * (warp - 2) + (use & 1)) * L.stg_bytes;
-      if (lane == 0) bulk_wait_group_read<1>();   // its store from two uses ago has read it
+      uint8_t* buf = smem + L.stg_off + (warp - 2) * L.stg_bytes;
+      if (lane == 0) bulk_wait_group_read<0>();   // its store of the previous stage has read it
       __syncwarp();
       {
         const uint32_t row_addr = smem_u32(buf) + lane * RB;
