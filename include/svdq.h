@@ -251,13 +251,15 @@ SVDQ_API int svdq_set_gemm_raster(int group_m);
  * tuning and testing aid): 1 = one CTA per 128 x 256 output tile, 2 = a pair of
  * CTAs (a cluster of two) per 256 x 256 tile, each CTA staging its own 128 rows
  * of the activations and half of the weight columns for tcgen05 MMAs that span
- * both, 3 = a pair of CTAs per 256 x 192 tile with two accumulators in TMEM (the
- * next tile's MMAs do not wait for the epilogue); 0 restores the automatic
- * choice (3 for K <= 4096, else 2).  All give the same Y bit for bit (the same
- * products summed in the same order).  The INT4 and W8A8 formats have one
- * kernel each and ignore it.  With kinds 2 and 3 the raster group of
- * svdq_set_gemm_raster counts 128-row blocks and is rounded up to pairs.
- * SVDQ_ERR_INVALID_ARG for other values. */
+ * both; when the tiles left after the last full round of the pairs are at most
+ * half as many as the pairs, each of them is computed as two 256 x 128 halves
+ * on two pairs, 3 = a pair of CTAs per 256 x 192 tile with two accumulators in
+ * TMEM (the next tile's MMAs do not wait for the epilogue), 4 = as 2 with whole
+ * tiles only; 0 restores the automatic choice (3 for K <= 4096, else 2).  All
+ * give the same Y bit for bit (the same products summed in the same order).
+ * The INT4 and W8A8 formats have one kernel each and ignore it.  With kinds 2
+ * to 4 the raster group of svdq_set_gemm_raster counts 128-row blocks and is
+ * rounded up to pairs.  SVDQ_ERR_INVALID_ARG for other values. */
 SVDQ_API int svdq_set_gemm_kernel(int kind);
 
 SVDQ_API const char* svdq_status_string(int status);

@@ -256,22 +256,23 @@ def test_forced_launch_shapes(S, M, K, N, rank, fmt):
 ])
 def test_forced_gemm_kernel(S, M, K, N, rank, fmt):
     """The FP4 GEMM on single CTAs (128 x 256 tiles), on CTA pairs with 256 x 256
-    tiles and on CTA pairs with 256 x 192 tiles and two accumulators (cta_group::2
-    MMAs) sums the same products in the same order: Y bit for bit the same,
-    within tolerance of the oracle."""
+    tiles (at these sizes every tile as two 256 x 128 halves, kind 2, or whole,
+    kind 4) and on CTA pairs with 256 x 192 tiles and two accumulators
+    (cta_group::2 MMAs) sums the same products in the same order: Y bit for bit
+    the same, within tolerance of the oracle."""
     data = WL.make_small(M, K, N, rank=rank, fmt=fmt, seed=M + K)
     ref = oracle_layer(fmt, data, rank)
     w = load_from_oracle(S, fmt, ref["prep"])
     try:
         Ys = {}
-        for kind in (1, 2, 3):
+        for kind in (1, 2, 3, 4):
             S.svdq_set_gemm_kernel(kind)
             _, Y = _run_layer(S, w, WL.bf16_bits(data["X"]))
             ok, info = y_within_tol(bits(Y), ref["Y"])
             assert ok, (kind, info)
             Ys[kind] = bits(Y)
-        assert np.array_equal(Ys[1], Ys[2])
-        assert np.array_equal(Ys[1], Ys[3])
+        for kind in (2, 3, 4):
+            assert np.array_equal(Ys[1], Ys[kind]), kind
     finally:
         S.svdq_set_gemm_kernel(0)
         w.close()

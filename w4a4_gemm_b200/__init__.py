@@ -355,8 +355,9 @@ def svdq_set_quant_split(S: int = 0, C: int = 0):
 
 
 def svdq_set_gemm_kernel(kind: int = 0):
-    """Force the FP4 GEMM kernel: 1 = one CTA per tile, 2 = CTA pairs on 256 x 256 tiles,
-    3 = CTA pairs on 256 x 192 tiles with two accumulators; 0 = automatic (see include/svdq.h)."""
+    """Force the FP4 GEMM kernel: 1 = one CTA per tile, 2 = CTA pairs on 256 x 256 tiles (the
+    tiles of a short last round as 256 x 128 halves), 3 = CTA pairs on 256 x 192 tiles with two
+    accumulators, 4 = as 2 with whole tiles only; 0 = automatic (see include/svdq.h)."""
     _check(lib().svdq_set_gemm_kernel(int(kind)), "svdq_set_gemm_kernel")
 
 

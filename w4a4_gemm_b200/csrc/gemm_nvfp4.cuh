@@ -63,6 +63,8 @@ struct GemmParams {
   int kt_total;        // ceil(K / 256)
   int m_tiles, n_tiles, num_tiles;
   int group_m;         // tile order: groups of group_m row blocks, see gemm_tile_coords
+  int wide_tiles;      // CTA-pair kernels: tiles taken whole; each later one as two half-width units
+  int num_units;       // CTA-pair kernels: wide_tiles + 2 (num_tiles - wide_tiles)
   int r_tail;          // tail K: 2 r_pad (X_hat L1 as hi | lo against L2^T | L2^T), 0 = none
   const uint8_t* sfa;  // activation scale atoms [M_pad/128][sf_kcols][512]
   const uint8_t* sfb;  // weight scale atoms     [N_pad/128][sf_kcols][512]

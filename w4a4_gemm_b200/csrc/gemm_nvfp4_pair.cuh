@@ -15,6 +15,13 @@
 //
 // BN = 256 leaves room in TMEM for one accumulator: the MMAs of a tile wait
 // until the epilogue has copied the previous tile's accumulator to registers.
+//
+// The pairs walk units: the first wide_tiles are whole tiles; when the tiles
+// left over after the last full round are at most half as many as the pairs,
+// each of them is split into two units of half its width (256 x 128, BN = 256
+// only), so that twice as many pairs share that round, in half the time.  A
+// half-width unit computes its columns exactly as the whole tile would: the
+// same products, summed in the same order.
 // BN = 192 fits two accumulators (TMEM columns 0 and 256) beside the scale
 // factors, so the MMAs run on into the next tile while the epilogue drains the
 // last one; it moves more operand bytes per MMA and pays where the K loop of a
@@ -120,11 +127,26 @@ __device__ __forceinline__ void epi_store_32(const uint32_t* r, uint8_t* buf, co
   }
 }
 
+// Unit u of a pair's walk: units below p.wide_tiles are whole tiles in
+// gemm_tile_coords order; tile p.wide_tiles + v / 2 of that order gives the
+// units p.wide_tiles + v, the half v % 2 of its columns each.  Returns that
+// half, or -1 for a whole tile.
+__device__ __forceinline__ int pair_unit_coords(const GemmParams& p, int u, int& mp, int& nb) {
+  if (u < p.wide_tiles) {
+    gemm_tile_coords(p.m_tiles, p.n_tiles, p.group_m, u, mp, nb);
+    return -1;
+  }
+  const int v = u - p.wide_tiles;
+  gemm_tile_coords(p.m_tiles, p.n_tiles, p.group_m, p.wide_tiles + (v >> 1), mp, nb);
+  return v & 1;
+}
+
 // p.m_tiles counts pair row blocks (256 rows), p.n_tiles weight column blocks
 // of BN; p.sfa / p.sfb are unused (the scale atoms come through tm_sfa / tm_sfb:
 // [atoms][128 x 32-bit words]; for tm_sfb, atom slot 2 nb + a of a K step holds
 // the scales of weight columns nb BN + 128 a .. + 127).  tm_b and tm_l2t have
-// boxes of BN / 2 rows.
+// boxes of BN / 2 rows; a half-width unit loads the same boxes from its own
+// first column on and its MMAs read the first BN / 4 rows of each CTA's half.
 template <int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_nvfp4_pair_kernel(const __grid_constant__ CUtensorMap tm_a,
@@ -199,12 +221,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint32_t lr_tx = 2 * (128 + Sh::kBH) * static_cast<uint32_t>(lr_cols) * 2;
       int it = 0;
       bool ok = true;
-      for (int tile = pair; tile < p.num_tiles && ok; tile += n_pairs) {
+      for (int u = pair; u < p.num_units && ok; u += n_pairs) {
         int mp, nb;
-        gemm_tile_coords(p.m_tiles, p.n_tiles, p.group_m, tile, mp, nb);
+        const int half = pair_unit_coords(p, u, mp, nb);
         const int m_blk = 2 * mp + static_cast<int>(rank);    // this CTA's 128-row block
         const int m0 = m_blk * 128;
-        const int nh0 = nb * BN + Sh::kBH * static_cast<int>(rank);
+        // this CTA's first weight column; the B scale atoms of the columns
+        const int nh0 = half < 0 ? nb * BN + Sh::kBH * static_cast<int>(rank)
+                                 : nb * BN + Sh::kBH * half + (Sh::kBH / 2) * static_cast<int>(rank);
+        const int sfb0 = half < 0 ? 2 * nb : 2 * nb + half;
+        const int sfb1 = half < 0 ? 2 * nb + 1 : 2 * nb + half;
         for (int step = 0; step < steps_per_tile; ++step, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
@@ -222,8 +248,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             tma_load_2d_pair(st + Sh::kAOff, &tm_a, fb, kt * kGemmBKB, m0);
             tma_load_2d_pair(st + Sh::kBOff, &tm_b, fb, kt * kGemmBKB, nh0);
             tma_load_2d_pair(st + Sh::kSfaOff, &tm_sfa, fb, 0, m_blk * p.sf_kcols + 4 * kt);
-            tma_load_2d_pair(st + Sh::kSfbOff, &tm_sfb, fb, 0, (2 * nb) * p.sf_kcols + 4 * kt);
-            tma_load_2d_pair(st + Sh::kSfbOff + 2048, &tm_sfb, fb, 0, (2 * nb + 1) * p.sf_kcols + 4 * kt);
+            tma_load_2d_pair(st + Sh::kSfbOff, &tm_sfb, fb, 0, sfb0 * p.sf_kcols + 4 * kt);
+            tma_load_2d_pair(st + Sh::kSfbOff + 2048, &tm_sfb, fb, 0, sfb1 * p.sf_kcols + 4 * kt);
           } else {
             const int c = step - p.kt_total;
             if (rank == 0) mbar_arrive_expect_tx(&full[s], lr_tx);
@@ -238,15 +264,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer (rank 0)
     if (rank == 0 && elect_one()) {
-      const uint32_t idesc_main = idesc_e2m1_ue4m3(kPairBM, BN);
-      const uint32_t idesc_lr = idesc_bf16_f32(kPairBM, BN);
+      const uint32_t idesc_main_w = idesc_e2m1_ue4m3(kPairBM, BN);
+      const uint32_t idesc_lr_w = idesc_bf16_f32(kPairBM, BN);
+      const uint32_t idesc_main_h = idesc_e2m1_ue4m3(kPairBM, BN / 2);   // half-width units
+      const uint32_t idesc_lr_h = idesc_bf16_f32(kPairBM, BN / 2);
       const uint32_t lr_row_bytes = static_cast<uint32_t>(lr_cols) * 2;
       const uint32_t sfa_col = tmem_base + Sh::kSfaCol;
       const uint32_t sfb_col = tmem_base + Sh::kSfbCol;
       int it = 0, t_local = 0;
       bool ok = true;
-      for (int tile = pair; tile < p.num_tiles && ok; tile += n_pairs, ++t_local) {
-        // accumulator b of this tile; its previous tile's epilogue must have emptied it
+      for (int u = pair; u < p.num_units && ok; u += n_pairs, ++t_local) {
+        int mp, nb;
+        const bool whole = pair_unit_coords(p, u, mp, nb) < 0;
+        const uint32_t idesc_main = whole ? idesc_main_w : idesc_main_h;
+        const uint32_t idesc_lr = whole ? idesc_lr_w : idesc_lr_h;
+        // accumulator b of this unit; its previous unit's epilogue must have emptied it
         const int b = t_local % ACC;
         const uint32_t d_tmem = tmem_base + Sh::kAccStride * static_cast<uint32_t>(b);
         if (!mbar_wait(&acc_empty[b], ((t_local / ACC) & 1) ^ 1, p.budget, abort_flag)) {
@@ -303,9 +335,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     constexpr int CH = Sh::kBH / 32;   // 32-column chunks of this warp's half of the tile
     uint8_t* ebuf = smem + Sh::kEpiOff + (warp - 2) * Sh::kEpiBufBytes;
     int t_local = 0;
-    for (int tile = pair; tile < p.num_tiles; tile += n_pairs, ++t_local) {
+    for (int u = pair; u < p.num_units; u += n_pairs, ++t_local) {
       int mp, nb;
-      gemm_tile_coords(p.m_tiles, p.n_tiles, p.group_m, tile, mp, nb);
+      const int half = pair_unit_coords(p, u, mp, nb);
+      // columns of this warp: half of the unit's BN (whole tile) or BN / 2 per CTA
+      const int wcols = half < 0 ? Sh::kBH : Sh::kBH / 2;
+      const int nch = wcols / 32;
       const int b = t_local % ACC;
       if (!warp_wait(&acc_full[b], (t_local / ACC) & 1, p.budget, abort_flag)) {
         if (lane == 0) raise_error(kErrWaitGemm);
@@ -315,19 +350,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       uint32_t v[CH][32];
       const uint32_t taddr = tmem_base + ((q * 32u) << 16) + Sh::kAccStride * static_cast<uint32_t>(b) +
-                             static_cast<uint32_t>(Sh::kBH) * h;
+                             static_cast<uint32_t>(wcols) * h;
 #pragma unroll
-      for (int c = 0; c < CH; ++c) tmem_ld32(taddr + 32 * c, v[c]);
+      for (int c = 0; c < CH; ++c)
+        if (c < nch) tmem_ld32(taddr + 32 * c, v[c]);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(map_shared_rank(smem_u32(&acc_empty[b]), 0));
       const int row0 = mp * kPairBM + 128 * static_cast<int>(rank) + static_cast<int>(q) * 32;
-      const int ncol = nb * BN + Sh::kBH * static_cast<int>(h);
+      const int ncol = nb * BN + (half < 0 ? 0 : Sh::kBH * half) + wcols * static_cast<int>(h);
       if (row0 < p.M) {
 #pragma unroll
         for (int c = 0; c < CH; ++c)
-          if (ncol + 32 * c < p.N)
+          if (c < nch && ncol + 32 * c < p.N)
             epi_store_32(v[c], ebuf, &tm_y, ncol + 32 * c, row0, p.N, p.bias, p.out_scale, lane);
       }
     }

@@ -316,7 +316,7 @@ constexpr double kQuantL1Cycles = 400.0;   // refitted with the hi + lo factor (
 std::atomic<int> g_forced_split{0};      // svdq_set_quant_split: 16 S + C; 0 = automatic
 std::atomic<int> g_forced_group_m{0};    // svdq_set_gemm_raster; 0 = automatic
 std::atomic<int> g_forced_gemm_kind{0};  // svdq_set_gemm_kernel; 0 = automatic, 1 = one CTA, 2 = CTA pairs,
-                                         // 3 = CTA pairs on 192-column tiles
+                                         // 3 = CTA pairs on 192-column tiles, 4 = 2 with whole tiles only
 
 QuantSplit quant_split_for(int fmt, int M, int K, int r_pad, const DeviceInfo& d) {
   const int smax = r_pad > 0 ? quant_stack_max(r_pad) : 8;
@@ -800,7 +800,7 @@ SVDQ_API int svdq_tensor_peak(int fmt, long long steps, void* stream) {
 }
 
 SVDQ_API int svdq_set_gemm_kernel(int kind) {
-  if (kind < 0 || kind > 3) return SVDQ_ERR_INVALID_ARG;
+  if (kind < 0 || kind > 4) return SVDQ_ERR_INVALID_ARG;
   g_forced_gemm_kind.store(kind, std::memory_order_relaxed);
   return SVDQ_OK;
 }
@@ -1125,7 +1125,7 @@ int fp4_gemm_kind(const svdq_weights* w, const DeviceInfo& d) {
   const int forced = g_forced_gemm_kind.load(std::memory_order_relaxed);
   int kind = forced != 0 ? forced : (w->K <= 4096 ? 3 : 2);
   if (kind == 3 && d.pair192_clusters <= 0) kind = 2;
-  if (kind == 2 && d.pair_clusters <= 0) kind = 1;
+  if ((kind == 2 || kind == 4) && d.pair_clusters <= 0) kind = 1;
   return kind;
 }
 
@@ -1163,8 +1163,8 @@ SVDQ_API int svdq_linear(const svdq_weights* w, const void* ws, int M, void* Y, 
     tm_xl1 = tm_a;
   }
   const int fp4_kind = is_fp4(w->fmt) ? fp4_gemm_kind(w, g_dev[dev]) : 0;
-  if (fp4_kind == 2 || fp4_kind == 3) {
-    const int bn = fp4_kind == 2 ? 256 : 192;
+  if (fp4_kind == 2 || fp4_kind == 3 || fp4_kind == 4) {
+    const int bn = fp4_kind == 3 ? 192 : 256;
     CUtensorMap tm_y, tm_sfa;
     if ((rc = make_map(&tm_y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Y, w->N, M, 32, 32))) return rc;
     if ((rc = make_atom_map(&tm_sfa, base + L.sf_off, static_cast<uint64_t>(L.M_pad / 128) * w->sf_kcols)))
@@ -1179,6 +1179,12 @@ SVDQ_API int svdq_linear(const svdq_weights* w, const void* ws, int M, void* Y, 
     p.num_tiles = p.m_tiles * p.n_tiles;
     const int forced_g = g_forced_group_m.load(std::memory_order_relaxed);
     p.group_m = forced_g > 0 ? std::min((forced_g + 1) / 2, p.m_tiles) : std::min(kPairGroupM, p.m_tiles);
+    // 256-column tiles left over after the last full round of the pairs, if at
+    // most half as many as the pairs, go as two 256 x 128 units each
+    const int pairs_max = bn == 256 ? g_dev[dev].pair_clusters : g_dev[dev].pair192_clusters;
+    const int left = p.num_tiles % pairs_max;
+    p.wide_tiles = (fp4_kind == 2 && left > 0 && 2 * left <= pairs_max) ? p.num_tiles - left : p.num_tiles;
+    p.num_units = p.wide_tiles + 2 * (p.num_tiles - p.wide_tiles);
     p.r_tail = 2 * w->r_pad;
     p.sfa = nullptr;
     p.sfb = nullptr;
@@ -1187,11 +1193,11 @@ SVDQ_API int svdq_linear(const svdq_weights* w, const void* ws, int M, void* Y, 
     p.out_scale = std::ldexp(1.0f, -w->w_exp);
     p.budget = wait_budget();
     if (bn == 256) {
-      const int pairs = std::min(p.num_tiles, g_dev[dev].pair_clusters);
+      const int pairs = std::min(p.num_units, g_dev[dev].pair_clusters);
       SVDQ_CUDA(launch_pdl(gemm_nvfp4_pair_kernel<256>, dim3(2 * pairs), dim3(kGemmThreads), kPairSmemBytes, st,
                            2u, tm_a, w->tm_b_half, tm_sfa, w->tm_sfb, tm_xl1, w->tm_l2t_half, tm_y, p));
     } else {
-      const int pairs = std::min(p.num_tiles, g_dev[dev].pair192_clusters);
+      const int pairs = std::min(p.num_units, g_dev[dev].pair192_clusters);
       SVDQ_CUDA(launch_pdl(gemm_nvfp4_pair_kernel<192>, dim3(2 * pairs), dim3(kGemmThreads), kPair192SmemBytes,
                            st, 2u, tm_a, w->tm_b_96, tm_sfa, w->tm_sfb192, tm_xl1, w->tm_l2t_96, tm_y, p));
     }
@@ -1207,6 +1213,8 @@ SVDQ_API int svdq_linear(const svdq_weights* w, const void* ws, int M, void* Y, 
     p.n_tiles = n_tiles;
     p.num_tiles = tiles;
     p.group_m = group_m;
+    p.wide_tiles = tiles;
+    p.num_units = tiles;
     p.r_tail = 2 * w->r_pad;
     p.sfa = base + L.sf_off;
     p.sfb = w->wsf;
