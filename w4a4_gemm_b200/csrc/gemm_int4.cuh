@@ -68,8 +68,8 @@ constexpr uint32_t kI4SmemBytes = kI4ConstOff + 12288 + kI4BarBytes + 1024;
 static_assert(kI4SwOff + kI4BN * 4 <= kI4StageBytes, "stage layout");
 static_assert((3 * kI4Stages + 2 * kI4Bufs + 1) * 8 + 8 <= kI4BarBytes, "barrier area");
 
-// Low-rank tail chunks of at most 32 bf16 columns (64-byte rows: they fit the
-// A and B regions of a stage).
+// Low-rank tail chunks of at most 64 bf16 columns (128-byte rows: 128 of them
+// fill the 16 KB A and B regions of a stage).
 __host__ __device__ inline int i4_lr_chunk_cols(int k_tail) { return k_tail < 64 ? k_tail : 64; }
 __host__ __device__ inline int i4_lr_num_chunks(int k_tail) {
   return k_tail == 0 ? 0 : (k_tail + 63) / 64;
