@@ -76,12 +76,10 @@ DATASHEET_FP4_TFLOPS = 9000.0
 DATASHEET_INT8_TOPS = 4500.0
 NOMINAL_HBM_GBS = 8000.0
 NCU_TRAFFIC = {
-    ("gemm_nvfp4_pair_kernel", "c5_block/fc2", 16384, "nvfp4"): (221565696, "97027a9e62004fde"),
-    ("quant_act_kernel", "c5_block/fc2", 16384, "nvfp4"): (499809792, "21b4a8dae4db57e2"),
-    ("gemm_int4_kernel", "c4_int4_lora/proj", 4608, "int4"): (21903616, "94d8e85b38a51e4a"),
-    ("gemm_nvfp4_pair_kernel", "c2_qkv/qkv", 4608, "nvfp4"): (64266752, "97027a9e62004fde"),
-    ("quant_act_kernel", "c2_qkv/qkv", 4608, "nvfp4"): (28757760, "21b4a8dae4db57e2"),
-    ("gemm_w8a8_kernel", "c2_qkv/qkv", 4608, "w8a8"): (93856256, "7bfa1387a77d1a37"),
+    ("gemm_nvfp4_pair_kernel", "c5_block/fc2", 16384, "nvfp4"): (222011392, "559ee5e39072da5f"),
+    ("quant_act_kernel", "c5_block/fc2", 16384, "nvfp4"): (499774208, "c3616c4fb90d854e"),
+    ("gemm_int4_kernel", "c4_int4_lora/proj", 4608, "int4"): (21903616, "05e99fde6326be6b"),
+    ("gemm_w8a8_kernel", "c2_qkv/qkv", 4608, "w8a8"): (93856256, "6fe3c9970eeb8a17"),
 }
 KERNEL_SOURCES = {
     "gemm_nvfp4_kernel": ("gemm_nvfp4.cuh", "svdq_ptx.cuh", "svdq_formats.cuh"),
