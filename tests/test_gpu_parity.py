@@ -253,6 +253,7 @@ def test_forced_launch_shapes(S, M, K, N, rank, fmt):
     (1000, 768, 272, 48, "nvfp4"),   # ragged last column block, 3 tail chunks
     (384, 320, 1024, 32, "nvfp4"),   # K below two K steps
     (520, 512, 208, 32, "nvfp4"),    # one 192-column tile and a 16-column one
+    (1792, 512, 3072, 32, "nvfp4"),  # 84 tiles of 256 x 256: a full round of the pairs, then halves
 ])
 def test_forced_gemm_kernel(S, M, K, N, rank, fmt):
     """The FP4 GEMM on single CTAs (128 x 256 tiles), on CTA pairs with 256 x 256
