@@ -186,6 +186,7 @@ SHAPES = [
     (96, 512, 256, 32, "int4", True),
     (200, 1024, 512, 48, "int4", False),
     (64, 256, 272, 0, "int4", False),
+    (130, 320, 256, 32, "int4", True),       # five groups of 64: the last stage holds one
     (77, 512, 384, 32, "fp4g32", True),      # one E4M3 scale per 32 values, stored per 16
     (300, 320, 272, 48, "fp4g32", False),
     (77, 512, 384, 16, "w8a8", True),        # int8, per-token / per-channel scales
