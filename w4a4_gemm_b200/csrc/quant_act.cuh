@@ -8,15 +8,17 @@
 // quantizer warps.  One bf16 rounding of the folded factor (2^-8 per term)
 // would move Y by several times the output tolerance where the branch and the
 // 4-bit part cancel, so the factor is carried as a bf16 pair L1s = hi + lo
-// (2^-16 per term) and each stage issues the MMAs twice, X hi then X lo, into
-// the same accumulator (bf16 x bf16 products are exact in fp32).
+// (2^-16 per term): the lo slices sit right after the hi slices in the stage,
+// and one MMA of twice the width (two where that exceeds N = 256) puts X hi and
+// X lo side by side in the accumulator, summed in fp32 at the end (bf16 x bf16
+// products are exact in fp32).
 //
 // A cluster of C CTAs owns BM = 128 / S token rows; its CTA of rank t takes
 // the t-th of C consecutive K ranges.  Each pipeline stage holds S consecutive
 // 64-wide K sub-tiles of those rows stacked on top of each other as the
 // 128-row A operand of one tcgen05 MMA, and the S matching 64 x r_pad slices
 // of the folded factor L1s side by side as its N = S * r_pad wide B operand
-// (once for hi, once for lo):
+// (once for hi, then once for lo, at column offset S * r_pad):
 //   D[j*BM + i, j'*r_pad + c] += sum_k x[i, sub-tile j, k] * L1s[sub-tile j', k, c]
 // Only the diagonal blocks j == j' are wanted; summing them over j and over
 // the cluster's K ranges gives X L1s = X_hat L1 for row i.  The partial sums
@@ -152,8 +154,9 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
   const int nkt = (p.K + kstep - 1) / kstep;            // stages over all of K
   const int i0 = min(rank * p.per, nkt);                // this CTA's stages: i0 .. i0 + n_local - 1
   const int n_local = min(nkt - i0, p.per);
-  const int n_mma = S * p.r_pad;                        // MMA N
-  const uint32_t tmem_cols = n_mma <= 32 ? 32u : (n_mma <= 64 ? 64u : (n_mma <= 128 ? 128u : 256u));
+  const int n_mma = S * p.r_pad;                        // columns of the hi (and of the lo) product
+  // the accumulator: hi products in columns 0 .. n_mma - 1, lo in n_mma .. 2 n_mma - 1
+  const uint32_t tmem_cols = n_mma <= 16 ? 32u : (n_mma <= 32 ? 64u : (n_mma <= 64 ? 128u : (n_mma <= 128 ? 256u : 512u)));
 
   griddep_launch_dependents();
   if (threadIdx.x == 0) {
@@ -215,7 +218,10 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (has_lr && elect_one()) {
-      const uint32_t idesc = idesc_bf16_f32(kQuantTileRows, n_mma);
+      // one MMA of N = 2 n_mma over the hi and lo slices (adjacent in the
+      // stage) where N fits, else one for each
+      const bool one = 2 * n_mma <= 256;
+      const uint32_t idesc = idesc_bf16_f32(kQuantTileRows, one ? 2 * n_mma : n_mma);
       for (int li = 0; li < n_local; ++li) {
         const int s = li % NS;
         const uint32_t ph = (li / NS) & 1;
@@ -233,9 +239,12 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
           mma_bf16(tmem_base, make_kmajor_desc(a0 + 32 * k, 128), make_kmajor_desc(b0 + 32 * k, 128),
                    idesc, (li > 0 || k > 0) ? 1u : 0u);
         }
+        if (!one) {
 #pragma unroll
-        for (int k = 0; k < kQuantBK / 16; ++k)
-          mma_bf16(tmem_base, make_kmajor_desc(a0 + 32 * k, 128), make_kmajor_desc(b1 + 32 * k, 128), idesc, 1u);
+          for (int k = 0; k < kQuantBK / 16; ++k)
+            mma_bf16(tmem_base + static_cast<uint32_t>(n_mma), make_kmajor_desc(a0 + 32 * k, 128),
+                     make_kmajor_desc(b1 + 32 * k, 128), idesc, (li > 0 || k > 0) ? 1u : 0u);
+        }
         tc_commit(&empty[s]);
       }
       tc_commit(acc_full);  // also covers an early exit: waits for every issued MMA
@@ -420,20 +429,23 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
     const int j_first = static_cast<int>(q * 32) / BM, j_last = static_cast<int>(q * 32 + 31) / BM;
     for (int jj = j_first; jj <= j_last; ++jj) {
       for (int c = 0; c < p.r_pad; c += 16) {
-        uint32_t r[16];
+        // the hi and the lo product of the block, summed in fp32
+        uint32_t r[16], rl[16];
         if (n_local > 0) {
           tmem_ld16(tmem_base + ((q * 32u) << 16) + jj * p.r_pad + c, r);
+          tmem_ld16(tmem_base + ((q * 32u) << 16) + n_mma + jj * p.r_pad + c, rl);
           tmem_wait_ld();
         } else {   // an empty K range contributes zero (its accumulator was never written)
 #pragma unroll
-          for (int e = 0; e < 16; ++e) r[e] = 0u;
+          for (int e = 0; e < 16; ++e) r[e] = rl[e] = 0u;
         }
         if (jj == j) {
+          float v[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) v[e] = __fadd_rn(__uint_as_float(r[e]), __uint_as_float(rl[e]));
 #pragma unroll
           for (int e = 0; e < 16; e += 4)
-            *reinterpret_cast<float4*>(red + R * rs + c + e) =
-                make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]),
-                            __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
+            *reinterpret_cast<float4*>(red + R * rs + c + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
         }
       }
     }
