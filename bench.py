@@ -77,11 +77,11 @@ DATASHEET_INT8_TOPS = 4500.0
 NOMINAL_HBM_GBS = 8000.0
 NCU_TRAFFIC = {
     ("gemm_nvfp4_pair_kernel", "c5_block/fc2", 16384, "nvfp4"): (222011392, "559ee5e39072da5f"),
-    ("quant_act_kernel", "c5_block/fc2", 16384, "nvfp4"): (499774208, "c3616c4fb90d854e"),
+    ("quant_act_kernel", "c5_block/fc2", 16384, "nvfp4"): (500727552, "07cf2606c82c7582"),
     ("gemm_int4_kernel", "c4_int4_lora/proj", 4608, "int4"): (21903616, "05e99fde6326be6b"),
     ("gemm_w8a8_kernel", "c2_qkv/qkv", 4608, "w8a8"): (93856256, "6fe3c9970eeb8a17"),
     ("gemm_nvfp4_pair_kernel", "c2_qkv/qkv", 4608, "nvfp4"): (63152896, "559ee5e39072da5f"),
-    ("quant_act_kernel", "c2_qkv/qkv", 4608, "nvfp4"): (28757760, "c3616c4fb90d854e"),
+    ("quant_act_kernel", "c2_qkv/qkv", 4608, "nvfp4"): (28758016, "07cf2606c82c7582"),
 }
 KERNEL_SOURCES = {
     "gemm_nvfp4_kernel": ("gemm_nvfp4.cuh", "svdq_ptx.cuh", "svdq_formats.cuh"),
