@@ -227,17 +227,13 @@ SVDQ_API int svdq_set_wait_budget(long long cycles);
  * (process-wide; a tuning and testing aid).  S = stacked 64-wide K sub-tiles
  * per pipeline stage (rows per CTA cluster = 128 / S), C = CTAs per cluster,
  * each on its own K range, whose partial X_hat L1 sums meet in distributed
- * shared memory.  S, C in {1, 2, 4, 8}; S = 1, C = 0 selects the streamed
- * launch (NVFP4, rank_padded <= 128): one CTA per SM, each taking an equal
- * run of the (128-row block, 64-wide stage) units in row-major order, the
- * partial X_hat L1 sums of a row block split between CTAs meeting in the
- * workspace.  0, 0 restores the automatic choice (a cost model over the SM
- * count and the resident clusters of each size).  A forced shape the layer
- * cannot use (S above 256 / rank_padded, C above 128 / S or above the number
- * of stages, no resident cluster of C CTAs, a streamed launch of another
- * format or rank) falls back to the automatic choice for that call.  The
- * results do not depend on the shape beyond the summation order of X_hat L1
- * (fp32).  SVDQ_ERR_INVALID_ARG for other values. */
+ * shared memory.  S, C in {1, 2, 4, 8}; 0, 0 restores the automatic choice
+ * (a cost model over the SM count and the resident clusters of each size).
+ * A forced shape the layer cannot use (S above 256 / rank_padded, C above
+ * 128 / S or above the number of stages, no resident cluster of C CTAs)
+ * falls back to the automatic choice for that call.  The results do not
+ * depend on the shape beyond the summation order of X_hat L1 (fp32).
+ * SVDQ_ERR_INVALID_ARG for other values. */
 SVDQ_API int svdq_set_quant_split(int S, int C);
 
 /* Tile order of the GEMM for every later svdq_linear (process-wide; a tuning

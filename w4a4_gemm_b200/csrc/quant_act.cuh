@@ -35,14 +35,6 @@
 //   warp 0      : TMA producer (S X boxes BM x 64, 2 S L1s^T boxes r_pad x 64
 //                 (hi, lo), 1/lambda)
 //   warp 1      : TMEM owner; one lane issues the kind::f16 MMAs
-// A streamed launch (S = C = 1) gives every CTA an equal run of (row block,
-// stage) units instead of whole row blocks: the run's stretch of each row
-// block (a segment) accumulates in one of two TMEM accumulators, and the
-// quantizer group that takes a segment's last stage reads it out while the
-// other accumulator already takes the next segment.  A row block that lies
-// in one run is written at once; otherwise each run leaves its fp32 partial
-// and the last to arrive sums the parts in the order of their K ranges.
-//
 //   warps 2..17 : quantizers in up to four groups of four (as many groups as
 //                 there are pipeline stages); group k takes every G-th stage,
 //                 and its warp w serves A-tile rows 32 (w % 4) .. + 31, one lane
@@ -68,10 +60,6 @@ constexpr int kQuantWarps = kQuantGroupWarps * kQuantGroups;
 constexpr int kQuantThreads = 32 * (2 + kQuantWarps);
 constexpr uint32_t kQuantSmemBudget = 220u * 1024u;    // shared memory for stages + code staging
 
-// barrier area at QuantSmem::bar_off: full and empty per stage, acc_full[2],
-// acc_empty[2], mma_done, the TMEM address and the abort flag
-static_assert((2 * kQuantMaxStages + 5) * 8 + 8 <= 256, "activation kernel barrier area");
-
 // Bytes of codes one row of a 64-wide sub-tile produces: 64 E2M1 (NVFP4, FP4 g32) or 64 int8 (INT4, W8A8).
 __host__ __device__ constexpr uint32_t quant_code_row_bytes(int fmt) { return (fmt == 1 || fmt == 3) ? 64u : 32u; }
 
@@ -87,15 +75,6 @@ struct QuantParams {
   uint8_t* sf;      // NVFP4: 512-byte atoms; INT4: fp16 [K/64][M_pad]
   __nv_bfloat16* xl1;  // M x 2 r_pad: X_hat L1 as a bf16 pair, hi | lo (hi + lo = fp32 value)
   long long budget;
-  // Streamed launch (NVFP4, S = C = 1, r_pad <= 128): the (row block,
-  // stage) units in row-major order are cut into gridDim.x equal runs, one per
-  // CTA, so that every SM gets the same share.  A row block split between
-  // runs meets in `part` (fp32 [128][r_pad] slot c + row block for CTA c) and
-  // `cnt` (arrivals per row block and lane quarter, zero before the launch).
-  int stream;
-  int units;        // row blocks x stages
-  float* part;
-  unsigned* cnt;
 };
 
 // Most sub-tiles that can be stacked for a given padded rank (N = S * r_pad <= 256).
@@ -147,21 +126,6 @@ __host__ __device__ inline QuantSmem quant_smem_layout(int fmt, int r_pad, int S
   return L;
 }
 
-// Eight fp32 X_hat L1 values of token row m, columns c .. c + 7, as the bf16
-// pair hi = bf16(v), lo = bf16(v - hi) (hi + lo carries v to ~2^-17): hi at
-// columns c .., lo at r_pad + c .. of the row's 2 r_pad.
-__device__ __forceinline__ void store_xl1_pair8(__nv_bfloat16* xl1, int m, int r_pad, int c, const float* v) {
-  uint32_t hi[4], lo[4];
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    hi[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
-    lo[e] = pack_bf16x2(v[2 * e] - bf16_lo(hi[e]), v[2 * e + 1] - bf16_hi(hi[e]));
-  }
-  __nv_bfloat16* dst = xl1 + static_cast<size_t>(m) * (2 * r_pad) + c;
-  *reinterpret_cast<uint4*>(dst) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-  *reinterpret_cast<uint4*>(dst + r_pad) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-}
-
 template <int FMT>  // 0 = NVFP4 (groups of 16), 1 = INT4 (groups of 64), 2 = FP4 g32 (groups of 32),
                     // 3 = W8A8 (int8, the per-token scale computed beforehand by w8_row_scale_kernel)
 __global__ void __launch_bounds__(kQuantThreads, 1)
@@ -174,10 +138,8 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
   const int NS = static_cast<int>(L.stages);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bar_off);
   uint64_t* empty = full + kQuantMaxStages;
-  uint64_t* acc_full = empty + kQuantMaxStages;   // [2]: the accumulator (streamed: of a segment) is complete
-  uint64_t* acc_empty = acc_full + 2;             // [2]: streamed: a segment's accumulator has been read
-  uint64_t* mma_done = acc_empty + 2;             // streamed: every MMA issued has retired
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
+  uint64_t* acc_full = empty + kQuantMaxStages;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_full + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   float* rcp_tab = reinterpret_cast<float*>(smem + L.bar_off + 256);   // 1/E4M3 value, 128 entries
 
@@ -190,27 +152,11 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
   const int m0 = (static_cast<int>(blockIdx.x) / p.C) * BM;
   const int kstep = S * kQuantBK;                       // K columns per stage
   const int nkt = (p.K + kstep - 1) / kstep;            // stages over all of K
-  const bool stream = FMT == 0 && p.stream != 0;        // NVFP4 only; then S = C = 1 and r_pad <= 128
-  // this CTA's units: stages i0 .. i0 + n_local - 1 of row block m0, or
-  // (streamed) the units u0 .. u0 + n_local - 1 of the row-major order, which
-  // start at stage i0 of the row block at row m0 (each role then steps its
-  // (row, stage) position forward without dividing)
-  int i0, n_local, m_first;
-  if (stream) {
-    const long long G = gridDim.x;
-    const int u0 = static_cast<int>(static_cast<long long>(blockIdx.x) * p.units / G);
-    n_local = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * p.units / G) - u0;
-    i0 = u0 % nkt;
-    m_first = (u0 / nkt) * BM;
-  } else {
-    i0 = min(rank * p.per, nkt);
-    n_local = min(nkt - i0, p.per);
-    m_first = m0;
-  }
+  const int i0 = min(rank * p.per, nkt);                // this CTA's stages: i0 .. i0 + n_local - 1
+  const int n_local = min(nkt - i0, p.per);
   const int n_mma = S * p.r_pad;                        // columns of the hi (and of the lo) product
-  // an accumulator: hi products in columns 0 .. n_mma - 1, lo in n_mma .. 2 n_mma - 1
+  // the accumulator: hi products in columns 0 .. n_mma - 1, lo in n_mma .. 2 n_mma - 1
   const uint32_t tmem_cols = n_mma <= 16 ? 32u : (n_mma <= 32 ? 64u : (n_mma <= 64 ? 128u : (n_mma <= 128 ? 256u : 512u)));
-  const uint32_t tmem_alloc_cols = stream ? 2u * tmem_cols : tmem_cols;   // streamed: two accumulators
 
   griddep_launch_dependents();
   if (threadIdx.x == 0) {
@@ -219,17 +165,13 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
       // released by the quantizer warps and, with a low-rank branch, the MMAs
       mbar_init(&empty[s], kQuantGroupWarps + (has_lr ? 1 : 0));
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], kQuantGroupWarps);
-    }
-    mbar_init(mma_done, 1);
+    mbar_init(acc_full, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
   if ((FMT == 0 || FMT == 2) && warp >= 2 && warp < 6) fill_e4m3_rcp_table(rcp_tab, threadIdx.x - 64, 128);
   if (warp == 1 && has_lr) {
-    tmem_alloc(tmem_holder, tmem_alloc_cols);
+    tmem_alloc(tmem_holder, tmem_cols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -246,12 +188,8 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
       if (has_lr) prefetch_tmap(&tm_l1t);
       const uint32_t tx = S * (BM * kQuantBK * 2 + (has_lr ? 2 * p.r_pad * 128 : 0) + kQuantBK * 4);
       int issued = 0;
-      int i = i0, mb = m_first;   // stage and first row of unit li
-      for (int li = 0; li < n_local; ++li, ++i) {
-        if (i == nkt) {   // streamed: the next row block
-          i = 0;
-          mb += BM;
-        }
+      for (int li = 0; li < n_local; ++li) {
+        const int i = i0 + li;
         const int s = li % NS;
         const uint32_t ph = (li / NS) & 1;
         if (!mbar_wait(&empty[s], ph ^ 1, p.budget, abort_flag)) {
@@ -263,7 +201,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
         mbar_arrive_expect_tx(&full[s], tx);
         for (int j = 0; j < S; ++j) {
           const int k = (i * S + j) * kQuantBK;   // may lie past K: the box is zero-filled
-          tma_load_2d(st + L.x_off + j * BM * 128, &tm_x, &full[s], k, mb);
+          tma_load_2d(st + L.x_off + j * BM * 128, &tm_x, &full[s], k, m0);
           if (has_lr) {   // rows 0 .. r_pad - 1 of the map hold hi, r_pad .. 2 r_pad - 1 lo
             tma_load_2d(st + L.l1_off + j * p.r_pad * 128, &tm_l1t, &full[s], k, 0);
             tma_load_2d(st + L.l1_off + (S + j) * p.r_pad * 128, &tm_l1t, &full[s], k, p.r_pad);
@@ -284,24 +222,9 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
       // stage) where N fits, else one for each
       const bool one = 2 * n_mma <= 256;
       const uint32_t idesc = idesc_bf16_f32(kQuantTileRows, one ? 2 * n_mma : n_mma);
-      int i = i0, seg = 0;   // stage of unit li; streamed, its segment (row blocks since the run's first)
-      for (int li = 0; li < n_local; ++li, ++i) {
-        if (i == nkt) {
-          i = 0;
-          ++seg;
-        }
+      for (int li = 0; li < n_local; ++li) {
         const int s = li % NS;
         const uint32_t ph = (li / NS) & 1;
-        const bool first = li == 0 || i == 0;   // the unit opens a segment
-        // streamed: segment seg accumulates in TMEM block seg % 2, read out by
-        // then for segment seg - 2
-        const uint32_t d = tmem_base + static_cast<uint32_t>(seg & 1) * tmem_cols;
-        if (stream && first && seg >= 2 &&
-            !mbar_wait(&acc_empty[seg & 1], ((seg >> 1) - 1) & 1, p.budget, abort_flag)) {
-          raise_error(kErrWaitQuant);
-          *abort_flag = 1;
-          break;
-        }
         if (!mbar_wait(&full[s], ph, p.budget, abort_flag)) {
           raise_error(kErrWaitQuant);
           *abort_flag = 1;
@@ -313,20 +236,18 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
         const uint32_t b1 = b0 + static_cast<uint32_t>(S * p.r_pad * 128);    // lo slices
 #pragma unroll
         for (int k = 0; k < kQuantBK / 16; ++k) {
-          mma_bf16(d, make_kmajor_desc(a0 + 32 * k, 128), make_kmajor_desc(b0 + 32 * k, 128),
-                   idesc, (!first || k > 0) ? 1u : 0u);
+          mma_bf16(tmem_base, make_kmajor_desc(a0 + 32 * k, 128), make_kmajor_desc(b0 + 32 * k, 128),
+                   idesc, (li > 0 || k > 0) ? 1u : 0u);
         }
         if (!one) {
 #pragma unroll
           for (int k = 0; k < kQuantBK / 16; ++k)
-            mma_bf16(d + static_cast<uint32_t>(n_mma), make_kmajor_desc(a0 + 32 * k, 128),
-                     make_kmajor_desc(b1 + 32 * k, 128), idesc, (!first || k > 0) ? 1u : 0u);
+            mma_bf16(tmem_base + static_cast<uint32_t>(n_mma), make_kmajor_desc(a0 + 32 * k, 128),
+                     make_kmajor_desc(b1 + 32 * k, 128), idesc, (li > 0 || k > 0) ? 1u : 0u);
         }
         tc_commit(&empty[s]);
-        if (stream && (li == n_local - 1 || i == nkt - 1)) tc_commit(&acc_full[seg & 1]);
       }
-      // both also cover an early exit: they wait for every issued MMA
-      tc_commit(stream ? mma_done : acc_full);
+      tc_commit(acc_full);  // also covers an early exit: waits for every issued MMA
     }
   } else {
     // ------------------------------------------------------------ quantizers
@@ -347,25 +268,18 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
     const uint32_t R = q * 32 + lane;          // row of the stacked A tile
     const int st_boxes = BM < 32 ? 2 : 1;                               // code stores per stage
     const int st_j0 = static_cast<int>(q * 32) / BM;                    // sub-tile of the first box
+    const int st_m0 = m0 + static_cast<int>(q * 32) % BM;               // its first token row
     const int j = static_cast<int>(R) / BM;    // K sub-tile
-    float w8_inv = 0.0f;   // W8A8 (never streamed): 1 / this row's token scale, fixed for every stage
+    const int m = m0 + static_cast<int>(R) % BM;
+    const bool row_ok = m < p.M;
+    float w8_inv = 0.0f;   // W8A8: 1 / this row's token scale, fixed for every stage
     if constexpr (FMT == 3) {
-      const int mw = m0 + static_cast<int>(R) % BM;
-      const float sd = reinterpret_cast<const float*>(p.sf)[mw < p.M ? mw : 0];
-      w8_inv = (sd == 0.0f || mw >= p.M) ? 0.0f : __frcp_rn(sd);
+      const float sd = reinterpret_cast<const float*>(p.sf)[row_ok ? m : 0];
+      w8_inv = (sd == 0.0f || !row_ok) ? 0.0f : __frcp_rn(sd);
     }
     const int G = static_cast<int>(L.groups);
-    // stage, first row and (streamed) segment of unit li, stepped G units at a time
-    int i = i0 + grp, mb = m_first, seg = 0;
-    while (i >= nkt) {
-      i -= nkt;
-      mb += BM;
-      ++seg;
-    }
     for (int li = grp < G ? grp : n_local; li < n_local; li += G) {
-      const int st_m0 = mb + static_cast<int>(q * 32) % BM;             // first token row of the code box
-      const int m = mb + static_cast<int>(R) % BM;
-      const bool row_ok = m < p.M;
+      const int i = i0 + li;
       const int s = li % NS;
       const uint32_t ph = (li / NS) & 1;
       const bool ok = warp_wait(&full[s], ph, p.budget, abort_flag);
@@ -482,87 +396,6 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
               row_ok ? static_cast<uint16_t>(sfw) : static_cast<uint16_t>(0);
         }
       }
-      if (stream && has_lr && (li == n_local - 1 || i == nkt - 1)) {
-        // streamed: this group took the segment's last stage, so its four
-        // warps read the segment's accumulator out (rows 32 q .. + 31 each)
-        bool eok = ok;
-        if (eok && !warp_wait(&acc_full[seg & 1], (seg >> 1) & 1, p.budget, abort_flag)) {
-          if (lane == 0) raise_error(kErrWaitQuant);
-          *abort_flag = 1;
-          eok = false;
-        }
-        tc_fence_after();
-        // the CTAs whose runs cover this row block: c_first .. c_last (the run
-        // of CTA c starts at unit floor(c units / G))
-        const int rb = mb / BM;
-        const long long U = p.units, Gr = gridDim.x;
-        const int c_first = static_cast<int>(((static_cast<long long>(rb) * nkt + 1) * Gr + U - 1) / U) - 1;
-        const int c_last = static_cast<int>((static_cast<long long>(rb + 1) * nkt * Gr + U - 1) / U) - 1;
-        const int parts = c_last - c_first + 1;
-        const uint32_t tb = tmem_base + static_cast<uint32_t>(seg & 1) * tmem_cols + ((q * 32u) << 16);
-        float* prow = p.part + (static_cast<size_t>(blockIdx.x + rb) * kQuantTileRows + R) * p.r_pad;
-        if (eok) {
-          for (int c = 0; c < p.r_pad; c += 16) {
-            uint32_t r[16], rl[16];
-            tmem_ld16(tb + c, r);                                      // X hi
-            tmem_ld16(tb + static_cast<uint32_t>(n_mma) + c, rl);      // X lo
-            tmem_wait_ld();
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              float v8[8];
-#pragma unroll
-              for (int e = 0; e < 8; ++e)
-                v8[e] = __fadd_rn(__uint_as_float(r[8 * h + e]), __uint_as_float(rl[8 * h + e]));
-              if (parts == 1) {
-                if (row_ok) {
-#pragma unroll
-                  for (int e = 0; e < 8; ++e) v8[e] = __fadd_rn(0.0f, v8[e]);   // as the parts' sum from 0
-                  store_xl1_pair8(p.xl1, m, p.r_pad, c + 8 * h, v8);
-                }
-              } else {
-                *reinterpret_cast<float4*>(prow + c + 8 * h) = make_float4(v8[0], v8[1], v8[2], v8[3]);
-                *reinterpret_cast<float4*>(prow + c + 8 * h + 4) = make_float4(v8[4], v8[5], v8[6], v8[7]);
-              }
-            }
-          }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[seg & 1]);
-        if (eok && parts > 1) {
-          // the last of the parts' warps for these rows sums them, in the order
-          // of their K ranges, and writes the pair
-          __threadfence();
-          __syncwarp();
-          unsigned prev = 0u;
-          if (lane == 0) prev = atomicAdd(p.cnt + rb * 4 + static_cast<int>(q), 1u);
-          prev = __shfl_sync(0xffffffffu, prev, 0);
-          if (prev == static_cast<unsigned>(parts - 1)) {
-            __threadfence();
-            if (row_ok) {
-              for (int c = 0; c < p.r_pad; c += 8) {
-                float v8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                for (int t = c_first; t <= c_last; ++t) {
-                  const float4* src = reinterpret_cast<const float4*>(
-                      p.part + (static_cast<size_t>(t + rb) * kQuantTileRows + R) * p.r_pad + c);
-                  const float4 a = __ldcg(src), b = __ldcg(src + 1);
-                  v8[0] = __fadd_rn(v8[0], a.x); v8[1] = __fadd_rn(v8[1], a.y);
-                  v8[2] = __fadd_rn(v8[2], a.z); v8[3] = __fadd_rn(v8[3], a.w);
-                  v8[4] = __fadd_rn(v8[4], b.x); v8[5] = __fadd_rn(v8[5], b.y);
-                  v8[6] = __fadd_rn(v8[6], b.z); v8[7] = __fadd_rn(v8[7], b.w);
-                }
-                store_xl1_pair8(p.xl1, m, p.r_pad, c, v8);
-              }
-            }
-          }
-        }
-      }
-      i += G;
-      while (i >= nkt) {
-        i -= nkt;
-        mb += BM;
-        ++seg;
-      }
     }
     if (lane == 0) bulk_wait_group_all();
   }
@@ -582,7 +415,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
   float* red = reinterpret_cast<float*>(smem);
   const int rs = p.r_pad + 4;
   __syncthreads();
-  if (has_lr && !stream && warp >= 2 && warp < 6) {
+  if (has_lr && warp >= 2 && warp < 6) {
     const uint32_t q = warp & 3u;
     const uint32_t R = q * 32 + lane;
     const int j = static_cast<int>(R) / BM;
@@ -619,7 +452,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
   }
   tc_fence_before();
   cluster_sync();   // every CTA of the cluster has parked its blocks (C = 1: the CTA)
-  if (has_lr && !stream) {
+  if (has_lr) {
     // this CTA's BM / C rows x r_pad columns, 8 columns per thread over all threads
     const int rows = BM / p.C;
     const int units = rows * (p.r_pad / 8);
@@ -636,17 +469,28 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
           for (int e = 0; e < 8; ++e) acc[e] = __fadd_rn(acc[e], v[e]);
         }
       }
-      if (m0 + i < p.M) store_xl1_pair8(p.xl1, m0 + i, p.r_pad, c, acc);
+      if (m0 + i < p.M) {
+        // hi = bf16(acc), lo = bf16(acc - hi): hi + lo carries acc to ~2^-17
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          hi[e] = pack_bf16x2(acc[2 * e], acc[2 * e + 1]);
+          lo[e] = pack_bf16x2(acc[2 * e] - bf16_lo(hi[e]), acc[2 * e + 1] - bf16_hi(hi[e]));
+        }
+        __nv_bfloat16* dst = p.xl1 + static_cast<size_t>(m0 + i) * (2 * p.r_pad) + c;
+        *reinterpret_cast<uint4*>(dst) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4*>(dst + p.r_pad) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      }
     }
   }
   // no CTA leaves while a peer may still read its shared memory
   if (p.C > 1) cluster_sync();
   if (warp == 1 && has_lr) {
     // every MMA this CTA issued has retired before its TMEM is released
-    mbar_wait(stream ? mma_done : acc_full, 0, drain_budget(p.budget), nullptr);
+    mbar_wait(acc_full, 0, drain_budget(p.budget), nullptr);
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, tmem_alloc_cols);
+    tmem_dealloc(tmem_base, tmem_cols);
   }
 }
 

@@ -305,25 +305,15 @@ int current_device(int* dev) {
 // peers' partial sums; stage and l1: one 128 x 64 stage, whose L1s share
 // (hi and lo: 2 r_pad / BM bytes per byte of X) travels and is read with it.  Ties go to
 // the smaller C, then the smaller S.
-// A streamed launch (NVFP4, S = C = 1, every CTA an equal run of the row
-// blocks' stages) is modelled as one wave of ceil(units / slots) stages plus
-// the extra read-out of the second segment a run usually holds; it is
-// considered only when the row blocks are at least half as many as the slots,
-// so that no row block is split in more than three parts.
 struct QuantSplit {
   int S, C;
-  bool stream;
 };
 constexpr double kQuantFixedCycles = 10000.0;
 constexpr double kQuantExchangeCycles = 2000.0;
 constexpr double kQuantPerPeerCycles = 1000.0;
 constexpr double kQuantStageCycles = 800.0;
 constexpr double kQuantL1Cycles = 400.0;   // refitted with the hi + lo factor (a forced-shape sweep on B200)
-// a run's second segment: its read-out holds up the quantizer group that
-// takes it (measured at M = 16384: 9k-12k cycles; streaming then wins at
-// K = 12288, 192 stages per row block, and loses at K = 3072)
-constexpr double kQuantSegCycles = 10000.0;
-std::atomic<int> g_forced_split{0};      // svdq_set_quant_split: 16 S + C (C = 0: streamed); 0 = automatic
+std::atomic<int> g_forced_split{0};      // svdq_set_quant_split: 16 S + C; 0 = automatic
 std::atomic<int> g_forced_group_m{0};    // svdq_set_gemm_raster; 0 = automatic
 std::atomic<int> g_forced_gemm_kind{0};  // svdq_set_gemm_kernel; 0 = automatic, 1 = one CTA, 2 = CTA pairs,
                                          // 3 = CTA pairs on 192-column tiles, 4 = 2 with whole tiles only
@@ -331,18 +321,11 @@ std::atomic<int> g_forced_gemm_kind{0};  // svdq_set_gemm_kernel; 0 = automatic,
 QuantSplit quant_split_for(int fmt, int M, int K, int r_pad, const DeviceInfo& d) {
   const int smax = r_pad > 0 ? quant_stack_max(r_pad) : 8;
   const int fs = g_forced_split.load(std::memory_order_relaxed);
-  // the streamed launch: NVFP4, two accumulators of 2 r_pad columns in TMEM
-  const bool can_stream = fmt == SVDQ_NVFP4 && r_pad <= 128 && d.qclusters[1] > 0;
-  const bool forced_stream = fs != 0 && fs % 16 == 0;
-  if (forced_stream) {
-    if (can_stream) return QuantSplit{1, 1, true};
-  } else {
-    const QuantSplit f{fs / 16, fs % 16, false};
-    if (f.S > 0 && f.S <= smax && f.C <= kQuantTileRows / f.S &&
-        f.C <= (K + f.S * kQuantBK - 1) / (f.S * kQuantBK) && d.qclusters[f.C] > 0)
-      return f;
-  }
-  QuantSplit best{1, 1, false};
+  const QuantSplit f{fs / 16, fs % 16};
+  if (f.S > 0 && f.S <= smax && f.C <= kQuantTileRows / f.S &&
+      f.C <= (K + f.S * kQuantBK - 1) / (f.S * kQuantBK) && d.qclusters[f.C] > 0)
+    return f;
+  QuantSplit best{1, 1};
   double best_t = 1e300;
   for (int C = 1; C <= kQuantMaxSplit; C *= 2) {
     const int slots = d.qclusters[C] * C;   // resident CTAs in clusters of C
@@ -362,27 +345,16 @@ QuantSplit quant_split_for(int fmt, int M, int K, int r_pad, const DeviceInfo& d
                         per * (kQuantStageCycles + kQuantL1Cycles * 2 * r_pad / BM));
       if (t < best_t * 0.98) {
         best_t = t;
-        best = {S, C, false};
+        best = {S, C};
       }
     }
-  }
-  const long long row_blocks = (M + kQuantTileRows - 1) / kQuantTileRows;
-  const long long slots = d.qclusters[1];
-  if (can_stream && 2 * row_blocks >= slots) {
-    const long long units = row_blocks * ((K + kQuantBK - 1) / kQuantBK);
-    const long long per = (units + slots - 1) / slots;
-    const double t = kQuantFixedCycles + (r_pad > 0 ? kQuantSegCycles : 0.0) +
-                     static_cast<double>(per) * (kQuantStageCycles + kQuantL1Cycles * 2 * r_pad / kQuantTileRows);
-    if (t < best_t * 0.98) best = {1, 1, true};
   }
   return best;
 }
 
 struct ActLayout {
   int M, M_pad;
-  size_t codes_off, codes_bytes, sf_off, sf_bytes, xl1_off, xl1_bytes;
-  size_t part_off, part_bytes, cnt_off, cnt_bytes;   // streamed activation kernel: partial X_hat L1, arrivals
-  size_t total;
+  size_t codes_off, codes_bytes, sf_off, sf_bytes, xl1_off, xl1_bytes, total;
 };
 
 ActLayout act_layout(const svdq_weights* w, int M) {
@@ -395,21 +367,10 @@ ActLayout act_layout(const svdq_weights* w, int M) {
                : w->fmt == SVDQ_W8A8 ? static_cast<size_t>(L.M_pad) * 4          // fp32 per token
                                      : static_cast<size_t>(w->K / 64) * L.M_pad * 2;
   L.xl1_bytes = static_cast<size_t>(M) * 2 * w->r_pad * 2;   // bf16 hi | lo
-  // streamed activation kernel (NVFP4, r_pad <= 128): one fp32 [128][r_pad]
-  // slot per (CTA, row block) pair a run can touch (slot c + row block: fewer
-  // than CTAs + row blocks), and four arrival counters per row block
-  const int row_blocks = L.M_pad / 128;
-  const int sms = (w->device >= 0 && w->device < kMaxDevices && g_dev[w->device].sms > 0)
-                      ? g_dev[w->device].sms : 1024;
-  const bool streamable = w->fmt == SVDQ_NVFP4 && w->r_pad > 0 && w->r_pad <= 128;
-  L.part_bytes = streamable ? static_cast<size_t>(sms + row_blocks) * 128 * w->r_pad * 4 : 0;
-  L.cnt_bytes = streamable ? static_cast<size_t>(row_blocks) * 4 * 4 : 0;
   L.codes_off = 0;
   L.sf_off = align256(L.codes_bytes);
   L.xl1_off = L.sf_off + align256(L.sf_bytes);
-  L.part_off = L.xl1_off + align256(L.xl1_bytes);
-  L.cnt_off = L.part_off + align256(L.part_bytes);
-  L.total = L.cnt_off + align256(L.cnt_bytes);
+  L.total = L.xl1_off + align256(L.xl1_bytes);
   return L;
 }
 
@@ -856,10 +817,6 @@ SVDQ_API int svdq_set_quant_split(int S, int C) {
     g_forced_split.store(0, std::memory_order_relaxed);
     return SVDQ_OK;
   }
-  if (S == 1 && C == 0) {   // streamed
-    g_forced_split.store(16, std::memory_order_relaxed);
-    return SVDQ_OK;
-  }
   if (!pow2_le8(S) || !pow2_le8(C)) return SVDQ_ERR_INVALID_ARG;
   g_forced_split.store(16 * S + C, std::memory_order_relaxed);
   return SVDQ_OK;
@@ -1117,11 +1074,6 @@ SVDQ_API int svdq_quantize_act(const svdq_weights* w, const void* X, int M, void
   p.sf = base + L.sf_off;
   p.xl1 = reinterpret_cast<__nv_bfloat16*>(base + L.xl1_off);
   p.budget = wait_budget();
-  const int row_blocks = (M + BM - 1) / BM;
-  p.stream = sp.stream ? 1 : 0;
-  p.units = row_blocks * ((w->K + S * kQuantBK - 1) / (S * kQuantBK));
-  p.part = reinterpret_cast<float*>(base + L.part_off);
-  p.cnt = reinterpret_cast<unsigned*>(base + L.cnt_off);
   const QuantSmem Q = quant_smem_layout(w->fmt, w->r_pad, S);
   if (Q.groups < 1 || Q.stages % Q.groups != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
   // the X_hat L1 epilogue parks [128][r_pad + 4] fp32 over the stage and staging buffers
@@ -1132,14 +1084,8 @@ SVDQ_API int svdq_quantize_act(const svdq_weights* w, const void* X, int M, void
     const size_t off = static_cast<size_t>(w->K / 64) * 512;
     SVDQ_CUDA(cudaMemset2DAsync(p.sf + off, pitch, 0, pitch - off, L.M_pad / 128, st));
   }
-  // clusters of C consecutive CTAs share a row block, one K range each; or
-  // (streamed) one CTA per resident slot, each an equal run of the units
-  const dim3 grid(sp.stream ? std::min(p.units, g_dev[dev].qclusters[1]) : row_blocks * sp.C);
-  if (sp.stream && w->r_pad > 0) {
-    if (grid.x + row_blocks > L.part_bytes / (static_cast<size_t>(128) * w->r_pad * 4))
-      return SVDQ_ERR_UNSUPPORTED_SHAPE;
-    SVDQ_CUDA(cudaMemsetAsync(p.cnt, 0, L.cnt_bytes, st));
-  }
+  // clusters of C consecutive CTAs share a row block, one K range each
+  const dim3 grid(((M + BM - 1) / BM) * sp.C);
   const unsigned C = static_cast<unsigned>(sp.C);
   const CUtensorMap& tm_l1t = w->r_pad > 0 ? w->tm_l1t : tm_x;
   const dim3 blk(kQuantThreads);
